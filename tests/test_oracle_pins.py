@@ -1,0 +1,365 @@
+"""Pins of the CPU oracle against what the source pages and the mathematics
+fix, independent of the oracle's own code.
+
+Page: "3比特逼近4比特精度？WARP残差向量量化VQ3R的完整测量实验"
+(xdnf.cn/news/289497), §2 (format, reconstruction rule, Lloyd codebooks),
+§3.1 (relative Frobenius error, rtn4-row, vq2), §4 (greedy single pass).
+"""
+import itertools
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+K, D = 256, 8
+
+
+# ---------------------------------------------------------------- helpers
+
+def sign_pattern_codebooks(a=1.0):
+    """C1 = all 256 sign patterns of +-a (bit k of j set <=> dim k negative),
+    C2 = same with a/2, C3 = same with a/4."""
+    j = np.arange(K)[:, None]
+    k = np.arange(D)[None, :]
+    sgn = np.where((j >> k) & 1, -1.0, 1.0)
+    return np.stack([sgn * a, sgn * a / 2, sgn * a / 4]).astype(np.float32)
+
+
+def energy8_vectors(rng, n):
+    """n vectors with entries k/4 (k integer in [-8, 8], zeros included) whose
+    8 squares sum to exactly 8, so a row made of them has RMS exactly 1."""
+    tuples = []
+    for combo in itertools.combinations_with_replacement(range(0, 9), D):
+        if sum(c * c for c in combo) == 128 and len(set(combo)) >= 3:
+            tuples.append(combo)
+    assert len(tuples) > 10
+    out = np.empty((n, D), dtype=np.float32)
+    for i in range(n):
+        t = np.array(tuples[rng.integers(len(tuples))], dtype=np.float64)
+        rng.shuffle(t)
+        t *= rng.choice([-1.0, 1.0], size=D)
+        out[i] = t / 4.0
+    return out
+
+
+# ---------------------------------------------------------------- generator
+
+def test_philox_known_answers():
+    """Philox4x32-10 known-answer vectors (Salmon et al., SC'11, Random123 KAT)."""
+    assert synth.philox([0, 0, 0, 0], [0, 0]) == [0x6627e8d5, 0xe169c58d, 0xbc57ac4c, 0x9b00dbd8]
+    assert synth.philox([0xffffffff] * 4, [0xffffffff] * 2) == [0x408f276d, 0x41c83b0e, 0xa20bc7c6, 0x6d5451fd]
+    assert synth.philox([0x243f6a88, 0x85a308d3, 0x13198a2e, 0x03707344], [0xa4093822, 0x299f31d0]) == \
+        [0xd16cfe09, 0x94fdcceb, 0x5001e420, 0x24126ea1]
+
+
+def test_generator_moments_and_row_independence():
+    d = synth.normal()
+    a = synth.fill_rows(4096, 0, 64, 7, 3, d, dtype="f32")
+    assert abs(a.mean()) < 0.01 and abs(a.std() - 1.0) < 0.01
+    # any row range regenerates the same values
+    b = synth.fill_rows(4096, 17, 5, 7, 3, d, dtype="f32")
+    np.testing.assert_array_equal(a[17:22], b)
+    c = synth.fill_row_list(4096, [40, 2, 40], 7, 3, d, dtype="f32")
+    np.testing.assert_array_equal(c[0], a[40])
+    np.testing.assert_array_equal(c[1], a[2])
+    t = synth.fill_rows(2048, 0, 64, 7, 3, synth.student_t(4), dtype="f32").astype(np.float64)
+    # Student-t(4) variance = df / (df - 2) = 2
+    assert abs(t.var() - 2.0) < 0.15
+
+
+def test_sample_without_replacement():
+    s = synth.sample(5, 9, 100000, 5000)
+    assert len(np.unique(s)) == 5000 and s.min() >= 0 and s.max() < 100000
+    assert abs(s.mean() - 50000) < 2000
+    np.testing.assert_array_equal(s[:100], synth.sample(5, 9, 100000, 100))
+
+
+# ---------------------------------------------------------------- conversions
+
+def test_fp16_rounding_matches_numpy():
+    rng = np.random.default_rng(0)
+    xs = np.concatenate([rng.standard_normal(2000) * 10.0 ** rng.integers(-8, 5, 2000),
+                         [0.0, -0.0, 1.0, 65504.0, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26, 2.0 ** -14]])
+    for x in xs:
+        assert oracle.fp16_from_double_sat(x) == int(np.float16(x).view(np.uint16)), x
+        h = int(np.float16(x).view(np.uint16))
+        assert oracle.fp16_to_double(h) == float(np.float16(x))
+
+
+def test_fp16_midpoints_and_saturation():
+    assert oracle.fp16_from_double_sat(1 + 2 ** -11) == 0x3C00          # tie -> even (1.0)
+    assert oracle.fp16_from_double_sat(1 + 3 * 2 ** -11) == 0x3C02      # tie -> even (1 + 2^-9)
+    assert oracle.fp16_from_double_sat(65520.0) == 0x7BFF               # saturating reading
+    assert oracle.fp16_from_double_sat(1e9) == 0x7BFF
+    assert oracle.fp16_from_float(65520.0) == 0x7C00                    # plain conversion: inf
+    assert oracle.fp16_from_double_sat(2.0 ** -25) == 0x0000            # tie -> even (0)
+    assert oracle.fp16_from_double_sat(3 * 2.0 ** -25) == 0x0002
+
+
+# ---------------------------------------------------------------- scale (§2)
+
+@pytest.mark.parametrize("cols", [8, 512, 2048, 7168])
+def test_scale_of_constant_magnitude_rows(cols):
+    rng = np.random.default_rng(cols)
+    for m in [2.0 ** -10, 0.25, 1.0, 4.0, 1024.0]:
+        W = (rng.choice([-1.0, 1.0], size=(3, cols)) * m).astype(np.float32)
+        sc = oracle.row_scales(W, "f32")
+        assert all(oracle.fp16_to_double(s) == m for s in sc)
+
+
+def test_scale_rne_midpoints_and_limits():
+    W = np.full((4, 1024), 1 + 2 ** -11, dtype=np.float32)
+    W[1] = 1 + 3 * 2 ** -11
+    W[2] = 70000.0
+    W[3] = 2.0 ** -20
+    sc = oracle.row_scales(W, "f32")
+    assert list(sc) == [0x3C00, 0x3C02, 0x7BFF, 0x0010]
+    assert oracle.row_scales(np.zeros((1, 64), np.float32), "f32")[0] == 0
+
+
+def test_scale_equals_correctly_rounded_rms():
+    """binary16(sqrt(mean w^2)) with the mean taken exactly (math.fsum)."""
+    rng = np.random.default_rng(1)
+    for cols in (8, 512, 7168):
+        W = (rng.standard_normal((16, cols)) * np.exp(rng.standard_normal((16, 1)))).astype(np.float32)
+        sc = oracle.row_scales(W, "f32")
+        for i in range(16):
+            ss = math.fsum(float(w) * float(w) for w in W[i])
+            ref = np.float16(math.sqrt(ss / cols))
+            assert sc[i] == int(ref.view(np.uint16))
+
+
+# ---------------------------------------------------------------- encode/decode closed forms
+
+def _greedy_scalar_levels(r):
+    """Per-dimension greedy binary expansion with step a, a/2, a/4 (a = 1),
+    exact in rationals; a zero residual takes the positive codeword."""
+    bits = np.zeros((3, D), dtype=np.int64)
+    w = np.zeros(D, dtype=np.float64)
+    for k in range(D):
+        e = Fraction(float(r[k]))
+        acc = Fraction(0)
+        for s, step in enumerate([Fraction(1), Fraction(1, 2), Fraction(1, 4)]):
+            neg = e < 0
+            bits[s, k] = 1 if neg else 0
+            c = -step if neg else step
+            e -= c
+            acc += c
+        w[k] = float(acc)
+    return bits, w
+
+
+def test_sign_pattern_codebooks_equal_scalar_quantizer():
+    """With sign-pattern codebooks (+-1, +-1/2, +-1/4) greedy RVQ is the uniform
+    8-level scalar quantizer +-{1.75, 1.25, 0.75, 0.25} per dimension, ties to
+    the lower index (positive codeword); all arithmetic is exact."""
+    rng = np.random.default_rng(2)
+    cb = sign_pattern_codebooks()
+    V, rows = 16, 24
+    W = energy8_vectors(rng, rows * V).reshape(rows, V * D)
+    idx, sc = oracle.encode(W, "f32", cb)
+    assert all(s == 0x3C00 for s in sc)  # RMS exactly 1
+    What = oracle.decode(idx, sc, cb)
+    for i in range(rows):
+        for v in range(V):
+            bits, w = _greedy_scalar_levels(W[i, v * D:(v + 1) * D])
+            for s in range(3):
+                assert idx[s, i, v] == int(sum(int(b) << k for k, b in enumerate(bits[s])))
+            np.testing.assert_array_equal(What[i, v * D:(v + 1) * D], w.astype(np.float32))
+
+
+def test_permuted_sign_codebooks_tie_goes_to_lowest_index():
+    rng = np.random.default_rng(3)
+    cb = sign_pattern_codebooks()
+    perm = rng.permutation(K)
+    cbp = cb[:, perm, :]
+    r = energy8_vectors(rng, 200)
+    r[:, 0] = 0.0  # force a tie in dimension 0 at stage 1
+    idx, _ = oracle.encode_vectors(r, cbp, nstages=1)
+    for i in range(200):
+        # codewords whose signs match every nonzero dimension all tie; lowest position wins
+        cand = []
+        for pos in range(K):
+            j = perm[pos]
+            ok = all(r[i, k] == 0 or ((j >> k) & 1) == (1 if r[i, k] < 0 else 0) for k in range(D))
+            if ok:
+                cand.append(pos)
+        assert idx[i, 0] == min(cand)
+
+
+def test_planted_exact_reconstruction():
+    """Rows s * C1[pi(v)] with +-1 sign-pattern C1 and zero codeword 0 in C2, C3:
+    scale = s exactly, indices (pi(v), 0, 0), decode exact, error 0."""
+    rng = np.random.default_rng(4)
+    cb = sign_pattern_codebooks()
+    cb[0] = cb[0][rng.permutation(K)]
+    cb[1] = rng.standard_normal((K, D)).astype(np.float32) * 0.3
+    cb[2] = rng.standard_normal((K, D)).astype(np.float32) * 0.1
+    cb[1, 0] = 0.0
+    cb[2, 0] = 0.0
+    rows, V = 12, 32
+    pi = rng.integers(0, K, size=(rows, V))
+    svals = np.array([0.75, 3.0, 2.0 ** -6, 1.5, 40.0, 0.125] * 2, dtype=np.float32)
+    W = (cb[0][pi].reshape(rows, V * D) * svals[:, None]).astype(np.float32)
+    Wb = synth.bf16_bits_to_f32((W.view(np.uint32) >> 16).astype(np.uint16))
+    np.testing.assert_array_equal(Wb, W)  # exactly representable in bf16 too
+    for dt, Win in (("f32", W), ("bf16", (W.view(np.uint32) >> 16).astype(np.uint16))):
+        idx, sc = oracle.encode(Win, dt, cb)
+        np.testing.assert_array_equal([oracle.fp16_to_double(s) for s in sc], svals.astype(np.float64))
+        np.testing.assert_array_equal(idx[0], pi)
+        assert not idx[1].any() and not idx[2].any()
+        What = oracle.decode(idx, sc, cb)
+        np.testing.assert_array_equal(What, W)
+        assert oracle.rel_frobenius(Win, dt, What) == 0.0
+
+
+def test_zero_row_and_zero_scale():
+    cb = sign_pattern_codebooks()
+    W = np.zeros((2, 16), np.float32)
+    W[1] = 2.0 ** -30  # RMS underflows binary16 -> scale 0 -> r = 0
+    idx, sc = oracle.encode(W, "f32", cb)
+    assert list(sc) == [0, 0]
+    What = oracle.decode(idx, sc, cb)
+    assert not What.any()
+
+
+def test_bits_per_weight_is_three():
+    rng = np.random.default_rng(5)
+    cb = rng.standard_normal((3, K, D)).astype(np.float32)
+    for rows, cols in ((3, 8), (5, 512), (2, 7168)):
+        W = rng.standard_normal((rows, cols)).astype(np.float32)
+        idx, sc = oracle.encode(W, "f32", cb)
+        assert idx.nbytes == 3 * rows * cols // 8
+        assert idx.nbytes * 8 / (rows * cols) == 3.0
+        assert sc.nbytes * 8 / (rows * cols) == 16 / cols
+
+
+# ---------------------------------------------------------------- greedy vs exhaustive
+
+def test_exhaustive_joint_search_lower_bounds_greedy():
+    rng = np.random.default_rng(6)
+    cb = (rng.standard_normal((3, K, D)) * np.array([1.0, 0.5, 0.25])[:, None, None]).astype(np.float32)
+    r = rng.standard_normal((6, D)).astype(np.float32)
+    idx, _ = oracle.encode_vectors(r, cb)
+    g = cb[0][idx[:, 0]].astype(np.float64) + cb[1][idx[:, 1]] + cb[2][idx[:, 2]]
+    greedy_err = ((r.astype(np.float64) - g) ** 2).sum(1)
+    bidx, berr = oracle.bruteforce_joint(r, cb)
+    assert np.all(berr <= greedy_err + 1e-12)
+    # the exhaustive result is the reported triple's error
+    bj = cb[0][bidx[:, 0]].astype(np.float64) + cb[1][bidx[:, 1]] + cb[2][bidx[:, 2]]
+    np.testing.assert_allclose(((r.astype(np.float64) - bj) ** 2).sum(1), berr, rtol=1e-12)
+
+
+def test_exhaustive_equals_greedy_when_later_stages_are_zero():
+    rng = np.random.default_rng(7)
+    cb = np.zeros((3, K, D), np.float32)
+    cb[0] = rng.standard_normal((K, D))
+    r = rng.standard_normal((4, D)).astype(np.float32)
+    idx, _ = oracle.encode_vectors(r, cb)
+    bidx, _ = oracle.bruteforce_joint(r, cb)
+    np.testing.assert_array_equal(bidx[:, 0], idx[:, 0])
+
+
+# ---------------------------------------------------------------- Lloyd (§2, §4)
+
+def test_lloyd_recovers_separated_centres():
+    rng = np.random.default_rng(8)
+    centres = (rng.integers(-64, 64, size=(K, D)) * 4.0).astype(np.float32)
+    centres[:, 0] = np.arange(K) * 8.0  # all distinct and far apart
+    off = np.zeros((4, D), np.float32)
+    off[0, 1], off[1, 1], off[2, 2], off[3, 2] = 0.125, -0.125, 0.25, -0.25
+    pts = (centres[None, :, :] + off[:, None, :]).reshape(-1, D)  # first 256 = one per cluster
+    cb, tr = oracle.lloyd_train(pts, iters=2, nstages=1)
+    np.testing.assert_array_equal(cb[0], centres)
+    assert tr[0, -1] == pytest.approx(K * (2 * 0.125 ** 2 + 2 * 0.25 ** 2))
+
+
+def test_lloyd_matches_sklearn_lloyd():
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(9)
+    X = rng.standard_normal((2048, D)).astype(np.float32)
+    cb, _ = oracle.lloyd_train(X, iters=3, nstages=1)
+    km = KMeans(n_clusters=K, init=X[:K].astype(np.float64), n_init=1, max_iter=3, tol=0.0,
+                algorithm="lloyd").fit(X.astype(np.float64))
+    close = np.all(np.abs(km.cluster_centers_ - cb[0]) < 1e-5, axis=1)
+    assert close.mean() > 0.95
+
+
+def test_lloyd_distortion_non_increasing_and_stages_reduce_error():
+    rng = np.random.default_rng(10)
+    X = rng.standard_normal((8192, D)).astype(np.float32)
+    cb, tr = oracle.lloyd_train(X, iters=6)
+    for s in range(3):
+        assert np.all(np.diff(tr[s]) <= 1e-6 * tr[s][0])
+    # on the training set each stage lowers total distortion (cluster means
+    # minimise squared error; zero is always a worse candidate centre)
+    e = []
+    for ns in (1, 2, 3):
+        _, res = oracle.encode_vectors(X, cb[:ns], nstages=ns)
+        e.append(float((res.astype(np.float64) ** 2).sum()))
+    assert e[0] > e[1] > e[2]
+    assert e[0] < float((X.astype(np.float64) ** 2).sum())
+    # stage s training distortion equals the encoder's residual energy
+    np.testing.assert_allclose(tr[2, -1], e[2], rtol=1e-6)
+
+
+# ---------------------------------------------------------------- metric, GEMV, rtn4-row (§3.1)
+
+def test_rel_frobenius_closed_forms():
+    rng = np.random.default_rng(11)
+    Wf = rng.standard_normal((8, 64)).astype(np.float32)
+    W = (Wf.view(np.uint32) >> 16).astype(np.uint16)
+    Wx = synth.bf16_bits_to_f32(W)
+    assert oracle.rel_frobenius(W, "bf16", Wx) == 0.0
+    assert oracle.rel_frobenius(W, "bf16", np.zeros_like(Wx)) == 1.0
+    assert oracle.rel_frobenius(W, "bf16", Wx * np.float32(0.875)) == 0.125
+
+
+def test_gemv_matches_float64_matmul():
+    rng = np.random.default_rng(12)
+    What = rng.standard_normal((33, 520)).astype(np.float32)
+    x = rng.standard_normal((5, 520)).astype(np.float32)
+    y = oracle.gemv(What, x, "f32")
+    ref = x.astype(np.float64) @ What.astype(np.float64).T
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_rtn4_row_exact_grid_and_clamp():
+    rng = np.random.default_rng(13)
+    s = np.float32(0.375)
+    q = rng.integers(-7, 8, size=(4, 64)).astype(np.float32)
+    q[:, 0] = 7
+    W = q * s
+    What, sc = oracle.rtn4_row(W, "f32")
+    assert all(oracle.fp16_to_double(h) == 0.375 for h in sc)
+    np.testing.assert_array_equal(What, W)
+    # a value of -7.6 scales rounds to -8 (inside the int4 range); with max |w| = 7.6 s the
+    # scale is fp16(7.6 s / 7) and the extreme maps to +-7
+    W2 = np.array([[7.0, -3.0, 1.0, 0.0] * 2], np.float32)
+    W2[0, 1] = -7.6
+    What2, sc2 = oracle.rtn4_row(W2, "f32")
+    s2 = oracle.fp16_to_double(sc2[0])
+    assert s2 == float(np.float16(7.6 / 7))
+    assert What2[0, 1] == np.float32(-7 * s2)
+
+
+# ---------------------------------------------------------------- sanity bands (not pins)
+
+def test_tiny_pipeline_sanity_bands():
+    """The tiny N(0,1) 256 x 512 case: errors in the expected bands and ordered
+    rtn4-row < vq3 < vq2, the pattern of the Gate 3 table (§3.1)."""
+    W = synth.fill_rows(512, 0, 256, 0, 0, synth.normal(), dtype="f32")
+    sc = oracle.row_scales(W, "f32")
+    vecs = oracle.normalize_rows(W, "f32", sc)
+    cb, _ = oracle.lloyd_train(vecs, iters=10)
+    idx3, sc3 = oracle.encode(W, "f32", cb)
+    e3 = oracle.rel_frobenius(W, "f32", oracle.decode(idx3, sc3, cb))
+    idx2, sc2 = oracle.encode(W, "f32", cb[:2], nstages=2)
+    e2 = oracle.rel_frobenius(W, "f32", oracle.decode(idx2, sc2, cb[:2]))
+    rt, _ = oracle.rtn4_row(W, "f32")
+    e4 = oracle.rel_frobenius(W, "f32", rt)
+    assert 0.10 < e3 < 0.26 and e2 > e3 and 0.10 < e4 < 0.18, (e4, e3, e2)
