@@ -1,0 +1,165 @@
+/*
+ * vq3r.h -- C ABI of the VQ3R codec library for NVIDIA B200 (sm_100a).
+ *
+ * VQ3R (page "3比特逼近4比特精度？WARP残差向量量化VQ3R的完整测量实验",
+ * xdnf.cn/news/289497, §2) stores a weight matrix W (rows x cols, a row being
+ * one output channel) as
+ *   - one FP16 scale per row, and
+ *   - for each 8-wide vector W[i, 8v : 8v+8], three uint8 indices i1, i2, i3
+ *     into three 256-entry codebooks C1, C2, C3 of 8-dim fp32 vectors,
+ * so that W[i, 8v+k] ~ scale_i * (C1[i1][k] + C2[i2][k] + C3[i3][k]):
+ * 3 index bytes per 8 weights = exactly 3.00 bits/weight.
+ *
+ * Layouts (all row-major, no padding):
+ *   W          [rows][cols]             f32, bf16 or f16
+ *   codebooks  [3][256][8] float        stage-major (C1, then C2, then C3), 24 KiB
+ *   idx        [3][rows][cols/8] uint8  three index planes, plane s = stage s+1
+ *   scales     [rows] uint16            IEEE binary16 bit patterns
+ *   x          [B][cols]                activations, f32, bf16 or f16
+ *   y          [B][rows] float
+ *
+ * Conventions shared by every call:
+ *   - Every data pointer is DEVICE memory owned by the caller, 16-byte
+ *     aligned (VQ3R_ERR_ALIGN otherwise).  The library never allocates or
+ *     frees device memory; temporary storage is the caller's `workspace`.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and return after enqueuing the work.
+ *   - Argument errors are detected before anything is launched and nothing
+ *     is written.  A failed launch returns VQ3R_ERR_CUDA.
+ *   - cols must be a positive multiple of 8 (VQ3R_ERR_SHAPE).
+ *   - Calls that overlap on the GPU must not share output or workspace
+ *     buffers.
+ */
+#ifndef VQ3R_H
+#define VQ3R_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VQ3R_OK = 0,
+  VQ3R_ERR_NULL = 1,      /* a required pointer is NULL */
+  VQ3R_ERR_SHAPE = 2,     /* rows < 0 (or < 1 where stated), cols < 8, cols % 8 != 0, size overflow */
+  VQ3R_ERR_ALIGN = 3,     /* a device pointer is not 16-byte aligned */
+  VQ3R_ERR_DTYPE = 4,     /* unsupported dtype for this argument */
+  VQ3R_ERR_BATCH = 5,     /* B outside [1, 32], or n_mats outside [1, VQ3R_GEMV_MAX_MATS] */
+  VQ3R_ERR_CUDA = 6,      /* a CUDA call or kernel launch failed (see vq3r_last_cuda_error) */
+  VQ3R_ERR_WORKSPACE = 7  /* workspace NULL or smaller than the *_workspace_size result */
+} vq3r_status;
+
+typedef enum { VQ3R_F32 = 0, VQ3R_BF16 = 1, VQ3R_F16 = 2 } vq3r_dtype;
+
+typedef void* vq3r_stream; /* cudaStream_t */
+
+#define VQ3R_STAGES 3
+#define VQ3R_CODEWORDS 256
+#define VQ3R_DIM 8
+#define VQ3R_GEMV_MAX_B 32
+#define VQ3R_GEMV_MAX_MATS 32
+
+/*
+ * vq3r_encode -- per-row FP16 scale and greedy 3-stage residual assignment.
+ *
+ * Page §2 (per-row FP16 scale, 3 stages of 256 x 8-dim codebooks, stage s
+ * quantises the residual left by stage s-1) and §4 (one pass over the three
+ * stages writing only the winning indices).  For row i:
+ *   scale_i = binary16(sqrt(ss_i / cols)), RNE, saturating at 65504, where
+ *     ss_i is the binary64 sum of w^2 taken in a fixed order: per 8-vector
+ *     q_v = ((w0^2 + w1^2) + ...) + w7^2, partials t_p = sum over v = p mod 128
+ *     (v ascending), then t_p += t_{p+h} for h = 64, 32, ..., 1.
+ *   r = (float)w / (float)scale_i (IEEE division; r = 0 if scale_i = 0).
+ * For each stage s = 1..3: d_j = sum_{k=0..7} (r_k - C_s[j][k])^2 in binary32,
+ * k ascending, every operation rounded (no fused multiply-add); i_s = the
+ * j with the smallest d_j, the lowest j on ties; r -= C_s[i_s].
+ * Results are bit-identical to that definition.
+ *
+ *   W         [rows][cols], w_dtype in {F32, BF16, F16}
+ *   codebooks [3][256][8] float
+ *   idx       out, [3][rows][cols/8] uint8
+ *   scales    out, [rows] binary16 bits
+ * rows == 0 is a no-op (pointers may then be NULL).  Non-finite weights give
+ * unspecified (but in-bounds) indices.
+ */
+vq3r_status vq3r_encode(const void* W, vq3r_dtype w_dtype, int64_t rows, int64_t cols, const float* codebooks,
+                        uint8_t* idx, uint16_t* scales, vq3r_stream stream);
+
+/*
+ * vq3r_decode -- reconstruct the weights (page §2 reconstruction rule).
+ *   w_hat[i][8v+k] = (float)scale_i * ((C1[i1][k] + C2[i2][k]) + C3[i3][k])
+ * in binary32, every operation rounded; an F16 output is the RNE conversion
+ * of that binary32 value (overflow to +-inf).
+ *
+ *   idx, scales, codebooks as written by vq3r_encode
+ *   out       [rows][cols], out_dtype in {F32, F16}
+ * rows == 0 is a no-op (pointers may then be NULL).
+ */
+vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float* codebooks, int64_t rows,
+                        int64_t cols, void* out, vq3r_dtype out_dtype, vq3r_stream stream);
+
+/*
+ * vq3r_gemv -- y = W_hat . x for a group of VQ3R matrices, B = 1..32 tokens
+ * (the MoE decode step, page §1: a few experts' matrices per token).
+ *   y[b][i] = sum_c w_hat[i][c] * x[b][c], fp32 accumulation, w_hat as in
+ *   vq3r_decode.  Summation order is the library's own: results agree with
+ *   an exact (binary64) product to about 1e-4 relative to rms(y), not bit
+ *   for bit.
+ *
+ * One descriptor per matrix; matrices may differ in shape, codebooks and x.
+ * Matrices that share (codebooks, x, cols) share one x-projected table in
+ * the workspace, so one call over the gate and up matrices of all active
+ * experts reads x once.  y must not overlap any input.
+ *   mats      HOST array of n_mats descriptors (copied before return)
+ *   B         tokens, 1..32
+ *   x_dtype   dtype of every x, {F32, BF16, F16}
+ *   workspace device scratch of at least vq3r_gemv_workspace_size() bytes
+ * A matrix with rows == 0 contributes nothing (its pointers may be NULL).
+ */
+typedef struct {
+  const uint8_t* idx;       /* [3][rows][cols/8] */
+  const uint16_t* scales;   /* [rows] binary16 */
+  const float* codebooks;   /* [3][256][8] */
+  int64_t rows, cols;
+  const void* x;            /* [B][cols] */
+  float* y;                 /* [B][rows] */
+} vq3r_gemv_desc;
+
+size_t vq3r_gemv_workspace_size(const vq3r_gemv_desc* mats, int n_mats, int B);
+vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype x_dtype, void* workspace,
+                      size_t ws_bytes, vq3r_stream stream);
+
+/*
+ * vq3r_rel_frobenius_error -- the Gate 3 metric of page §3.1:
+ *   err = sqrt( sum (w - w_hat)^2 / sum w^2 ),
+ * w the original weight widened to binary64, w_hat the binary32 decode of
+ * vq3r_decode, both sums accumulated in binary64 (library order; agrees with
+ * a sequential binary64 sum to ~1e-12 relative).
+ *
+ *   W, w_dtype   original weights [rows][cols]
+ *   err_out      DEVICE pointer to one double (written asynchronously)
+ *   workspace    at least vq3r_rel_frobenius_workspace_size() bytes
+ * rows must be >= 1.  An all-zero W gives NaN (0/0).
+ */
+size_t vq3r_rel_frobenius_workspace_size(int64_t rows, int64_t cols);
+vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const uint8_t* idx, const uint16_t* scales,
+                                     const float* codebooks, int64_t rows, int64_t cols, double* err_out,
+                                     void* workspace, size_t ws_bytes, vq3r_stream stream);
+
+/* Human-readable name of a status code (static string). */
+const char* vq3r_status_string(vq3r_status s);
+
+/* cudaError_t value of the most recent VQ3R_ERR_CUDA on the calling thread (0 if none). */
+int vq3r_last_cuda_error(void);
+
+/* Device-side error word, set by a kernel whose bounded wait on an
+ * asynchronous copy gave up (0 = none).  Synchronises the current device;
+ * reading it clears it. */
+vq3r_status vq3r_device_error(int* code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VQ3R_H */

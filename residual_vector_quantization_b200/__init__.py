@@ -1,0 +1,163 @@
+"""VQ3R codec for NVIDIA B200: thin Python binding of libvq3r.so.
+
+The names mirror the C ABI in include/vq3r.h (vq3r_encode, vq3r_decode,
+vq3r_gemv, vq3r_rel_frobenius_error).  This module only marshals arguments:
+torch supplies device memory and the current stream; every step of the
+codec runs in the library's CUDA kernels.  There is no CPU fallback: if
+the library is missing, importing a function raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_DIR, "csrc", "libvq3r.so")
+
+VQ3R_F32, VQ3R_BF16, VQ3R_F16 = 0, 1, 2
+_DT = {torch.float32: VQ3R_F32, torch.bfloat16: VQ3R_BF16, torch.float16: VQ3R_F16}
+STAGES, CODEWORDS, DIM = 3, 256, 8
+GEMV_MAX_B = 32
+GEMV_MAX_MATS = 32
+
+EXPORTED = ["vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_gemv_workspace_size", "vq3r_rel_frobenius_error",
+            "vq3r_rel_frobenius_workspace_size", "vq3r_status_string", "vq3r_last_cuda_error",
+            "vq3r_device_error"]
+
+
+class VQ3RError(RuntimeError):
+    def __init__(self, status, where):
+        msg = _lib().vq3r_status_string(status).decode()
+        if status == 6:
+            msg += " (cudaError %d)" % _lib().vq3r_last_cuda_error()
+        super().__init__("%s: %s" % (where, msg))
+        self.status = status
+
+
+class GemvDesc(ctypes.Structure):
+    _fields_ = [("idx", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("codebooks", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
+
+
+_L = None
+
+
+def _lib():
+    global _L
+    if _L is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libvq3r.so is not built (run residual_vector_quantization_b200.build.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.vq3r_encode.argtypes = [P, I32, I64, I64, P, P, P, P]
+        L.vq3r_decode.argtypes = [P, P, P, I64, I64, P, I32, P]
+        L.vq3r_gemv.argtypes = [P, I32, I32, I32, P, SZ, P]
+        L.vq3r_gemv_workspace_size.argtypes = [P, I32, I32]
+        L.vq3r_gemv_workspace_size.restype = SZ
+        L.vq3r_rel_frobenius_error.argtypes = [P, I32, P, P, P, I64, I64, P, P, SZ, P]
+        L.vq3r_rel_frobenius_workspace_size.argtypes = [I64, I64]
+        L.vq3r_rel_frobenius_workspace_size.restype = SZ
+        L.vq3r_status_string.argtypes = [I32]
+        L.vq3r_status_string.restype = ctypes.c_char_p
+        L.vq3r_last_cuda_error.restype = I32
+        L.vq3r_device_error.argtypes = [P]
+        for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error"):
+            getattr(L, f).restype = I32
+        _L = L
+    return _L
+
+
+def lib():
+    """The loaded ctypes handle of libvq3r.so."""
+    return _lib()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(st, where):
+    if st != 0:
+        raise VQ3RError(st, where)
+
+
+def _dev(t, name):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.is_contiguous()):
+        raise ValueError("%s must be a contiguous CUDA tensor" % name)
+    return t.data_ptr()
+
+
+def vq3r_encode(W, codebooks, idx=None, scales=None, stream=None):
+    """Encode W [rows][cols] (f32/bf16/f16) -> (idx uint8 [3][rows][cols/8], scales int16 [rows] fp16 bits)."""
+    rows, cols = W.shape
+    if idx is None:
+        idx = torch.empty((STAGES, rows, cols // DIM), dtype=torch.uint8, device=W.device)
+    if scales is None:
+        scales = torch.empty(rows, dtype=torch.int16, device=W.device)
+    if W.dtype not in _DT:
+        raise ValueError("W dtype must be float32, bfloat16 or float16")
+    _check(_lib().vq3r_encode(_dev(W, "W"), _DT[W.dtype], rows, cols, _dev(codebooks, "codebooks"),
+                              _dev(idx, "idx"), _dev(scales, "scales"), _stream(stream)), "vq3r_encode")
+    return idx, scales
+
+
+def vq3r_decode(idx, scales, codebooks, out_dtype=torch.float32, out=None, stream=None):
+    """Reconstruct W_hat [rows][cols] as float32 or float16."""
+    _, rows, V = idx.shape
+    if out is None:
+        out = torch.empty((rows, V * DIM), dtype=out_dtype, device=idx.device)
+    _check(_lib().vq3r_decode(_dev(idx, "idx"), _dev(scales, "scales"), _dev(codebooks, "codebooks"), rows,
+                              V * DIM, _dev(out, "out"), _DT[out.dtype], _stream(stream)), "vq3r_decode")
+    return out
+
+
+def _descs(mats):
+    arr = (GemvDesc * len(mats))()
+    for i, m in enumerate(mats):
+        idx, scales, cb, x, y = m["idx"], m["scales"], m["codebooks"], m["x"], m["y"]
+        arr[i] = GemvDesc(_dev(idx, "idx"), _dev(scales, "scales"), _dev(cb, "codebooks"), idx.shape[1],
+                          idx.shape[2] * DIM, _dev(x, "x"), _dev(y, "y"))
+    return arr
+
+
+def vq3r_gemv_workspace_size(mats, B):
+    arr = _descs(mats)
+    return _lib().vq3r_gemv_workspace_size(arr, len(mats), B)
+
+
+def vq3r_gemv(mats, B, workspace=None, stream=None):
+    """y = W_hat . x for each descriptor dict {idx, scales, codebooks, x [B][cols], y [B][rows] float32}."""
+    arr = _descs(mats)
+    ws = _lib().vq3r_gemv_workspace_size(arr, len(mats), B)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=mats[0]["idx"].device)
+    xdt = _DT[mats[0]["x"].dtype]
+    _check(_lib().vq3r_gemv(arr, len(mats), B, xdt, _dev(workspace, "workspace"), workspace.numel(),
+                            _stream(stream)), "vq3r_gemv")
+    return [m["y"] for m in mats]
+
+
+def vq3r_rel_frobenius_workspace_size(rows, cols):
+    return _lib().vq3r_rel_frobenius_workspace_size(rows, cols)
+
+
+def vq3r_rel_frobenius_error(W, idx, scales, codebooks, out=None, workspace=None, stream=None):
+    """Device float64 tensor [1] holding sqrt(sum (w - w_hat)^2 / sum w^2)."""
+    rows, cols = W.shape
+    if out is None:
+        out = torch.empty(1, dtype=torch.float64, device=W.device)
+    if workspace is None:
+        workspace = torch.empty(vq3r_rel_frobenius_workspace_size(rows, cols), dtype=torch.uint8, device=W.device)
+    _check(_lib().vq3r_rel_frobenius_error(_dev(W, "W"), _DT[W.dtype], _dev(idx, "idx"), _dev(scales, "scales"),
+                                           _dev(codebooks, "codebooks"), rows, cols, _dev(out, "out"),
+                                           _dev(workspace, "workspace"), workspace.numel(), _stream(stream)),
+           "vq3r_rel_frobenius_error")
+    return out
+
+
+def vq3r_device_error():
+    code = ctypes.c_int(0)
+    _check(_lib().vq3r_device_error(ctypes.byref(code)), "vq3r_device_error")
+    return code.value

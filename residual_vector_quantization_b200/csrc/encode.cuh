@@ -1,0 +1,174 @@
+// VQ3R encoder: per-row FP16 scale and greedy 3-stage residual assignment.
+//
+// Page "3比特逼近4比特精度？WARP残差向量量化VQ3R的完整测量实验", §2: one FP16
+// scale per row; three stages of 256-entry codebooks of 8-dim vectors; stage
+// s quantises the residual left by stage s-1.  §4: a single pass over the
+// three stages that writes only the winning indices.
+//
+// The work is FP32-pipe bound: per 8-weight vector and stage, 256 distances
+// of 8 (sub, mul, add).  The distance d_j = sum_k (r_k - c_jk)^2 is formed
+// with every operation rounded in k order (no fused multiply-add) so the
+// argmin is bit-identical to the definition; packed f32x2 instructions
+// (add.rn.f32x2 / mul.rn.f32x2) evaluate two vectors per instruction, which
+// leaves issue slots for the argmin compare/select while the FP32 pipe stays
+// full.
+#pragma once
+
+#include "vq3r_common.cuh"
+
+namespace vq3r {
+
+// ---------------- K1: row scale ----------------
+//
+// scale_i = binary16(sqrt(ss_i / cols)) with ss_i in binary64 in the fixed
+// order: thread p (of 128) sums q_v = ((w0^2 + w1^2) + ...) + w7^2 over
+// v = p, p+128, ... ascending; then a halving tree t_p += t_{p+h},
+// h = 64 .. 1.  __dmul_rn / __dadd_rn keep every product and sum rounded
+// separately.
+constexpr int kScaleThreads = 128;
+
+template <int DT>
+__global__ void __launch_bounds__(kScaleThreads) row_scale_kernel(const void* __restrict__ W, int64_t rows,
+                                                                   int64_t cols, uint16_t* __restrict__ scales) {
+  __shared__ double t[kScaleThreads];
+  const int p = threadIdx.x;
+  const int64_t V = cols / kDim;
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    double acc = 0.0;
+    for (int64_t v = p; v < V; v += kScaleThreads) {
+      float w[8];
+      load8<DT>(W, row * cols + v * kDim, w);
+      double q = __dmul_rn((double)w[0], (double)w[0]);
+#pragma unroll
+      for (int k = 1; k < 8; k++) q = __dadd_rn(q, __dmul_rn((double)w[k], (double)w[k]));
+      acc = __dadd_rn(acc, q);
+    }
+    t[p] = acc;
+    __syncthreads();
+#pragma unroll
+    for (int h = 64; h >= 1; h >>= 1) {
+      if (p < h) t[p] = __dadd_rn(t[p], t[p + h]);
+      __syncthreads();
+    }
+    if (p == 0) {
+      const double rms = __dsqrt_rn(__ddiv_rn(t[0], (double)cols));
+      scales[row] = f64_to_f16_sat_rne(rms);
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------- K2: greedy 3-stage assignment ----------------
+
+constexpr int kEncThreads = 256;
+constexpr int kEncPairs = 2;                            // vector pairs per thread
+constexpr int kEncVecPerThread = 2 * kEncPairs;         // 4
+constexpr int kEncTile = kEncThreads * kEncVecPerThread; // vectors per CTA iteration
+
+struct __align__(16) EncSmem {
+  float2 ncb[kStages][kCodewords][kDim];  // (-c, -c) duplicated for the packed subtract (48 KiB)
+  float raw[kCodebookFloats];              // TMA staging of the caller's codebooks (24 KiB)
+  uint64_t mbar;
+};
+
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 f2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+template <int DT>
+__global__ void __launch_bounds__(kEncThreads, 2)
+    encode_kernel(const void* __restrict__ W, int64_t cols, int64_t nvec, const float* __restrict__ codebooks,
+                  const uint16_t* __restrict__ scales, uint8_t* __restrict__ idx) {
+  extern __shared__ __align__(16) unsigned char enc_smem_raw[];
+  EncSmem& sm = *reinterpret_cast<EncSmem*>(enc_smem_raw);
+  const int tid = threadIdx.x;
+
+  // Stage the 24 KiB codebooks with one bulk asynchronous copy, then expand
+  // to negated, lane-duplicated pairs.
+  if (tid == 0) {
+    mbar_init(&sm.mbar, 1);
+    mbar_arrive_expect_tx(&sm.mbar, kCodebookBytes);
+    bulk_copy_g2s(sm.raw, codebooks, kCodebookBytes, &sm.mbar);
+  }
+  __syncthreads();
+  if (!mbar_wait_bounded(&sm.mbar, 0)) return;
+  for (int i = tid; i < kCodebookFloats; i += kEncThreads) {
+    const float c = -sm.raw[i];
+    (&sm.ncb[0][0][0])[i] = make_float2(c, c);
+  }
+  __syncthreads();
+
+  const int64_t V = cols / kDim;
+  const int64_t ntiles = (nvec + kEncTile - 1) / kEncTile;
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    // Vector q of this thread: g = tile * kEncTile + q * kEncThreads + tid.
+    float2 r[kEncPairs][kDim];
+    int64_t g[kEncVecPerThread];
+#pragma unroll
+    for (int q = 0; q < kEncVecPerThread; q++) {
+      g[q] = tile * kEncTile + (int64_t)q * kEncThreads + tid;
+      float w[8];
+      float rq[8];
+      if (g[q] < nvec) {
+        const int64_t row = g[q] / V;
+        const int64_t v = g[q] - row * V;
+        load8<DT>(W, row * cols + v * kDim, w);
+        const float s = f16_bits_to_f32(scales[row]);
+#pragma unroll
+        for (int k = 0; k < 8; k++) rq[k] = (s == 0.0f) ? 0.0f : __fdiv_rn(w[k], s);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; k++) rq[k] = 0.0f;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; k++) {
+        if (q & 1) r[q >> 1][k].y = rq[k];
+        else r[q >> 1][k].x = rq[k];
+      }
+    }
+
+#pragma unroll 1
+    for (int s = 0; s < kStages; s++) {
+      float best[kEncVecPerThread];
+      int bi[kEncVecPerThread];
+#pragma unroll
+      for (int q = 0; q < kEncVecPerThread; q++) { best[q] = __int_as_float(0x7F800000); bi[q] = 0; }
+      const float4* cw = reinterpret_cast<const float4*>(&sm.ncb[s][0][0]);
+#pragma unroll 4
+      for (int j = 0; j < kCodewords; j++) {
+        // (-c_k, -c_k) for k = 0..7: four broadcast 16-byte shared loads
+        float2 c[kDim];
+#pragma unroll
+        for (int k2 = 0; k2 < 4; k2++) {
+          const float4 t = cw[j * 4 + k2];
+          c[2 * k2] = make_float2(t.x, t.y);
+          c[2 * k2 + 1] = make_float2(t.z, t.w);
+        }
+#pragma unroll
+        for (int pr = 0; pr < kEncPairs; pr++) {
+          float2 e = f2add(r[pr][0], c[0]);
+          float2 d = f2mul(e, e);
+#pragma unroll
+          for (int k = 1; k < kDim; k++) {
+            e = f2add(r[pr][k], c[k]);
+            d = f2add(d, f2mul(e, e));
+          }
+          if (d.x < best[2 * pr]) { best[2 * pr] = d.x; bi[2 * pr] = j; }
+          if (d.y < best[2 * pr + 1]) { best[2 * pr + 1] = d.y; bi[2 * pr + 1] = j; }
+        }
+      }
+      // write the winning indices and update the residuals
+#pragma unroll
+      for (int q = 0; q < kEncVecPerThread; q++) {
+        if (g[q] < nvec) idx[(int64_t)s * nvec + g[q]] = (uint8_t)bi[q];
+        const float2* cwin = &sm.ncb[s][bi[q]][0];
+#pragma unroll
+        for (int k = 0; k < kDim; k++) {
+          if (q & 1) r[q >> 1][k].y = __fadd_rn(r[q >> 1][k].y, cwin[k].x);
+          else r[q >> 1][k].x = __fadd_rn(r[q >> 1][k].x, cwin[k].x);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace vq3r

@@ -1,0 +1,307 @@
+// C ABI of the VQ3R library (declared in include/vq3r.h): argument checks,
+// launch configuration and status codes.  All arithmetic runs in the
+// kernels of encode.cuh, decode.cuh and gemv.cuh.
+#include <mutex>
+
+#include "decode.cuh"
+#include "encode.cuh"
+#include "gemv.cuh"
+#include "vq3r_common.cuh"
+
+using namespace vq3r;
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+vq3r_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = (int)e;
+  return VQ3R_ERR_CUDA;
+}
+
+vq3r_status check_launch() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? VQ3R_OK : cuda_fail(e);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_dtype(int d) { return d == VQ3R_F32 || d == VQ3R_BF16 || d == VQ3R_F16; }
+
+vq3r_status check_shape(int64_t rows, int64_t cols, int64_t min_rows) {
+  if (rows < min_rows || cols < kDim || cols % kDim) return VQ3R_ERR_SHAPE;
+  if (rows > 0 && cols > INT64_MAX / 8 / rows) return VQ3R_ERR_SHAPE;
+  return VQ3R_OK;
+}
+
+// Per-device launch setup: SM count and the dynamic shared-memory opt-ins.
+constexpr int kMaxDevices = 64;
+std::once_flag g_dev_once[kMaxDevices];
+int g_dev_sms[kMaxDevices];
+cudaError_t g_dev_err[kMaxDevices];
+
+cudaError_t device_setup(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_dev_once[dev], [dev]() {
+    cudaError_t r = cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    const int enc = (int)sizeof(EncSmem);
+    const int gv = (int)kSlabBytes + 16;
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
+    g_dev_err[dev] = r;
+  });
+  *sms = g_dev_sms[dev];
+  return g_dev_err[dev];
+}
+
+constexpr size_t kWsAlign = 256;
+size_t align_up(size_t x) { return (x + kWsAlign - 1) / kWsAlign * kWsAlign; }
+
+constexpr int kErrMaxBlocks = 4096;
+
+// ---- GEMV schedule (host) ----
+
+struct GemvPlan {
+  GvParams P;
+  size_t ws_bytes;
+  bool aligned4;
+};
+
+// Groups matrices sharing (codebooks, x, cols), lays out the workspace and
+// numbers the work units.  Returns false on an invalid descriptor.
+vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_base, GemvPlan* plan) {
+  GvParams& P = plan->P;
+  memset(&P, 0, sizeof(P));
+  P.n_mats = n_mats;
+  P.B = B;
+  plan->aligned4 = true;
+  int n_groups = 0;
+  for (int i = 0; i < n_mats; i++) {
+    const vq3r_gemv_desc& d = mats[i];
+    vq3r_status st = check_shape(d.rows, d.cols, 0);
+    if (st != VQ3R_OK) return st;
+    if (d.cols / kDim > (int64_t)kSlabV * (1 << 20)) return VQ3R_ERR_SHAPE;
+    if (d.rows > 0) {  // an empty matrix may carry NULL pointers
+      if (!d.idx || !d.scales || !d.codebooks || !d.x || !d.y) return VQ3R_ERR_NULL;
+      if (!aligned16(d.idx) || !aligned16(d.scales) || !aligned16(d.codebooks) || !aligned16(d.x) ||
+          !aligned16(d.y))
+        return VQ3R_ERR_ALIGN;
+    }
+    if ((d.cols / kDim) % 4) plan->aligned4 = false;
+    int g = 0;
+    while (g < n_groups && !(P.g[g].codebooks == d.codebooks && P.g[g].x == d.x && P.g[g].cols == d.cols)) g++;
+    if (g == n_groups) {
+      P.g[g].codebooks = d.codebooks;
+      P.g[g].x = d.x;
+      P.g[g].cols = d.cols;
+      P.g[g].n_slabs = (int32_t)((d.cols / kDim + kSlabV - 1) / kSlabV);
+      P.g[g].tiles = 0;
+      n_groups++;
+    }
+    GvMat& M = P.m[i];
+    M.idx = d.idx;
+    M.scales = d.scales;
+    M.y = d.y;
+    M.rows = d.rows;
+    M.group = g;
+    M.n_tiles = (int32_t)((d.rows + kGvTileRows - 1) / kGvTileRows);
+    M.tile_prefix = P.g[g].tiles;
+    P.g[g].tiles += M.n_tiles;
+  }
+  P.n_groups = n_groups;
+  size_t off = 0;
+  int64_t units = 0;
+  int32_t images = 0;
+  for (int g = 0; g < n_groups; g++) {
+    GvGroup& G = P.g[g];
+    G.lut = reinterpret_cast<float*>(ws_base + off);
+    off = align_up(off + (size_t)B * G.n_slabs * kSlabBytes);
+    G.unit_begin = units;
+    units += (int64_t)G.n_slabs * B * G.tiles;
+    G.image_begin = images;
+    images += B * G.n_slabs;
+  }
+  for (int i = 0; i < n_mats; i++) {
+    GvMat& M = P.m[i];
+    M.partial = reinterpret_cast<float*>(ws_base + off);
+    off = align_up(off + (size_t)B * P.g[M.group].n_slabs * (size_t)M.rows * sizeof(float));
+  }
+  P.total_units = units;
+  P.total_images = images;
+  plan->ws_bytes = off;
+  return VQ3R_OK;
+}
+
+template <int DT>
+vq3r_status launch_encode(const void* W, int64_t rows, int64_t cols, const float* cb, uint8_t* idx,
+                          uint16_t* scales, cudaStream_t s, int sms) {
+  const int64_t nvec = rows * (cols / kDim);
+  const int g1 = (int)(rows < (int64_t)sms * 16 ? rows : (int64_t)sms * 16);
+  row_scale_kernel<DT><<<g1, kScaleThreads, 0, s>>>(W, rows, cols, scales);
+  const int64_t ntiles = (nvec + kEncTile - 1) / kEncTile;
+  const int g2 = (int)(ntiles < (int64_t)sms * 2 ? ntiles : (int64_t)sms * 2);
+  encode_kernel<DT><<<g2, kEncThreads, sizeof(EncSmem), s>>>(W, cols, nvec, cb, scales, idx);
+  return check_launch();
+}
+
+template <int DT>
+vq3r_status launch_relfro(const void* W, const uint8_t* idx, const uint16_t* scales, const float* cb, int64_t cols,
+                          int64_t nvec, double* err_out, double* partial, cudaStream_t s, int sms) {
+  int64_t blocks = (nvec + kErrThreads - 1) / kErrThreads;
+  const int64_t cap = (int64_t)sms * 8 < kErrMaxBlocks ? (int64_t)sms * 8 : kErrMaxBlocks;
+  if (blocks > cap) blocks = cap;
+  relfro_partial_kernel<DT><<<(int)blocks, kErrThreads, 0, s>>>(W, idx, scales, cb, cols, nvec, partial);
+  relfro_final_kernel<<<1, 256, 0, s>>>(partial, (int)blocks, err_out);
+  return check_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+vq3r_status vq3r_encode(const void* W, vq3r_dtype w_dtype, int64_t rows, int64_t cols, const float* codebooks,
+                        uint8_t* idx, uint16_t* scales, vq3r_stream stream) {
+  vq3r_status st = check_shape(rows, cols, 0);
+  if (st != VQ3R_OK) return st;
+  if (!valid_dtype(w_dtype)) return VQ3R_ERR_DTYPE;
+  if (rows == 0) return VQ3R_OK;
+  if (!W || !codebooks || !idx || !scales) return VQ3R_ERR_NULL;
+  if (!aligned16(W) || !aligned16(codebooks) || !aligned16(idx) || !aligned16(scales)) return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (w_dtype) {
+    case VQ3R_F32: return launch_encode<VQ3R_F32>(W, rows, cols, codebooks, idx, scales, s, sms);
+    case VQ3R_BF16: return launch_encode<VQ3R_BF16>(W, rows, cols, codebooks, idx, scales, s, sms);
+    default: return launch_encode<VQ3R_F16>(W, rows, cols, codebooks, idx, scales, s, sms);
+  }
+}
+
+vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float* codebooks, int64_t rows,
+                        int64_t cols, void* out, vq3r_dtype out_dtype, vq3r_stream stream) {
+  vq3r_status st = check_shape(rows, cols, 0);
+  if (st != VQ3R_OK) return st;
+  if (out_dtype != VQ3R_F32 && out_dtype != VQ3R_F16) return VQ3R_ERR_DTYPE;
+  if (rows == 0) return VQ3R_OK;
+  if (!idx || !scales || !codebooks || !out) return VQ3R_ERR_NULL;
+  if (!aligned16(idx) || !aligned16(scales) || !aligned16(codebooks) || !aligned16(out)) return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nvec = rows * (cols / kDim);
+  int64_t blocks = (nvec + kDecThreads - 1) / kDecThreads;
+  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+  if (out_dtype == VQ3R_F32)
+    decode_kernel<VQ3R_F32><<<(int)blocks, kDecThreads, 0, s>>>(idx, scales, codebooks, cols, nvec, out);
+  else
+    decode_kernel<VQ3R_F16><<<(int)blocks, kDecThreads, 0, s>>>(idx, scales, codebooks, cols, nvec, out);
+  return check_launch();
+}
+
+size_t vq3r_gemv_workspace_size(const vq3r_gemv_desc* mats, int n_mats, int B) {
+  if (!mats || n_mats < 1 || n_mats > VQ3R_GEMV_MAX_MATS || B < 1 || B > VQ3R_GEMV_MAX_B) return 0;
+  GemvPlan plan;
+  if (plan_gemv(mats, n_mats, B, nullptr, &plan) != VQ3R_OK) return 0;
+  return plan.ws_bytes;
+}
+
+vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype x_dtype, void* workspace,
+                      size_t ws_bytes, vq3r_stream stream) {
+  if (!mats) return VQ3R_ERR_NULL;
+  if (n_mats < 1 || n_mats > VQ3R_GEMV_MAX_MATS || B < 1 || B > VQ3R_GEMV_MAX_B) return VQ3R_ERR_BATCH;
+  if (!valid_dtype(x_dtype)) return VQ3R_ERR_DTYPE;
+  GemvPlan plan;
+  vq3r_status st = plan_gemv(mats, n_mats, B, static_cast<char*>(workspace), &plan);
+  if (st != VQ3R_OK) return st;
+  if (plan.P.total_units == 0) return VQ3R_OK;
+  if (!workspace || ws_bytes < plan.ws_bytes) return VQ3R_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return VQ3R_ERR_ALIGN;
+  plan.P.x_dtype = x_dtype;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const GvParams& P = plan.P;
+  const int build_blocks = P.total_images * kLutBuildBlocksPerImage;
+  switch (x_dtype) {
+    case VQ3R_F32: lut_build_kernel<VQ3R_F32><<<build_blocks, kGvThreads, 0, s>>>(P); break;
+    case VQ3R_BF16: lut_build_kernel<VQ3R_BF16><<<build_blocks, kGvThreads, 0, s>>>(P); break;
+    default: lut_build_kernel<VQ3R_F16><<<build_blocks, kGvThreads, 0, s>>>(P); break;
+  }
+  const int grid = (int)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms);
+  const size_t smem = kSlabBytes + 16;
+  if (plan.aligned4) gemv_lut_kernel<true><<<grid, kGvThreads, smem, s>>>(P);
+  else gemv_lut_kernel<false><<<grid, kGvThreads, smem, s>>>(P);
+  int64_t maxrows = 0;
+  for (int i = 0; i < n_mats; i++) maxrows = P.m[i].rows * B > maxrows ? P.m[i].rows * B : maxrows;
+  int64_t gx = (maxrows + 255) / 256;
+  if (gx > (int64_t)sms * 4) gx = (int64_t)sms * 4;
+  if (gx < 1) gx = 1;
+  gemv_reduce_kernel<<<dim3((unsigned)gx, (unsigned)n_mats), 256, 0, s>>>(P);
+  return check_launch();
+}
+
+size_t vq3r_rel_frobenius_workspace_size(int64_t rows, int64_t cols) {
+  (void)rows;
+  (void)cols;
+  return (size_t)kErrMaxBlocks * 2 * sizeof(double);
+}
+
+vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const uint8_t* idx, const uint16_t* scales,
+                                     const float* codebooks, int64_t rows, int64_t cols, double* err_out,
+                                     void* workspace, size_t ws_bytes, vq3r_stream stream) {
+  if (!W || !idx || !scales || !codebooks || !err_out) return VQ3R_ERR_NULL;
+  vq3r_status st = check_shape(rows, cols, 1);
+  if (st != VQ3R_OK) return st;
+  if (!valid_dtype(w_dtype)) return VQ3R_ERR_DTYPE;
+  if (!workspace || ws_bytes < vq3r_rel_frobenius_workspace_size(rows, cols)) return VQ3R_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(idx) || !aligned16(scales) || !aligned16(codebooks) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(err_out) & 7u))
+    return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nvec = rows * (cols / kDim);
+  double* partial = static_cast<double*>(workspace);
+  switch (w_dtype) {
+    case VQ3R_F32: return launch_relfro<VQ3R_F32>(W, idx, scales, codebooks, cols, nvec, err_out, partial, s, sms);
+    case VQ3R_BF16: return launch_relfro<VQ3R_BF16>(W, idx, scales, codebooks, cols, nvec, err_out, partial, s, sms);
+    default: return launch_relfro<VQ3R_F16>(W, idx, scales, codebooks, cols, nvec, err_out, partial, s, sms);
+  }
+}
+
+const char* vq3r_status_string(vq3r_status s) {
+  switch (s) {
+    case VQ3R_OK: return "VQ3R_OK";
+    case VQ3R_ERR_NULL: return "VQ3R_ERR_NULL: a required pointer is NULL";
+    case VQ3R_ERR_SHAPE: return "VQ3R_ERR_SHAPE: rows/cols invalid (cols must be a positive multiple of 8)";
+    case VQ3R_ERR_ALIGN: return "VQ3R_ERR_ALIGN: device pointers must be 16-byte aligned";
+    case VQ3R_ERR_DTYPE: return "VQ3R_ERR_DTYPE: unsupported dtype";
+    case VQ3R_ERR_BATCH: return "VQ3R_ERR_BATCH: B must be in [1, 32] and n_mats in [1, 32]";
+    case VQ3R_ERR_CUDA: return "VQ3R_ERR_CUDA: CUDA launch or call failed";
+    case VQ3R_ERR_WORKSPACE: return "VQ3R_ERR_WORKSPACE: workspace missing or too small";
+    default: return "VQ3R: unknown status";
+  }
+}
+
+int vq3r_last_cuda_error(void) { return t_last_cuda_error; }
+
+vq3r_status vq3r_device_error(int* code) {
+  if (!code) return VQ3R_ERR_NULL;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(code, g_device_error, sizeof(int));
+  const int zero = 0;
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  return e == cudaSuccess ? VQ3R_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+"""The C-ABI library loads and exports every entry point include/vq3r.h
+declares; host-side argument checks and workspace sizing (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import residual_vector_quantization_b200 as vq
+from residual_vector_quantization_b200.build import SO
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "vq3r.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(vq3r_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(SO):
+        from residual_vector_quantization_b200.build import build
+        build()
+    return vq.lib()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert set(vq.EXPORTED) <= set(declared_functions())
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert lib.vq3r_status_string(s).decode().startswith("VQ3R")
+    assert lib.vq3r_last_cuda_error() == 0
+
+
+def test_null_and_shape_errors_return_before_any_launch(lib):
+    fake = 0x100000  # never dereferenced: the checks fail first
+    assert lib.vq3r_encode(None, 1, 4, 16, fake, fake, fake, None) == 1
+    assert lib.vq3r_encode(fake, 1, 4, 12, fake, fake, fake, None) == 2
+    assert lib.vq3r_encode(fake, 1, -1, 16, fake, fake, fake, None) == 2
+    assert lib.vq3r_encode(fake, 1, 4, 0, fake, fake, fake, None) == 2
+    assert lib.vq3r_encode(fake, 7, 4, 16, fake, fake, fake, None) == 4
+    assert lib.vq3r_encode(fake + 2, 1, 4, 16, fake, fake, fake, None) == 3
+    assert lib.vq3r_encode(fake, 1, 0, 16, fake, fake, fake, None) == 0  # empty: no-op
+    assert lib.vq3r_decode(fake, fake, fake, 4, 16, fake, 1, None) == 4   # bf16 output unsupported
+    assert lib.vq3r_decode(fake, fake, fake, 4, 16, None, 0, None) == 1
+    assert lib.vq3r_rel_frobenius_error(fake, 1, fake, fake, fake, 0, 16, fake, fake, 1 << 20, None) == 2
+    assert lib.vq3r_rel_frobenius_error(fake, 1, fake, fake, fake, 4, 16, fake, fake, 16, None) == 7
+
+
+def _descs(specs):
+    arr = (vq.GemvDesc * len(specs))()
+    for i, (rows, cols, cb, x) in enumerate(specs):
+        arr[i] = vq.GemvDesc(0x200000 + 0x1000 * i, 0x300000 + 0x1000 * i, cb, rows, cols, x, 0x400000 + 0x1000 * i)
+    return arr
+
+
+def test_gemv_batch_and_workspace_checks(lib):
+    arr = _descs([(2048, 7168, 0x10000, 0x20000)])
+    assert lib.vq3r_gemv(arr, 1, 0, 1, 0x500000, 1 << 30, None) == 5
+    assert lib.vq3r_gemv(arr, 1, 33, 1, 0x500000, 1 << 30, None) == 5
+    assert lib.vq3r_gemv(arr, 0, 1, 1, 0x500000, 1 << 30, None) == 5
+    assert lib.vq3r_gemv(arr, 1, 1, 9, 0x500000, 1 << 30, None) == 4
+    assert lib.vq3r_gemv(arr, 1, 1, 1, 0x500000, 16, None) == 7
+    assert lib.vq3r_gemv(arr, 1, 1, 1, None, 0, None) == 7
+    assert lib.vq3r_gemv_workspace_size(arr, 1, 0) == 0
+
+
+def test_gemv_workspace_groups_shared_tables(lib):
+    slab = 3 * 256 * 64 * 4
+    # 16 gate/up matrices sharing x and codebooks: one set of tables (14 slabs)
+    specs = [(2048, 7168, 0x10000, 0x20000)] * 16
+    for B in (1, 4, 32):
+        ws = lib.vq3r_gemv_workspace_size(_descs(specs), 16, B)
+        assert ws == B * 14 * slab + 16 * B * 14 * 2048 * 4
+    # 8 down matrices with their own inputs: 8 groups of 4 slabs
+    specs = [(7168, 2048, 0x10000, 0x20000 + 0x10000 * i) for i in range(8)]
+    ws = lib.vq3r_gemv_workspace_size(_descs(specs), 8, 1)
+    assert ws == 8 * 4 * slab + 8 * 4 * 7168 * 4

@@ -1,0 +1,319 @@
+"""CUDA path vs the CPU oracle, through the C ABI (residual_vector_quantization_b200).
+
+Bars: indices, scales and decoded weights bit-exact; relative Frobenius
+error within 1e-9 relative; GEMV within 2e-3 max relative error (rms(y)
+floor) against the binary64 oracle GEMV.  Every oracle input comes from the
+host generator (synth) or from the oracle itself, never from the GPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import workloads as wl
+from vq3r_cases import (GEMV_TOL, RELFRO_TOL, energy8_vectors, f32_to_bf16_bits, gemv_rel_err, random_codebooks,
+                        sign_pattern_codebooks)
+
+pytestmark = pytest.mark.gpu
+
+vq = pytest.importorskip("residual_vector_quantization_b200")
+DEV = "cuda"
+
+
+def to_dev(a, dtype):
+    """numpy host array -> device tensor: f32 as float32, bf16/f16 from uint16 bit patterns."""
+    if dtype == "f32":
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(DEV)
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).to(DEV)
+    return t.view(torch.bfloat16 if dtype == "bf16" else torch.float16)
+
+
+def host_bits(t):
+    """device bf16/f16 tensor -> numpy uint16 bit patterns."""
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def gpu_encode(W_t, cb):
+    idx, sc = vq.vq3r_encode(W_t, torch.from_numpy(cb).to(DEV))
+    torch.cuda.synchronize()
+    return idx, sc
+
+
+def check_encode_decode(Wnp, dtype, cb):
+    """Full bit-exact parity of encode and decode on one matrix; returns device tensors."""
+    W_t = to_dev(Wnp, dtype)
+    idx_t, sc_t = gpu_encode(W_t, cb)
+    idx_o, sc_o = oracle.encode(Wnp, dtype, cb)
+    np.testing.assert_array_equal(sc_t.cpu().numpy().view(np.uint16), sc_o)
+    np.testing.assert_array_equal(idx_t.cpu().numpy(), idx_o)
+    cb_t = torch.from_numpy(cb).to(DEV)
+    d32 = vq.vq3r_decode(idx_t, sc_t, cb_t, torch.float32).cpu().numpy()
+    np.testing.assert_array_equal(d32.view(np.uint32), oracle.decode(idx_o, sc_o, cb).view(np.uint32))
+    d16 = vq.vq3r_decode(idx_t, sc_t, cb_t, torch.float16)
+    np.testing.assert_array_equal(host_bits(d16), oracle.decode(idx_o, sc_o, cb, out="f16"))
+    return W_t, idx_t, sc_t, cb_t, idx_o, sc_o
+
+
+# ------------------------------------------------------------------ tiny workload, end to end
+
+@pytest.fixture(scope="module")
+def tiny():
+    cfg = wl.TINY
+    W = synth.fill_rows(cfg["cols"], 0, cfg["rows"], cfg["seed"], wl.tag(0, wl.W1), synth.normal(), dtype="f32")
+    sc = oracle.row_scales(W, "f32")
+    cb, _ = oracle.lloyd_train(oracle.normalize_rows(W, "f32", sc), cfg["lloyd_iters"])
+    return W, cb
+
+
+def test_tiny_encode_decode_bit_exact(tiny):
+    W, cb = tiny
+    check_encode_decode(W, "f32", cb)
+
+
+def test_tiny_rel_frobenius(tiny):
+    W, cb = tiny
+    W_t, idx_t, sc_t, cb_t, idx_o, sc_o = check_encode_decode(W, "f32", cb)
+    e_gpu = float(vq.vq3r_rel_frobenius_error(W_t, idx_t, sc_t, cb_t).cpu()[0])
+    e_ref = oracle.rel_frobenius(W, "f32", oracle.decode(idx_o, sc_o, cb))
+    assert abs(e_gpu - e_ref) <= RELFRO_TOL * e_ref
+
+
+@pytest.mark.parametrize("B", [1, 4, 8, 32])
+def test_tiny_gemv(tiny, B):
+    W, cb = tiny
+    W_t, idx_t, sc_t, cb_t, idx_o, sc_o = check_encode_decode(W, "f32", cb)
+    x = synth.fill_rows(W.shape[1], 0, B, wl.TINY_SEED, wl.tag(0, wl.X_GATEUP), synth.normal(), dtype="f32")
+    y_t = torch.empty((B, W.shape[0]), dtype=torch.float32, device=DEV)
+    vq.vq3r_gemv([dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=to_dev(x, "f32"), y=y_t)], B)
+    y_ref = oracle.gemv(oracle.decode(idx_o, sc_o, cb), x, "f32")
+    assert gemv_rel_err(y_t.cpu().numpy(), y_ref) <= GEMV_TOL
+
+
+# ------------------------------------------------------------------ shapes, dtypes, ragged tails
+
+@pytest.mark.parametrize("rows,cols,dtype", [(1, 8, "f32"), (3, 40, "bf16"), (130, 800, "bf16"), (257, 1032, "f16"),
+                                             (64, 7168, "bf16"), (1025, 2048, "bf16"), (5, 4104, "f32")])
+def test_shapes_and_dtypes(rows, cols, dtype):
+    rng = np.random.default_rng(rows * 7 + cols)
+    cb = random_codebooks(rows + cols)
+    Wf = (rng.standard_normal((rows, cols)) * np.exp(rng.standard_normal((rows, 1)))).astype(np.float32)
+    if dtype == "f32":
+        W = Wf
+    elif dtype == "bf16":
+        W = f32_to_bf16_bits(Wf)
+    else:
+        W = Wf.astype(np.float16).view(np.uint16)
+    W_t, idx_t, sc_t, cb_t, idx_o, sc_o = check_encode_decode(W, dtype, cb)
+    for B in (1, 3):
+        x = rng.standard_normal((B, cols)).astype(np.float32)
+        xb = f32_to_bf16_bits(x)
+        y_t = torch.empty((B, rows), dtype=torch.float32, device=DEV)
+        vq.vq3r_gemv([dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=to_dev(xb, "bf16"), y=y_t)], B)
+        y_ref = oracle.gemv(oracle.decode(idx_o, sc_o, cb), xb, "bf16")
+        assert gemv_rel_err(y_t.cpu().numpy(), y_ref) <= GEMV_TOL
+    e_gpu = float(vq.vq3r_rel_frobenius_error(W_t, idx_t, sc_t, cb_t).cpu()[0])
+    e_ref = oracle.rel_frobenius(W, dtype, oracle.decode(idx_o, sc_o, cb))
+    assert abs(e_gpu - e_ref) <= RELFRO_TOL * e_ref
+
+
+def test_ties_take_the_lowest_index():
+    """Sign-pattern codebooks and residual components that are exactly 0: every
+    tie is exact, and the lowest index must win on the GPU as in the oracle."""
+    rng = np.random.default_rng(21)
+    cb = sign_pattern_codebooks()
+    V, rows = 64, 96
+    W = energy8_vectors(rng, rows * V).reshape(rows, V * 8)
+    W[:, ::3] = 0.0  # more ties (rows keep a nonzero RMS)
+    check_encode_decode(W, "f32", cb)
+    perm = rng.permutation(256)
+    check_encode_decode(W, "f32", np.ascontiguousarray(cb[:, perm, :]))
+
+
+def test_scale_limits_zero_rows_and_subnormals():
+    rng = np.random.default_rng(22)
+    cb = random_codebooks(5)
+    W = rng.standard_normal((8, 512)).astype(np.float32)
+    W[0] = 0.0                       # zero row -> scale 0, r = 0
+    W[1] *= 1e6                      # RMS above 65504 -> saturated scale
+    W[2] *= 2.0 ** -20               # binary16 subnormal scale
+    W[3] *= 2.0 ** -30               # scale underflows to 0
+    W[4] = 1 + 2.0 ** -11            # RMS on a binary16 midpoint (ties to even)
+    W[5] = 1 + 3 * 2.0 ** -11
+    check_encode_decode(W, "f32", cb)
+
+
+def test_planted_exact_case():
+    rng = np.random.default_rng(23)
+    cb = sign_pattern_codebooks()
+    cb[0] = cb[0][rng.permutation(256)]
+    cb[1] = rng.standard_normal((256, 8)).astype(np.float32) * 0.3
+    cb[2] = rng.standard_normal((256, 8)).astype(np.float32) * 0.1
+    cb[1, 0] = 0.0
+    cb[2, 0] = 0.0
+    pi = rng.integers(0, 256, size=(16, 64))
+    s = np.array([0.75, 3.0, 2.0 ** -6, 1.5] * 4, dtype=np.float32)
+    W = (cb[0][pi].reshape(16, 512) * s[:, None]).astype(np.float32)
+    W_t, idx_t, sc_t, cb_t, idx_o, _ = check_encode_decode(W, "f32", cb)
+    np.testing.assert_array_equal(idx_t.cpu().numpy()[0], pi)
+    assert float(vq.vq3r_rel_frobenius_error(W_t, idx_t, sc_t, cb_t).cpu()[0]) == 0.0
+
+
+def test_empty_matrix_is_a_noop():
+    W_t = torch.empty((0, 64), dtype=torch.bfloat16, device=DEV)
+    idx, sc = vq.vq3r_encode(W_t, torch.zeros((3, 256, 8), device=DEV))
+    assert idx.shape == (3, 0, 8) and sc.shape == (0,)
+
+
+def test_grouped_gemv_mixed_matrices():
+    """One call over matrices of different shapes, codebooks and inputs."""
+    rng = np.random.default_rng(24)
+    specs = [(300, 1024, 0, 0), (129, 1024, 0, 0), (64, 512, 1, 1), (200, 1024, 2, 0), (33, 1024, 0, 2)]
+    B = 4
+    xs = {}
+    mats, refs = [], []
+    for rows, cols, cbk, xk in specs:
+        cb = random_codebooks(100 + cbk)
+        if (xk, cols) not in xs:
+            xs[(xk, cols)] = f32_to_bf16_bits(rng.standard_normal((B, cols)).astype(np.float32))
+        x = xs[(xk, cols)]
+        W = f32_to_bf16_bits(rng.standard_normal((rows, cols)).astype(np.float32))
+        W_t, idx_t, sc_t, cb_t, idx_o, sc_o = check_encode_decode(W, "bf16", cb)
+        y_t = torch.empty((B, rows), dtype=torch.float32, device=DEV)
+        mats.append(dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=None, y=y_t, key=(xk, cols)))
+        refs.append(oracle.gemv(oracle.decode(idx_o, sc_o, cb), x, "bf16"))
+    xdev = {k: to_dev(v, "bf16") for k, v in xs.items()}
+    for m in mats:
+        m["x"] = xdev[m.pop("key")]
+    vq.vq3r_gemv(mats, B)
+    for m, ref in zip(mats, refs):
+        assert gemv_rel_err(m["y"].cpu().numpy(), ref) <= GEMV_TOL
+
+
+# ------------------------------------------------------------------ error statuses
+
+def test_error_statuses():
+    cb = torch.zeros((3, 256, 8), device=DEV)
+    with pytest.raises(vq.VQ3RError) as e:
+        vq.vq3r_encode(torch.zeros((4, 12), device=DEV), cb)
+    assert e.value.status == 2
+    buf = torch.zeros(4 * 16 + 1, device=DEV)
+    with pytest.raises(vq.VQ3RError) as e:
+        vq.vq3r_encode(buf[1:].view(4, 16), cb)  # 4-byte offset: not 16-byte aligned
+    assert e.value.status == 3
+    W = torch.zeros((4, 16), device=DEV)
+    idx, sc = vq.vq3r_encode(W, cb)
+    y = torch.empty((1, 4), device=DEV)
+    m = [dict(idx=idx, scales=sc, codebooks=cb, x=torch.zeros((1, 16), device=DEV), y=y)]
+    with pytest.raises(vq.VQ3RError) as e:
+        vq.vq3r_gemv(m, 33)
+    assert e.value.status == 5
+    with pytest.raises(vq.VQ3RError) as e:
+        vq.vq3r_gemv(m, 1, workspace=torch.empty(16, dtype=torch.uint8, device=DEV))
+    assert e.value.status == 7
+    assert vq.vq3r_device_error() == 0
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled rows
+
+def load_codebooks(name):
+    import importlib.util
+    import os
+    p = os.path.join(os.path.dirname(__file__), "golden", "make_codebooks.py")
+    spec = importlib.util.spec_from_file_location("make_codebooks", p)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return np.ascontiguousarray(mod.load(name))
+
+
+def device_matrix(experts, kind, seed, dist):
+    """Rows of `kind` for the listed experts stacked into one bf16 device tensor."""
+    rows, cols = wl.mat_shape(kind)
+    W = torch.empty((len(experts) * rows, cols), dtype=torch.bfloat16, device=DEV)
+    for i, e in enumerate(experts):
+        synth.fill_rows_device(W[i * rows:(i + 1) * rows].data_ptr(), cols, 0, rows, seed, wl.tag(e, kind), dist,
+                               stream=torch.cuda.current_stream().cuda_stream)
+    return W
+
+
+def host_rows(experts, kind, seed, dist, stacked_rows):
+    rows, cols = wl.mat_shape(kind)
+    out = np.empty((len(stacked_rows), cols), dtype=np.uint16)
+    for i, r in enumerate(stacked_rows):
+        e = experts[r // rows]
+        out[i] = synth.fill_row_list(cols, [r % rows], seed, wl.tag(e, kind), dist)[0]
+    return out
+
+
+@pytest.mark.parametrize("kind", [wl.W1, wl.W2])
+def test_layer_stacked_encode_sampled_rows(kind):
+    """Encode of a 64-expert layer matrix stacked into one call (the benchmark's
+    launch), bit-exact against the oracle on 256 sampled rows."""
+    cfg = wl.LAYER
+    cb = load_codebooks("layer")
+    experts = list(range(cfg["experts"]))
+    W_t = device_matrix(experts, kind, cfg["seed"], wl.expert_dist())
+    idx_t, sc_t = gpu_encode(W_t, cb)
+    rng = np.random.default_rng(kind)
+    sample = np.sort(rng.choice(W_t.shape[0], 256, replace=False))
+    Wh = host_rows(experts, kind, cfg["seed"], wl.expert_dist(), sample)
+    np.testing.assert_array_equal(host_bits(W_t[torch.from_numpy(sample).to(DEV)]), Wh)  # generators agree
+    idx_o, sc_o = oracle.encode(Wh, "bf16", cb)
+    sel = torch.from_numpy(sample).to(DEV)
+    np.testing.assert_array_equal(sc_t[sel].cpu().numpy().view(np.uint16), sc_o)
+    np.testing.assert_array_equal(idx_t[:, sel, :].cpu().numpy(), idx_o)
+
+
+def test_expert_full_matrix_rel_frobenius_consistent():
+    """Single-expert w2 at full size: the error kernel agrees with the decode kernel
+    (binary64 torch sums of its output), and both sit in the expected band."""
+    cfg = wl.EXPERT
+    cb = load_codebooks("expert")
+    W_t = device_matrix([0], wl.W2, cfg["seed"], wl.expert_dist())
+    idx_t, sc_t = gpu_encode(W_t, cb)
+    cb_t = torch.from_numpy(cb).to(DEV)
+    e = float(vq.vq3r_rel_frobenius_error(W_t, idx_t, sc_t, cb_t).cpu()[0])
+    Wd = vq.vq3r_decode(idx_t, sc_t, cb_t).double()
+    w = W_t.double()
+    e2 = float(torch.sqrt(((w - Wd) ** 2).sum() / (w ** 2).sum()))
+    assert abs(e - e2) <= 1e-9 * e2
+    assert 0.1 < e < 0.3
+
+
+@pytest.mark.parametrize("B", [1, 4, 8, 32])
+def test_moe_decode_step_gemv_sampled_rows(B):
+    """The MoE decode step (8 experts of the layer; gate/up in one call, down in
+    one call) at full size against the binary64 oracle on sampled rows."""
+    cfg = wl.LAYER
+    cb = load_codebooks("layer")
+    cb_t = torch.from_numpy(cb).to(DEV)
+    experts = list(range(8))
+    x_up = synth.fill_rows(wl.HIDDEN, 0, B, wl.ACT_SEED, wl.tag(0, wl.X_GATEUP), synth.normal())
+    x_dn = [synth.fill_rows(wl.INTER, 0, B, wl.ACT_SEED, wl.tag(e, wl.X_DOWN), synth.normal()) for e in experts]
+    x_up_t = to_dev(x_up, "bf16")
+    phase1, phase2, checks = [], [], []
+    rng = np.random.default_rng(B)
+    for e in experts:
+        for kind in (wl.W1, wl.W3, wl.W2):
+            rows, cols = wl.mat_shape(kind)
+            W_t = device_matrix([e], kind, cfg["seed"], wl.expert_dist())
+            idx_t, sc_t = gpu_encode(W_t, cb)
+            del W_t
+            y_t = torch.empty((B, rows), dtype=torch.float32, device=DEV)
+            if kind == wl.W2:
+                phase2.append(dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=to_dev(x_dn[e], "bf16"), y=y_t))
+            else:
+                phase1.append(dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=x_up_t, y=y_t))
+            sample = np.sort(rng.choice(rows, 24, replace=False))
+            checks.append((y_t, e, kind, sample, x_dn[e] if kind == wl.W2 else x_up))
+    vq.vq3r_gemv(phase1, B)
+    vq.vq3r_gemv(phase2, B)
+    torch.cuda.synchronize()
+    worst = 0.0
+    for y_t, e, kind, sample, x in checks:
+        Wh = host_rows([e], kind, cfg["seed"], wl.expert_dist(), sample)
+        idx_o, sc_o = oracle.encode(Wh, "bf16", cb)
+        y_ref = oracle.gemv(oracle.decode(idx_o, sc_o, cb), x, "bf16")
+        y = y_t.cpu().numpy()[:, sample]
+        worst = max(worst, gemv_rel_err(y, y_ref))
+    assert worst <= GEMV_TOL, worst

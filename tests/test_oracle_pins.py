@@ -5,7 +5,6 @@ Page: "3比特逼近4比特精度？WARP残差向量量化VQ3R的完整测量实
 (xdnf.cn/news/289497), §2 (format, reconstruction rule, Lloyd codebooks),
 §3.1 (relative Frobenius error, rtn4-row, vq2), §4 (greedy single pass).
 """
-import itertools
 import math
 from fractions import Fraction
 
@@ -18,32 +17,7 @@ import synth
 K, D = 256, 8
 
 
-# ---------------------------------------------------------------- helpers
-
-def sign_pattern_codebooks(a=1.0):
-    """C1 = all 256 sign patterns of +-a (bit k of j set <=> dim k negative),
-    C2 = same with a/2, C3 = same with a/4."""
-    j = np.arange(K)[:, None]
-    k = np.arange(D)[None, :]
-    sgn = np.where((j >> k) & 1, -1.0, 1.0)
-    return np.stack([sgn * a, sgn * a / 2, sgn * a / 4]).astype(np.float32)
-
-
-def energy8_vectors(rng, n):
-    """n vectors with entries k/4 (k integer in [-8, 8], zeros included) whose
-    8 squares sum to exactly 8, so a row made of them has RMS exactly 1."""
-    tuples = []
-    for combo in itertools.combinations_with_replacement(range(0, 9), D):
-        if sum(c * c for c in combo) == 128 and len(set(combo)) >= 3:
-            tuples.append(combo)
-    assert len(tuples) > 10
-    out = np.empty((n, D), dtype=np.float32)
-    for i in range(n):
-        t = np.array(tuples[rng.integers(len(tuples))], dtype=np.float64)
-        rng.shuffle(t)
-        t *= rng.choice([-1.0, 1.0], size=D)
-        out[i] = t / 4.0
-    return out
+from vq3r_cases import energy8_vectors, sign_pattern_codebooks  # noqa: E402
 
 
 # ---------------------------------------------------------------- generator
