@@ -1,0 +1,490 @@
+#!/usr/bin/env python
+"""Benchmark of the VQ3R hot path on B200.
+
+One step = one pass of the whole path over a 64-expert MoE layer
+(w1, w3: 2048 x 7168; w2: 7168 x 2048 per expert, bf16, Student-t(4) rows
+with log-normal row factors; 2.82 G weights):
+  encode (row scale + greedy 3-stage assignment), decode to fp32,
+  relative Frobenius error of each matrix, and the MoE decode step
+  (8 active experts: gate/up GEMV in one call, down GEMV in one call, B = 1).
+Each matrix kind of the layer is stacked into one call.  The decode step
+rotates over the 8 disjoint 8-expert groups of the layer so that its 132 MB
+of indices per step come from HBM, not L2 (the layer's 5.6 GB of weights
+exceed L2 as well).
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from synth import workloads as wl  # noqa: E402
+
+METRIC = "VQ3R encode Gweights/s (vs fp32 peak); decode-GEMV GB/s vs HBM roofline, 1 B200"
+FLOPS_PER_WEIGHT = 2304  # 3 stages x 256 codewords x 8 dims x (sub, mul, add) / 8 weights
+SM_COUNT_NOMINAL = 148
+FP32_LANES_PER_SM = 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="vq3r", choices=["vq3r", "reference"])
+    ap.add_argument("--experts", type=int, default=64)
+    ap.add_argument("--gemv-iters", type=int, default=40)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_codebooks(name):
+    """Codebooks written by tests/golden/make_codebooks.py (hex float32 text)."""
+    rows = []
+    with open(os.path.join(ROOT, "tests", "golden", "codebooks_%s.txt" % name)) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            rows.append([int(t, 16) for t in line.split()])
+    return np.array(rows, dtype=np.uint32).view(np.float32).reshape(3, 256, 8)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", 1965.0)), "measured"
+    except Exception:
+        return 6650.0, 1965.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+def moe_step_bytes(B, n_exp=8):
+    """Algorithmic bytes of one MoE decode step: index planes, scales, x, y."""
+    gu_rows, gu_cols = wl.mat_shape(wl.W1)
+    dn_rows, dn_cols = wl.mat_shape(wl.W2)
+    idx = n_exp * (2 * 3 * gu_rows * gu_cols // 8 + 3 * dn_rows * dn_cols // 8)
+    scales = n_exp * 2 * (2 * gu_rows + dn_rows)
+    x = 2 * B * gu_cols + 2 * n_exp * B * dn_cols
+    y = 4 * B * n_exp * (2 * gu_rows + dn_rows)
+    return idx + scales + x + y
+
+
+class Layer:
+    """The layer on one GPU: inputs, outputs, workspaces and the step."""
+
+    def __init__(self, torch, vq, dev, experts, expert0, B_list):
+        self.torch, self.vq, self.dev = torch, vq, dev
+        self.E = experts
+        seed, dist = wl.LAYER["seed"], wl.expert_dist()
+        stream = torch.cuda.current_stream().cuda_stream
+        self.cb = torch.from_numpy(load_codebooks("layer")).to(dev)
+        self.kinds = (wl.W1, wl.W3, wl.W2)
+        self.W, self.idx, self.sc, self.dec, self.err, self.err_ws = {}, {}, {}, {}, {}, {}
+        for k in self.kinds:
+            rows, cols = wl.mat_shape(k)
+            W = torch.empty((experts * rows, cols), dtype=torch.bfloat16, device=dev)
+            for e in range(experts):
+                synth.fill_rows_device(W[e * rows:(e + 1) * rows].data_ptr(), cols, 0, rows, seed,
+                                       wl.tag(expert0 + e, k), dist, stream=stream)
+            self.W[k] = W
+            self.idx[k] = torch.empty((3, experts * rows, cols // 8), dtype=torch.uint8, device=dev)
+            self.sc[k] = torch.empty(experts * rows, dtype=torch.int16, device=dev)
+            self.dec[k] = torch.empty((experts * rows, cols), dtype=torch.float32, device=dev)
+            self.err[k] = torch.empty(1, dtype=torch.float64, device=dev)
+            self.err_ws[k] = torch.empty(vq.vq3r_rel_frobenius_workspace_size(experts * rows, cols),
+                                         dtype=torch.uint8, device=dev)
+        self.weights = sum(self.W[k].numel() for k in self.kinds)
+        # decode-step inputs and outputs per batch size
+        self.groups = max(1, experts // 8)
+        self.moe = {}
+        for B in B_list:
+            xu = torch.empty((B, wl.HIDDEN), dtype=torch.bfloat16, device=dev)
+            synth.fill_rows_device(xu.data_ptr(), wl.HIDDEN, 0, B, wl.ACT_SEED, wl.tag(0, wl.X_GATEUP),
+                                   synth.normal(), stream=stream)
+            xd = torch.empty((8, B, wl.INTER), dtype=torch.bfloat16, device=dev)
+            for j in range(8):
+                synth.fill_rows_device(xd[j].data_ptr(), wl.INTER, 0, B, wl.ACT_SEED, wl.tag(j, wl.X_DOWN),
+                                       synth.normal(), stream=stream)
+            plans = []
+            for g in range(self.groups):
+                ex = [g * 8 + j for j in range(min(8, experts))]
+                p1, p2 = [], []
+                for j, e in enumerate(ex):
+                    for k in (wl.W1, wl.W3):
+                        rows, _ = wl.mat_shape(k)
+                        p1.append(dict(idx=self.idx[k], scales=self.sc[k], codebooks=self.cb, x=xu, row0=e * rows,
+                                       rows=rows, y=torch.empty((B, rows), dtype=torch.float32, device=dev)))
+                    rows, _ = wl.mat_shape(wl.W2)
+                    p2.append(dict(idx=self.idx[wl.W2], scales=self.sc[wl.W2], codebooks=self.cb, x=xd[j],
+                                   row0=e * rows, rows=rows,
+                                   y=torch.empty((B, rows), dtype=torch.float32, device=dev)))
+                d1, d2 = vq._descs(p1), vq._descs(p2)
+                ws1 = vq.lib().vq3r_gemv_workspace_size(d1, len(p1), B)
+                ws2 = vq.lib().vq3r_gemv_workspace_size(d2, len(p2), B)
+                plans.append((d1, len(p1), d2, len(p2), p1, p2, ws1, ws2))
+            wsz = max(max(p[6], p[7]) for p in plans)
+            ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+            self.moe[B] = (plans, ws, xu, xd)
+
+    # --- the parts of a step (each enqueues on the current stream) ---
+
+    def encode(self):
+        for k in self.kinds:
+            self.vq.vq3r_encode(self.W[k], self.cb, self.idx[k], self.sc[k])
+
+    def decode(self):
+        for k in self.kinds:
+            self.vq.vq3r_decode(self.idx[k], self.sc[k], self.cb, out=self.dec[k])
+
+    def errors(self):
+        for k in self.kinds:
+            self.vq.vq3r_rel_frobenius_error(self.W[k], self.idx[k], self.sc[k], self.cb, out=self.err[k],
+                                             workspace=self.err_ws[k])
+
+    def gemv(self, B, group):
+        plans, ws, _, _ = self.moe[B]
+        d1, n1, d2, n2 = plans[group % len(plans)][:4]
+        L, s = self.vq.lib(), self.torch.cuda.current_stream().cuda_stream
+        for d, n in ((d1, n1), (d2, n2)):
+            st = L.vq3r_gemv(d, n, B, 1, ws.data_ptr(), ws.numel(), s)
+            if st:
+                raise self.vq.VQ3RError(st, "vq3r_gemv")
+
+    LAUNCHES_PER_STEP = 3 * 2 + 3 * 1 + 3 * 2 + 2 * 3  # encode, decode, error, gemv (kernels)
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+
+def cpu_oracle_sample(seconds, experts=64):
+    """Time the oracle (as it stands) on a bounded row sample of the same layer:
+    encode + decode + error + GEMV of sampled rows of each matrix kind."""
+    import oracle
+    seed, dist = wl.LAYER["seed"], wl.expert_dist()
+    cb = load_codebooks("layer")
+    rng = np.random.default_rng(0)
+
+    def run(nrows):
+        t_work, n_w = 0.0, 0
+        for k in (wl.W1, wl.W3, wl.W2):
+            rows, cols = wl.mat_shape(k)
+            picks = rng.integers(0, experts * rows, size=nrows)
+            W = np.stack([synth.fill_row_list(cols, [r % rows], seed, wl.tag(int(r // rows), k), dist)[0]
+                          for r in picks])
+            x = synth.fill_rows(cols, 0, 1, wl.ACT_SEED, wl.tag(0, wl.X_GATEUP), synth.normal())
+            t0 = time.perf_counter()
+            idx, sc = oracle.encode(W, "bf16", cb)
+            Wd = oracle.decode(idx, sc, cb)
+            oracle.rel_frobenius(W, "bf16", Wd)
+            oracle.gemv(Wd, x, "bf16")
+            t_work += time.perf_counter() - t0
+            n_w += W.size
+        return t_work, n_w
+
+    t, n = run(16)
+    per_w = t / n
+    nrows = max(16, int(seconds / (per_w * (2 * 7168 + 2048))))
+    t, n = run(nrows)
+    return {"value": n / t / 1e9, "unit": "Gweights/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": "%d sampled rows of each of w1, w3, w2 of the 64-expert layer (%d weights): encode + decode + "
+                      "rel-Frobenius + binary64 GEMV, %.1f s" % (nrows, n, t)}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle on a bounded sample, same metric and config."""
+    if rank != 0:
+        return
+    import oracle
+    cb = load_codebooks("layer")
+    seed, dist = wl.LAYER["seed"], wl.expert_dist()
+    rng = np.random.default_rng(1)
+    rows_per_step = 128
+    samples = []
+    for it in range(args.warmup + args.steps):
+        mats = []
+        for k in (wl.W1, wl.W3, wl.W2):
+            rows, cols = wl.mat_shape(k)
+            picks = rng.integers(0, args.experts * rows, size=rows_per_step)
+            W = np.stack([synth.fill_row_list(cols, [r % rows], seed, wl.tag(int(r // rows), k), dist)[0]
+                          for r in picks])
+            mats.append((W, synth.fill_rows(cols, 0, 1, wl.ACT_SEED, wl.tag(0, wl.X_GATEUP), synth.normal())))
+        t0 = time.perf_counter()
+        n = 0
+        for W, x in mats:
+            idx, sc = oracle.encode(W, "bf16", cb)
+            Wd = oracle.decode(idx, sc, cb)
+            oracle.rel_frobenius(W, "bf16", Wd)
+            oracle.gemv(Wd, x, "bf16")
+            n += W.size
+        dt = time.perf_counter() - t0
+        if it >= args.warmup:
+            samples.append((dt, n))
+    t = sum(s[0] for s in samples)
+    n = sum(s[1] for s in samples)
+    v = n / t / 1e9
+    desc = ("each step: %d sampled rows of each of w1, w3, w2 of the 64-expert layer (%d weights): encode + decode + "
+            "rel-Frobenius + binary64 GEMV" % (rows_per_step, samples[0][1]))
+    out = {"metric": METRIC, "value": v, "unit": "Gweights/s", "impl": "reference", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / len(samples),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+           "config": {"workload": "moe-layer-64x3-bf16 (sampled rows) + moe-decode-step", "experts": args.experts},
+           "cpu_baseline": {"value": v, "unit": "Gweights/s", "cores": oracle.max_threads(), "kind": "oracle",
+                            "sample": desc},
+           "e2e": {"value": v, "unit": "Gweights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d: launch N>1 with torchrun" % (args.gpus, world))
+
+    # CPU baseline first (the oracle on host cores, before CUDA starts)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(args.cpu_seconds, args.experts)
+
+    import torch
+    import residual_vector_quantization_b200 as vq
+    from datetime import timedelta
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    B_list = (1, 4, 8, 32)
+    layer = Layer(torch, vq, dev, args.experts, rank * args.experts, B_list)
+    torch.cuda.synchronize()
+    hbm_gbs, sm_max_mhz, peak_src = peaks()
+    props = torch.cuda.get_device_properties(dev)
+    sms = props.multi_processor_count
+    fp32_peak_tflops = sms * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(i, marks=None):
+        if marks: marks[0].record()
+        layer.encode()
+        if marks: marks[1].record()
+        layer.decode()
+        if marks: marks[2].record()
+        layer.errors()
+        if marks: marks[3].record()
+        layer.gemv(1, i)
+        if marks: marks[4].record()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    marks = [[ev() for _ in range(5)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = ev(), ev()
+    t0.record()
+    for i in range(args.steps):
+        step(args.warmup + i, marks[i])
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    part = lambda a, b: [marks[i][a].elapsed_time(marks[i][b]) for i in range(args.steps)]  # noqa: E731
+    enc_ms = statistics.mean(part(0, 1))
+    dec_ms = statistics.mean(part(1, 2))
+    err_ms = statistics.mean(part(2, 3))
+    gv1_ms = statistics.mean(part(3, 4))
+
+    # decode-step GEMV sweep over batch sizes (not part of the step), rotating expert groups
+    gemv = {}
+    for B in B_list:
+        for i in range(3):
+            layer.gemv(B, i)
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record()
+        for i in range(args.gemv_iters):
+            layer.gemv(B, i)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / args.gemv_iters
+        gbs = moe_step_bytes(B) / ms / 1e6
+        gemv[str(B)] = {"us_per_step": 1e3 * ms, "GB/s": gbs, "frac_hbm": gbs / hbm_gbs,
+                        "tokens_per_s": B / ms * 1e3}
+
+    # end to end through the public API with host buffers: H2D of the layer, the step, D2H of the results
+    e2e = None
+    if args.e2e_steps > 0:
+        hostW = {k: torch.empty(layer.W[k].shape, dtype=layer.W[k].dtype, pin_memory=True) for k in layer.kinds}
+        hostI = {k: torch.empty(layer.idx[k].shape, dtype=torch.uint8, pin_memory=True) for k in layer.kinds}
+        hostS = {k: torch.empty(layer.sc[k].shape, dtype=torch.int16, pin_memory=True) for k in layer.kinds}
+        hostE = torch.empty(3, dtype=torch.float64, pin_memory=True)
+        hostY = torch.empty((8 * 7168 + 16 * 2048,), dtype=torch.float32, pin_memory=True)
+        for k in layer.kinds:
+            hostW[k].copy_(layer.W[k])
+        torch.cuda.synchronize()
+        h2d = sum(hostW[k].numel() * hostW[k].element_size() for k in layer.kinds)
+        d2h = sum(hostI[k].numel() + 2 * hostS[k].numel() for k in layer.kinds) + 24 + 4 * hostY.numel()
+        barrier()
+        a, b = ev(), ev()
+        a.record()
+        for i in range(args.e2e_steps):
+            for k in layer.kinds:
+                layer.W[k].copy_(hostW[k], non_blocking=True)
+            step(i)
+            for k in layer.kinds:
+                hostI[k].copy_(layer.idx[k], non_blocking=True)
+                hostS[k].copy_(layer.sc[k], non_blocking=True)
+            for j, k in enumerate(layer.kinds):
+                hostE[j:j + 1].copy_(layer.err[k], non_blocking=True)
+            plans = layer.moe[1][0][i % layer.groups]
+            off = 0
+            for m in plans[4] + plans[5]:
+                n = m["y"].numel()
+                hostY[off:off + n].copy_(m["y"].view(-1), non_blocking=True)
+                off += n
+        b.record()
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / args.e2e_steps
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": world * layer.weights / e2e_ms / 1e6, "unit": "Gweights/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    errs = {str(k): float(layer.err[k].item()) for k in layer.kinds}
+    ms_step = total_ms / args.steps
+    value = world * layer.weights / ms_step / 1e6  # Gweights/s over the whole path
+    enc_tflops = FLOPS_PER_WEIGHT * layer.weights / enc_ms / 1e9
+    dev_err = vq.vq3r_device_error()
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": "Gweights/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "moe-layer-64x3-bf16: encode + decode(fp32) + rel-Frobenius of the layer, "
+                                   "then moe-decode-step-8-experts GEMV (B=1)",
+                       "experts_per_gpu": args.experts, "weights_per_gpu": layer.weights,
+                       "matrices": "w1,w3 2048x7168; w2 7168x2048 per expert, stacked per kind",
+                       "l2": "inputs larger than L2 (5.6 GB layer); GEMV rotates 8 disjoint 8-expert groups "
+                             "(1.06 GB of indices)"},
+            "roofline": {"bound": "alu", "achieved": enc_tflops, "peak": fp32_peak_tflops, "unit": "TFLOP/s",
+                         "frac": enc_tflops / fp32_peak_tflops, "traffic": None,
+                         "kernel": "vq3r_encode (row scale + greedy assignment), %d algorithmic flops/weight; "
+                                   "peak = %d SMs x 128 FP32 lanes x 2 (FMA-counted) x %.0f MHz" %
+                                   (FLOPS_PER_WEIGHT, sms, sm_max_mhz),
+                         "frac_of_non_fma_ceiling": 2 * enc_tflops / fp32_peak_tflops * 23 / 24},
+            "kernels": {
+                "encode": {"ms": enc_ms, "Gweights/s": layer.weights / enc_ms / 1e6, "TFLOP/s": enc_tflops},
+                "decode_f32": {"ms": dec_ms, "GB/s": layer.weights * (4 + 0.375) / dec_ms / 1e6,
+                               "frac_hbm": layer.weights * 4.375 / dec_ms / 1e6 / hbm_gbs},
+                "rel_frobenius": {"ms": err_ms, "GB/s": layer.weights * (2 + 0.375) / err_ms / 1e6,
+                                  "frac_hbm": layer.weights * 2.375 / err_ms / 1e6 / hbm_gbs, "errors": errs},
+                "gemv_in_step_B1": {"us": 1e3 * gv1_ms, "GB/s": moe_step_bytes(1) / gv1_ms / 1e6,
+                                    "frac_hbm": moe_step_bytes(1) / gv1_ms / 1e6 / hbm_gbs},
+                "gemv_sweep": gemv,
+                "hbm_peak_gbs": hbm_gbs, "peak_source": peak_src},
+            "e2e": e2e,
+            "gpu_launches": Layer.LAUNCHES_PER_STEP * args.steps,
+            "clocks": clk,
+            "device_error": dev_err,
+        }
+        if cpu is not None:
+            out["cpu_baseline"] = cpu
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

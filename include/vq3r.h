@@ -119,12 +119,17 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
  * A matrix with rows == 0 contributes nothing (its pointers may be NULL).
  */
 typedef struct {
-  const uint8_t* idx;       /* [3][rows][cols/8] */
+  const uint8_t* idx;       /* plane 0 of [3][rows][cols/8]; planes plane_stride bytes apart */
   const uint16_t* scales;   /* [rows] binary16 */
   const float* codebooks;   /* [3][256][8] */
   int64_t rows, cols;
   const void* x;            /* [B][cols] */
   float* y;                 /* [B][rows] */
+  int64_t plane_stride;     /* bytes from one index plane to the next; 0 = rows * cols / 8.
+                               A row range [r0, r0 + rows) of a larger encoded matrix
+                               (e.g. one expert of a stacked layer) is described by
+                               idx + r0 * cols / 8, scales + r0 and that matrix's
+                               plane size; it must be a multiple of 16. */
 } vq3r_gemv_desc;
 
 size_t vq3r_gemv_workspace_size(const vq3r_gemv_desc* mats, int n_mats, int B);

@@ -36,7 +36,8 @@ class VQ3RError(RuntimeError):
 
 class GemvDesc(ctypes.Structure):
     _fields_ = [("idx", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("codebooks", ctypes.c_void_p),
-                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("plane_stride", ctypes.c_int64)]
 
 
 _L = None
@@ -117,8 +118,17 @@ def _descs(mats):
     arr = (GemvDesc * len(mats))()
     for i, m in enumerate(mats):
         idx, scales, cb, x, y = m["idx"], m["scales"], m["codebooks"], m["x"], m["y"]
-        arr[i] = GemvDesc(_dev(idx, "idx"), _dev(scales, "scales"), _dev(cb, "codebooks"), idx.shape[1],
-                          idx.shape[2] * DIM, _dev(x, "x"), _dev(y, "y"))
+        if "rows" in m:
+            # a row range of a larger encoded matrix: idx is the full [3][R][V] tensor
+            r0, rows = m.get("row0", 0), m["rows"]
+            V = idx.shape[2]
+            if not (idx.is_cuda and idx.is_contiguous()):
+                raise ValueError("idx must be a contiguous CUDA tensor")
+            arr[i] = GemvDesc(idx.data_ptr() + r0 * V, scales.data_ptr() + 2 * r0, _dev(cb, "codebooks"), rows,
+                              V * DIM, _dev(x, "x"), _dev(y, "y"), idx.shape[1] * V)
+        else:
+            arr[i] = GemvDesc(_dev(idx, "idx"), _dev(scales, "scales"), _dev(cb, "codebooks"), idx.shape[1],
+                              idx.shape[2] * DIM, _dev(x, "x"), _dev(y, "y"), 0)
     return arr
 
 
@@ -128,7 +138,10 @@ def vq3r_gemv_workspace_size(mats, B):
 
 
 def vq3r_gemv(mats, B, workspace=None, stream=None):
-    """y = W_hat . x for each descriptor dict {idx, scales, codebooks, x [B][cols], y [B][rows] float32}."""
+    """y = W_hat . x for each descriptor dict {idx, scales, codebooks, x [B][cols], y [B][rows] float32}.
+
+    With keys "row0" and "rows" the descriptor covers rows [row0, row0 + rows) of the
+    encoded matrix (idx [3][R][V], scales [R]), e.g. one expert of a stacked layer."""
     arr = _descs(mats)
     ws = _lib().vq3r_gemv_workspace_size(arr, len(mats), B)
     if workspace is None:

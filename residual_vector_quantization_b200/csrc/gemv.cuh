@@ -49,6 +49,7 @@ struct GvMat {
   float* y;
   float* partial;     // [B][n_slabs][rows]
   int64_t rows;
+  int64_t plane_stride;  // bytes between index planes
   int32_t group;
   int32_t n_tiles;     // ceil(rows / kGvTileRows)
   int32_t tile_prefix; // tiles of the earlier matrices of the same group
@@ -203,7 +204,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_lut_kernel(const __grid_co
     const int64_t V = G.cols / kDim;
     const int64_t v0 = (int64_t)U.slab * kSlabV + 4 * l16;
     const int64_t row0 = (int64_t)U.tile * kGvTileRows + warp * (2 * kGvRowPairs) + h;
-    const int64_t plane_stride = M.rows * V;
+    const int64_t plane_stride = M.plane_stride;
 
     uint32_t wd[kGvRowPairs][kStages];
 #pragma unroll

@@ -87,10 +87,12 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
     vq3r_status st = check_shape(d.rows, d.cols, 0);
     if (st != VQ3R_OK) return st;
     if (d.cols / kDim > (int64_t)kSlabV * (1 << 20)) return VQ3R_ERR_SHAPE;
+    const int64_t plane = d.rows * (d.cols / kDim);
+    if (d.plane_stride != 0 && d.plane_stride < plane) return VQ3R_ERR_SHAPE;
     if (d.rows > 0) {  // an empty matrix may carry NULL pointers
       if (!d.idx || !d.scales || !d.codebooks || !d.x || !d.y) return VQ3R_ERR_NULL;
       if (!aligned16(d.idx) || !aligned16(d.scales) || !aligned16(d.codebooks) || !aligned16(d.x) ||
-          !aligned16(d.y))
+          !aligned16(d.y) || ((d.plane_stride ? d.plane_stride : plane) & 15))
         return VQ3R_ERR_ALIGN;
     }
     if ((d.cols / kDim) % 4) plan->aligned4 = false;
@@ -109,6 +111,7 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
     M.scales = d.scales;
     M.y = d.y;
     M.rows = d.rows;
+    M.plane_stride = d.plane_stride ? d.plane_stride : plane;
     M.group = g;
     M.n_tiles = (int32_t)((d.rows + kGvTileRows - 1) / kGvTileRows);
     M.tile_prefix = P.g[g].tiles;

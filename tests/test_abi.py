@@ -62,7 +62,7 @@ def test_null_and_shape_errors_return_before_any_launch(lib):
 def _descs(specs):
     arr = (vq.GemvDesc * len(specs))()
     for i, (rows, cols, cb, x) in enumerate(specs):
-        arr[i] = vq.GemvDesc(0x200000 + 0x1000 * i, 0x300000 + 0x1000 * i, cb, rows, cols, x, 0x400000 + 0x1000 * i)
+        arr[i] = vq.GemvDesc(0x200000 + 0x1000 * i, 0x300000 + 0x1000 * i, cb, rows, cols, x, 0x400000 + 0x1000 * i, 0)
     return arr
 
 
@@ -88,3 +88,11 @@ def test_gemv_workspace_groups_shared_tables(lib):
     specs = [(7168, 2048, 0x10000, 0x20000 + 0x10000 * i) for i in range(8)]
     ws = lib.vq3r_gemv_workspace_size(_descs(specs), 8, 1)
     assert ws == 8 * 4 * slab + 8 * 4 * 7168 * 4
+
+
+def test_gemv_plane_stride_checks(lib):
+    arr = _descs([(2048, 7168, 0x10000, 0x20000)])
+    arr[0].plane_stride = 2048 * 896 - 16  # smaller than one plane
+    assert lib.vq3r_gemv(arr, 1, 1, 1, 0x500000, 1 << 30, None) == 2
+    arr[0].plane_stride = 64 * 2048 * 896 + 8  # not a multiple of 16
+    assert lib.vq3r_gemv(arr, 1, 1, 1, 0x500000, 1 << 30, None) == 3
