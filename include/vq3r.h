@@ -129,7 +129,7 @@ typedef struct {
                                A row range [r0, r0 + rows) of a larger encoded matrix
                                (e.g. one expert of a stacked layer) is described by
                                idx + r0 * cols / 8, scales + r0 and that matrix's
-                               plane size; it must be a multiple of 16. */
+                               plane size (VQ3R_ERR_SHAPE if below rows * cols / 8). */
 } vq3r_gemv_desc;
 
 size_t vq3r_gemv_workspace_size(const vq3r_gemv_desc* mats, int n_mats, int B);

@@ -33,38 +33,50 @@ constexpr int kSlabWords = kStages * kCodewords * kSlabV;   // 49152 floats
 constexpr uint32_t kSlabBytes = kSlabWords * 4u;            // 192 KiB
 constexpr int kGvThreads = 512;
 constexpr int kGvWarps = kGvThreads / 32;
-constexpr int kGvRowPairs = 4;                              // row pairs per warp per unit
-constexpr int kGvTileRows = kGvWarps * kGvRowPairs * 2;     // 128 rows per unit
+constexpr int kGvRowsPerWarp = 8;                           // 4 lanes per row, 16 columns per lane
+constexpr int kGvTileRows = kGvWarps * kGvRowsPerWarp;      // 128 rows per unit
+constexpr int kGvRing = 3;                                  // units of index words held per lane
+constexpr int kSlabGroup = 2;                               // CTAs walking adjacent slabs in step
 constexpr int kLutBuildBlocksPerImage = 12;                 // 64 (stage, codeword) rows per block
 
-// Word offset of T_s[v][j] inside a slab image:
-//   s * 16384 + j * 64 + (v & 1) * 32 + bank(v),  bank(v) = 16 * ((v >> 1) & 1) + (v >> 2).
+// Word offset of T_s[v][j] inside a slab image (v = column within the slab):
+//   s * 16384 + j * 64 + slot(v) * 32 + bank(v),
+//   slot(v) = (v >> 2) & 1,  bank(v) = 8 * (v >> 4) + (v & 3) + 4 * ((v >> 3) & 1).
+// Lane (g, a) of a warp (g = lane / 4 picks one of 8 rows, a = lane % 4 the
+// 16 columns [16a, 16a + 16)) visits its columns in the order o = m ^ d(g),
+// d(g) = (g & 3) | ((g >> 2) << 3), m = 0..15.  At step m its bank is
+// 8a + ((m ^ g) & 3) + 4 * ((m >> 3) ^ (g >> 2)), so the 32 lanes hit 32
+// distinct banks whatever the indices, and the slot ((m >> 2) & 1) is the
+// same for all lanes.  The column's index byte sits in register m >> 2 when
+// the lane loads its two 8-byte halves in the order (g >> 2, 1 - (g >> 2)).
 __host__ __device__ __forceinline__ int slab_word(int s, int v, int j) {
-  return s * (kCodewords * kSlabV) + j * kSlabV + (v & 1) * 32 + 16 * ((v >> 1) & 1) + (v >> 2);
+  return s * (kCodewords * kSlabV) + j * kSlabV + ((v >> 2) & 1) * 32 + 8 * (v >> 4) + (v & 3) + 4 * ((v >> 3) & 1);
 }
 
 struct GvMat {
   const uint8_t* idx;
   const uint16_t* scales;
   float* y;
-  float* partial;     // [B][n_slabs][rows]
+  float* partial;        // [B][n_slabs][rows]
   int64_t rows;
   int64_t plane_stride;  // bytes between index planes
   int32_t group;
-  int32_t n_tiles;     // ceil(rows / kGvTileRows)
-  int32_t tile_prefix; // tiles of the earlier matrices of the same group
+  int32_t n_tiles;       // ceil(rows / kGvTileRows) >= 1
+  int32_t tile_prefix;   // tiles of the earlier matrices of the same group
   int32_t pad_;
 };
 
 struct GvGroup {
   const float* codebooks;
-  const void* x;       // [B][cols]
-  float* lut;          // [B][n_slabs] slab images
+  const void* x;         // [B][cols]
+  float* lut;            // [B][n_slabs] slab images
   int64_t cols;
-  int64_t unit_begin;  // first work unit of this group
+  int64_t unit_begin;    // first work unit of this group
   int32_t n_slabs;
-  int32_t tiles;       // tiles of all matrices of the group (units per (slab, token))
-  int32_t image_begin; // first slab image (for the build kernel)
+  int32_t n_sgroups;     // ceil(n_slabs / kSlabGroup)
+  int32_t tiles;         // tiles of all matrices of the group (units per (slab, token))
+  int32_t image_begin;   // first slab image (for the build kernel)
+  int16_t mat_begin, mat_end;  // the group's matrices are P.m[mat_begin .. mat_end)
   int32_t pad_;
 };
 
@@ -74,14 +86,23 @@ struct GvParams {
   int32_t n_mats, n_groups, B, x_dtype;
   int64_t total_units;
   int32_t total_images;
-  int32_t pad_;
+  int32_t vec8;          // 1: index rows and planes are 8-byte aligned (64-bit loads)
 };
+
+// Programmatic dependent launch: wait until the preceding kernel in the
+// stream has completed and its writes are visible / let the next kernel's
+// CTAs launch early (they wait at their own griddep_wait).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // ---------------- table build ----------------
 
 template <int XDT>
 __global__ void __launch_bounds__(kGvThreads) lut_build_kernel(const __grid_constant__ GvParams P) {
   __shared__ float xs[kSlabV][kDim];
+  griddep_launch_dependents();
   const int image = blockIdx.x / kLutBuildBlocksPerImage;
   const int part = blockIdx.x - image * kLutBuildBlocksPerImage;
   int gi = 0;
@@ -123,128 +144,180 @@ __global__ void __launch_bounds__(kGvThreads) lut_build_kernel(const __grid_cons
 
 // ---------------- main kernel ----------------
 
-// Unit u of the schedule: (group, slab, token, matrix, row tile), ordered so
-// that consecutive units share a slab image.
-struct GvUnit {
-  int g, slab, b, m, tile;
+// Work unit: (group, slab group, token, matrix, row tile of 128 rows),
+// ordered so that consecutive units share a slab image.  The kSlabGroup CTAs
+// of a CTA group take the same units, each its own slab of the slab group:
+// they read adjacent 64-byte pieces of the same index rows at about the same
+// time, so each 128-byte line fetched from DRAM serves both.
+struct GvCursor {
+  int g, sg, b, m, tile;
 };
 
-__device__ __forceinline__ GvUnit decode_unit(const GvParams& P, int64_t u) {
-  GvUnit r;
+__device__ __forceinline__ GvCursor unit_cursor(const GvParams& P, int64_t u) {
+  GvCursor c;
   int g = 0;
   while (g + 1 < P.n_groups && P.g[g + 1].unit_begin <= u) g++;
   const GvGroup& G = P.g[g];
   const int64_t lu = u - G.unit_begin;
   const int64_t sb = lu / G.tiles;  // slab * B + b
-  int t = (int)(lu - sb * G.tiles);
-  r.g = g;
-  r.slab = (int)(sb / P.B);
-  r.b = (int)(sb - (int64_t)r.slab * P.B);
-  int m = 0;
-  while (m < P.n_mats && !(P.m[m].group == g && t >= P.m[m].tile_prefix && t < P.m[m].tile_prefix + P.m[m].n_tiles))
-    m++;
-  r.m = m;
-  r.tile = t - P.m[m].tile_prefix;
-  return r;
+  const int t = (int)(lu - sb * G.tiles);
+  c.g = g;
+  c.sg = (int)(sb / P.B);
+  c.b = (int)(sb - (int64_t)c.sg * P.B);
+  int m = G.mat_begin;
+  while (m + 1 < G.mat_end && P.m[m + 1].tile_prefix <= t) m++;
+  c.m = m;
+  c.tile = t - P.m[m].tile_prefix;
+  return c;
 }
 
-template <bool ALIGNED4>
-__device__ __forceinline__ uint32_t load_idx_word(const uint8_t* plane, int64_t off, int64_t v0, int64_t V) {
-  if (ALIGNED4) {
-    return (v0 < V) ? __ldcs(reinterpret_cast<const unsigned int*>(plane + off)) : 0u;
-  } else {
-    uint32_t w = 0;
+__device__ __forceinline__ void unit_advance(const GvParams& P, GvCursor& c) {
+  if (++c.tile < P.m[c.m].n_tiles) return;
+  c.tile = 0;
+  if (++c.m < P.g[c.g].mat_end) return;
+  c.m = P.g[c.g].mat_begin;
+  if (++c.b < P.B) return;
+  c.b = 0;
+  if (++c.sg < P.g[c.g].n_sgroups) return;
+  c.sg = 0;
+  if (++c.g < P.n_groups) c.m = P.g[c.g].mat_begin;
+}
+
+// The 12 index words of one lane for one unit: for plane s, registers 0-1
+// hold bytes [8h, 8h + 8) and registers 2-3 bytes [8(1-h), 8(1-h) + 8) of the
+// lane's 16 columns, h = g >> 2 (zero past the matrix's end).
+__device__ __forceinline__ void load_unit_words(const GvParams& P, const GvCursor& c, int member, int warp, int g,
+                                                int a, uint32_t wd[kStages][4]) {
+  const GvMat& M = P.m[c.m];
+  const int64_t V = P.g[c.g].cols / kDim;
+  const int64_t row0 = (int64_t)c.tile * kGvTileRows;
+  const int64_t row = row0 + warp * kGvRowsPerWarp + g;
+  const int64_t col0 = (int64_t)(c.sg * kSlabGroup + member) * kSlabV;
+  const int h = g >> 2;
+  const uint8_t* base = M.idx + row * V + col0 + 16 * a;
+  if (P.vec8 && row0 + kGvTileRows <= M.rows && col0 + kSlabV <= V) {
 #pragma unroll
-    for (int i = 0; i < 4; i++)
-      if (v0 + i < V) w |= (uint32_t)__ldcs(plane + off + i) << (8 * i);
-    return w;
+    for (int s = 0; s < kStages; s++) {
+      const uint8_t* p = base + s * M.plane_stride;
+      const uint2 x0 = __ldg(reinterpret_cast<const uint2*>(p + 8 * h));
+      const uint2 x1 = __ldg(reinterpret_cast<const uint2*>(p + 8 * (1 - h)));
+      wd[s][0] = x0.x;
+      wd[s][1] = x0.y;
+      wd[s][2] = x1.x;
+      wd[s][3] = x1.y;
+    }
+  } else {  // edge of the matrix or unaligned rows: byte loads with bounds checks
+    const bool row_ok = row < M.rows;
+#pragma unroll
+    for (int s = 0; s < kStages; s++) {
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        const int cw = 4 * (k ^ (2 * h));  // first column of the word held in register k
+        uint32_t x = 0;
+#pragma unroll 1
+        for (int i = 0; i < 4; i++)
+          if (row_ok && col0 + 16 * a + cw + i < V) x |= (uint32_t)__ldg(base + s * M.plane_stride + cw + i) << (8 * i);
+        wd[s][k] = x;
+      }
+    }
   }
 }
 
-template <bool ALIGNED4>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_lut_kernel(const __grid_constant__ GvParams P) {
   extern __shared__ __align__(128) unsigned char gv_smem[];
-  unsigned char* lut_s = gv_smem;                                  // kSlabBytes
+  unsigned char* lut_s = gv_smem;  // kSlabBytes
   uint64_t* mbar = reinterpret_cast<uint64_t*>(gv_smem + kSlabBytes);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = lane >> 4, l16 = lane & 15;
-  // PRMT operands: byte 0 = bank byte offset of this lane's column, byte 1 = index byte.
-  const uint32_t lc0 = 64u * h + 4u * l16;        // steps m = 0, 1
-  const uint32_t lc1 = 64u * (1 - h) + 4u * l16;  // steps m = 2, 3
+  const int g = lane >> 2, a = lane & 3;
+  // PRMT operands: byte 0 = byte offset of the bank of the current column, byte 1 = its index.
+  // lc[q], q = (m & 3) | ((m >> 3) << 2); sel[m & 3] picks the index byte (m ^ g) & 3.
+  uint32_t lc[8];
+#pragma unroll
+  for (int q = 0; q < 8; q++)
+    lc[q] = 4u * (8u * a + (uint32_t)((q & 3) ^ (g & 3)) + 4u * (uint32_t)((q >> 2) ^ (g >> 2)));
   uint32_t sel[4];
 #pragma unroll
-  for (int m = 0; m < 4; m++) sel[m] = 0x5504u | ((uint32_t)((m + 2 * h) & 3) << 4);
+  for (int q = 0; q < 4; q++) sel[q] = 0x5504u | ((uint32_t)((q ^ g) & 3) << 4);
 
-  const int64_t u0 = (int64_t)blockIdx.x * P.total_units / gridDim.x;
-  const int64_t u1 = (int64_t)(blockIdx.x + 1) * P.total_units / gridDim.x;
+  const int member = blockIdx.x % kSlabGroup;  // which slab of each slab group
+  const int64_t cg = blockIdx.x / kSlabGroup, ncg = gridDim.x / kSlabGroup;
+  const int64_t u0 = cg * P.total_units / ncg;
+  const int64_t u1 = (cg + 1) * P.total_units / ncg;
+  griddep_launch_dependents();  // the reduction kernel may be scheduled now; it waits for us
+  if (u0 >= u1) return;
   if (tid == 0) mbar_init(mbar, 1);
   __syncthreads();
 
-  const float* cur = nullptr;
+  // Ring of kGvRing units of index words: while unit u is looked up, the
+  // loads of units u+1 .. u+kGvRing-1 are in flight.
+  GvCursor c0 = unit_cursor(P, u0), c1 = c0, c2;
+  unit_advance(P, c1);
+  c2 = c1;
+  unit_advance(P, c2);
+  uint32_t w0[kStages][4], w1[kStages][4], w2[kStages][4];
+  load_unit_words(P, c0, member, warp, g, a, w0);
+  if (u0 + 1 < u1) load_unit_words(P, c1, member, warp, g, a, w1);
+  if (u0 + 2 < u1) load_unit_words(P, c2, member, warp, g, a, w2);
+
+  griddep_wait();  // the slab tables written by the build kernel are complete
+
+  const float* loaded = nullptr;
   uint32_t phase = 0;
-  for (int64_t u = u0; u < u1; u++) {
-    const GvUnit U = decode_unit(P, u);
-    const GvGroup& G = P.g[U.g];
-    const GvMat& M = P.m[U.m];
-    const float* img = G.lut + ((size_t)U.b * G.n_slabs + U.slab) * kSlabWords;
-    if (img != cur) {
+  auto step = [&](int64_t u, GvCursor& c, uint32_t (&wa)[kStages][4]) -> bool {
+    const GvGroup& G = P.g[c.g];
+    const int slab = c.sg * kSlabGroup + member;
+    if (slab >= G.n_slabs) {  // odd slab count: this CTA has no slab in the last group
+#pragma unroll
+      for (int i = 0; i < kGvRing; i++) unit_advance(P, c);
+      if (u + kGvRing < u1) load_unit_words(P, c, member, warp, g, a, wa);
+      return true;
+    }
+    const float* img = G.lut + ((size_t)c.b * G.n_slabs + slab) * kSlabWords;
+    if (img != loaded) {
       __syncthreads();  // every warp is done with the previous image
       if (tid == 0) {
         mbar_arrive_expect_tx(mbar, kSlabBytes);
 #pragma unroll
-        for (int c = 0; c < 4; c++)
-          bulk_copy_g2s(lut_s + c * (kSlabBytes / 4), reinterpret_cast<const unsigned char*>(img) + c * (kSlabBytes / 4),
-                        kSlabBytes / 4, mbar);
+        for (int q = 0; q < 4; q++)
+          bulk_copy_g2s(lut_s + q * (kSlabBytes / 4),
+                        reinterpret_cast<const unsigned char*>(img) + q * (kSlabBytes / 4), kSlabBytes / 4, mbar);
       }
-      if (!mbar_wait_bounded(mbar, phase)) return;
+      if (!mbar_wait_bounded(mbar, phase)) return false;
       phase ^= 1u;
-      cur = img;
+      loaded = img;
     }
-    const int64_t V = G.cols / kDim;
-    const int64_t v0 = (int64_t)U.slab * kSlabV + 4 * l16;
-    const int64_t row0 = (int64_t)U.tile * kGvTileRows + warp * (2 * kGvRowPairs) + h;
-    const int64_t plane_stride = M.plane_stride;
-
-    uint32_t wd[kGvRowPairs][kStages];
+    float acc = 0.0f;
 #pragma unroll
-    for (int p = 0; p < kGvRowPairs; p++) {
-      const int64_t row = row0 + 2 * p;
+    for (int m = 0; m < 16; m++) {
 #pragma unroll
-      for (int s = 0; s < kStages; s++)
-        wd[p][s] = (row < M.rows) ? load_idx_word<ALIGNED4>(M.idx + s * plane_stride, row * V + v0, v0, V) : 0u;
-    }
-    float acc[kGvRowPairs];
-#pragma unroll
-    for (int p = 0; p < kGvRowPairs; p++) {
-      float a = 0.0f;
-#pragma unroll
-      for (int m = 0; m < 4; m++) {
-        const uint32_t lc = (m < 2) ? lc0 : lc1;
-#pragma unroll
-        for (int s = 0; s < kStages; s++) {
-          const uint32_t off = __byte_perm(wd[p][s], lc, sel[m]);
-          a += *reinterpret_cast<const float*>(lut_s + off + s * 65536 + (m & 1) * 128);
-        }
+      for (int s = 0; s < kStages; s++) {
+        const uint32_t off = __byte_perm(wa[s][m >> 2], lc[(m & 3) | ((m >> 3) << 2)], sel[m & 3]);
+        acc += *reinterpret_cast<const float*>(lut_s + off + s * 65536 + ((m >> 2) & 1) * 128);
       }
-      acc[p] = a;
     }
+    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
+    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 2);
+    const GvMat& M = P.m[c.m];
+    const int64_t row = (int64_t)c.tile * kGvTileRows + warp * kGvRowsPerWarp + g;
+    if (a == 0 && row < M.rows) M.partial[((int64_t)c.b * G.n_slabs + slab) * M.rows + row] = acc;
+    // this buffer now takes unit u + kGvRing
 #pragma unroll
-    for (int p = 0; p < kGvRowPairs; p++) {
-      float a = acc[p];
-      a += __shfl_xor_sync(0xFFFFFFFFu, a, 8);
-      a += __shfl_xor_sync(0xFFFFFFFFu, a, 4);
-      a += __shfl_xor_sync(0xFFFFFFFFu, a, 2);
-      a += __shfl_xor_sync(0xFFFFFFFFu, a, 1);
-      const int64_t row = row0 + 2 * p;
-      if (l16 == 0 && row < M.rows) M.partial[((int64_t)U.b * G.n_slabs + U.slab) * M.rows + row] = a;
-    }
+    for (int i = 0; i < kGvRing; i++) unit_advance(P, c);
+    if (u + kGvRing < u1) load_unit_words(P, c, member, warp, g, a, wa);
+    return true;
+  };
+  for (int64_t u = u0; u < u1; u += kGvRing) {
+    if (!step(u, c0, w0)) return;
+    if (u + 1 < u1 && !step(u + 1, c1, w1)) return;
+    if (u + 2 < u1 && !step(u + 2, c2, w2)) return;
   }
 }
 
 // y[b][i] = scale_i * sum_slab partial[b][slab][i], slabs in ascending order.
 __global__ void __launch_bounds__(256) gemv_reduce_kernel(const __grid_constant__ GvParams P) {
   // blockIdx.y = matrix
+  griddep_wait();
   const GvMat& M = P.m[blockIdx.y];
   const GvGroup& G = P.g[M.group];
   const int64_t n = (int64_t)P.B * M.rows;

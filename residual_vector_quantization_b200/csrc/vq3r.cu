@@ -52,8 +52,7 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     g_dev_err[dev] = r;
   });
   *sms = g_dev_sms[dev];
@@ -70,18 +69,18 @@ constexpr int kErrMaxBlocks = 4096;
 struct GemvPlan {
   GvParams P;
   size_t ws_bytes;
-  bool aligned4;
 };
 
 // Groups matrices sharing (codebooks, x, cols), lays out the workspace and
-// numbers the work units.  Returns false on an invalid descriptor.
+// numbers the work units.  Matrices are stored grouped (each group's
+// matrices contiguous in P.m); empty matrices are dropped.
 vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_base, GemvPlan* plan) {
   GvParams& P = plan->P;
   memset(&P, 0, sizeof(P));
-  P.n_mats = n_mats;
   P.B = B;
-  plan->aligned4 = true;
+  P.vec8 = 1;
   int n_groups = 0;
+  int group_of[VQ3R_GEMV_MAX_MATS];
   for (int i = 0; i < n_mats; i++) {
     const vq3r_gemv_desc& d = mats[i];
     vq3r_status st = check_shape(d.rows, d.cols, 0);
@@ -89,13 +88,14 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
     if (d.cols / kDim > (int64_t)kSlabV * (1 << 20)) return VQ3R_ERR_SHAPE;
     const int64_t plane = d.rows * (d.cols / kDim);
     if (d.plane_stride != 0 && d.plane_stride < plane) return VQ3R_ERR_SHAPE;
-    if (d.rows > 0) {  // an empty matrix may carry NULL pointers
-      if (!d.idx || !d.scales || !d.codebooks || !d.x || !d.y) return VQ3R_ERR_NULL;
-      if (!aligned16(d.idx) || !aligned16(d.scales) || !aligned16(d.codebooks) || !aligned16(d.x) ||
-          !aligned16(d.y) || ((d.plane_stride ? d.plane_stride : plane) & 15))
-        return VQ3R_ERR_ALIGN;
-    }
-    if ((d.cols / kDim) % 4) plan->aligned4 = false;
+    group_of[i] = -1;
+    if (d.rows == 0) continue;  // an empty matrix may carry NULL pointers
+    if (!d.idx || !d.scales || !d.codebooks || !d.x || !d.y) return VQ3R_ERR_NULL;
+    if (!aligned16(d.idx) || !aligned16(d.scales) || !aligned16(d.codebooks) || !aligned16(d.x) || !aligned16(d.y))
+      return VQ3R_ERR_ALIGN;
+    const int64_t stride = d.plane_stride ? d.plane_stride : plane;
+    // 64-bit index loads need 8-byte aligned rows and planes; otherwise bytes are loaded one by one
+    if ((d.cols / kDim) % 8 || (stride & 7)) P.vec8 = 0;
     int g = 0;
     while (g < n_groups && !(P.g[g].codebooks == d.codebooks && P.g[g].x == d.x && P.g[g].cols == d.cols)) g++;
     if (g == n_groups) {
@@ -103,21 +103,33 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
       P.g[g].x = d.x;
       P.g[g].cols = d.cols;
       P.g[g].n_slabs = (int32_t)((d.cols / kDim + kSlabV - 1) / kSlabV);
-      P.g[g].tiles = 0;
+      P.g[g].n_sgroups = (P.g[g].n_slabs + kSlabGroup - 1) / kSlabGroup;
       n_groups++;
     }
-    GvMat& M = P.m[i];
-    M.idx = d.idx;
-    M.scales = d.scales;
-    M.y = d.y;
-    M.rows = d.rows;
-    M.plane_stride = d.plane_stride ? d.plane_stride : plane;
-    M.group = g;
-    M.n_tiles = (int32_t)((d.rows + kGvTileRows - 1) / kGvTileRows);
-    M.tile_prefix = P.g[g].tiles;
-    P.g[g].tiles += M.n_tiles;
+    group_of[i] = g;
   }
   P.n_groups = n_groups;
+  int nm = 0;
+  for (int g = 0; g < n_groups; g++) {
+    P.g[g].mat_begin = (int16_t)nm;
+    P.g[g].tiles = 0;
+    for (int i = 0; i < n_mats; i++) {
+      if (group_of[i] != g) continue;
+      const vq3r_gemv_desc& d = mats[i];
+      GvMat& M = P.m[nm++];
+      M.idx = d.idx;
+      M.scales = d.scales;
+      M.y = d.y;
+      M.rows = d.rows;
+      M.plane_stride = d.plane_stride ? d.plane_stride : d.rows * (d.cols / kDim);
+      M.group = g;
+      M.n_tiles = (int32_t)((d.rows + kGvTileRows - 1) / kGvTileRows);
+      M.tile_prefix = P.g[g].tiles;
+      P.g[g].tiles += M.n_tiles;
+    }
+    P.g[g].mat_end = (int16_t)nm;
+  }
+  P.n_mats = nm;
   size_t off = 0;
   int64_t units = 0;
   int32_t images = 0;
@@ -126,11 +138,11 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
     G.lut = reinterpret_cast<float*>(ws_base + off);
     off = align_up(off + (size_t)B * G.n_slabs * kSlabBytes);
     G.unit_begin = units;
-    units += (int64_t)G.n_slabs * B * G.tiles;
+    units += (int64_t)G.n_sgroups * B * G.tiles;
     G.image_begin = images;
     images += B * G.n_slabs;
   }
-  for (int i = 0; i < n_mats; i++) {
+  for (int i = 0; i < nm; i++) {
     GvMat& M = P.m[i];
     M.partial = reinterpret_cast<float*>(ws_base + off);
     off = align_up(off + (size_t)B * P.g[M.group].n_slabs * (size_t)M.rows * sizeof(float));
@@ -239,16 +251,34 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
     case VQ3R_BF16: lut_build_kernel<VQ3R_BF16><<<build_blocks, kGvThreads, 0, s>>>(P); break;
     default: lut_build_kernel<VQ3R_F16><<<build_blocks, kGvThreads, 0, s>>>(P); break;
   }
-  const int grid = (int)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms);
-  const size_t smem = kSlabBytes + 16;
-  if (plan.aligned4) gemv_lut_kernel<true><<<grid, kGvThreads, smem, s>>>(P);
-  else gemv_lut_kernel<false><<<grid, kGvThreads, smem, s>>>(P);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  // The main and reduction kernels are launched with programmatic stream
+  // serialization: each may start while its predecessor finishes and waits
+  // (griddepcontrol.wait) before reading the predecessor's results.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  const int64_t groups = (sms / kSlabGroup) < P.total_units ? (sms / kSlabGroup) : P.total_units;
+  cfg.gridDim = dim3((unsigned)(groups * kSlabGroup));
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = kSlabBytes + 16;
+  cfg.stream = s;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel, P);
+  if (e != cudaSuccess) return cuda_fail(e);
   int64_t maxrows = 0;
-  for (int i = 0; i < n_mats; i++) maxrows = P.m[i].rows * B > maxrows ? P.m[i].rows * B : maxrows;
+  for (int i = 0; i < P.n_mats; i++) maxrows = P.m[i].rows * B > maxrows ? P.m[i].rows * B : maxrows;
   int64_t gx = (maxrows + 255) / 256;
   if (gx > (int64_t)sms * 4) gx = (int64_t)sms * 4;
   if (gx < 1) gx = 1;
-  gemv_reduce_kernel<<<dim3((unsigned)gx, (unsigned)n_mats), 256, 0, s>>>(P);
+  cfg.gridDim = dim3((unsigned)gx, (unsigned)P.n_mats);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  e = cudaLaunchKernelEx(&cfg, gemv_reduce_kernel, P);
+  if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
 
