@@ -153,6 +153,34 @@ vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const ui
                                      const float* codebooks, int64_t rows, int64_t cols, double* err_out,
                                      void* workspace, size_t ws_bytes, vq3r_stream stream);
 
+/*
+ * vq3r_gemv_noalloc -- vq3r_gemv for callers that cannot allocate device
+ * memory: a decode loop running under a memory pool that forbids new
+ * allocations after warm-up, code that must not trigger the implicit device
+ * synchronisation of cudaMalloc/cudaFree, or a host that simply has no
+ * allocator to offer.  The paper has no counterpart; this is a library
+ * convenience.
+ *
+ * Same arguments and results as vq3r_gemv, minus the workspace: the scratch
+ * is one array of VQ3R_GEMV_NOALLOC_BYTES (16 MiB) in the library's device
+ * image, which every GPU that loads the library holds until the process
+ * exits.  The call allocates nothing (no cudaMalloc, cudaFree or allocating
+ * library routine).
+ *   - A call whose vq3r_gemv_workspace_size() exceeds 16 MiB returns
+ *     VQ3R_ERR_WORKSPACE before launching anything (the 8-expert MoE decode
+ *     step of 2048 x 7168 / 7168 x 2048 matrices fits for B = 1 and 2).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before capturing a stream into a graph.
+ *   - All calls share the one array: calls that overlap on the GPU (different
+ *     streams, or different host threads on the same device) race and must be
+ *     serialised by the caller.  Every byte the kernels read from it is
+ *     written earlier in the same call, so nothing needs clearing between
+ *     calls.
+ */
+#define VQ3R_GEMV_NOALLOC_BYTES (16u << 20)
+vq3r_status vq3r_gemv_noalloc(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype x_dtype, vq3r_stream stream);
+
 /* Human-readable name of a status code (static string). */
 const char* vq3r_status_string(vq3r_status s);
 

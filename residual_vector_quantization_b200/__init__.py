@@ -22,7 +22,7 @@ GEMV_MAX_MATS = 32
 
 EXPORTED = ["vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_gemv_workspace_size", "vq3r_rel_frobenius_error",
             "vq3r_rel_frobenius_workspace_size", "vq3r_status_string", "vq3r_last_cuda_error",
-            "vq3r_device_error"]
+            "vq3r_device_error", "vq3r_gemv_noalloc"]
 
 
 class VQ3RError(RuntimeError):
@@ -54,6 +54,7 @@ def _lib():
         L.vq3r_decode.argtypes = [P, P, P, I64, I64, P, I32, P]
         L.vq3r_gemv.argtypes = [P, I32, I32, I32, P, SZ, P]
         L.vq3r_gemv_workspace_size.argtypes = [P, I32, I32]
+        L.vq3r_gemv_noalloc.argtypes = [P, I32, I32, I32, P]
         L.vq3r_gemv_workspace_size.restype = SZ
         L.vq3r_rel_frobenius_error.argtypes = [P, I32, P, P, P, I64, I64, P, P, SZ, P]
         L.vq3r_rel_frobenius_workspace_size.argtypes = [I64, I64]
@@ -62,7 +63,8 @@ def _lib():
         L.vq3r_status_string.restype = ctypes.c_char_p
         L.vq3r_last_cuda_error.restype = I32
         L.vq3r_device_error.argtypes = [P]
-        for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error"):
+        for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error",
+                  "vq3r_gemv_noalloc"):
             getattr(L, f).restype = I32
         _L = L
     return _L
@@ -149,6 +151,16 @@ def vq3r_gemv(mats, B, workspace=None, stream=None):
     xdt = _DT[mats[0]["x"].dtype]
     _check(_lib().vq3r_gemv(arr, len(mats), B, xdt, _dev(workspace, "workspace"), workspace.numel(),
                             _stream(stream)), "vq3r_gemv")
+    return [m["y"] for m in mats]
+
+
+def vq3r_gemv_noalloc(mats, B, stream=None):
+    """vq3r_gemv without a workspace argument: the library's own static device
+    scratch (16 MiB, shared by all calls; overlapping calls race) is used and
+    nothing is allocated, here or in the library."""
+    arr = _descs(mats)
+    xdt = _DT[mats[0]["x"].dtype]
+    _check(_lib().vq3r_gemv_noalloc(arr, len(mats), B, xdt, _stream(stream)), "vq3r_gemv_noalloc")
     return [m["y"] for m in mats]
 
 

@@ -312,6 +312,51 @@ vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const ui
   }
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch of vq3r_gemv_noalloc: file-scope device array, one per GPU that
+// loads the library.  Host code must not pass the symbol itself to a kernel
+// (in host code it names a host-side stand-in); the device address comes
+// from cudaGetSymbolAddress, looked up once per device with that device
+// current.
+static __device__ __align__(256) unsigned char g_gemv_noalloc_scratch[VQ3R_GEMV_NOALLOC_BYTES];
+
+std::once_flag g_noalloc_once[kMaxDevices];
+void* g_noalloc_ptr[kMaxDevices];
+cudaError_t g_noalloc_err[kMaxDevices];
+
+cudaError_t noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_noalloc_once[dev], [dev]() {
+    void* p = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_gemv_noalloc_scratch);
+    g_noalloc_ptr[dev] = p;
+  });
+  *ptr = g_noalloc_ptr[dev];
+  return g_noalloc_err[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+vq3r_status vq3r_gemv_noalloc(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype x_dtype,
+                              vq3r_stream stream) {
+  if (!mats) return VQ3R_ERR_NULL;
+  if (n_mats < 1 || n_mats > VQ3R_GEMV_MAX_MATS || B < 1 || B > VQ3R_GEMV_MAX_B) return VQ3R_ERR_BATCH;
+  const size_t need = vq3r_gemv_workspace_size(mats, n_mats, B);
+  if (need > (size_t)VQ3R_GEMV_NOALLOC_BYTES) return VQ3R_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return vq3r_gemv(mats, n_mats, B, x_dtype, scratch, VQ3R_GEMV_NOALLOC_BYTES, stream);
+}
+
 const char* vq3r_status_string(vq3r_status s) {
   switch (s) {
     case VQ3R_OK: return "VQ3R_OK";
