@@ -4,9 +4,10 @@
 One step = one pass of the whole path over a 64-expert MoE layer
 (w1, w3: 2048 x 7168; w2: 7168 x 2048 per expert, bf16, Student-t(4) rows
 with log-normal row factors; 2.82 G weights):
-  encode (row scale + greedy 3-stage assignment), decode to fp32,
-  relative Frobenius error of each matrix, and the MoE decode step
-  (8 active experts: gate/up GEMV in one call, down GEMV in one call, B = 1).
+  encode (row scale + greedy 3-stage assignment), repack of the indices into
+  the tiled GEMV layout, decode to fp32, relative Frobenius error of each
+  matrix, and the MoE decode step (8 active experts: gate/up GEMV in one
+  call, down GEMV in one call, B = 1).
 Each matrix kind of the layer is stacked into one call.  The decode step
 rotates over the 8 disjoint 8-expert groups of the layer so that its 132 MB
 of indices per step come from HBM, not L2 (the layer's 5.6 GB of weights
@@ -148,7 +149,7 @@ class Layer:
         stream = torch.cuda.current_stream().cuda_stream
         self.cb = torch.from_numpy(load_codebooks("layer")).to(dev)
         self.kinds = (wl.W1, wl.W3, wl.W2)
-        self.W, self.idx, self.sc, self.dec, self.err, self.err_ws = {}, {}, {}, {}, {}, {}
+        self.W, self.idx, self.sc, self.dec, self.err, self.err_ws, self.tiles = {}, {}, {}, {}, {}, {}, {}
         for k in self.kinds:
             rows, cols = wl.mat_shape(k)
             W = torch.empty((experts * rows, cols), dtype=torch.bfloat16, device=dev)
@@ -157,6 +158,7 @@ class Layer:
                                        wl.tag(expert0 + e, k), dist, stream=stream)
             self.W[k] = W
             self.idx[k] = torch.empty((3, experts * rows, cols // 8), dtype=torch.uint8, device=dev)
+            self.tiles[k] = torch.empty(vq.vq3r_tiles_size(experts * rows, cols), dtype=torch.uint8, device=dev)
             self.sc[k] = torch.empty(experts * rows, dtype=torch.int16, device=dev)
             self.dec[k] = torch.empty((experts * rows, cols), dtype=torch.float32, device=dev)
             self.err[k] = torch.empty(1, dtype=torch.float64, device=dev)
@@ -180,12 +182,13 @@ class Layer:
                 p1, p2 = [], []
                 for j, e in enumerate(ex):
                     for k in (wl.W1, wl.W3):
-                        rows, _ = wl.mat_shape(k)
-                        p1.append(dict(idx=self.idx[k], scales=self.sc[k], codebooks=self.cb, x=xu, row0=e * rows,
-                                       rows=rows, y=torch.empty((B, rows), dtype=torch.float32, device=dev)))
-                    rows, _ = wl.mat_shape(wl.W2)
-                    p2.append(dict(idx=self.idx[wl.W2], scales=self.sc[wl.W2], codebooks=self.cb, x=xd[j],
-                                   row0=e * rows, rows=rows,
+                        rows, cols = wl.mat_shape(k)
+                        p1.append(dict(idx=self.tiles[k], scales=self.sc[k], codebooks=self.cb, x=xu, row0=e * rows,
+                                       rows=rows, layout="tiles", cols=cols,
+                                       y=torch.empty((B, rows), dtype=torch.float32, device=dev)))
+                    rows, cols = wl.mat_shape(wl.W2)
+                    p2.append(dict(idx=self.tiles[wl.W2], scales=self.sc[wl.W2], codebooks=self.cb, x=xd[j],
+                                   row0=e * rows, rows=rows, layout="tiles", cols=cols,
                                    y=torch.empty((B, rows), dtype=torch.float32, device=dev)))
                 d1, d2 = vq._descs(p1), vq._descs(p2)
                 ws1 = vq.lib().vq3r_gemv_workspace_size(d1, len(p1), B)
@@ -200,6 +203,10 @@ class Layer:
     def encode(self):
         for k in self.kinds:
             self.vq.vq3r_encode(self.W[k], self.cb, self.idx[k], self.sc[k])
+
+    def pack(self):
+        for k in self.kinds:
+            self.vq.vq3r_pack_tiles(self.idx[k], out=self.tiles[k])
 
     def decode(self):
         for k in self.kinds:
@@ -219,7 +226,7 @@ class Layer:
             if st:
                 raise self.vq.VQ3RError(st, "vq3r_gemv")
 
-    LAUNCHES_PER_STEP = 3 * 2 + 3 * 1 + 3 * 2 + 2 * 3  # encode, decode, error, gemv (kernels)
+    LAUNCHES_PER_STEP = 3 * 2 + 3 + 3 * 1 + 3 * 2 + 2 * 2  # encode, pack, decode, error, gemv (kernels)
 
 
 # ----------------------------------------------------------------------------- CPU oracle sample
@@ -347,12 +354,14 @@ def main():
         if marks: marks[0].record()
         layer.encode()
         if marks: marks[1].record()
-        layer.decode()
+        layer.pack()
         if marks: marks[2].record()
-        layer.errors()
+        layer.decode()
         if marks: marks[3].record()
-        layer.gemv(1, i)
+        layer.errors()
         if marks: marks[4].record()
+        layer.gemv(1, i)
+        if marks: marks[5].record()
 
     for i in range(args.warmup):
         step(i)
@@ -361,7 +370,7 @@ def main():
 
     clocks = ClockSampler(local)
     clocks.start()
-    marks = [[ev() for _ in range(5)] for _ in range(args.steps)]
+    marks = [[ev() for _ in range(6)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     t0, t1 = ev(), ev()
@@ -379,9 +388,10 @@ def main():
         total_ms = float(tt.item())
     part = lambda a, b: [marks[i][a].elapsed_time(marks[i][b]) for i in range(args.steps)]  # noqa: E731
     enc_ms = statistics.mean(part(0, 1))
-    dec_ms = statistics.mean(part(1, 2))
-    err_ms = statistics.mean(part(2, 3))
-    gv1_ms = statistics.mean(part(3, 4))
+    pack_ms = statistics.mean(part(1, 2))
+    dec_ms = statistics.mean(part(2, 3))
+    err_ms = statistics.mean(part(3, 4))
+    gv1_ms = statistics.mean(part(4, 5))
 
     # decode-step GEMV sweep over batch sizes (not part of the step), rotating expert groups
     gemv = {}
@@ -451,8 +461,8 @@ def main():
             "metric": METRIC, "value": value, "unit": "Gweights/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "moe-layer-64x3-bf16: encode + decode(fp32) + rel-Frobenius of the layer, "
-                                   "then moe-decode-step-8-experts GEMV (B=1)",
+            "config": {"workload": "moe-layer-64x3-bf16: encode + tile repack + decode(fp32) + rel-Frobenius of "
+                                   "the layer, then moe-decode-step-8-experts GEMV (B=1)",
                        "experts_per_gpu": args.experts, "weights_per_gpu": layer.weights,
                        "matrices": "w1,w3 2048x7168; w2 7168x2048 per expert, stacked per kind",
                        "l2": "inputs larger than L2 (5.6 GB layer); GEMV rotates 8 disjoint 8-expert groups "
@@ -465,6 +475,7 @@ def main():
                          "frac_of_non_fma_ceiling": 2 * enc_tflops / fp32_peak_tflops * 23 / 24},
             "kernels": {
                 "encode": {"ms": enc_ms, "Gweights/s": layer.weights / enc_ms / 1e6, "TFLOP/s": enc_tflops},
+                "pack_tiles": {"ms": pack_ms, "GB/s": 2 * 0.375 * layer.weights / pack_ms / 1e6},
                 "decode_f32": {"ms": dec_ms, "GB/s": layer.weights * (4 + 0.375) / dec_ms / 1e6,
                                "frac_hbm": layer.weights * 4.375 / dec_ms / 1e6 / hbm_gbs},
                 "rel_frobenius": {"ms": err_ms, "GB/s": layer.weights * (2 + 0.375) / err_ms / 1e6,

@@ -116,23 +116,55 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
  *   B         tokens, 1..32
  *   x_dtype   dtype of every x, {F32, BF16, F16}
  *   workspace device scratch of at least vq3r_gemv_workspace_size() bytes
- * A matrix with rows == 0 contributes nothing (its pointers may be NULL).
+ * A matrix with rows == 0 contributes nothing (its pointers may be NULL);
+ * rows must be below 2^31 and cols / 8 at most 2^26 (VQ3R_ERR_SHAPE).
+ * TILES descriptors need plane_stride a multiple of 32768 and at least
+ * ceil(rows / 512) * 32768; mixing layouts in one call is VQ3R_ERR_SHAPE.
  */
+/* Index layouts accepted by vq3r_gemv (the encoder writes VQ3R_LAYOUT_PLANES). */
+typedef enum {
+  VQ3R_LAYOUT_PLANES = 0, /* [3][rows][cols/8], as written by vq3r_encode */
+  VQ3R_LAYOUT_TILES = 1   /* blocks of 512 rows x 64 columns, see vq3r_pack_tiles */
+} vq3r_layout;
+
 typedef struct {
-  const uint8_t* idx;       /* plane 0 of [3][rows][cols/8]; planes plane_stride bytes apart */
+  const uint8_t* idx;       /* PLANES: plane 0 of [3][rows][cols/8]; TILES: first block, see below */
   const uint16_t* scales;   /* [rows] binary16 */
   const float* codebooks;   /* [3][256][8] */
   int64_t rows, cols;
   const void* x;            /* [B][cols] */
   float* y;                 /* [B][rows] */
-  int64_t plane_stride;     /* bytes from one index plane to the next; 0 = rows * cols / 8.
+  int64_t plane_stride;     /* PLANES: bytes from one index plane to the next; 0 = rows * cols / 8.
                                A row range [r0, r0 + rows) of a larger encoded matrix
                                (e.g. one expert of a stacked layer) is described by
                                idx + r0 * cols / 8, scales + r0 and that matrix's
-                               plane size (VQ3R_ERR_SHAPE if below rows * cols / 8). */
+                               plane size (VQ3R_ERR_SHAPE if below rows * cols / 8).
+                               TILES: bytes from one (stage, slab) column of blocks to
+                               the next, i.e. n_tiles * 32768 of the packed matrix; 0 =
+                               ceil(rows / 512) * 32768.  A row range starting at a
+                               multiple of 512 is idx + (r0 / 512) * 32768, scales + r0. */
+  int32_t layout;           /* vq3r_layout; all descriptors of one call use the same one */
+  int32_t reserved;         /* must be 0 */
 } vq3r_gemv_desc;
 
 size_t vq3r_gemv_workspace_size(const vq3r_gemv_desc* mats, int n_mats, int B);
+
+/*
+ * vq3r_pack_tiles -- repack encoded index planes into the tiled layout that
+ * lets vq3r_gemv stream each work unit as one contiguous block (a one-time
+ * conversion of static weights; results of vq3r_gemv are the same for both
+ * layouts).  Layout: for stage s (0..2), slab (64 index columns, n_slabs =
+ * ceil(cols / 512)) and tile (512 rows, n_tiles = ceil(rows / 512)), a block
+ * of 512 x 64 bytes at ((s * n_slabs + slab) * n_tiles + tile) * 32768; row r
+ * of a block at r * 64, index column c at
+ *   16 * (c >> 4) + 8 * (((c >> 3) & 1) ^ ((r >> 2) & 1)) + (c & 7).
+ * Rows and columns past the matrix are zero.
+ *   idx          [3][rows][cols/8] planes, plane_stride bytes apart (0 = rows * cols / 8)
+ *   packed       out, vq3r_tiles_size(rows, cols) bytes, 16-byte aligned
+ */
+size_t vq3r_tiles_size(int64_t rows, int64_t cols);
+vq3r_status vq3r_pack_tiles(const uint8_t* idx, int64_t rows, int64_t cols, int64_t plane_stride, uint8_t* packed,
+                            vq3r_stream stream);
 vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype x_dtype, void* workspace,
                       size_t ws_bytes, vq3r_stream stream);
 

@@ -19,10 +19,12 @@ _DT = {torch.float32: VQ3R_F32, torch.bfloat16: VQ3R_BF16, torch.float16: VQ3R_F
 STAGES, CODEWORDS, DIM = 3, 256, 8
 GEMV_MAX_B = 32
 GEMV_MAX_MATS = 32
+LAYOUT_PLANES, LAYOUT_TILES = 0, 1
+TILE_ROWS, TILE_BYTES, SLAB_COLS = 512, 32768, 512
 
 EXPORTED = ["vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_gemv_workspace_size", "vq3r_rel_frobenius_error",
             "vq3r_rel_frobenius_workspace_size", "vq3r_status_string", "vq3r_last_cuda_error",
-            "vq3r_device_error", "vq3r_gemv_noalloc"]
+            "vq3r_device_error", "vq3r_gemv_noalloc", "vq3r_tiles_size", "vq3r_pack_tiles"]
 
 
 class VQ3RError(RuntimeError):
@@ -37,7 +39,7 @@ class VQ3RError(RuntimeError):
 class GemvDesc(ctypes.Structure):
     _fields_ = [("idx", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("codebooks", ctypes.c_void_p),
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
-                ("plane_stride", ctypes.c_int64)]
+                ("plane_stride", ctypes.c_int64), ("layout", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 _L = None
@@ -55,6 +57,9 @@ def _lib():
         L.vq3r_gemv.argtypes = [P, I32, I32, I32, P, SZ, P]
         L.vq3r_gemv_workspace_size.argtypes = [P, I32, I32]
         L.vq3r_gemv_noalloc.argtypes = [P, I32, I32, I32, P]
+        L.vq3r_tiles_size.argtypes = [I64, I64]
+        L.vq3r_tiles_size.restype = SZ
+        L.vq3r_pack_tiles.argtypes = [P, I64, I64, I64, P, P]
         L.vq3r_gemv_workspace_size.restype = SZ
         L.vq3r_rel_frobenius_error.argtypes = [P, I32, P, P, P, I64, I64, P, P, SZ, P]
         L.vq3r_rel_frobenius_workspace_size.argtypes = [I64, I64]
@@ -64,7 +69,7 @@ def _lib():
         L.vq3r_last_cuda_error.restype = I32
         L.vq3r_device_error.argtypes = [P]
         for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error",
-                  "vq3r_gemv_noalloc"):
+                  "vq3r_gemv_noalloc", "vq3r_pack_tiles"):
             getattr(L, f).restype = I32
         _L = L
     return _L
@@ -117,21 +122,52 @@ def vq3r_decode(idx, scales, codebooks, out_dtype=torch.float32, out=None, strea
 
 
 def _descs(mats):
+    """ctypes descriptor array for vq3r_gemv.  Each entry is a dict with
+    idx, scales, codebooks, x [B][cols], y [B][rows] and optionally:
+      layout "tiles": idx is a tiled tensor from vq3r_pack_tiles (1-D uint8)
+                      and "cols" gives the matrix width;
+      row0, rows:     a row range of a larger encoded (or packed) matrix; for
+                      tiles row0 must be a multiple of 512."""
     arr = (GemvDesc * len(mats))()
     for i, m in enumerate(mats):
         idx, scales, cb, x, y = m["idx"], m["scales"], m["codebooks"], m["x"], m["y"]
-        if "rows" in m:
+        if not (idx.is_cuda and idx.is_contiguous() and scales.is_cuda and scales.is_contiguous()):
+            raise ValueError("idx and scales must be contiguous CUDA tensors")
+        if m.get("layout", "planes") == "tiles":
+            cols = m["cols"]
+            total_rows = scales.shape[0]
+            r0, rows = m.get("row0", 0), m.get("rows", total_rows)
+            if r0 % TILE_ROWS:
+                raise ValueError("row0 of a tiled matrix must be a multiple of 512")
+            n_tiles = (total_rows + TILE_ROWS - 1) // TILE_ROWS
+            arr[i] = GemvDesc(idx.data_ptr() + (r0 // TILE_ROWS) * TILE_BYTES, scales.data_ptr() + 2 * r0,
+                              _dev(cb, "codebooks"), rows, cols, _dev(x, "x"), _dev(y, "y"), n_tiles * TILE_BYTES,
+                              LAYOUT_TILES, 0)
+        elif "rows" in m:
             # a row range of a larger encoded matrix: idx is the full [3][R][V] tensor
             r0, rows = m.get("row0", 0), m["rows"]
             V = idx.shape[2]
-            if not (idx.is_cuda and idx.is_contiguous()):
-                raise ValueError("idx must be a contiguous CUDA tensor")
             arr[i] = GemvDesc(idx.data_ptr() + r0 * V, scales.data_ptr() + 2 * r0, _dev(cb, "codebooks"), rows,
-                              V * DIM, _dev(x, "x"), _dev(y, "y"), idx.shape[1] * V)
+                              V * DIM, _dev(x, "x"), _dev(y, "y"), idx.shape[1] * V, LAYOUT_PLANES, 0)
         else:
             arr[i] = GemvDesc(_dev(idx, "idx"), _dev(scales, "scales"), _dev(cb, "codebooks"), idx.shape[1],
-                              idx.shape[2] * DIM, _dev(x, "x"), _dev(y, "y"), 0)
+                              idx.shape[2] * DIM, _dev(x, "x"), _dev(y, "y"), 0, LAYOUT_PLANES, 0)
     return arr
+
+
+def vq3r_tiles_size(rows, cols):
+    return _lib().vq3r_tiles_size(rows, cols)
+
+
+def vq3r_pack_tiles(idx, out=None, stream=None):
+    """Repack index planes [3][rows][cols/8] into the tiled layout (1-D uint8 tensor)."""
+    _, rows, V = idx.shape
+    n = vq3r_tiles_size(rows, V * DIM)
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=idx.device)
+    _check(_lib().vq3r_pack_tiles(_dev(idx, "idx"), rows, V * DIM, 0, _dev(out, "out"), _stream(stream)),
+           "vq3r_pack_tiles")
+    return out
 
 
 def vq3r_gemv_workspace_size(mats, B):

@@ -48,11 +48,16 @@ cudaError_t device_setup(int* sms) {
   std::call_once(g_dev_once[dev], [dev]() {
     cudaError_t r = cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev);
     const int enc = (int)sizeof(EncSmem);
-    const int gv = (int)kSlabBytes + 16;
+    const int gv = (int)kGvSmemBytes;
     if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     g_dev_err[dev] = r;
   });
   *sms = g_dev_sms[dev];
@@ -79,15 +84,20 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
   memset(&P, 0, sizeof(P));
   P.B = B;
   P.vec8 = 1;
+  P.layout = mats[0].layout;
+  if (P.layout != VQ3R_LAYOUT_PLANES && P.layout != VQ3R_LAYOUT_TILES) return VQ3R_ERR_SHAPE;
+  const bool tiles = P.layout == VQ3R_LAYOUT_TILES;
+  P.tile_rows = tiles ? kTileRows : kGvTileRows;
   int n_groups = 0;
   int group_of[VQ3R_GEMV_MAX_MATS];
   for (int i = 0; i < n_mats; i++) {
     const vq3r_gemv_desc& d = mats[i];
     vq3r_status st = check_shape(d.rows, d.cols, 0);
     if (st != VQ3R_OK) return st;
-    if (d.cols / kDim > (int64_t)kSlabV * (1 << 20)) return VQ3R_ERR_SHAPE;
-    const int64_t plane = d.rows * (d.cols / kDim);
-    if (d.plane_stride != 0 && d.plane_stride < plane) return VQ3R_ERR_SHAPE;
+    if (d.cols / kDim > (int64_t)kSlabV * (1 << 20) || d.rows >= ((int64_t)1 << 31)) return VQ3R_ERR_SHAPE;
+    if (d.layout != P.layout || d.reserved != 0) return VQ3R_ERR_SHAPE;
+    const int64_t plane = tiles ? (d.rows + kTileRows - 1) / kTileRows * kTileBytes : d.rows * (d.cols / kDim);
+    if (d.plane_stride != 0 && (d.plane_stride < plane || (tiles && d.plane_stride % kTileBytes))) return VQ3R_ERR_SHAPE;
     group_of[i] = -1;
     if (d.rows == 0) continue;  // an empty matrix may carry NULL pointers
     if (!d.idx || !d.scales || !d.codebooks || !d.x || !d.y) return VQ3R_ERR_NULL;
@@ -103,7 +113,6 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
       P.g[g].x = d.x;
       P.g[g].cols = d.cols;
       P.g[g].n_slabs = (int32_t)((d.cols / kDim + kSlabV - 1) / kSlabV);
-      P.g[g].n_sgroups = (P.g[g].n_slabs + kSlabGroup - 1) / kSlabGroup;
       n_groups++;
     }
     group_of[i] = g;
@@ -121,9 +130,11 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
       M.scales = d.scales;
       M.y = d.y;
       M.rows = d.rows;
-      M.plane_stride = d.plane_stride ? d.plane_stride : d.rows * (d.cols / kDim);
+      M.plane_stride = d.plane_stride ? d.plane_stride
+                                      : (tiles ? (d.rows + kTileRows - 1) / kTileRows * kTileBytes
+                                               : d.rows * (d.cols / kDim));
       M.group = g;
-      M.n_tiles = (int32_t)((d.rows + kGvTileRows - 1) / kGvTileRows);
+      M.n_tiles = (int32_t)((d.rows + P.tile_rows - 1) / P.tile_rows);
       M.tile_prefix = P.g[g].tiles;
       P.g[g].tiles += M.n_tiles;
     }
@@ -132,23 +143,17 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
   P.n_mats = nm;
   size_t off = 0;
   int64_t units = 0;
-  int32_t images = 0;
   for (int g = 0; g < n_groups; g++) {
     GvGroup& G = P.g[g];
-    G.lut = reinterpret_cast<float*>(ws_base + off);
-    off = align_up(off + (size_t)B * G.n_slabs * kSlabBytes);
     G.unit_begin = units;
-    units += (int64_t)G.n_sgroups * B * G.tiles;
-    G.image_begin = images;
-    images += B * G.n_slabs;
+    units += (int64_t)G.n_slabs * kStages * B * G.tiles;
   }
   for (int i = 0; i < nm; i++) {
     GvMat& M = P.m[i];
     M.partial = reinterpret_cast<float*>(ws_base + off);
-    off = align_up(off + (size_t)B * P.g[M.group].n_slabs * (size_t)M.rows * sizeof(float));
+    off = align_up(off + (size_t)B * kStages * P.g[M.group].n_slabs * (size_t)M.rows * sizeof(float));
   }
   P.total_units = units;
-  P.total_images = images;
   plan->ws_bytes = off;
   return VQ3R_OK;
 }
@@ -239,39 +244,41 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   if (plan.P.total_units == 0) return VQ3R_OK;
   if (!workspace || ws_bytes < plan.ws_bytes) return VQ3R_ERR_WORKSPACE;
   if (!aligned16(workspace)) return VQ3R_ERR_ALIGN;
-  plan.P.x_dtype = x_dtype;
   int sms = 0;
   cudaError_t e = device_setup(&sms);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const GvParams& P = plan.P;
-  const int build_blocks = P.total_images * kLutBuildBlocksPerImage;
-  switch (x_dtype) {
-    case VQ3R_F32: lut_build_kernel<VQ3R_F32><<<build_blocks, kGvThreads, 0, s>>>(P); break;
-    case VQ3R_BF16: lut_build_kernel<VQ3R_BF16><<<build_blocks, kGvThreads, 0, s>>>(P); break;
-    default: lut_build_kernel<VQ3R_F16><<<build_blocks, kGvThreads, 0, s>>>(P); break;
+  if (P.layout == VQ3R_LAYOUT_TILES) {  // one CTA per SM
+    const int grid = (int)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms);
+    switch (x_dtype) {
+      case VQ3R_F32: gemv_tiles_kernel<VQ3R_F32><<<grid, kGvThreads, kGvSmemBytes, s>>>(P); break;
+      case VQ3R_BF16: gemv_tiles_kernel<VQ3R_BF16><<<grid, kGvThreads, kGvSmemBytes, s>>>(P); break;
+      default: gemv_tiles_kernel<VQ3R_F16><<<grid, kGvThreads, kGvSmemBytes, s>>>(P); break;
+    }
+  } else {  // two CTAs per SM
+    const int grid = (int)(P.total_units < 2 * (int64_t)sms ? P.total_units : 2 * (int64_t)sms);
+    switch (x_dtype) {
+      case VQ3R_F32: gemv_lut_kernel<VQ3R_F32><<<grid, kGvThreads, kGvSmemBytes, s>>>(P); break;
+      case VQ3R_BF16: gemv_lut_kernel<VQ3R_BF16><<<grid, kGvThreads, kGvSmemBytes, s>>>(P); break;
+      default: gemv_lut_kernel<VQ3R_F16><<<grid, kGvThreads, kGvSmemBytes, s>>>(P); break;
+    }
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
-  // The main and reduction kernels are launched with programmatic stream
-  // serialization: each may start while its predecessor finishes and waits
-  // (griddepcontrol.wait) before reading the predecessor's results.
+  // The reduction kernel is launched with programmatic stream serialization:
+  // its CTAs may start while the main kernel runs and wait (griddepcontrol.wait)
+  // for its partial sums.
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  const int64_t groups = (sms / kSlabGroup) < P.total_units ? (sms / kSlabGroup) : P.total_units;
-  cfg.gridDim = dim3((unsigned)(groups * kSlabGroup));
-  cfg.blockDim = dim3(kGvThreads);
-  cfg.dynamicSmemBytes = kSlabBytes + 16;
   cfg.stream = s;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemv_lut_kernel, P);
-  if (e != cudaSuccess) return cuda_fail(e);
   int64_t maxrows = 0;
   for (int i = 0; i < P.n_mats; i++) maxrows = P.m[i].rows * B > maxrows ? P.m[i].rows * B : maxrows;
-  int64_t gx = (maxrows + 255) / 256;
+  int64_t gx = (maxrows * 4 + 255) / 256;  // four lanes per output
   if (gx > (int64_t)sms * 4) gx = (int64_t)sms * 4;
   if (gx < 1) gx = 1;
   cfg.gridDim = dim3((unsigned)gx, (unsigned)P.n_mats);
@@ -279,6 +286,36 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   cfg.dynamicSmemBytes = 0;
   e = cudaLaunchKernelEx(&cfg, gemv_reduce_kernel, P);
   if (e != cudaSuccess) return cuda_fail(e);
+  return check_launch();
+}
+
+size_t vq3r_tiles_size(int64_t rows, int64_t cols) {
+  if (check_shape(rows, cols, 0) != VQ3R_OK) return 0;
+  const int64_t n_slabs = (cols / kDim + kSlabV - 1) / kSlabV;
+  const int64_t n_tiles = (rows + kTileRows - 1) / kTileRows;
+  return (size_t)kStages * n_slabs * n_tiles * kTileBytes;
+}
+
+vq3r_status vq3r_pack_tiles(const uint8_t* idx, int64_t rows, int64_t cols, int64_t plane_stride, uint8_t* packed,
+                            vq3r_stream stream) {
+  vq3r_status st = check_shape(rows, cols, 0);
+  if (st != VQ3R_OK) return st;
+  if (cols / kDim > (int64_t)kSlabV * (1 << 20)) return VQ3R_ERR_SHAPE;
+  const int64_t plane = rows * (cols / kDim);
+  if (plane_stride != 0 && plane_stride < plane) return VQ3R_ERR_SHAPE;
+  if (rows == 0) return VQ3R_OK;
+  if (!idx || !packed) return VQ3R_ERR_NULL;
+  if (!aligned16(packed)) return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int32_t n_slabs = (int32_t)((cols / kDim + kSlabV - 1) / kSlabV);
+  const int64_t n_tiles = (rows + kTileRows - 1) / kTileRows;
+  const int64_t chunks = (int64_t)kStages * n_slabs * n_tiles * (kTileBytes / 16);
+  int64_t blocks = (chunks + 255) / 256;
+  if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+  pack_tiles_kernel<<<(int)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      idx, rows, cols / kDim, plane_stride ? plane_stride : plane, n_slabs, n_tiles, packed);
   return check_launch();
 }
 

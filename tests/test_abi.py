@@ -62,7 +62,7 @@ def test_null_and_shape_errors_return_before_any_launch(lib):
 def _descs(specs):
     arr = (vq.GemvDesc * len(specs))()
     for i, (rows, cols, cb, x) in enumerate(specs):
-        arr[i] = vq.GemvDesc(0x200000 + 0x1000 * i, 0x300000 + 0x1000 * i, cb, rows, cols, x, 0x400000 + 0x1000 * i, 0)
+        arr[i] = vq.GemvDesc(0x200000 + 0x1000 * i, 0x300000 + 0x1000 * i, cb, rows, cols, x, 0x400000 + 0x1000 * i, 0, 0, 0)
     return arr
 
 
@@ -77,17 +77,15 @@ def test_gemv_batch_and_workspace_checks(lib):
     assert lib.vq3r_gemv_workspace_size(arr, 1, 0) == 0
 
 
-def test_gemv_workspace_groups_shared_tables(lib):
-    slab = 3 * 256 * 64 * 4
-    # 16 gate/up matrices sharing x and codebooks: one set of tables (14 slabs)
+def test_gemv_workspace_holds_the_partial_sums(lib):
+    # per matrix: B tokens x 3 stages x ceil(cols / 512) slabs x rows fp32 partial sums (256-byte aligned)
     specs = [(2048, 7168, 0x10000, 0x20000)] * 16
     for B in (1, 4, 32):
         ws = lib.vq3r_gemv_workspace_size(_descs(specs), 16, B)
-        assert ws == B * 14 * slab + 16 * B * 14 * 2048 * 4
-    # 8 down matrices with their own inputs: 8 groups of 4 slabs
+        assert ws == 16 * B * 3 * 14 * 2048 * 4
     specs = [(7168, 2048, 0x10000, 0x20000 + 0x10000 * i) for i in range(8)]
     ws = lib.vq3r_gemv_workspace_size(_descs(specs), 8, 1)
-    assert ws == 8 * 4 * slab + 8 * 4 * 7168 * 4
+    assert ws == 8 * 3 * 4 * 7168 * 4
 
 
 def test_gemv_plane_stride_checks(lib):
@@ -96,3 +94,20 @@ def test_gemv_plane_stride_checks(lib):
     assert lib.vq3r_gemv(arr, 1, 1, 1, 0x500000, 1 << 30, None) == 2
     arr[0].plane_stride = 64 * 2048 * 896 + 8
     assert lib.vq3r_gemv_workspace_size(arr, 1, 1) > 0  # any stride >= one plane is accepted
+
+
+def test_tiles_size_and_layout_checks(lib):
+    assert lib.vq3r_tiles_size(2048, 7168) == 3 * 14 * 4 * 32768
+    assert lib.vq3r_tiles_size(7168, 2048) == 3 * 4 * 14 * 32768
+    assert lib.vq3r_tiles_size(5, 40) == 3 * 1 * 1 * 32768
+    arr = _descs([(2048, 7168, 0x10000, 0x20000), (2048, 7168, 0x10000, 0x20000)])
+    arr[1].layout = 1  # mixed layouts in one call
+    assert lib.vq3r_gemv_workspace_size(arr, 2, 1) == 0
+    assert lib.vq3r_gemv(arr, 2, 1, 1, 0x500000, 1 << 30, None) == 2
+    arr[0].layout = 1
+    arr[0].plane_stride = arr[1].plane_stride = 4 * 32768 + 16  # not a whole number of blocks
+    assert lib.vq3r_gemv(arr, 2, 1, 1, 0x500000, 1 << 30, None) == 2
+    arr[0].plane_stride = arr[1].plane_stride = 0
+    assert lib.vq3r_gemv_workspace_size(arr, 2, 1) == 2 * 3 * 14 * 2048 * 4
+    assert lib.vq3r_pack_tiles(None, 4, 16, 0, 0x100000, None) == 1
+    assert lib.vq3r_pack_tiles(0x100000, 4, 12, 0, 0x100000, None) == 2

@@ -55,6 +55,35 @@ def check_encode_decode(Wnp, dtype, cb):
     return W_t, idx_t, sc_t, cb_t, idx_o, sc_o
 
 
+def as_layout(mats, layout):
+    """GEMV descriptors in the requested index layout (tiles: packed with vq3r_pack_tiles)."""
+    if layout == "planes":
+        return mats
+    out = []
+    for m in mats:
+        idx = m["idx"]
+        out.append(dict(m, idx=vq.vq3r_pack_tiles(idx), layout="tiles", cols=idx.shape[2] * 8))
+    return out
+
+
+def tiles_reference(idx):
+    """The tiled layout of index planes [3][rows][V], written out from its definition."""
+    _, rows, V = idx.shape
+    n_slabs, n_tiles = -(-V // 64), -(-rows // 512)
+    out = np.zeros((3, n_slabs, n_tiles, 512, 64), dtype=np.uint8)
+    for s in range(3):
+        for slab in range(n_slabs):
+            for t in range(n_tiles):
+                blk = np.zeros((512, 64), np.uint8)
+                src = idx[s, t * 512:(t + 1) * 512, slab * 64:(slab + 1) * 64]
+                blk[:src.shape[0], :src.shape[1]] = src
+                swap = (np.arange(512) >> 2) & 1
+                for c in range(64):
+                    dst = 16 * (c >> 4) + 8 * (((c >> 3) & 1) ^ swap) + (c & 7)
+                    out[s, slab, t, np.arange(512), dst] = blk[:, c]
+    return out.reshape(-1)
+
+
 # ------------------------------------------------------------------ tiny workload, end to end
 
 @pytest.fixture(scope="module")
@@ -79,13 +108,14 @@ def test_tiny_rel_frobenius(tiny):
     assert abs(e_gpu - e_ref) <= RELFRO_TOL * e_ref
 
 
+@pytest.mark.parametrize("layout", ["planes", "tiles"])
 @pytest.mark.parametrize("B", [1, 4, 8, 32])
-def test_tiny_gemv(tiny, B):
+def test_tiny_gemv(tiny, B, layout):
     W, cb = tiny
     W_t, idx_t, sc_t, cb_t, idx_o, sc_o = check_encode_decode(W, "f32", cb)
     x = synth.fill_rows(W.shape[1], 0, B, wl.TINY_SEED, wl.tag(0, wl.X_GATEUP), synth.normal(), dtype="f32")
     y_t = torch.empty((B, W.shape[0]), dtype=torch.float32, device=DEV)
-    vq.vq3r_gemv([dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=to_dev(x, "f32"), y=y_t)], B)
+    vq.vq3r_gemv(as_layout([dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=to_dev(x, "f32"), y=y_t)], layout), B)
     y_ref = oracle.gemv(oracle.decode(idx_o, sc_o, cb), x, "f32")
     assert gemv_rel_err(y_t.cpu().numpy(), y_ref) <= GEMV_TOL
 
@@ -108,10 +138,12 @@ def test_shapes_and_dtypes(rows, cols, dtype):
     for B in (1, 3):
         x = rng.standard_normal((B, cols)).astype(np.float32)
         xb = f32_to_bf16_bits(x)
-        y_t = torch.empty((B, rows), dtype=torch.float32, device=DEV)
-        vq.vq3r_gemv([dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=to_dev(xb, "bf16"), y=y_t)], B)
         y_ref = oracle.gemv(oracle.decode(idx_o, sc_o, cb), xb, "bf16")
-        assert gemv_rel_err(y_t.cpu().numpy(), y_ref) <= GEMV_TOL
+        for layout in ("planes", "tiles"):
+            y_t = torch.empty((B, rows), dtype=torch.float32, device=DEV)
+            vq.vq3r_gemv(as_layout([dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=to_dev(xb, "bf16"), y=y_t)],
+                                   layout), B)
+            assert gemv_rel_err(y_t.cpu().numpy(), y_ref) <= GEMV_TOL, layout
     e_gpu = float(vq.vq3r_rel_frobenius_error(W_t, idx_t, sc_t, cb_t).cpu()[0])
     e_ref = oracle.rel_frobenius(W, dtype, oracle.decode(idx_o, sc_o, cb))
     assert abs(e_gpu - e_ref) <= RELFRO_TOL * e_ref
@@ -165,7 +197,17 @@ def test_empty_matrix_is_a_noop():
     assert idx.shape == (3, 0, 8) and sc.shape == (0,)
 
 
-def test_grouped_gemv_mixed_matrices():
+@pytest.mark.parametrize("rows,cols", [(3, 40), (130, 800), (1025, 2048), (600, 7168)])
+def test_pack_tiles_layout(rows, cols):
+    rng = np.random.default_rng(rows + cols)
+    idx = rng.integers(0, 256, size=(3, rows, cols // 8), dtype=np.uint8)
+    packed = vq.vq3r_pack_tiles(torch.from_numpy(idx).to(DEV)).cpu().numpy()
+    assert packed.size == vq.vq3r_tiles_size(rows, cols)
+    np.testing.assert_array_equal(packed, tiles_reference(idx))
+
+
+@pytest.mark.parametrize("layout", ["planes", "tiles"])
+def test_grouped_gemv_mixed_matrices(layout):
     """One call over matrices of different shapes, codebooks and inputs."""
     rng = np.random.default_rng(24)
     specs = [(300, 1024, 0, 0), (129, 1024, 0, 0), (64, 512, 1, 1), (200, 1024, 2, 0), (33, 1024, 0, 2)]
@@ -185,7 +227,7 @@ def test_grouped_gemv_mixed_matrices():
     xdev = {k: to_dev(v, "bf16") for k, v in xs.items()}
     for m in mats:
         m["x"] = xdev[m.pop("key")]
-    vq.vq3r_gemv(mats, B)
+    vq.vq3r_gemv(as_layout(mats, layout), B)
     for m, ref in zip(mats, refs):
         assert gemv_rel_err(m["y"].cpu().numpy(), ref) <= GEMV_TOL
 
@@ -280,8 +322,9 @@ def test_expert_full_matrix_rel_frobenius_consistent():
     assert 0.1 < e < 0.3
 
 
+@pytest.mark.parametrize("layout", ["planes", "tiles"])
 @pytest.mark.parametrize("B", [1, 4, 8, 32])
-def test_moe_decode_step_gemv_sampled_rows(B):
+def test_moe_decode_step_gemv_sampled_rows(B, layout):
     """The MoE decode step (8 experts of the layer; gate/up in one call, down in
     one call) at full size against the binary64 oracle on sampled rows."""
     cfg = wl.LAYER
@@ -306,8 +349,8 @@ def test_moe_decode_step_gemv_sampled_rows(B):
                 phase1.append(dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=x_up_t, y=y_t))
             sample = np.sort(rng.choice(rows, 24, replace=False))
             checks.append((y_t, e, kind, sample, x_dn[e] if kind == wl.W2 else x_up))
-    vq.vq3r_gemv(phase1, B)
-    vq.vq3r_gemv(phase2, B)
+    vq.vq3r_gemv(as_layout(phase1, layout), B)
+    vq.vq3r_gemv(as_layout(phase2, layout), B)
     torch.cuda.synchronize()
     worst = 0.0
     for y_t, e, kind, sample, x in checks:

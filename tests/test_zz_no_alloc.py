@@ -59,7 +59,14 @@ def test_noalloc_matches_gemv_on_two_calls_in_a_row(B):
 
 def test_noalloc_rejects_calls_that_need_more_scratch():
     B = 32
-    mats = [dict(m, y=torch.empty((B, m["idx"].shape[1]), device=DEV)) for m in _matrices(B, 3)]
+    cb = torch.zeros((3, 256, 8), device=DEV)
+    x = torch.zeros((B, 4096), dtype=torch.bfloat16, device=DEV)
+    mats = []
+    for _ in range(2):
+        rows, cols = 8192, 4096
+        mats.append(dict(idx=torch.zeros((3, rows, cols // 8), dtype=torch.uint8, device=DEV),
+                         scales=torch.zeros(rows, dtype=torch.int16, device=DEV), codebooks=cb, x=x,
+                         y=torch.empty((B, rows), device=DEV)))
     descs = vq._descs(mats)
     L = vq.lib()
     assert L.vq3r_gemv_workspace_size(descs, len(mats), B) > (16 << 20)
