@@ -35,6 +35,10 @@ from synth import workloads as wl  # noqa: E402
 
 METRIC = "VQ3R encode Gweights/s (vs fp32 peak); decode-GEMV GB/s vs HBM roofline, 1 B200"
 FLOPS_PER_WEIGHT = 2304  # 3 stages x 256 codewords x 8 dims x (sub, mul, add) / 8 weights
+# DRAM bytes (read + write) per weight of the encode kernel, from an ncu capture
+# of this kernel (dram__bytes_read.sum + dram__bytes_write.sum over 117.4 M
+# weights); None once the kernel changes and until it is captured again.
+ENCODE_DRAM_BYTES_PER_WEIGHT = (235124480 + 7574784) / 117440512
 SM_COUNT_NOMINAL = 148
 FP32_LANES_PER_SM = 128
 
@@ -468,9 +472,12 @@ def main():
                        "l2": "inputs larger than L2 (5.6 GB layer); GEMV rotates 8 disjoint 8-expert groups "
                              "(1.06 GB of indices)"},
             "roofline": {"bound": "alu", "achieved": enc_tflops, "peak": fp32_peak_tflops, "unit": "TFLOP/s",
-                         "frac": enc_tflops / fp32_peak_tflops, "traffic": None,
-                         "kernel": "vq3r_encode (row scale + greedy assignment), %d algorithmic flops/weight; "
-                                   "peak = %d SMs x 128 FP32 lanes x 2 (FMA-counted) x %.0f MHz" %
+                         "frac": enc_tflops / fp32_peak_tflops,
+                         "traffic": (None if ENCODE_DRAM_BYTES_PER_WEIGHT is None
+                                     else ENCODE_DRAM_BYTES_PER_WEIGHT * layer.weights / 3),
+                         "kernel": "vq3r_encode (row scale + greedy assignment; per launch = one stacked matrix "
+                                   "kind, 3 per step), %d algorithmic flops/weight; peak = %d SMs x 128 FP32 lanes x "
+                                   "2 (FMA-counted) x %.0f MHz; traffic = DRAM bytes per launch" %
                                    (FLOPS_PER_WEIGHT, sms, sm_max_mhz),
                          "frac_of_non_fma_ceiling": 2 * enc_tflops / fp32_peak_tflops * 23 / 24},
             "kernels": {
