@@ -46,6 +46,7 @@ constexpr size_t kGvSmemBytes = kTabBytes + (size_t)(kSlabV * kDim + kCodewords 
 // order the lookup schedule wants, so a 16-byte load needs no shuffling.
 constexpr int kTileRows = 512;
 constexpr int kTileBytes = kTileRows * kSlabV;  // 32 KiB
+constexpr int kTileSlots = 2;                   // units of index registers per lane in the tiled kernel
 __host__ __device__ __forceinline__ int tile_byte(int r, int c) {
   return r * kSlabV + 16 * (c >> 4) + 8 * (((c >> 3) & 1) ^ ((r >> 2) & 1)) + (c & 7);
 }
@@ -312,86 +313,341 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_lut_kernel(const __grid_co
   }
 }
 
-// Decode-GEMV over the tiled index layout: the 32 KiB block of a unit is
-// contiguous, so each lane reads the 16 bytes of its 4 rows with four 16-byte
-// loads and keeps the next unit's loads in flight (two-deep register ring).
+// ---------------------------------------------------------------------------
+// Decode-GEMV over the tiled index layout.
+//
+// A unit is one 32 KiB block (stage s, slab, 512-row tile); lane (warp, g, a)
+// owns rows warp*32 + 8t + g, t = 0..3, and the lane's 16 index bytes of each
+// row arrive as one 16-byte load.  Each slot of the register ring holds one
+// unit; a slot is refilled quarter by quarter (one row t at a time) as soon as
+// that quarter has been looked up, so about NSLOT - 1/2 units per SM stay in
+// flight while the lookups run.
+//
+// Table key of a unit: slab | s << 20 | b << 22 | group << 27 (slab < 2^20,
+// s < 3, b < 32, group < 32), so one 32-bit compare detects a table switch.
+__host__ __device__ __forceinline__ uint32_t table_key(int g, int slab, int s, int b) {
+  return (uint32_t)slab | ((uint32_t)s << 20) | ((uint32_t)b << 22) | ((uint32_t)g << 27);
+}
+
+// Position of the next unit to load: the index block, the partial sums of
+// its tile (row 0), the matrix rows from the tile's first row on, the table
+// key, and the coordinates needed for the carry to the next matrix or table.
+struct TileCursor {
+  const uint8_t* p;
+  float* q;
+  int32_t rows_left;
+  uint32_t tkey;
+  int32_t m, tile, ntiles;
+};
+
+__device__ __forceinline__ void tcur_fill(const GvParams& P, TileCursor& c) {
+  const uint32_t k = c.tkey;
+  const int slab = (int)(k & 0xFFFFFu), s = (int)((k >> 20) & 3u), b = (int)((k >> 22) & 31u), g = (int)(k >> 27);
+  const GvMat& M = P.m[c.m];
+  const int64_t n_slabs = P.g[g].n_slabs;
+  c.ntiles = M.n_tiles;
+  c.p = M.idx + ((int64_t)s * n_slabs + slab) * M.plane_stride + (int64_t)c.tile * kTileBytes;
+  c.q = M.partial + (((int64_t)b * kStages + s) * n_slabs + slab) * M.rows + (int64_t)c.tile * kTileRows;
+  c.rows_left = (int32_t)(M.rows - (int64_t)c.tile * kTileRows);
+}
+
+__device__ __forceinline__ TileCursor tcur_at(const GvParams& P, int64_t u) {
+  const GvCursor g = unit_cursor(P, u);
+  TileCursor c;
+  c.tkey = table_key(g.g, g.slab, g.s, g.b);
+  c.m = g.m;
+  c.tile = g.tile;
+  tcur_fill(P, c);
+  return c;
+}
+
+// Next unit in (group, slab, stage, token, matrix, tile) order.  The common
+// case, the next tile of the same matrix, is three increments.
+__device__ __forceinline__ void tcur_next(const GvParams& P, TileCursor& c) {
+  if (++c.tile < c.ntiles) {
+    c.p += kTileBytes;
+    c.q += kTileRows;
+    c.rows_left -= kTileRows;
+    return;
+  }
+  c.tile = 0;
+  int g = (int)(c.tkey >> 27);
+  if (++c.m >= P.g[g].mat_end) {
+    int slab = (int)(c.tkey & 0xFFFFFu), s = (int)((c.tkey >> 20) & 3u), b = (int)((c.tkey >> 22) & 31u);
+    if (++b >= P.B) {
+      b = 0;
+      if (++s >= kStages) {
+        s = 0;
+        if (++slab >= P.g[g].n_slabs) {
+          slab = 0;
+          if (++g >= P.n_groups) return;  // past the last unit: never loaded
+        }
+      }
+    }
+    c.m = P.g[g].mat_begin;
+    c.tkey = table_key(g, slab, s, b);
+  }
+  tcur_fill(P, c);
+}
+
+// Table pipeline of the tiled kernel.  A CTA walks its units table by table
+// (table = group, slab, stage, token).  Table t lives in tab[t & 1]; its
+// inputs (the x slab as stored and the stage's 8 KiB codebook) are brought
+// into xraw[t & 1] / cb[t & 1] by bulk asynchronous copies completing on
+// mbar[t & 1], issued one table ahead, so they never wait behind the index
+// stream.  While the units of table t run, table t + 1 is computed in
+// kBuildChunks pieces, one piece per unit; the switch only finishes what is
+// left.
+constexpr int kBuildChunks = 8;
+constexpr int kChunkCw = kCodewords / kBuildChunks;  // 32 codewords per piece
+constexpr uint32_t kNoTable = 0xFFFFFFFFu;           // no key has all bits set (group < 32, s < 3)
+
+struct TilesSmem {
+  float tab[2][kTabWords];                       // 2 x 64 KiB
+  float cb[2][kCodewords * kDim];                // 2 x 8 KiB
+  unsigned char xraw[2][kSlabV * kDim * 4];      // 2 x 2 KiB (f32; 16-bit types use half)
+  uint64_t mbar[2];
+};
+constexpr size_t kTilesSmemBytes = sizeof(TilesSmem);
+
 template <int XDT>
+__host__ __device__ constexpr int x_elt_bytes() {
+  return XDT == VQ3R_F32 ? 4 : 2;
+}
+
+__device__ __forceinline__ uint32_t next_table_key(const GvParams& P, uint32_t k) {
+  int slab = (int)(k & 0xFFFFFu), s = (int)((k >> 20) & 3u), b = (int)((k >> 22) & 31u), g = (int)(k >> 27);
+  if (++b < P.B) return table_key(g, slab, s, b);
+  b = 0;
+  if (++s < kStages) return table_key(g, slab, s, b);
+  s = 0;
+  if (++slab < P.g[g].n_slabs) return table_key(g, slab, s, b);
+  return table_key(g + 1, 0, 0, 0);
+}
+
+// Vector columns of the slab that exist in the matrix (the last slab may be short).
+__device__ __forceinline__ int slab_columns(const GvParams& P, uint32_t k) {
+  const GvGroup& G = P.g[k >> 27];
+  const int64_t left = G.cols / kDim - (int64_t)(k & 0xFFFFFu) * kSlabV;
+  return left < kSlabV ? (int)left : kSlabV;
+}
+
+// Issued by one thread: copy table k's inputs into staging buffer i.
+template <int XDT>
+__device__ __forceinline__ void stage_table(const GvParams& P, uint32_t k, TilesSmem& S, int i) {
+  const GvGroup& G = P.g[k >> 27];
+  const int slab = (int)(k & 0xFFFFFu), s = (int)((k >> 20) & 3u), b = (int)((k >> 22) & 31u);
+  const uint32_t xbytes = (uint32_t)(slab_columns(P, k) * kDim * x_elt_bytes<XDT>());
+  const unsigned char* xsrc = static_cast<const unsigned char*>(G.x) +
+                              ((int64_t)b * G.cols + (int64_t)slab * kSlabV * kDim) * x_elt_bytes<XDT>();
+  mbar_arrive_expect_tx(&S.mbar[i], xbytes + (uint32_t)(kCodewords * kDim * 4));
+  bulk_copy_g2s(S.xraw[i], xsrc, xbytes, &S.mbar[i]);
+  bulk_copy_g2s(S.cb[i], G.codebooks + (size_t)s * kCodewords * kDim, kCodewords * kDim * 4, &S.mbar[i]);
+}
+
+// The 8 x values of slab column v widened to float (zero for columns past the row end).
+template <int XDT>
+__device__ __forceinline__ void staged_x(const unsigned char* xr, int v, int nv, float x[8]) {
+  if (v >= nv) {
+#pragma unroll
+    for (int k = 0; k < 8; k++) x[k] = 0.0f;
+    return;
+  }
+  if constexpr (XDT == VQ3R_F32) {
+    const float4 a = reinterpret_cast<const float4*>(xr)[2 * v], b = reinterpret_cast<const float4*>(xr)[2 * v + 1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  } else {
+    const uint4 w = reinterpret_cast<const uint4*>(xr)[v];
+    const uint32_t h[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+      if constexpr (XDT == VQ3R_BF16) {
+        x[2 * q] = bf16_bits_to_f32(h[q] & 0xFFFFu);
+        x[2 * q + 1] = bf16_bits_to_f32(h[q] >> 16);
+      } else {
+        x[2 * q] = f16_bits_to_f32(h[q] & 0xFFFFu);
+        x[2 * q + 1] = f16_bits_to_f32(h[q] >> 16);
+      }
+    }
+  }
+}
+
+// Piece c of a table: warp w computes codewords 32c + w and 32c + w + 16 for
+// slab columns lane and lane + 32, T[v][j] = C[j] . x[v] in k order.
+template <int XDT>
+__device__ __forceinline__ void build_piece(float* tab, const float* cb, const unsigned char* xr, int nv, int c,
+                                            int warp, int lane) {
+  float xa[8], xb[8];
+  staged_x<XDT>(xr, lane, nv, xa);
+  staged_x<XDT>(xr, lane + 32, nv, xb);
+  const float4* c4 = reinterpret_cast<const float4*>(cb);
+#pragma unroll
+  for (int h = 0; h < 2; h++) {
+    const int j = c * kChunkCw + warp + 16 * h;
+    const float4 c0 = c4[2 * j], c1 = c4[2 * j + 1];
+    const float cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    float ta = cw[0] * xa[0], tb = cw[0] * xb[0];
+#pragma unroll
+    for (int k = 1; k < 8; k++) {
+      ta = fmaf(cw[k], xa[k], ta);
+      tb = fmaf(cw[k], xb[k], tb);
+    }
+    tab[tab_word(lane, j)] = ta;
+    tab[tab_word(lane + 32, j)] = tb;
+  }
+}
+
+// Table key of unit u (divisions; used once per CTA).
+__device__ __forceinline__ uint32_t unit_table_key(const GvParams& P, int64_t u) {
+  const GvCursor c = unit_cursor(P, u);
+  return table_key(c.g, c.slab, c.s, c.b);
+}
+
+template <int XDT, int NSLOT>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_constant__ GvParams P) {
   extern __shared__ __align__(128) unsigned char gv_smem[];
-  float* tab = reinterpret_cast<float*>(gv_smem);
-  float* xs = reinterpret_cast<float*>(gv_smem + kTabBytes);
-  float* cbs = xs + kSlabV * kDim;
+  TilesSmem& S = *reinterpret_cast<TilesSmem*>(gv_smem);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, a = lane & 3;
+  // PRMT operands: byte 0 = byte offset of the bank of the current column,
+  // byte 2 = table buffer (tab[1] starts 64 KiB after tab[0]); the index
+  // byte lands in byte 1, i.e. at j * 256.
   uint32_t lc[8];
 #pragma unroll
   for (int q = 0; q < 8; q++)
     lc[q] = 4u * (8u * a + (uint32_t)((q & 3) ^ (g & 3)) + 4u * (uint32_t)((q >> 2) ^ (g >> 2)));
   uint32_t sel[4];
 #pragma unroll
-  for (int q = 0; q < 4; q++) sel[q] = 0x5504u | ((uint32_t)((q ^ g) & 3) << 4);
+  for (int q = 0; q < 4; q++) sel[q] = 0x7604u | ((uint32_t)((q ^ g) & 3) << 4);
   constexpr int kRowsPerWarpT = kTileRows / kGvWarps;  // 32: rows warp*32 + 8t + g, t = 0..3
   const int lane_off = (warp * kRowsPerWarpT + g) * kSlabV + 16 * a;
+  const int out_row = warp * kRowsPerWarpT + 8 * a + g;  // row whose sum this lane holds after the reduction
+  const bool hi2 = (a & 2) != 0, hi1 = (a & 1) != 0;
+  const uint64_t pol = l2_policy_evict_first();
 
   const int64_t u0 = (int64_t)blockIdx.x * P.total_units / gridDim.x;
   const int64_t u1 = (int64_t)(blockIdx.x + 1) * P.total_units / gridDim.x;
   griddep_launch_dependents();
   if (u0 >= u1) return;
-
-  auto load = [&](const GvCursor& c, uint4 (&w)[4]) {
-    const GvMat& M = P.m[c.m];
-    const uint8_t* base = M.idx + ((int64_t)c.s * P.g[c.g].n_slabs + c.slab) * M.plane_stride +
-                          (int64_t)c.tile * kTileBytes + lane_off;
-#pragma unroll
-    for (int t = 0; t < 4; t++) w[t] = __ldg(reinterpret_cast<const uint4*>(base + t * 8 * kSlabV));
-  };
-  GvCursor ci = unit_cursor(P, u0);
-  GvCursor c0 = ci, c1;
-  uint4 r0[4], r1[4];
-  load(ci, r0);
-  unit_advance(P, ci);
-  c1 = ci;
-  if (u0 + 1 < u1) load(ci, r1);
-  unit_advance(P, ci);
-
-  int loaded_g = -1, loaded_tab = -1;
-  const unsigned char* tb = reinterpret_cast<const unsigned char*>(tab);
-  auto step = [&](int64_t u, GvCursor& c, uint4 (&wr)[4]) {
-    const GvGroup& G = P.g[c.g];
-    const int tab_id = (c.slab * kStages + c.s) * P.B + c.b;
-    if (c.g != loaded_g || tab_id != loaded_tab) {
-      build_table<XDT>(G, c, tab, xs, cbs, tid);
-      loaded_g = c.g;
-      loaded_tab = tab_id;
-    }
-    const GvMat& M = P.m[c.m];
-    const int row = c.tile * kTileRows + warp * kRowsPerWarpT + g;
-    float* part = M.partial + (((int64_t)c.b * kStages + c.s) * G.n_slabs + c.slab) * M.rows + row;
-#pragma unroll
-    for (int t = 0; t < 4; t++) {
-      const uint32_t w[4] = {wr[t].x, wr[t].y, wr[t].z, wr[t].w};
-      float acc0 = 0.0f, acc1 = 0.0f;
-#pragma unroll
-      for (int m = 0; m < 16; m++) {
-        const uint32_t off = __byte_perm(w[m >> 2], lc[(m & 3) | ((m >> 3) << 2)], sel[m & 3]);
-        const float tv = *reinterpret_cast<const float*>(tb + off + ((m >> 2) & 1) * 128);
-        if (m & 1) acc1 += tv;
-        else acc0 += tv;
-      }
-      float sum = acc0 + acc1;
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-      if (a == 0 && row + 8 * t < M.rows) part[8 * t] = sum;
-    }
-    c = ci;
-    if (u + 2 < u1) load(ci, wr);
-    unit_advance(P, ci);
-  };
-  for (int64_t u = u0; u < u1; u += 2) {
-    step(u, c0, r0);
-    if (u + 1 < u1) step(u + 1, c1, r1);
+  TileCursor ci = tcur_at(P, u0);
+  const uint32_t key_last = unit_table_key(P, u1 - 1);
+  if (tid == 0) {
+    mbar_init(&S.mbar[0], 1);
+    mbar_init(&S.mbar[1], 1);
   }
+  __syncthreads();
+  griddep_wait();  // inputs may be written by the preceding kernel in the stream
+
+  // Inputs of the first two tables go out before the index stream.
+  uint32_t key_cur = ci.tkey;
+  uint32_t key_next = key_cur == key_last ? kNoTable : next_table_key(P, key_cur);
+  if (tid == 0) {
+    stage_table<XDT>(P, key_cur, S, 0);
+    if (key_next != kNoTable) stage_table<XDT>(P, key_next, S, 1);
+  }
+
+  uint4 r[NSLOT][4];
+  float* sq[NSLOT];
+  int32_t srows[NSLOT];
+  uint32_t skey[NSLOT];
+#pragma unroll
+  for (int i = 0; i < NSLOT; i++) {
+    if (u0 + i < u1) {
+#pragma unroll
+      for (int t = 0; t < 4; t++) r[i][t] = ldg_stream16(ci.p + lane_off + t * 8 * kSlabV, pol);
+      sq[i] = ci.q;
+      srows[i] = ci.rows_left;
+      skey[i] = ci.tkey;
+      tcur_next(P, ci);
+    } else {
+      sq[i] = nullptr;
+      srows[i] = 0;
+      skey[i] = kNoTable;
+    }
+  }
+
+  // The first table is built at once, while the first index loads are in flight.
+  bool ok = mbar_wait_bounded(&S.mbar[0], 0);
+  {
+    const int nv = slab_columns(P, key_cur);
+#pragma unroll 1
+    for (int c = 0; c < kBuildChunks; c++) build_piece<XDT>(S.tab[0], S.cb[0], S.xraw[0], nv, c, warp, lane);
+  }
+  __syncthreads();
+  int tno = 0;              // number of the current table within this CTA; it lives in tab[tno & 1]
+  int pieces = 0;           // pieces of table tno + 1 this warp has built
+  bool next_ready = false;  // the inputs of table tno + 1 have landed
+  const unsigned char* tb = reinterpret_cast<const unsigned char*>(S.tab[0]);
+
+  for (int64_t u = u0; u < u1; u += NSLOT) {
+#pragma unroll
+    for (int i = 0; i < NSLOT; i++) {
+      if (u + i < u1) {
+        const int nb = (tno + 1) & 1;
+        const uint32_t nparity = (uint32_t)((tno + 1) >> 1) & 1u;
+        if (skey[i] != key_cur) {  // switch to table tno + 1 (= key_next)
+          if (!next_ready) ok = mbar_wait_bounded(&S.mbar[nb], nparity) && ok;
+          const int nv = slab_columns(P, key_next);
+#pragma unroll 1
+          for (; pieces < kBuildChunks; pieces++) build_piece<XDT>(S.tab[nb], S.cb[nb], S.xraw[nb], nv, pieces, warp, lane);
+          __syncthreads();  // table complete; every warp is done with table tno - 1's buffers
+          tno++;
+          key_cur = key_next;
+          key_next = key_cur == key_last ? kNoTable : next_table_key(P, key_cur);
+          pieces = 0;
+          next_ready = false;
+#pragma unroll
+          for (int q = 0; q < 8; q++) lc[q] ^= 0x10000u;
+          if (tid == 0 && key_next != kNoTable) {
+            fence_proxy_async_smem();  // generic reads of the staging buffer precede the async refill
+            stage_table<XDT>(P, key_next, S, (tno + 1) & 1);
+          }
+        } else if (key_next != kNoTable && pieces < kBuildChunks) {
+          if (!next_ready) next_ready = __all_sync(0xFFFFFFFFu, mbar_test_wait(&S.mbar[nb], nparity));
+          if (next_ready) {
+            build_piece<XDT>(S.tab[nb], S.cb[nb], S.xraw[nb], slab_columns(P, key_next), pieces, warp, lane);
+            pieces++;
+          }
+        }
+        float* const q = sq[i];
+        const int32_t rows_valid = srows[i];
+        const bool refill = u + i + NSLOT < u1;
+        const uint8_t* const pn = ci.p + lane_off;
+        float acc[4];
+#pragma unroll
+        for (int t = 0; t < 4; t++) {
+          const uint32_t w[4] = {r[i][t].x, r[i][t].y, r[i][t].z, r[i][t].w};
+          float sum = 0.0f;
+#pragma unroll
+          for (int m = 0; m < 16; m++) {
+            const uint32_t off = __byte_perm(w[m >> 2], lc[(m & 3) | ((m >> 3) << 2)], sel[m & 3]);
+            sum += *reinterpret_cast<const float*>(tb + off + ((m >> 2) & 1) * 128);
+          }
+          acc[t] = sum;
+          if (refill) r[i][t] = ldg_stream16(pn + t * 8 * kSlabV, pol);
+        }
+        if (refill) {
+          sq[i] = ci.q;
+          srows[i] = ci.rows_left;
+          skey[i] = ci.tkey;
+          tcur_next(P, ci);
+        }
+        // Four lanes (a = 0..3) hold partial sums of rows t = 0..3 over
+        // their column quarters; two exchange steps leave lane a with the
+        // full sum of row t = a.
+        float k0 = hi2 ? acc[2] : acc[0], k1 = hi2 ? acc[3] : acc[1];
+        const float s0 = hi2 ? acc[0] : acc[2], s1 = hi2 ? acc[1] : acc[3];
+        k0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 2);
+        k1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
+        float kk = hi1 ? k1 : k0;
+        kk += __shfl_xor_sync(0xFFFFFFFFu, hi1 ? k0 : k1, 1);
+        if (out_row < rows_valid) q[out_row] = kk;
+      }
+    }
+  }
+  (void)ok;  // a timed-out wait has recorded kDevErrMbarTimeout in the device error word
 }
 
 // Repack the index planes [3][rows][cols/8] (plane_stride bytes apart) into
@@ -423,32 +679,51 @@ __global__ void __launch_bounds__(256) pack_tiles_kernel(const uint8_t* __restri
   }
 }
 
-// y[b][i] = scale_i * sum_s sum_slab partial[b][s][slab][i].  Four lanes share
-// an output: lane k of the group adds partials k, k+4, k+8, ... in order, then
-// two butterfly steps combine the four sums, so the order is fixed.
+// y[b][i] = scale_i * sum_s sum_slab partial[b][s][slab][i].  Two lanes share
+// an output: lane k (k = 0, 1) adds partials k, k + 2, k + 4, ... in order and
+// one butterfly step combines the two sums, so the order is fixed.  Each lane
+// issues the loads of up to kRedPer partials before adding any, so an output
+// with up to 2 * kRedPer partials costs one round trip to L2.  CTA (x, y)
+// takes rows [128x, 128x + 128) of matrix y for every token.
+constexpr int kRedPer = 24;
+constexpr int kRedRows = 128;  // rows per CTA (256 threads, two lanes per row)
+
+// Sum, in order, of partials k0, k0 + 2, ... (N of them, those below np) of
+// one output.  The loads are unconditional (past-the-end ones re-read the
+// last partial) so that all N are in flight at once; the sum masks them.
+template <int N>
+__device__ __forceinline__ float sum_partials(const float* pp, int64_t stride, int np, int k0) {
+  float v[N];
+#pragma unroll
+  for (int j = 0; j < N; j++) v[j] = __ldcg(pp + (int64_t)min(k0 + 2 * j, np - 1) * stride);
+  float acc = 0.0f;
+#pragma unroll
+  for (int j = 0; j < N; j++)
+    if (k0 + 2 * j < np) acc += v[j];
+  return acc;
+}
+
 __global__ void __launch_bounds__(256) gemv_reduce_kernel(const __grid_constant__ GvParams P) {
-  griddep_wait();  // the partial sums of the main kernel are complete
+  griddep_launch_dependents();
   const GvMat& M = P.m[blockIdx.y];
-  const GvGroup& G = P.g[M.group];
-  const int64_t n = (int64_t)P.B * M.rows;
-  const int np = kStages * G.n_slabs;
-  const int sub = threadIdx.x & 3;
-  const int64_t per_pass = (int64_t)gridDim.x * (blockDim.x / 4);
-  for (int64_t base = (int64_t)blockIdx.x * (blockDim.x / 4); base < n; base += per_pass) {
-    const int64_t i = base + (threadIdx.x >> 2);
+  const int64_t row = (int64_t)blockIdx.x * kRedRows + (threadIdx.x >> 1);
+  if ((int64_t)blockIdx.x * kRedRows >= M.rows) return;  // past this matrix's rows (whole CTA)
+  griddep_wait();  // the partial sums of the main kernel are complete
+  const int sub = threadIdx.x & 1;
+  const int np = kStages * P.g[M.group].n_slabs;
+  const bool valid = row < M.rows;
+  const float scale = valid ? f16_bits_to_f32(__ldg(M.scales + row)) : 0.0f;
+  for (int b = 0; b < P.B; b++) {
     float acc = 0.0f;
-    if (i < n) {
-      const int64_t b = i / M.rows, row = i - b * M.rows;
-      const float* pp = M.partial + b * np * M.rows + row;
-#pragma unroll 4
-      for (int k = sub; k < np; k += 4) acc += __ldg(pp + (int64_t)k * M.rows);
+    if (valid) {
+      const float* pp = M.partial + (int64_t)b * np * M.rows + row;
+      if (np <= 16)
+        acc = sum_partials<8>(pp, M.rows, np, sub);
+      else
+        for (int k0 = sub; k0 < np; k0 += 2 * kRedPer) acc += sum_partials<kRedPer>(pp, M.rows, np, k0);
     }
     acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
-    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 2);
-    if (i < n && sub == 0) {
-      const int64_t row = i - (i / M.rows) * M.rows;
-      M.y[i] = f16_bits_to_f32(__ldg(M.scales + row)) * acc;
-    }
+    if (valid && sub == 0) M.y[(int64_t)b * M.rows + row] = scale * acc;
   }
 }
 

@@ -49,15 +49,16 @@ cudaError_t device_setup(int* sms) {
     cudaError_t r = cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev);
     const int enc = (int)sizeof(EncSmem);
     const int gv = (int)kGvSmemBytes;
+    const int gt = (int)kTilesSmemBytes;
     if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F32, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_BF16, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
     g_dev_err[dev] = r;
   });
   *sms = g_dev_sms[dev];
@@ -249,13 +250,27 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   if (e != cudaSuccess) return cuda_fail(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const GvParams& P = plan.P;
+  // Both kernels are launched with programmatic stream serialization: the
+  // main kernel's CTAs may be scheduled while the preceding kernel drains
+  // (they wait at griddepcontrol.wait before reading any input), and the
+  // reduction's CTAs wait the same way for the partial sums.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = s;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
   if (P.layout == VQ3R_LAYOUT_TILES) {  // one CTA per SM
-    const int grid = (int)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms);
+    cfg.gridDim = dim3((unsigned)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms));
+    cfg.blockDim = dim3(kGvThreads);
+    cfg.dynamicSmemBytes = kTilesSmemBytes;
     switch (x_dtype) {
-      case VQ3R_F32: gemv_tiles_kernel<VQ3R_F32><<<grid, kGvThreads, kGvSmemBytes, s>>>(P); break;
-      case VQ3R_BF16: gemv_tiles_kernel<VQ3R_BF16><<<grid, kGvThreads, kGvSmemBytes, s>>>(P); break;
-      default: gemv_tiles_kernel<VQ3R_F16><<<grid, kGvThreads, kGvSmemBytes, s>>>(P); break;
+      case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, kTileSlots>, P); break;
+      case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, kTileSlots>, P); break;
+      default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, kTileSlots>, P); break;
     }
+    if (e != cudaSuccess) return cuda_fail(e);
   } else {  // two CTAs per SM
     const int grid = (int)(P.total_units < 2 * (int64_t)sms ? P.total_units : 2 * (int64_t)sms);
     switch (x_dtype) {
@@ -266,23 +281,10 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
-  // The reduction kernel is launched with programmatic stream serialization:
-  // its CTAs may start while the main kernel runs and wait (griddepcontrol.wait)
-  // for its partial sums.
-  cudaLaunchAttribute pdl[1];
-  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.stream = s;
-  cfg.attrs = pdl;
-  cfg.numAttrs = 1;
-  int64_t maxrows = 0;
-  for (int i = 0; i < P.n_mats; i++) maxrows = P.m[i].rows * B > maxrows ? P.m[i].rows * B : maxrows;
-  int64_t gx = (maxrows * 4 + 255) / 256;  // four lanes per output
-  if (gx > (int64_t)sms * 4) gx = (int64_t)sms * 4;
-  if (gx < 1) gx = 1;
-  cfg.gridDim = dim3((unsigned)gx, (unsigned)P.n_mats);
-  cfg.blockDim = dim3(256);
+  int64_t maxrows = 1;
+  for (int i = 0; i < P.n_mats; i++) maxrows = P.m[i].rows > maxrows ? P.m[i].rows : maxrows;
+  cfg.gridDim = dim3((unsigned)((maxrows + kRedRows - 1) / kRedRows), (unsigned)P.n_mats);
+  cfg.blockDim = dim3(2 * kRedRows);
   cfg.dynamicSmemBytes = 0;
   e = cudaLaunchKernelEx(&cfg, gemv_reduce_kernel, P);
   if (e != cudaSuccess) return cuda_fail(e);

@@ -90,6 +90,26 @@ __device__ __forceinline__ uint16_t f64_to_f16_sat_rne(double x) {
   return sign | (uint16_t)q;
 }
 
+// ---- streaming loads ----
+
+// L2 cache policy that makes lines the first candidates for eviction: used
+// for data read exactly once (the index stream), so that it does not push
+// out what is read again (tables' inputs, partial sums).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 16-byte read-only load that allocates in neither L1 nor (preferentially) L2.
+__device__ __forceinline__ uint4 ldg_stream16(const void* p, uint64_t pol) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p), "l"(pol));
+  return v;
+}
+
 // ---- shared-memory mbarrier and bulk asynchronous copy (TMA, no multicast) ----
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -121,6 +141,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* mbar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(mbar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Orders this thread's earlier generic-proxy accesses of shared memory before
+// later asynchronous-proxy (bulk copy) writes to it.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* mbar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(mbar)), "r"(parity)
