@@ -6,8 +6,8 @@ One step = one pass of the whole path over a 64-expert MoE layer
 with log-normal row factors; 2.82 G weights):
   encode (row scale + greedy 3-stage assignment), repack of the indices into
   the tiled GEMV layout, decode to fp32, relative Frobenius error of each
-  matrix, and the MoE decode step (8 active experts: gate/up GEMV in one
-  call, down GEMV in one call, B = 1).
+  matrix, and the MoE decode step (8 active experts: gate/up and down GEMV
+  of all 8 experts in one grouped call, B = 1).
 Each matrix kind of the layer is stacked into one call.  The decode step
 rotates over the 8 disjoint 8-expert groups of the layer so that its 132 MB
 of indices per step come from HBM, not L2 (the layer's 5.6 GB of weights
@@ -194,11 +194,10 @@ class Layer:
                     p2.append(dict(idx=self.tiles[wl.W2], scales=self.sc[wl.W2], codebooks=self.cb, x=xd[j],
                                    row0=e * rows, rows=rows, layout="tiles", cols=cols,
                                    y=torch.empty((B, rows), dtype=torch.float32, device=dev)))
-                d1, d2 = vq._descs(p1), vq._descs(p2)
-                ws1 = vq.lib().vq3r_gemv_workspace_size(d1, len(p1), B)
-                ws2 = vq.lib().vq3r_gemv_workspace_size(d2, len(p2), B)
-                plans.append((d1, len(p1), d2, len(p2), p1, p2, ws1, ws2))
-            wsz = max(max(p[6], p[7]) for p in plans)
+                # the whole step (gate/up and down of the 8 experts) is one grouped call
+                d = vq._descs(p1 + p2)
+                plans.append((d, len(p1) + len(p2), p1 + p2, vq.lib().vq3r_gemv_workspace_size(d, len(p1) + len(p2), B)))
+            wsz = max(p[3] for p in plans)
             ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
             self.moe[B] = (plans, ws, xu, xd)
 
@@ -223,14 +222,13 @@ class Layer:
 
     def gemv(self, B, group):
         plans, ws, _, _ = self.moe[B]
-        d1, n1, d2, n2 = plans[group % len(plans)][:4]
+        d, n = plans[group % len(plans)][:2]
         L, s = self.vq.lib(), self.torch.cuda.current_stream().cuda_stream
-        for d, n in ((d1, n1), (d2, n2)):
-            st = L.vq3r_gemv(d, n, B, 1, ws.data_ptr(), ws.numel(), s)
-            if st:
-                raise self.vq.VQ3RError(st, "vq3r_gemv")
+        st = L.vq3r_gemv(d, n, B, 1, ws.data_ptr(), ws.numel(), s)
+        if st:
+            raise self.vq.VQ3RError(st, "vq3r_gemv")
 
-    LAUNCHES_PER_STEP = 3 * 2 + 3 + 3 * 1 + 3 * 2 + 2 * 2  # encode, pack, decode, error, gemv (kernels)
+    LAUNCHES_PER_STEP = 3 * 2 + 3 + 3 * 1 + 3 * 2 + 2  # encode, pack, decode, error, gemv (kernels)
 
 
 # ----------------------------------------------------------------------------- CPU oracle sample
@@ -441,7 +439,7 @@ def main():
                 hostE[j:j + 1].copy_(layer.err[k], non_blocking=True)
             plans = layer.moe[1][0][i % layer.groups]
             off = 0
-            for m in plans[4] + plans[5]:
+            for m in plans[2]:
                 n = m["y"].numel()
                 hostY[off:off + n].copy_(m["y"].view(-1), non_blocking=True)
                 off += n
