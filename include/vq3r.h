@@ -109,9 +109,18 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
  *   for bit.
  *
  * One descriptor per matrix; matrices may differ in shape, codebooks and x.
- * Matrices that share (codebooks, x, cols) share one x-projected table in
- * the workspace, so one call over the gate and up matrices of all active
- * experts reads x once.  y must not overlap any input.
+ * Matrices that share (codebooks, x, cols) share the x-projected tables the
+ * kernel builds in shared memory, so one call over the gate and up matrices
+ * of all active experts builds each table once per SM that needs it.  y must
+ * not overlap any input.
+ *
+ * Workspace: one partial sum per (token, stage, 64-column slab, row); PLANES
+ * stores floats and adds them in a second kernel, TILES stores 64-bit slots
+ * (call tag, float) and reduces them in the same kernel, each SM waiting
+ * until the slots it adds carry this call's tag.  Nothing needs clearing
+ * between calls.  The TILES kernel runs one CTA per SM and needs all of them
+ * resident together: if another workload holds SMs for more than about a
+ * second, the call finishes with vq3r_device_error() = 2 and y undefined.
  *   mats      HOST array of n_mats descriptors (copied before return)
  *   B         tokens, 1..32
  *   x_dtype   dtype of every x, {F32, BF16, F16}
@@ -219,8 +228,9 @@ const char* vq3r_status_string(vq3r_status s);
 /* cudaError_t value of the most recent VQ3R_ERR_CUDA on the calling thread (0 if none). */
 int vq3r_last_cuda_error(void);
 
-/* Device-side error word, set by a kernel whose bounded wait on an
- * asynchronous copy gave up (0 = none).  Synchronises the current device;
+/* Device-side error word, set by a kernel whose bounded wait gave up
+ * (0 = none; 1 = a shared-memory bulk copy did not complete; 2 = vq3r_gemv
+ * TILES partial sums did not all appear).  Synchronises the current device;
  * reading it clears it. */
 vq3r_status vq3r_device_error(int* code);
 

@@ -70,13 +70,13 @@ struct GvMat {
   const uint8_t* idx;
   const uint16_t* scales;
   float* y;
-  float* partial;        // [B][3][n_slabs][rows]
+  void* partial;         // [B][3][n_slabs][rows]: float (planes) or 64-bit slots (tiles)
   int64_t rows;
   int64_t plane_stride;  // bytes between index planes
   int32_t group;
   int32_t n_tiles;       // ceil(rows / kGvTileRows) >= 1
   int32_t tile_prefix;   // tiles of the earlier matrices of the same group
-  int32_t pad_;
+  int32_t red_begin;     // first block (kRedRows rows) of this matrix in the tiled kernel's reduction
 };
 
 struct GvGroup {
@@ -97,6 +97,8 @@ struct GvParams {
   int64_t total_units;
   int32_t tile_rows;     // rows per work unit: kGvTileRows (planes) or kTileRows (tiles)
   int32_t layout;        // VQ3R_LAYOUT_PLANES or VQ3R_LAYOUT_TILES
+  uint32_t epoch;        // tiles: tag of this call's partial-sum slots (never 0)
+  int32_t red_blocks;    // tiles: output blocks of kRedRows rows over all matrices
 };
 
 // Programmatic dependent launch: wait until the preceding kernel in the
@@ -282,7 +284,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_lut_kernel(const __grid_co
     }
     const GvMat& M = P.m[c.m];
     const int row = c.tile * kGvTileRows + warp * kGvRowsPerWarp + g;
-    float* part = M.partial + (((int64_t)c.b * kStages + c.s) * G.n_slabs + c.slab) * M.rows + row;
+    float* part = static_cast<float*>(M.partial) + (((int64_t)c.b * kStages + c.s) * G.n_slabs + c.slab) * M.rows + row;
     const bool w_ok0 = a == 0 && row < M.rows, w_ok1 = a == 0 && row + 8 < M.rows;
 #pragma unroll
     for (int q = 0; q < 2; q++) {
@@ -334,7 +336,7 @@ __host__ __device__ __forceinline__ uint32_t table_key(int g, int slab, int s, i
 // key, and the coordinates needed for the carry to the next matrix or table.
 struct TileCursor {
   const uint8_t* p;
-  float* q;
+  unsigned long long* q;
   int32_t rows_left;
   uint32_t tkey;
   int32_t m, tile, ntiles;
@@ -347,7 +349,8 @@ __device__ __forceinline__ void tcur_fill(const GvParams& P, TileCursor& c) {
   const int64_t n_slabs = P.g[g].n_slabs;
   c.ntiles = M.n_tiles;
   c.p = M.idx + ((int64_t)s * n_slabs + slab) * M.plane_stride + (int64_t)c.tile * kTileBytes;
-  c.q = M.partial + (((int64_t)b * kStages + s) * n_slabs + slab) * M.rows + (int64_t)c.tile * kTileRows;
+  c.q = static_cast<unsigned long long*>(M.partial) + (((int64_t)b * kStages + s) * n_slabs + slab) * M.rows +
+        (int64_t)c.tile * kTileRows;
   c.rows_left = (int32_t)(M.rows - (int64_t)c.tile * kTileRows);
 }
 
@@ -498,6 +501,95 @@ __device__ __forceinline__ void build_piece(float* tab, const float* cb, const u
   }
 }
 
+// ---------------------------------------------------------------------------
+// Stage reduction inside the tiled kernel.
+//
+// Each unit leaves one partial sum per row in a 64-bit slot: the high word is
+// the call's epoch (a per-call tag chosen by the host, never 0), the low word
+// the float.  One aligned 64-bit store is single-copy atomic, so a reader that
+// sees this call's epoch also sees the value written with it; slots left by
+// earlier calls (or never written) carry another tag.  After its own units,
+// each warp reduces output blocks of kRedRows rows of one matrix (block
+// numbers warp, warp + all warps of the grid, ...): it waits, with a time
+// bound, until every slot of a row carries the epoch and adds them in a fixed
+// order.  This needs no counter, no cleared workspace and no second kernel.
+// Every CTA of the grid must be resident at once (one CTA per SM, grid <=
+// SMs), or the bound fires and the call reports kDevErrSlotTimeout.
+constexpr int kRedRows = 16;  // rows per warp block: two lanes per row
+
+__device__ __forceinline__ void slot_store(unsigned long long* p, uint32_t epoch, float v) {
+  const unsigned long long w = ((unsigned long long)epoch << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long slot_load(const unsigned long long* p) {
+  unsigned long long w;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+
+// In-order sum of slots k0, k0 + 2, ... (N of them, those below np) of one
+// output, once all of them carry the epoch.  Past-the-end positions re-read
+// the last slot so that all N loads are issued together.
+template <int N>
+__device__ __forceinline__ float sum_slots(const unsigned long long* sp, int64_t stride, int np, int k0,
+                                           uint32_t epoch) {
+  unsigned long long w[N];
+  uint64_t t0 = 0;
+  for (;;) {
+#pragma unroll
+    for (int j = 0; j < N; j++) w[j] = slot_load(sp + (int64_t)min(k0 + 2 * j, np - 1) * stride);
+    bool ready = true;
+#pragma unroll
+    for (int j = 0; j < N; j++) ready = ready && (uint32_t)(w[j] >> 32) == epoch;
+    if (ready) break;
+    const uint64_t now = global_timer_ns();
+    if (t0 == 0) {
+      t0 = now;
+    } else if (now - t0 > 1000000000ull) {
+      set_device_error(kDevErrSlotTimeout);
+      break;
+    }
+    __nanosleep(128);
+  }
+  float acc = 0.0f;
+#pragma unroll
+  for (int j = 0; j < N; j++)
+    if (k0 + 2 * j < np) acc += __uint_as_float((uint32_t)w[j]);
+  return acc;
+}
+
+// y[b][i] = scale_i * sum over (stage, slab) of the slots of row i.  Lane k of
+// a row's two lanes adds slots k, k + 2, ... in order (one load batch sized to
+// the number of slots); one butterfly step combines the two sums.
+__device__ __forceinline__ void reduce_slots(const GvParams& P, int tid) {
+  const int lane = tid & 31, sub = lane & 1;
+  const int warps = gridDim.x * kGvWarps;
+  for (int blk = blockIdx.x * kGvWarps + (tid >> 5); blk < P.red_blocks; blk += warps) {
+    int m = 0;
+    while (m + 1 < P.n_mats && P.m[m + 1].red_begin <= blk) m++;
+    const GvMat& M = P.m[m];
+    const int64_t row = (int64_t)(blk - M.red_begin) * kRedRows + (lane >> 1);
+    const bool valid = row < M.rows;
+    const int np = kStages * P.g[M.group].n_slabs;
+    const float scale = valid ? f16_bits_to_f32(__ldg(M.scales + row)) : 0.0f;
+    for (int b = 0; b < P.B; b++) {
+      float acc = 0.0f;
+      if (valid) {
+        const unsigned long long* sp = static_cast<const unsigned long long*>(M.partial) + (int64_t)b * np * M.rows + row;
+        if (np <= 12)
+          acc = sum_slots<6>(sp, M.rows, np, sub, P.epoch);
+        else if (np <= 24)
+          acc = sum_slots<12>(sp, M.rows, np, sub, P.epoch);
+        else
+          for (int k0 = sub; k0 < np; k0 += 48) acc += sum_slots<24>(sp, M.rows, np, k0, P.epoch);
+      }
+      acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
+      if (valid && sub == 0) M.y[(int64_t)b * M.rows + row] = scale * acc;
+    }
+  }
+}
+
 // Table key of unit u (divisions; used once per CTA).
 __device__ __forceinline__ uint32_t unit_table_key(const GvParams& P, int64_t u) {
   const GvCursor c = unit_cursor(P, u);
@@ -530,7 +622,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   const int64_t u0 = (int64_t)blockIdx.x * P.total_units / gridDim.x;
   const int64_t u1 = (int64_t)(blockIdx.x + 1) * P.total_units / gridDim.x;
   griddep_launch_dependents();
-  if (u0 >= u1) return;
+  if (u0 >= u1) {  // no units (cannot happen with grid <= units): only the reduction share
+    griddep_wait();
+    reduce_slots(P, tid);
+    return;
+  }
   TileCursor ci = tcur_at(P, u0);
   const uint32_t key_last = unit_table_key(P, u1 - 1);
   if (tid == 0) {
@@ -549,7 +645,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   }
 
   uint4 r[NSLOT][4];
-  float* sq[NSLOT];
+  unsigned long long* sq[NSLOT];
   int32_t srows[NSLOT];
   uint32_t skey[NSLOT];
 #pragma unroll
@@ -611,7 +707,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
             pieces++;
           }
         }
-        float* const q = sq[i];
+        unsigned long long* const q = sq[i];
         const int32_t rows_valid = srows[i];
         const bool refill = u + i + NSLOT < u1;
         const uint8_t* const pn = ci.p + lane_off;
@@ -643,11 +739,12 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
         k1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
         float kk = hi1 ? k1 : k0;
         kk += __shfl_xor_sync(0xFFFFFFFFu, hi1 ? k0 : k1, 1);
-        if (out_row < rows_valid) q[out_row] = kk;
+        if (out_row < rows_valid) slot_store(q + out_row, P.epoch, kk);
       }
     }
   }
   (void)ok;  // a timed-out wait has recorded kDevErrMbarTimeout in the device error word
+  reduce_slots(P, tid);
 }
 
 // Repack the index planes [3][rows][cols/8] (plane_stride bytes apart) into
@@ -686,7 +783,7 @@ __global__ void __launch_bounds__(256) pack_tiles_kernel(const uint8_t* __restri
 // with up to 2 * kRedPer partials costs one round trip to L2.  CTA (x, y)
 // takes rows [128x, 128x + 128) of matrix y for every token.
 constexpr int kRedPer = 24;
-constexpr int kRedRows = 128;  // rows per CTA (256 threads, two lanes per row)
+constexpr int kPlanesRedRows = 128;  // rows per CTA of the reduction kernel (256 threads)
 
 // Sum, in order, of partials k0, k0 + 2, ... (N of them, those below np) of
 // one output.  The loads are unconditional (past-the-end ones re-read the
@@ -706,8 +803,8 @@ __device__ __forceinline__ float sum_partials(const float* pp, int64_t stride, i
 __global__ void __launch_bounds__(256) gemv_reduce_kernel(const __grid_constant__ GvParams P) {
   griddep_launch_dependents();
   const GvMat& M = P.m[blockIdx.y];
-  const int64_t row = (int64_t)blockIdx.x * kRedRows + (threadIdx.x >> 1);
-  if ((int64_t)blockIdx.x * kRedRows >= M.rows) return;  // past this matrix's rows (whole CTA)
+  const int64_t row = (int64_t)blockIdx.x * kPlanesRedRows + (threadIdx.x >> 1);
+  if ((int64_t)blockIdx.x * kPlanesRedRows >= M.rows) return;  // past this matrix's rows (whole CTA)
   griddep_wait();  // the partial sums of the main kernel are complete
   const int sub = threadIdx.x & 1;
   const int np = kStages * P.g[M.group].n_slabs;
@@ -716,7 +813,7 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const __grid_constant_
   for (int b = 0; b < P.B; b++) {
     float acc = 0.0f;
     if (valid) {
-      const float* pp = M.partial + (int64_t)b * np * M.rows + row;
+      const float* pp = static_cast<const float*>(M.partial) + (int64_t)b * np * M.rows + row;
       if (np <= 16)
         acc = sum_partials<8>(pp, M.rows, np, sub);
       else

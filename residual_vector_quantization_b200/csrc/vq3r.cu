@@ -1,6 +1,7 @@
 // C ABI of the VQ3R library (declared in include/vq3r.h): argument checks,
 // launch configuration and status codes.  All arithmetic runs in the
 // kernels of encode.cuh, decode.cuh and gemv.cuh.
+#include <atomic>
 #include <mutex>
 
 #include "decode.cuh"
@@ -149,11 +150,19 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
     G.unit_begin = units;
     units += (int64_t)G.n_slabs * kStages * B * G.tiles;
   }
+  // Partial sums: one float per (token, stage, slab, row) for the planes
+  // kernel, one 64-bit (epoch, float) slot for the tiled kernel.
+  const size_t part_bytes = tiles ? sizeof(unsigned long long) : sizeof(float);
+  int64_t red_blocks = 0;
   for (int i = 0; i < nm; i++) {
     GvMat& M = P.m[i];
-    M.partial = reinterpret_cast<float*>(ws_base + off);
-    off = align_up(off + (size_t)B * kStages * P.g[M.group].n_slabs * (size_t)M.rows * sizeof(float));
+    M.partial = ws_base + off;
+    off = align_up(off + (size_t)B * kStages * P.g[M.group].n_slabs * (size_t)M.rows * part_bytes);
+    M.red_begin = (int32_t)red_blocks;
+    red_blocks += (M.rows + kRedRows - 1) / kRedRows;
   }
+  if (red_blocks >= ((int64_t)1 << 31)) return VQ3R_ERR_SHAPE;
+  P.red_blocks = (int32_t)red_blocks;
   P.total_units = units;
   plan->ws_bytes = off;
   return VQ3R_OK;
@@ -249,11 +258,18 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   cudaError_t e = device_setup(&sms);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Tag of this call's partial-sum slots: distinct from the previous calls'
+  // (a 32-bit counter per process, skipping 0).
+  static std::atomic<uint32_t> g_epoch{0};
+  uint32_t ep = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (ep == 0) ep = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+  plan.P.epoch = ep;
   const GvParams& P = plan.P;
-  // Both kernels are launched with programmatic stream serialization: the
-  // main kernel's CTAs may be scheduled while the preceding kernel drains
-  // (they wait at griddepcontrol.wait before reading any input), and the
-  // reduction's CTAs wait the same way for the partial sums.
+  // Kernels are launched with programmatic stream serialization: their CTAs
+  // may be scheduled while the preceding kernel drains and wait
+  // (griddepcontrol.wait) before reading any input.  The tiled kernel reduces
+  // its own partial sums; the planes kernel is followed by the reduction
+  // kernel, whose CTAs wait the same way for the partial sums.
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
@@ -271,6 +287,7 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
       default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, kTileSlots>, P); break;
     }
     if (e != cudaSuccess) return cuda_fail(e);
+    return check_launch();  // the tiled kernel reduces its partial sums itself
   } else {  // two CTAs per SM
     const int grid = (int)(P.total_units < 2 * (int64_t)sms ? P.total_units : 2 * (int64_t)sms);
     switch (x_dtype) {
@@ -283,8 +300,8 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   if (e != cudaSuccess) return cuda_fail(e);
   int64_t maxrows = 1;
   for (int i = 0; i < P.n_mats; i++) maxrows = P.m[i].rows > maxrows ? P.m[i].rows : maxrows;
-  cfg.gridDim = dim3((unsigned)((maxrows + kRedRows - 1) / kRedRows), (unsigned)P.n_mats);
-  cfg.blockDim = dim3(2 * kRedRows);
+  cfg.gridDim = dim3((unsigned)((maxrows + kPlanesRedRows - 1) / kPlanesRedRows), (unsigned)P.n_mats);
+  cfg.blockDim = dim3(2 * kPlanesRedRows);
   cfg.dynamicSmemBytes = 0;
   e = cudaLaunchKernelEx(&cfg, gemv_reduce_kernel, P);
   if (e != cudaSuccess) return cuda_fail(e);
