@@ -90,15 +90,19 @@ struct GvGroup {
   int32_t pad_;
 };
 
+constexpr int kMaxSplit = 256;  // CTAs whose unit ranges the host can set (tiled kernel)
+
 struct GvParams {
   GvMat m[VQ3R_GEMV_MAX_MATS];
   GvGroup g[VQ3R_GEMV_MAX_MATS];
+  int64_t cta_begin[kMaxSplit + 1];  // tiles: CTA c takes units [cta_begin[c], cta_begin[c + 1]) when n_split == grid
   int32_t n_mats, n_groups, B, vec8;  // vec8: rows and planes 8-byte aligned (64-bit index loads)
   int64_t total_units;
   int32_t tile_rows;     // rows per work unit: kGvTileRows (planes) or kTileRows (tiles)
   int32_t layout;        // VQ3R_LAYOUT_PLANES or VQ3R_LAYOUT_TILES
   uint32_t epoch;        // tiles: tag of this call's partial-sum slots (never 0)
   int32_t red_blocks;    // tiles: output blocks of kRedRows rows over all matrices
+  int32_t n_split;       // tiles: entries of cta_begin in use minus one (0: equal split)
 };
 
 // Programmatic dependent launch: wait until the preceding kernel in the
@@ -510,12 +514,12 @@ __device__ __forceinline__ void build_piece(float* tab, const float* cb, const u
 // sees this call's epoch also sees the value written with it; slots left by
 // earlier calls (or never written) carry another tag.  After its own units,
 // each warp reduces output blocks of kRedRows rows of one matrix (block
-// numbers warp, warp + all warps of the grid, ...): it waits, with a time
-// bound, until every slot of a row carries the epoch and adds them in a fixed
-// order.  This needs no counter, no cleared workspace and no second kernel.
+// numbers warp, warp + all warps of the grid, ...), one lane per row: it
+// waits, with a time bound, until every slot of its row carries the epoch
+// and adds them in a fixed order.  This needs no counter, no cleared workspace and no second kernel.
 // Every CTA of the grid must be resident at once (one CTA per SM, grid <=
 // SMs), or the bound fires and the call reports kDevErrSlotTimeout.
-constexpr int kRedRows = 16;  // rows per warp block: two lanes per row
+constexpr int kRedRows = 32;  // rows per warp block: one lane per row
 
 __device__ __forceinline__ void slot_store(unsigned long long* p, uint32_t epoch, float v) {
   const unsigned long long w = ((unsigned long long)epoch << 32) | __float_as_uint(v);
@@ -528,9 +532,9 @@ __device__ __forceinline__ unsigned long long slot_load(const unsigned long long
   return w;
 }
 
-// In-order sum of slots k0, k0 + 2, ... (N of them, those below np) of one
-// output, once all of them carry the epoch.  Past-the-end positions re-read
-// the last slot so that all N loads are issued together.
+// In-order sum of slots k0 .. k0 + N - 1 (those below np) of one output, once
+// all of them carry the epoch.  Past-the-end positions re-read the last slot
+// so that all N loads are issued together.
 template <int N>
 __device__ __forceinline__ float sum_slots(const unsigned long long* sp, int64_t stride, int np, int k0,
                                            uint32_t epoch) {
@@ -538,7 +542,7 @@ __device__ __forceinline__ float sum_slots(const unsigned long long* sp, int64_t
   uint64_t t0 = 0;
   for (;;) {
 #pragma unroll
-    for (int j = 0; j < N; j++) w[j] = slot_load(sp + (int64_t)min(k0 + 2 * j, np - 1) * stride);
+    for (int j = 0; j < N; j++) w[j] = slot_load(sp + (int64_t)min(k0 + j, np - 1) * stride);
     bool ready = true;
 #pragma unroll
     for (int j = 0; j < N; j++) ready = ready && (uint32_t)(w[j] >> 32) == epoch;
@@ -550,42 +554,38 @@ __device__ __forceinline__ float sum_slots(const unsigned long long* sp, int64_t
       set_device_error(kDevErrSlotTimeout);
       break;
     }
-    __nanosleep(128);
+    __nanosleep(64);
   }
   float acc = 0.0f;
 #pragma unroll
   for (int j = 0; j < N; j++)
-    if (k0 + 2 * j < np) acc += __uint_as_float((uint32_t)w[j]);
+    if (k0 + j < np) acc += __uint_as_float((uint32_t)w[j]);
   return acc;
 }
 
-// y[b][i] = scale_i * sum over (stage, slab) of the slots of row i.  Lane k of
-// a row's two lanes adds slots k, k + 2, ... in order (one load batch sized to
-// the number of slots); one butterfly step combines the two sums.
+// y[b][i] = scale_i * sum over k = s * n_slabs + slab of the slots of row i,
+// added in k order by the row's lane, in load batches of up to 24 slots.
 __device__ __forceinline__ void reduce_slots(const GvParams& P, int tid) {
-  const int lane = tid & 31, sub = lane & 1;
+  const int lane = tid & 31;
   const int warps = gridDim.x * kGvWarps;
   for (int blk = blockIdx.x * kGvWarps + (tid >> 5); blk < P.red_blocks; blk += warps) {
     int m = 0;
     while (m + 1 < P.n_mats && P.m[m + 1].red_begin <= blk) m++;
     const GvMat& M = P.m[m];
-    const int64_t row = (int64_t)(blk - M.red_begin) * kRedRows + (lane >> 1);
-    const bool valid = row < M.rows;
+    const int64_t row = (int64_t)(blk - M.red_begin) * kRedRows + lane;
+    if (row >= M.rows) continue;
     const int np = kStages * P.g[M.group].n_slabs;
-    const float scale = valid ? f16_bits_to_f32(__ldg(M.scales + row)) : 0.0f;
+    const float scale = f16_bits_to_f32(__ldg(M.scales + row));
     for (int b = 0; b < P.B; b++) {
-      float acc = 0.0f;
-      if (valid) {
-        const unsigned long long* sp = static_cast<const unsigned long long*>(M.partial) + (int64_t)b * np * M.rows + row;
-        if (np <= 12)
-          acc = sum_slots<6>(sp, M.rows, np, sub, P.epoch);
-        else if (np <= 24)
-          acc = sum_slots<12>(sp, M.rows, np, sub, P.epoch);
-        else
-          for (int k0 = sub; k0 < np; k0 += 48) acc += sum_slots<24>(sp, M.rows, np, k0, P.epoch);
+      const unsigned long long* sp = static_cast<const unsigned long long*>(M.partial) + (int64_t)b * np * M.rows + row;
+      float acc;
+      if (np <= 12) {
+        acc = sum_slots<12>(sp, M.rows, np, 0, P.epoch);
+      } else {
+        acc = 0.0f;
+        for (int k0 = 0; k0 < np; k0 += 24) acc += sum_slots<24>(sp, M.rows, np, k0, P.epoch);
       }
-      acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
-      if (valid && sub == 0) M.y[(int64_t)b * M.rows + row] = scale * acc;
+      M.y[(int64_t)b * M.rows + row] = scale * acc;
     }
   }
 }
@@ -619,10 +619,14 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   const bool hi2 = (a & 2) != 0, hi1 = (a & 1) != 0;
   const uint64_t pol = l2_policy_evict_first();
 
-  const int64_t u0 = (int64_t)blockIdx.x * P.total_units / gridDim.x;
-  const int64_t u1 = (int64_t)(blockIdx.x + 1) * P.total_units / gridDim.x;
+  int64_t u0 = (int64_t)blockIdx.x * P.total_units / gridDim.x;
+  int64_t u1 = (int64_t)(blockIdx.x + 1) * P.total_units / gridDim.x;
+  if (P.n_split == (int)gridDim.x) {  // ranges balanced by the host for units and table builds
+    u0 = P.cta_begin[blockIdx.x];
+    u1 = P.cta_begin[blockIdx.x + 1];
+  }
   griddep_launch_dependents();
-  if (u0 >= u1) {  // no units (cannot happen with grid <= units): only the reduction share
+  if (u0 >= u1) {  // no units: only the reduction share
     griddep_wait();
     reduce_slots(P, tid);
     return;
@@ -636,13 +640,15 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   __syncthreads();
   griddep_wait();  // inputs may be written by the preceding kernel in the stream
 
-  // Inputs of the first two tables go out before the index stream.
+  // The first table's inputs arrive before the index stream is started (so
+  // they do not queue behind it); its build then overlaps the first loads.
   uint32_t key_cur = ci.tkey;
   uint32_t key_next = key_cur == key_last ? kNoTable : next_table_key(P, key_cur);
   if (tid == 0) {
     stage_table<XDT>(P, key_cur, S, 0);
     if (key_next != kNoTable) stage_table<XDT>(P, key_next, S, 1);
   }
+  bool ok = mbar_wait_bounded(&S.mbar[0], 0);
 
   uint4 r[NSLOT][4];
   unsigned long long* sq[NSLOT];
@@ -665,7 +671,6 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   }
 
   // The first table is built at once, while the first index loads are in flight.
-  bool ok = mbar_wait_bounded(&S.mbar[0], 0);
   {
     const int nv = slab_columns(P, key_cur);
 #pragma unroll 1

@@ -168,6 +168,61 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
   return VQ3R_OK;
 }
 
+// Split the tiled kernel's units into n contiguous CTA ranges that balance
+// cost = units + kTableCost * tables built, a table being the (group, slab,
+// stage, token) run of G.tiles consecutive units.  Binary search on the
+// largest range cost; for a given budget, ranges are filled greedily table by
+// table.  Writes P.cta_begin[0..n] and P.n_split = n (ranges past the last
+// unit are empty).
+constexpr int64_t kTableCost = 2;  // one table build costs about two units of streaming and lookups
+
+int64_t split_ranges(const GvParams& P, int64_t budget, int n, int64_t* begin) {
+  int used = 0;
+  int64_t unit = 0, cost = budget;  // cost of the open range; budget forces a new range first
+  for (int g = 0; g < P.n_groups; g++) {
+    const GvGroup& G = P.g[g];
+    const int64_t n_tables = (int64_t)G.n_slabs * kStages * P.B;
+    for (int64_t t = 0; t < n_tables; t++) {
+      int64_t left = G.tiles;
+      bool fresh = true;  // this table not yet charged to the open range
+      while (left > 0) {
+        if (cost + (fresh ? kTableCost : 0) + 1 > budget) {  // open a new range here
+          if (begin && used <= n) begin[used] = unit;
+          used++;
+          cost = 0;
+          fresh = true;
+        }
+        if (fresh) {
+          cost += kTableCost;
+          fresh = false;
+        }
+        int64_t take = budget - cost;
+        if (take > left) take = left;
+        if (take < 1) take = 1;
+        cost += take;
+        unit += take;
+        left -= take;
+      }
+    }
+  }
+  return used;
+}
+
+void balance_split(GvParams& P, int n) {
+  P.n_split = 0;
+  if (n < 1 || n > kMaxSplit) return;
+  int64_t lo = (P.total_units + n - 1) / n + kTableCost;  // no range can cost less
+  int64_t hi = P.total_units + kTableCost * P.total_units;  // one range holds everything
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo) / 2;
+    if (split_ranges(P, mid, n, nullptr) <= n) hi = mid;
+    else lo = mid + 1;
+  }
+  const int64_t used = split_ranges(P, lo, n, P.cta_begin);
+  for (int64_t c = used; c <= n; c++) P.cta_begin[c] = P.total_units;
+  P.n_split = n;
+}
+
 template <int DT>
 vq3r_status launch_encode(const void* W, int64_t rows, int64_t cols, const float* cb, uint8_t* idx,
                           uint16_t* scales, cudaStream_t s, int sms) {
@@ -278,7 +333,9 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
   if (P.layout == VQ3R_LAYOUT_TILES) {  // one CTA per SM
-    cfg.gridDim = dim3((unsigned)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms));
+    const int grid = (int)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms);
+    balance_split(plan.P, grid);
+    cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kGvThreads);
     cfg.dynamicSmemBytes = kTilesSmemBytes;
     switch (x_dtype) {
