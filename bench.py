@@ -132,6 +132,15 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workload
 
+def layer_gemv_bytes(B, experts):
+    """Algorithmic bytes of one GEMV call over the stacked matrices of every expert of the layer."""
+    total = 0
+    for k in (wl.W1, wl.W3, wl.W2):
+        rows, cols = wl.mat_shape(k)
+        total += experts * (3 * rows * cols // 8 + 2 * rows + 4 * B * rows) + 2 * B * cols
+    return total
+
+
 def moe_step_bytes(B, n_exp=8):
     """Algorithmic bytes of one MoE decode step: index planes, scales, x, y."""
     gu_rows, gu_cols = wl.mat_shape(wl.W1)
@@ -228,7 +237,28 @@ class Layer:
         if st:
             raise self.vq.VQ3RError(st, "vq3r_gemv")
 
-    LAUNCHES_PER_STEP = 3 * 2 + 3 + 3 * 1 + 3 * 2 + 2  # encode, pack, decode, error, gemv (kernels)
+    def layer_gemv_plan(self, B):
+        """One grouped call over the stacked w1, w3, w2 of every expert of the layer (shared x per kind):
+        the steady-state rate of the GEMV kernel, with the per-call start and reduction amortised."""
+        _, _, xu, xd = self.moe[B]
+        mats = []
+        for k in self.kinds:
+            rows, cols = wl.mat_shape(k)
+            mats.append(dict(idx=self.tiles[k], scales=self.sc[k], codebooks=self.cb, x=xu if cols == wl.HIDDEN else xd[0],
+                             rows=self.E * rows, layout="tiles", cols=cols,
+                             y=self.torch.empty((B, self.E * rows), dtype=self.torch.float32, device=self.dev)))
+        d = self.vq._descs(mats)
+        ws = self.torch.empty(self.vq.lib().vq3r_gemv_workspace_size(d, len(mats), B), dtype=self.torch.uint8,
+                              device=self.dev)
+        return d, len(mats), ws, mats
+
+    def layer_gemv(self, plan, B):
+        d, n, ws, _ = plan
+        st = self.vq.lib().vq3r_gemv(d, n, B, 1, ws.data_ptr(), ws.numel(), self.torch.cuda.current_stream().cuda_stream)
+        if st:
+            raise self.vq.VQ3RError(st, "vq3r_gemv")
+
+    LAUNCHES_PER_STEP = 3 * 2 + 3 + 3 * 1 + 3 * 2 + 1  # encode, pack, decode, error, gemv (kernels)
 
 
 # ----------------------------------------------------------------------------- CPU oracle sample
@@ -412,6 +442,25 @@ def main():
         gemv[str(B)] = {"us_per_step": 1e3 * ms, "GB/s": gbs, "frac_hbm": gbs / hbm_gbs,
                         "tokens_per_s": B / ms * 1e3}
 
+    # the same kernel over the whole layer in one call (all experts' indices, 3 stacked matrices)
+    layer_sweep = {}
+    for B in B_list:
+        plan = layer.layer_gemv_plan(B)
+        for i in range(2):
+            layer.layer_gemv(plan, B)
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        iters = 10 if B <= 8 else 3
+        a.record()
+        for i in range(iters):
+            layer.layer_gemv(plan, B)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / iters
+        nbytes = layer_gemv_bytes(B, layer.E)
+        layer_sweep[str(B)] = {"us_per_call": 1e3 * ms, "GB/s": nbytes / ms / 1e6, "frac_hbm": nbytes / ms / 1e6 / hbm_gbs}
+        del plan
+
     # end to end through the public API with host buffers: H2D of the layer, the step, D2H of the results
     e2e = None
     if args.e2e_steps > 0:
@@ -488,6 +537,7 @@ def main():
                 "gemv_in_step_B1": {"us": 1e3 * gv1_ms, "GB/s": moe_step_bytes(1) / gv1_ms / 1e6,
                                     "frac_hbm": moe_step_bytes(1) / gv1_ms / 1e6 / hbm_gbs},
                 "gemv_sweep": gemv,
+                "gemv_layer_sweep": layer_sweep,
                 "hbm_peak_gbs": hbm_gbs, "peak_source": peak_src},
             "e2e": e2e,
             "gpu_launches": Layer.LAUNCHES_PER_STEP * args.steps,

@@ -565,28 +565,28 @@ __device__ __forceinline__ float sum_slots(const unsigned long long* sp, int64_t
 
 // y[b][i] = scale_i * sum over k = s * n_slabs + slab of the slots of row i,
 // added in k order by the row's lane, in load batches of up to 24 slots.
+// Work items are (output block, token) pairs dealt to warps round-robin.
 __device__ __forceinline__ void reduce_slots(const GvParams& P, int tid) {
   const int lane = tid & 31;
   const int warps = gridDim.x * kGvWarps;
-  for (int blk = blockIdx.x * kGvWarps + (tid >> 5); blk < P.red_blocks; blk += warps) {
+  const int64_t items = (int64_t)P.red_blocks * P.B;  // (block, token) pairs
+  for (int64_t it = (int64_t)blockIdx.x * kGvWarps + (tid >> 5); it < items; it += warps) {
+    const int blk = (int)(it / P.B), b = (int)(it - (int64_t)blk * P.B);
     int m = 0;
     while (m + 1 < P.n_mats && P.m[m + 1].red_begin <= blk) m++;
     const GvMat& M = P.m[m];
     const int64_t row = (int64_t)(blk - M.red_begin) * kRedRows + lane;
     if (row >= M.rows) continue;
     const int np = kStages * P.g[M.group].n_slabs;
-    const float scale = f16_bits_to_f32(__ldg(M.scales + row));
-    for (int b = 0; b < P.B; b++) {
-      const unsigned long long* sp = static_cast<const unsigned long long*>(M.partial) + (int64_t)b * np * M.rows + row;
-      float acc;
-      if (np <= 12) {
-        acc = sum_slots<12>(sp, M.rows, np, 0, P.epoch);
-      } else {
-        acc = 0.0f;
-        for (int k0 = 0; k0 < np; k0 += 24) acc += sum_slots<24>(sp, M.rows, np, k0, P.epoch);
-      }
-      M.y[(int64_t)b * M.rows + row] = scale * acc;
+    const unsigned long long* sp = static_cast<const unsigned long long*>(M.partial) + (int64_t)b * np * M.rows + row;
+    float acc;
+    if (np <= 12) {
+      acc = sum_slots<12>(sp, M.rows, np, 0, P.epoch);
+    } else {
+      acc = 0.0f;
+      for (int k0 = 0; k0 < np; k0 += 24) acc += sum_slots<24>(sp, M.rows, np, k0, P.epoch);
     }
+    M.y[(int64_t)b * M.rows + row] = f16_bits_to_f32(__ldg(M.scales + row)) * acc;
   }
 }
 
