@@ -209,7 +209,8 @@ vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const ui
  * library routine).
  *   - A call whose vq3r_gemv_workspace_size() exceeds 16 MiB returns
  *     VQ3R_ERR_WORKSPACE before launching anything (the 8-expert MoE decode
- *     step of 2048 x 7168 / 7168 x 2048 matrices fits for B = 1 and 2).
+ *     step of 2048 x 7168 / 7168 x 2048 matrices in the TILES layout needs
+ *     15.75 MiB at B = 1 as one call, 10.5 MiB for its gate/up half).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before capturing a stream into a graph.
