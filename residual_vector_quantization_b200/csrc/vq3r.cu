@@ -7,6 +7,7 @@
 #include "decode.cuh"
 #include "encode.cuh"
 #include "gemv.cuh"
+#include "gemv_mma.cuh"
 #include "vq3r_common.cuh"
 
 using namespace vq3r;
@@ -60,6 +61,11 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F32, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_BF16, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
+    const int gm = (int)kMmaSmemBytes;
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     g_dev_err[dev] = r;
   });
   *sms = g_dev_sms[dev];
@@ -332,6 +338,27 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   cfg.stream = s;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
+  if (P.layout == VQ3R_LAYOUT_TILES && x_dtype == VQ3R_BF16 && B >= kMmaMinB) {
+    // Several tokens: rebuild the weights and contract on the tensor cores.
+    // One CTA per 128 rows of a matrix; red_begin numbers those blocks.
+    int64_t blocks = 0;
+    for (int i = 0; i < P.n_mats; i++) {
+      plan.P.m[i].red_begin = (int32_t)blocks;
+      blocks += (P.m[i].rows + kMmaRows - 1) / kMmaRows;
+    }
+    if (blocks >= ((int64_t)1 << 31)) return VQ3R_ERR_SHAPE;
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(kMmaThreads);
+    cfg.dynamicSmemBytes = kMmaSmemBytes;
+    switch ((B + 7) / 8) {
+      case 1: e = cudaLaunchKernelEx(&cfg, gemv_mma_kernel<1>, P); break;
+      case 2: e = cudaLaunchKernelEx(&cfg, gemv_mma_kernel<2>, P); break;
+      case 3: e = cudaLaunchKernelEx(&cfg, gemv_mma_kernel<3>, P); break;
+      default: e = cudaLaunchKernelEx(&cfg, gemv_mma_kernel<4>, P); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
+    return check_launch();
+  }
   if (P.layout == VQ3R_LAYOUT_TILES) {  // one CTA per SM
     const int grid = (int)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms);
     balance_split(plan.P, grid);

@@ -232,6 +232,34 @@ def test_grouped_gemv_mixed_matrices(layout):
         assert gemv_rel_err(m["y"].cpu().numpy(), ref) <= GEMV_TOL
 
 
+@pytest.mark.parametrize("B", [8, 9, 24, 32])
+def test_grouped_gemv_many_tokens(B):
+    """B >= 8 with bf16 x in the tiled layout runs on the tensor cores (weights rebuilt in bf16 hi + lo):
+    ragged rows (not multiples of 128), partial last slabs, partly filled 8-token tiles, mixed groups."""
+    rng = np.random.default_rng(80 + B)
+    specs = [(300, 1032, 0, 0), (129, 1032, 0, 0), (64, 200, 1, 1), (513, 2048, 2, 0), (33, 1032, 0, 2)]
+    xs = {}
+    mats, refs = [], []
+    for rows, cols, cbk, xk in specs:
+        cb = random_codebooks(300 + cbk)
+        if (xk, cols) not in xs:
+            xs[(xk, cols)] = f32_to_bf16_bits(rng.standard_normal((B, cols)).astype(np.float32))
+        x = xs[(xk, cols)]
+        W = f32_to_bf16_bits(rng.standard_normal((rows, cols)).astype(np.float32))
+        W_t, idx_t, sc_t, cb_t, idx_o, sc_o = check_encode_decode(W, "bf16", cb)
+        y_t = torch.full((B, rows), float("nan"), dtype=torch.float32, device=DEV)
+        mats.append(dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=None, y=y_t, key=(xk, cols)))
+        refs.append(oracle.gemv(oracle.decode(idx_o, sc_o, cb), x, "bf16"))
+    xdev = {k: to_dev(v, "bf16") for k, v in xs.items()}
+    for m in mats:
+        m["x"] = xdev[m.pop("key")]
+    vq.vq3r_gemv(as_layout(mats, "tiles"), B)
+    for m, ref in zip(mats, refs):
+        y = m["y"].cpu().numpy()
+        assert np.isfinite(y).all()  # every output written
+        assert gemv_rel_err(y, ref) <= GEMV_TOL
+
+
 # ------------------------------------------------------------------ error statuses
 
 def test_error_statuses():
