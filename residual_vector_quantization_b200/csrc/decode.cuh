@@ -15,66 +15,124 @@
 
 namespace vq3r {
 
-constexpr int kDecThreads = 256;
+constexpr int kDecThreads = 512;
 
-// Codebooks staged in shared memory (plain loads: 24 KiB, once per CTA).
-__device__ __forceinline__ void load_codebooks_smem(float* cb, const float* __restrict__ codebooks) {
+// Codebooks for gathers by 32 lanes: every codeword stored four times side by
+// side in a 128-byte row, cbr[s][j][copy][8].  Lane L reads copy (L >> 1) & 3,
+// half L & 1, so the eight lanes of a quarter-warp hit eight distinct 16-byte
+// bank groups whatever the indices are.  96 KiB.
+constexpr int kCbrFloats = kStages * kCodewords * 4 * kDim;
+__device__ __forceinline__ void load_codebooks_replicated(float* cbr, const float* __restrict__ codebooks) {
   const float4* src = reinterpret_cast<const float4*>(codebooks);
-  float4* dst = reinterpret_cast<float4*>(cb);
-  for (int i = threadIdx.x; i < kCodebookFloats / 4; i += blockDim.x) dst[i] = __ldg(src + i);
+  float4* dst = reinterpret_cast<float4*>(cbr);
+  for (int i = threadIdx.x; i < kCodebookFloats / 4; i += blockDim.x) {  // i: half of codeword i >> 1
+    const float4 v = __ldg(src + i);
+#pragma unroll
+    for (int c = 0; c < 4; c++) dst[((i >> 1) * 4 + c) * 2 + (i & 1)] = v;
+  }
   __syncthreads();
 }
 
-// w_hat of one vector: (float)scale * ((C1 + C2) + C3), each operation rounded.
-__device__ __forceinline__ void decode_vector(const float* cb, uint32_t i1, uint32_t i2, uint32_t i3, float s,
-                                              float out[8]) {
-  const float4* c1 = reinterpret_cast<const float4*>(cb + (0 * kCodewords + i1) * kDim);
-  const float4* c2 = reinterpret_cast<const float4*>(cb + (1 * kCodewords + i2) * kDim);
-  const float4* c3 = reinterpret_cast<const float4*>(cb + (2 * kCodewords + i3) * kDim);
-#pragma unroll
-  for (int h = 0; h < 2; h++) {
-    const float4 a = c1[h], b = c2[h], c = c3[h];
-    out[4 * h + 0] = __fmul_rn(s, __fadd_rn(__fadd_rn(a.x, b.x), c.x));
-    out[4 * h + 1] = __fmul_rn(s, __fadd_rn(__fadd_rn(a.y, b.y), c.y));
-    out[4 * h + 2] = __fmul_rn(s, __fadd_rn(__fadd_rn(a.z, b.z), c.z));
-    out[4 * h + 3] = __fmul_rn(s, __fadd_rn(__fadd_rn(a.w, b.w), c.w));
+// Half h = L & 1 (elements 4h .. 4h + 3) of w_hat for one vector:
+// (float)scale * ((C1 + C2) + C3), each operation rounded.
+__device__ __forceinline__ float4 decode_half_r(const float* cbr, uint32_t i1, uint32_t i2, uint32_t i3, float s,
+                                                int lane) {
+  const int off = ((lane >> 1) & 3) * kDim + 4 * (lane & 1);
+  const float4 a = *reinterpret_cast<const float4*>(cbr + (0 * kCodewords + i1) * 4 * kDim + off);
+  const float4 b = *reinterpret_cast<const float4*>(cbr + (1 * kCodewords + i2) * 4 * kDim + off);
+  const float4 c = *reinterpret_cast<const float4*>(cbr + (2 * kCodewords + i3) * 4 * kDim + off);
+  return make_float4(__fmul_rn(s, __fadd_rn(__fadd_rn(a.x, b.x), c.x)), __fmul_rn(s, __fadd_rn(__fadd_rn(a.y, b.y), c.y)),
+                     __fmul_rn(s, __fadd_rn(__fadd_rn(a.z, b.z), c.z)), __fmul_rn(s, __fadd_rn(__fadd_rn(a.w, b.w), c.w)));
+}
+
+// Traversal shared by decode and the error kernel.  Rows are split evenly over
+// the CTAs.  Two lanes take one vector (lane parity = half), so a warp covers
+// 16 consecutive vectors and its 16-byte stores form one 512-byte span.  The
+// CTA's threads / 2 vectors per step walk its rows in order; (row, v) advance
+// by that many vectors per step with no division.
+struct RowWalk {
+  int64_t row, v;     // current vector of this thread
+  int64_t V, dq, dr;  // vectors per row; step = dq * V + dr
+  __device__ __forceinline__ void init(int64_t r0, int64_t V_, int tid, int threads) {
+    V = V_;
+    const int64_t step = threads / 2, v0 = tid >> 1;
+    row = r0 + v0 / V;
+    v = v0 - (v0 / V) * V;
+    dq = step / V;
+    dr = step - dq * V;
   }
+  __device__ __forceinline__ void next() {
+    row += dq;
+    v += dr;
+    if (v >= V) {
+      v -= V;
+      row++;
+    }
+  }
+};
+
+constexpr int kWalkUnroll = 4;  // walk positions per thread whose loads are issued together
+
+// The next kWalkUnroll positions of a walk (rows at or past r1 are marked
+// invalid) with their index bytes and row scales, all loads issued before use.
+struct WalkBatch {
+  int64_t g[kWalkUnroll];
+  uint32_t e[kWalkUnroll][3];
+  float s[kWalkUnroll];
+  bool ok[kWalkUnroll];
+};
+__device__ __forceinline__ bool walk_batch(RowWalk& it, int64_t r1, const uint8_t* __restrict__ idx, int64_t nvec,
+                                           const uint16_t* __restrict__ scales, WalkBatch& wb) {
+  if (it.row >= r1) return false;
+#pragma unroll
+  for (int u = 0; u < kWalkUnroll; u++) {
+    wb.ok[u] = it.row < r1;
+    const int64_t row = wb.ok[u] ? it.row : r1 - 1, v = wb.ok[u] ? it.v : 0;  // clamped: always a valid address
+    wb.g[u] = row * it.V + v;
+    wb.e[u][0] = __ldcs(idx + wb.g[u]);
+    wb.e[u][1] = __ldcs(idx + nvec + wb.g[u]);
+    wb.e[u][2] = __ldcs(idx + 2 * nvec + wb.g[u]);
+    wb.s[u] = f16_bits_to_f32(__ldg(scales + row));
+    it.next();
+  }
+  return true;
 }
 
 template <int OUT_DT>
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(const uint8_t* __restrict__ idx,
-                                                              const uint16_t* __restrict__ scales,
-                                                              const float* __restrict__ codebooks, int64_t cols,
-                                                              int64_t nvec, void* __restrict__ out) {
-  __shared__ __align__(16) float cb[kCodebookFloats];
-  load_codebooks_smem(cb, codebooks);
-  const int64_t V = cols / kDim;
-  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < nvec; g += (int64_t)gridDim.x * blockDim.x) {
-    const uint32_t i1 = __ldcs(idx + g), i2 = __ldcs(idx + nvec + g), i3 = __ldcs(idx + 2 * nvec + g);
-    const int64_t row = g / V;
-    const float s = f16_bits_to_f32(__ldg(scales + row));
-    float w[8];
-    decode_vector(cb, i1, i2, i3, s, w);
-    if constexpr (OUT_DT == VQ3R_F32) {
-      float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + g * kDim);
-      __stcs(o, make_float4(w[0], w[1], w[2], w[3]));
-      __stcs(o + 1, make_float4(w[4], w[5], w[6], w[7]));
-    } else {
-      uint32_t u[4];
+__global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const uint8_t* __restrict__ idx,
+                                                                 const uint16_t* __restrict__ scales,
+                                                                 const float* __restrict__ codebooks, int64_t rows,
+                                                                 int64_t cols, void* __restrict__ out) {
+  extern __shared__ __align__(16) float cbr[];
+  load_codebooks_replicated(cbr, codebooks);
+  const int lane = threadIdx.x & 31, h = lane & 1;
+  const int64_t V = cols / kDim, nvec = rows * V;
+  const int64_t r0 = (int64_t)blockIdx.x * rows / gridDim.x, r1 = (int64_t)(blockIdx.x + 1) * rows / gridDim.x;
+  RowWalk it;
+  it.init(r0, V, threadIdx.x, kDecThreads);
+  WalkBatch wb;
+  while (walk_batch(it, r1, idx, nvec, scales, wb)) {
 #pragma unroll
-      for (int i = 0; i < 4; i++) {
-        const uint32_t lo = __half_as_ushort(__float2half_rn(w[2 * i]));
-        const uint32_t hi = __half_as_ushort(__float2half_rn(w[2 * i + 1]));
-        u[i] = lo | (hi << 16);
+    for (int u = 0; u < kWalkUnroll; u++) {
+      if (!wb.ok[u]) continue;
+      const int64_t g = wb.g[u];
+      const float4 o = decode_half_r(cbr, wb.e[u][0], wb.e[u][1], wb.e[u][2], wb.s[u], lane);
+      if constexpr (OUT_DT == VQ3R_F32) {
+        __stcs(reinterpret_cast<float4*>(static_cast<float*>(out) + g * kDim + 4 * h), o);
+      } else {
+        const uint32_t u0 = (uint32_t)__half_as_ushort(__float2half_rn(o.x)) |
+                            ((uint32_t)__half_as_ushort(__float2half_rn(o.y)) << 16);
+        const uint32_t u1 = (uint32_t)__half_as_ushort(__float2half_rn(o.z)) |
+                            ((uint32_t)__half_as_ushort(__float2half_rn(o.w)) << 16);
+        __stcs(reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + g * kDim + 4 * h), make_uint2(u0, u1));
       }
-      __stcs(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + g * kDim), make_uint4(u[0], u[1], u[2], u[3]));
     }
   }
 }
 
 // ---- relative Frobenius error: per-CTA binary64 partials, then one CTA ----
 
-constexpr int kErrThreads = 256;
+constexpr int kErrThreads = 512;
 
 __device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
@@ -82,35 +140,93 @@ __device__ __forceinline__ double warp_sum_f64(double v) {
   return v;
 }
 
+// Whole w_hat vector for one lane: both halves, the lane's copy of each
+// codeword, half L & 1 first (conflict-free order for a quarter-warp).
+__device__ __forceinline__ void decode_vector_r(const float* cbr, uint32_t i1, uint32_t i2, uint32_t i3, float s,
+                                                int lane, float4& lo, float4& hi) {
+  const int copy = (lane >> 1) & 3, h0 = lane & 1;
+  const float4* c1 = reinterpret_cast<const float4*>(cbr + ((0 * kCodewords + i1) * 4 + copy) * kDim);
+  const float4* c2 = reinterpret_cast<const float4*>(cbr + ((1 * kCodewords + i2) * 4 + copy) * kDim);
+  const float4* c3 = reinterpret_cast<const float4*>(cbr + ((2 * kCodewords + i3) * 4 + copy) * kDim);
+  const float4 a0 = c1[h0], b0 = c2[h0], d0 = c3[h0];
+  const float4 a1 = c1[h0 ^ 1], b1 = c2[h0 ^ 1], d1 = c3[h0 ^ 1];
+  const float4 first = make_float4(__fmul_rn(s, __fadd_rn(__fadd_rn(a0.x, b0.x), d0.x)), __fmul_rn(s, __fadd_rn(__fadd_rn(a0.y, b0.y), d0.y)),
+                                   __fmul_rn(s, __fadd_rn(__fadd_rn(a0.z, b0.z), d0.z)), __fmul_rn(s, __fadd_rn(__fadd_rn(a0.w, b0.w), d0.w)));
+  const float4 second = make_float4(__fmul_rn(s, __fadd_rn(__fadd_rn(a1.x, b1.x), d1.x)), __fmul_rn(s, __fadd_rn(__fadd_rn(a1.y, b1.y), d1.y)),
+                                    __fmul_rn(s, __fadd_rn(__fadd_rn(a1.z, b1.z), d1.z)), __fmul_rn(s, __fadd_rn(__fadd_rn(a1.w, b1.w), d1.w)));
+  lo = h0 ? second : first;
+  hi = h0 ? first : second;
+}
+
+__device__ __forceinline__ void acc_err(double& num, double& den, float w, float wh) {
+  const double e = (double)w - (double)wh;
+  num = fma(e, e, num);
+  den = fma((double)w, (double)w, den);
+}
+
+constexpr int kErrVecs = 4;  // consecutive vectors per thread and step
+
+// Rows are split evenly over the CTAs.  A CTA numbers the 4-vector groups of
+// its rows consecutively (row-major, at most 2^31 of them) and thread t takes
+// groups t, t + 512, ...: the index bytes of a group are one 32-bit word per
+// plane when V is a multiple of 4, and a warp's 16-byte W loads are 512
+// contiguous bytes.  Each thread keeps two binary64 sums, reduced per CTA.
 template <int DT>
-__global__ void __launch_bounds__(kErrThreads) relfro_partial_kernel(const void* __restrict__ W,
-                                                                      const uint8_t* __restrict__ idx,
-                                                                      const uint16_t* __restrict__ scales,
-                                                                      const float* __restrict__ codebooks,
-                                                                      int64_t cols, int64_t nvec,
-                                                                      double* __restrict__ partial) {
-  __shared__ __align__(16) float cb[kCodebookFloats];
+__global__ void __launch_bounds__(kErrThreads, 2) relfro_partial_kernel(const void* __restrict__ W,
+                                                                         const uint8_t* __restrict__ idx,
+                                                                         const uint16_t* __restrict__ scales,
+                                                                         const float* __restrict__ codebooks,
+                                                                         int64_t rows, int64_t cols,
+                                                                         double* __restrict__ partial) {
+  extern __shared__ __align__(16) float cbr[];
   __shared__ double red[2][kErrThreads / 32];
-  load_codebooks_smem(cb, codebooks);
-  const int64_t V = cols / kDim;
+  load_codebooks_replicated(cbr, codebooks);
+  const int lane = threadIdx.x & 31;
+  const int64_t V = cols / kDim, nvec = rows * V;
+  const uint32_t gpr = (uint32_t)((V + kErrVecs - 1) / kErrVecs);  // groups per row
+  const bool vec4 = (V % kErrVecs) == 0;
+  const int64_t r0 = (int64_t)blockIdx.x * rows / gridDim.x, r1 = (int64_t)(blockIdx.x + 1) * rows / gridDim.x;
+  const uint32_t nf = (uint32_t)((r1 - r0) * gpr);
   double num = 0.0, den = 0.0;
-  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < nvec; g += (int64_t)gridDim.x * blockDim.x) {
-    const uint32_t i1 = __ldcs(idx + g), i2 = __ldcs(idx + nvec + g), i3 = __ldcs(idx + 2 * nvec + g);
-    const int64_t row = g / V;
+  for (uint32_t f = threadIdx.x; f < nf; f += kErrThreads) {
+    const uint32_t rl = f / gpr, q = f - rl * gpr;
+    const int64_t row = r0 + rl;
+    const int64_t g = row * V + (int64_t)q * kErrVecs;
+    const int n = (int)((V - (int64_t)q * kErrVecs) < kErrVecs ? (V - (int64_t)q * kErrVecs) : kErrVecs);
     const float s = f16_bits_to_f32(__ldg(scales + row));
-    float wh[8], w[8];
-    decode_vector(cb, i1, i2, i3, s, wh);
-    load8<DT>(W, g * kDim, w);
+    uint32_t w3[3];
 #pragma unroll
-    for (int k = 0; k < 8; k++) {
-      const double e = (double)w[k] - (double)wh[k];
-      num = fma(e, e, num);
-      den = fma((double)w[k], (double)w[k], den);
+    for (int st = 0; st < kStages; st++) {
+      if (vec4) {
+        w3[st] = __ldcs(reinterpret_cast<const unsigned int*>(idx + st * nvec + g));
+      } else {
+        uint32_t x = 0;
+        for (int i = 0; i < n; i++) x |= (uint32_t)__ldcs(idx + st * nvec + g + i) << (8 * i);
+        w3[st] = x;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kErrVecs; i++) {
+      if (i < n) {
+        float4 lo, hi;
+        decode_vector_r(cbr, (w3[0] >> (8 * i)) & 0xFFu, (w3[1] >> (8 * i)) & 0xFFu, (w3[2] >> (8 * i)) & 0xFFu, s, lane,
+                        lo, hi);
+        float wv[8];
+        load8<DT>(W, (g + i) * kDim, wv);
+        acc_err(num, den, wv[0], lo.x);
+        acc_err(num, den, wv[1], lo.y);
+        acc_err(num, den, wv[2], lo.z);
+        acc_err(num, den, wv[3], lo.w);
+        acc_err(num, den, wv[4], hi.x);
+        acc_err(num, den, wv[5], hi.y);
+        acc_err(num, den, wv[6], hi.z);
+        acc_err(num, den, wv[7], hi.w);
+      }
     }
   }
   num = warp_sum_f64(num);
   den = warp_sum_f64(den);
-  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
   if (lane == 0) { red[0][wid] = num; red[1][wid] = den; }
   __syncthreads();
   if (threadIdx.x == 0) {

@@ -62,6 +62,12 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_BF16, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
     const int gm = (int)kMmaSmemBytes;
+    const int gc = (int)(kCbrFloats * sizeof(float));
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
@@ -241,13 +247,25 @@ vq3r_status launch_encode(const void* W, int64_t rows, int64_t cols, const float
   return check_launch();
 }
 
-template <int DT>
-vq3r_status launch_relfro(const void* W, const uint8_t* idx, const uint16_t* scales, const float* cb, int64_t cols,
-                          int64_t nvec, double* err_out, double* partial, cudaStream_t s, int sms) {
-  int64_t blocks = (nvec + kErrThreads - 1) / kErrThreads;
-  const int64_t cap = (int64_t)sms * 8 < kErrMaxBlocks ? (int64_t)sms * 8 : kErrMaxBlocks;
+// CTAs for the row-split decode and error kernels: two per SM (96 KiB of
+// replicated codebooks each), more when a CTA's share of 4-vector groups
+// would not fit 32 bits; never more than rows or cap.
+int64_t rowsplit_blocks(int64_t rows, int64_t cols, int sms, int64_t cap) {
+  int64_t blocks = 2 * (int64_t)sms;
+  // the error kernel counts a CTA's 4-vector groups in 32 bits
+  const int64_t need = rows * ((cols / kDim + kErrVecs - 1) / kErrVecs) / ((int64_t)1 << 30) + 1;
+  if (blocks < need) blocks = need;
   if (blocks > cap) blocks = cap;
-  relfro_partial_kernel<DT><<<(int)blocks, kErrThreads, 0, s>>>(W, idx, scales, cb, cols, nvec, partial);
+  if (blocks > rows) blocks = rows;
+  return blocks;
+}
+
+template <int DT>
+vq3r_status launch_relfro(const void* W, const uint8_t* idx, const uint16_t* scales, const float* cb, int64_t rows,
+                          int64_t cols, double* err_out, double* partial, cudaStream_t s, int sms) {
+  const int64_t blocks = rowsplit_blocks(rows, cols, sms, kErrMaxBlocks);
+  relfro_partial_kernel<DT><<<(int)blocks, kErrThreads, kCbrFloats * sizeof(float), s>>>(W, idx, scales, cb, rows,
+                                                                                          cols, partial);
   relfro_final_kernel<<<1, 256, 0, s>>>(partial, (int)blocks, err_out);
   return check_launch();
 }
@@ -287,13 +305,12 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
   cudaError_t e = device_setup(&sms);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int64_t nvec = rows * (cols / kDim);
-  int64_t blocks = (nvec + kDecThreads - 1) / kDecThreads;
-  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+  const int64_t blocks = rowsplit_blocks(rows, cols, sms, (int64_t)1 << 30);
+  const size_t smem = kCbrFloats * sizeof(float);
   if (out_dtype == VQ3R_F32)
-    decode_kernel<VQ3R_F32><<<(int)blocks, kDecThreads, 0, s>>>(idx, scales, codebooks, cols, nvec, out);
+    decode_kernel<VQ3R_F32><<<(int)blocks, kDecThreads, smem, s>>>(idx, scales, codebooks, rows, cols, out);
   else
-    decode_kernel<VQ3R_F16><<<(int)blocks, kDecThreads, 0, s>>>(idx, scales, codebooks, cols, nvec, out);
+    decode_kernel<VQ3R_F16><<<(int)blocks, kDecThreads, smem, s>>>(idx, scales, codebooks, rows, cols, out);
   return check_launch();
 }
 
@@ -443,12 +460,11 @@ vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const ui
   cudaError_t e = device_setup(&sms);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int64_t nvec = rows * (cols / kDim);
   double* partial = static_cast<double*>(workspace);
   switch (w_dtype) {
-    case VQ3R_F32: return launch_relfro<VQ3R_F32>(W, idx, scales, codebooks, cols, nvec, err_out, partial, s, sms);
-    case VQ3R_BF16: return launch_relfro<VQ3R_BF16>(W, idx, scales, codebooks, cols, nvec, err_out, partial, s, sms);
-    default: return launch_relfro<VQ3R_F16>(W, idx, scales, codebooks, cols, nvec, err_out, partial, s, sms);
+    case VQ3R_F32: return launch_relfro<VQ3R_F32>(W, idx, scales, codebooks, rows, cols, err_out, partial, s, sms);
+    case VQ3R_BF16: return launch_relfro<VQ3R_BF16>(W, idx, scales, codebooks, rows, cols, err_out, partial, s, sms);
+    default: return launch_relfro<VQ3R_F16>(W, idx, scales, codebooks, rows, cols, err_out, partial, s, sms);
   }
 }
 
