@@ -753,31 +753,41 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
 }
 
 // Repack the index planes [3][rows][cols/8] (plane_stride bytes apart) into
-// the tiled layout; one thread per 16-byte chunk of the output.
+// the tiled layout; one thread per 16-byte chunk of the output.  The chunk's 16
+// source columns are contiguous in the plane: one aligned 16-byte load when V
+// and plane_stride are multiples of 16 and the chunk lies inside the row,
+// byte loads otherwise.  Blocks are numbered below 2^32.
 __global__ void __launch_bounds__(256) pack_tiles_kernel(const uint8_t* __restrict__ idx, int64_t rows, int64_t V,
                                                           int64_t plane_stride, int32_t n_slabs, int64_t n_tiles,
                                                           uint8_t* __restrict__ out) {
   const int64_t n_chunks = (int64_t)kStages * n_slabs * n_tiles * (kTileBytes / 16);
+  const bool vec = (V % 16) == 0 && (plane_stride % 16) == 0 && (reinterpret_cast<uintptr_t>(idx) % 16) == 0;
+  const uint32_t nt = (uint32_t)n_tiles, ns = (uint32_t)n_slabs;
   for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < n_chunks; q += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t blk = q / (kTileBytes / 16);
-    const int within = (int)(q - blk * (kTileBytes / 16));
+    const uint32_t blk = (uint32_t)(q >> 11);  // kTileBytes / 16 = 2048 chunks per block
+    const int within = (int)(q & 2047);
     const int r = within >> 2, ch = within & 3;  // packed row, 16-byte chunk
-    const int64_t tile = blk % n_tiles;
-    const int64_t sc = blk / n_tiles;
-    const int slab = (int)(sc % n_slabs), s = (int)(sc / n_slabs);
-    const int64_t row = tile * kTileRows + r;
-    uint32_t h[4] = {0u, 0u, 0u, 0u};  // the chunk's 16 columns in source order
+    const uint32_t sc = blk / nt, tile = blk - sc * nt;
+    const uint32_t s = sc / ns, slab = sc - s * ns;
+    const int64_t row = (int64_t)tile * kTileRows + r;
+    const int64_t col0 = (int64_t)slab * kSlabV + 16 * ch;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);  // the chunk's 16 columns in source order
     if (row < rows) {
-      const uint8_t* src = idx + s * plane_stride + row * V;
+      const uint8_t* src = idx + s * plane_stride + row * V + col0;
+      if (vec && col0 + 16 <= V) {
+        v = __ldg(reinterpret_cast<const uint4*>(src));
+      } else {
+        uint32_t h[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int i = 0; i < 16; i++) {
-        const int64_t col = (int64_t)slab * kSlabV + 16 * ch + i;
-        const uint32_t v = col < V ? (uint32_t)__ldg(src + col) : 0u;
-        h[i >> 2] |= v << (8 * (i & 3));
+        for (int i = 0; i < 16; i++) {
+          const uint32_t b = col0 + i < V ? (uint32_t)__ldg(src + i) : 0u;
+          h[i >> 2] |= b << (8 * (i & 3));
+        }
+        v = make_uint4(h[0], h[1], h[2], h[3]);
       }
     }
     const bool swap = (r >> 2) & 1;  // rows whose two 8-byte halves are stored swapped
-    reinterpret_cast<uint4*>(out)[q] = swap ? make_uint4(h[2], h[3], h[0], h[1]) : make_uint4(h[0], h[1], h[2], h[3]);
+    reinterpret_cast<uint4*>(out)[q] = swap ? make_uint4(v.z, v.w, v.x, v.y) : v;
   }
 }
 

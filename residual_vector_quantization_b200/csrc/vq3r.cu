@@ -431,6 +431,7 @@ vq3r_status vq3r_pack_tiles(const uint8_t* idx, int64_t rows, int64_t cols, int6
   if (e != cudaSuccess) return cuda_fail(e);
   const int32_t n_slabs = (int32_t)((cols / kDim + kSlabV - 1) / kSlabV);
   const int64_t n_tiles = (rows + kTileRows - 1) / kTileRows;
+  if ((int64_t)kStages * n_slabs * n_tiles >= ((int64_t)1 << 32)) return VQ3R_ERR_SHAPE;  // block numbers are 32-bit
   const int64_t chunks = (int64_t)kStages * n_slabs * n_tiles * (kTileBytes / 16);
   int64_t blocks = (chunks + 255) / 256;
   if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
