@@ -341,6 +341,28 @@ def run_reference(args, rank, world):
     print(json.dumps(out), flush=True)
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_expert0(rank, experts):
+    """First expert of a rank's layer: rank r encodes experts experts*r .. experts*r + experts - 1 (weak scaling;
+    the shards are disjoint, and each is the same data a single process would generate for those experts)."""
+    return rank * experts
+
+
+def max_over_ranks(torch, value, world, device):
+    """The slowest rank's time (every rank takes the same collective step)."""
+    if world == 1:
+        return value
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, weights_per_rank, ms):
+    """Gweights/s of the whole job: every rank's weights over the slowest rank's time."""
+    return world * weights_per_rank / ms / 1e6
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -369,7 +391,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     B_list = (1, 4, 8, 32)
-    layer = Layer(torch, vq, dev, args.experts, rank * args.experts, B_list)
+    layer = Layer(torch, vq, dev, args.experts, rank_expert0(rank, args.experts), B_list)
     torch.cuda.synchronize()
     hbm_gbs, sm_max_mhz, peak_src = peaks()
     props = torch.cuda.get_device_properties(dev)
@@ -413,11 +435,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    total_ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(torch, t0.elapsed_time(t1), world, dev)
     part = lambda a, b: [marks[i][a].elapsed_time(marks[i][b]) for i in range(args.steps)]  # noqa: E731
     enc_ms = statistics.mean(part(0, 1))
     pack_ms = statistics.mean(part(1, 2))
@@ -494,17 +512,13 @@ def main():
                 off += n
         b.record()
         torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b) / args.e2e_steps
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": world * layer.weights / e2e_ms / 1e6, "unit": "Gweights/s", "h2d_bytes_per_step": h2d,
+        e2e_ms = max_over_ranks(torch, a.elapsed_time(b) / args.e2e_steps, world, dev)
+        e2e = {"value": whole_job_rate(world, layer.weights, e2e_ms), "unit": "Gweights/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     errs = {str(k): float(layer.err[k].item()) for k in layer.kinds}
     ms_step = total_ms / args.steps
-    value = world * layer.weights / ms_step / 1e6  # Gweights/s over the whole path
+    value = whole_job_rate(world, layer.weights, ms_step)  # Gweights/s over the whole path
     enc_tflops = FLOPS_PER_WEIGHT * layer.weights / enc_ms / 1e9
     dev_err = vq.vq3r_device_error()
     if rank == 0:
