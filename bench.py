@@ -207,7 +207,7 @@ class Layer:
                 d = vq._descs(p1 + p2)
                 plans.append((d, len(p1) + len(p2), p1 + p2, vq.lib().vq3r_gemv_workspace_size(d, len(p1) + len(p2), B)))
             wsz = max(p[3] for p in plans)
-            ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+            ws = torch.zeros(wsz, dtype=torch.uint8, device=dev)
             self.moe[B] = (plans, ws, xu, xd)
 
     # --- the parts of a step (each enqueues on the current stream) ---
@@ -248,7 +248,7 @@ class Layer:
                              rows=self.E * rows, layout="tiles", cols=cols,
                              y=self.torch.empty((B, self.E * rows), dtype=self.torch.float32, device=self.dev)))
         d = self.vq._descs(mats)
-        ws = self.torch.empty(self.vq.lib().vq3r_gemv_workspace_size(d, len(mats), B), dtype=self.torch.uint8,
+        ws = self.torch.zeros(self.vq.lib().vq3r_gemv_workspace_size(d, len(mats), B), dtype=self.torch.uint8,
                               device=self.dev)
         return d, len(mats), ws, mats
 

@@ -114,11 +114,16 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
  * of all active experts builds each table once per SM that needs it.  y must
  * not overlap any input.
  *
- * Workspace: one partial sum per (token, stage, 64-column slab, row); PLANES
- * stores floats and adds them in a second kernel, TILES stores 64-bit slots
- * (call tag, float) and reduces them in the same kernel, each SM waiting
- * until the slots it adds carry this call's tag.  Nothing needs clearing
- * between calls.  The TILES kernel runs one CTA per SM and needs all of them
+ * Workspace: a 256-byte header, then one partial sum per (token, stage,
+ * 64-column slab, row).  PLANES stores floats and adds them in a second
+ * kernel; TILES stores 64-bit slots (call tag, float) and reduces them in the
+ * same kernel, each SM waiting until the slots it adds carry this call's
+ * tag.  The tag comes from a generation counter in the header that the last
+ * CTA of each TILES call advances, so consecutive calls on one workspace,
+ * replays of a captured CUDA graph included, never take each other's slots.
+ * Fill a workspace with zeros once before its first call (e.g.
+ * cudaMemsetAsync after allocating it); nothing needs clearing between
+ * calls.  The TILES kernel runs one CTA per SM and needs all of them
  * resident together: if another workload holds SMs for more than about a
  * second, the call finishes with vq3r_device_error() = 2 and y undefined.
  *   mats      HOST array of n_mats descriptors (copied before return)
@@ -216,9 +221,8 @@ vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const ui
  *     before capturing a stream into a graph.
  *   - All calls share the one array: calls that overlap on the GPU (different
  *     streams, or different host threads on the same device) race and must be
- *     serialised by the caller.  Every byte the kernels read from it is
- *     written earlier in the same call, so nothing needs clearing between
- *     calls.
+ *     serialised by the caller.  The array is zeroed when the library is
+ *     loaded, as vq3r_gemv requires of a new workspace.
  */
 #define VQ3R_GEMV_NOALLOC_BYTES (16u << 20)
 vq3r_status vq3r_gemv_noalloc(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype x_dtype, vq3r_stream stream);

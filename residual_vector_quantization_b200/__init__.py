@@ -183,7 +183,7 @@ def vq3r_gemv(mats, B, workspace=None, stream=None):
     arr = _descs(mats)
     ws = _lib().vq3r_gemv_workspace_size(arr, len(mats), B)
     if workspace is None:
-        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=mats[0]["idx"].device)
+        workspace = torch.zeros(max(ws, 16), dtype=torch.uint8, device=mats[0]["idx"].device)
     xdt = _DT[mats[0]["x"].dtype]
     _check(_lib().vq3r_gemv(arr, len(mats), B, xdt, _dev(workspace, "workspace"), workspace.numel(),
                             _stream(stream)), "vq3r_gemv")

@@ -100,7 +100,7 @@ struct GvParams {
   int64_t total_units;
   int32_t tile_rows;     // rows per work unit: kGvTileRows (planes) or kTileRows (tiles)
   int32_t layout;        // VQ3R_LAYOUT_PLANES or VQ3R_LAYOUT_TILES
-  uint32_t epoch;        // tiles: tag of this call's partial-sum slots (never 0)
+  uint32_t* hdr;         // workspace header: [0] slot tag generation, [1] CTAs of the tiled kernel counted
   int32_t red_blocks;    // tiles: output blocks of kRedRows rows over all matrices
   int32_t n_split;       // tiles: entries of cta_begin in use minus one (0: equal split)
 };
@@ -414,6 +414,7 @@ struct TilesSmem {
   float cb[2][kCodewords * kDim];                // 2 x 8 KiB
   unsigned char xraw[2][kSlabV * kDim * 4];      // 2 x 2 KiB (f32; 16-bit types use half)
   uint64_t mbar[2];
+  uint32_t tag;                                  // this call's slot tag (tag_issue / tag_take)
 };
 constexpr size_t kTilesSmemBytes = sizeof(TilesSmem);
 
@@ -509,21 +510,48 @@ __device__ __forceinline__ void build_piece(float* tab, const float* cb, const u
 // Stage reduction inside the tiled kernel.
 //
 // Each unit leaves one partial sum per row in a 64-bit slot: the high word is
-// the call's epoch (a per-call tag chosen by the host, never 0), the low word
-// the float.  One aligned 64-bit store is single-copy atomic, so a reader that
-// sees this call's epoch also sees the value written with it; slots left by
-// earlier calls (or never written) carry another tag.  After its own units,
+// the call's tag, the low word the float.  One aligned 64-bit store is
+// single-copy atomic, so a reader that sees this call's tag also sees the
+// value written with it.  The tag is 2 * generation + 1 (never 0), the
+// generation being a word of the workspace header that each call advances
+// once (tag_issue / tag_take): consecutive calls on one workspace carry different tags,
+// also when they are replays of one captured CUDA graph, and a slot repeats
+// its tag only after 2^31 calls.  After its own units,
 // each warp reduces output blocks of kRedRows rows of one matrix (block
 // numbers warp, warp + all warps of the grid, ...), one lane per row: it
-// waits, with a time bound, until every slot of its row carries the epoch
-// and adds them in a fixed order.  This needs no counter, no cleared workspace and no second kernel.
-// Every CTA of the grid must be resident at once (one CTA per SM, grid <=
-// SMs), or the bound fires and the call reports kDevErrSlotTimeout.
+// waits, with a time bound, until every slot of its row carries the tag and
+// adds them in a fixed order.  No second kernel and no clearing of the slots
+// are needed.  Every CTA of the grid must be resident at once (one CTA per
+// SM, grid <= SMs), or the bound fires and the call reports
+// kDevErrSlotTimeout.
 constexpr int kRedRows = 32;  // rows per warp block: one lane per row
 
 __device__ __forceinline__ void slot_store(unsigned long long* p, uint32_t epoch, float v) {
   const unsigned long long w = ((unsigned long long)epoch << 32) | __float_as_uint(v);
   asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+
+// Tag of this call's slots, taken by one thread per CTA after griddep_wait
+// (the previous call on the workspace has completed) in two steps.
+// tag_issue reads the generation and counts the CTA on a counter that wraps
+// to 0 on the last CTA of the grid; tag_take, called once the two results
+// are needed, lets that last CTA (which comes after every CTA's read)
+// advance the generation for the next call.  Issued before the first table
+// build, the two accesses' latency is hidden behind it.
+struct TagTicket {
+  uint32_t gen, count;
+};
+
+__device__ __forceinline__ TagTicket tag_issue(uint32_t* hdr) {
+  TagTicket t;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t.gen) : "l"(hdr) : "memory");
+  t.count = atomicInc(hdr + 1, gridDim.x - 1);
+  return t;
+}
+
+__device__ __forceinline__ uint32_t tag_take(uint32_t* hdr, TagTicket t) {
+  if (t.count == gridDim.x - 1) asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(hdr) : "memory");
+  return 2u * t.gen + 1u;
 }
 
 __device__ __forceinline__ unsigned long long slot_load(const unsigned long long* p) {
@@ -566,7 +594,7 @@ __device__ __forceinline__ float sum_slots(const unsigned long long* sp, int64_t
 // y[b][i] = scale_i * sum over k = s * n_slabs + slab of the slots of row i,
 // added in k order by the row's lane, in load batches of up to 24 slots.
 // Work items are (output block, token) pairs dealt to warps round-robin.
-__device__ __forceinline__ void reduce_slots(const GvParams& P, int tid) {
+__device__ __forceinline__ void reduce_slots(const GvParams& P, int tid, uint32_t epoch) {
   const int lane = tid & 31;
   const int warps = gridDim.x * kGvWarps;
   const int64_t items = (int64_t)P.red_blocks * P.B;  // (block, token) pairs
@@ -581,10 +609,10 @@ __device__ __forceinline__ void reduce_slots(const GvParams& P, int tid) {
     const unsigned long long* sp = static_cast<const unsigned long long*>(M.partial) + (int64_t)b * np * M.rows + row;
     float acc;
     if (np <= 12) {
-      acc = sum_slots<12>(sp, M.rows, np, 0, P.epoch);
+      acc = sum_slots<12>(sp, M.rows, np, 0, epoch);
     } else {
       acc = 0.0f;
-      for (int k0 = 0; k0 < np; k0 += 24) acc += sum_slots<24>(sp, M.rows, np, k0, P.epoch);
+      for (int k0 = 0; k0 < np; k0 += 24) acc += sum_slots<24>(sp, M.rows, np, k0, epoch);
     }
     M.y[(int64_t)b * M.rows + row] = f16_bits_to_f32(__ldg(M.scales + row)) * acc;
   }
@@ -628,7 +656,9 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   griddep_launch_dependents();
   if (u0 >= u1) {  // no units: only the reduction share
     griddep_wait();
-    reduce_slots(P, tid);
+    if (tid == 0) S.tag = tag_take(P.hdr, tag_issue(P.hdr));
+    __syncthreads();
+    reduce_slots(P, tid, S.tag);
     return;
   }
   TileCursor ci = tcur_at(P, u0);
@@ -644,9 +674,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   // they do not queue behind it); its build then overlaps the first loads.
   uint32_t key_cur = ci.tkey;
   uint32_t key_next = key_cur == key_last ? kNoTable : next_table_key(P, key_cur);
+  TagTicket ticket = {0u, 0u};
   if (tid == 0) {
     stage_table<XDT>(P, key_cur, S, 0);
     if (key_next != kNoTable) stage_table<XDT>(P, key_next, S, 1);
+    ticket = tag_issue(P.hdr);
   }
   bool ok = mbar_wait_bounded(&S.mbar[0], 0);
 
@@ -676,7 +708,9 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
 #pragma unroll 1
     for (int c = 0; c < kBuildChunks; c++) build_piece<XDT>(S.tab[0], S.cb[0], S.xraw[0], nv, c, warp, lane);
   }
+  if (tid == 0) S.tag = tag_take(P.hdr, ticket);
   __syncthreads();
+  const uint32_t epoch = S.tag;
   int tno = 0;              // number of the current table within this CTA; it lives in tab[tno & 1]
   int pieces = 0;           // pieces of table tno + 1 this warp has built
   bool next_ready = false;  // the inputs of table tno + 1 have landed
@@ -744,12 +778,12 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
         k1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
         float kk = hi1 ? k1 : k0;
         kk += __shfl_xor_sync(0xFFFFFFFFu, hi1 ? k0 : k1, 1);
-        if (out_row < rows_valid) slot_store(q + out_row, P.epoch, kk);
+        if (out_row < rows_valid) slot_store(q + out_row, epoch, kk);
       }
     }
   }
   (void)ok;  // a timed-out wait has recorded kDevErrMbarTimeout in the device error word
-  reduce_slots(P, tid);
+  reduce_slots(P, tid, epoch);
 }
 
 // Repack the index planes [3][rows][cols/8] (plane_stride bytes apart) into

@@ -1,7 +1,6 @@
 // C ABI of the VQ3R library (declared in include/vq3r.h): argument checks,
 // launch configuration and status codes.  All arithmetic runs in the
 // kernels of encode.cuh, decode.cuh and gemv.cuh.
-#include <atomic>
 #include <mutex>
 
 #include "decode.cuh"
@@ -79,6 +78,7 @@ cudaError_t device_setup(int* sms) {
 }
 
 constexpr size_t kWsAlign = 256;
+constexpr size_t kWsHeaderBytes = 256;  // GEMV workspace header, see plan_gemv
 size_t align_up(size_t x) { return (x + kWsAlign - 1) / kWsAlign * kWsAlign; }
 
 constexpr int kErrMaxBlocks = 4096;
@@ -155,7 +155,11 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
     P.g[g].mat_end = (int16_t)nm;
   }
   P.n_mats = nm;
-  size_t off = 0;
+  // The workspace opens with a header (the tiled kernel's slot-tag
+  // generation and finished-CTA counter), kept out of every layout's
+  // partial sums so that calls of either layout may share a workspace.
+  P.hdr = reinterpret_cast<uint32_t*>(ws_base);
+  size_t off = kWsHeaderBytes;
   int64_t units = 0;
   for (int g = 0; g < n_groups; g++) {
     GvGroup& G = P.g[g];
@@ -336,12 +340,6 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   cudaError_t e = device_setup(&sms);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // Tag of this call's partial-sum slots: distinct from the previous calls'
-  // (a 32-bit counter per process, skipping 0).
-  static std::atomic<uint32_t> g_epoch{0};
-  uint32_t ep = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
-  if (ep == 0) ep = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
-  plan.P.epoch = ep;
   const GvParams& P = plan.P;
   // Kernels are launched with programmatic stream serialization: their CTAs
   // may be scheduled while the preceding kernel drains and wait

@@ -78,14 +78,15 @@ def test_gemv_batch_and_workspace_checks(lib):
 
 
 def test_gemv_workspace_holds_the_partial_sums(lib):
-    # per matrix: B tokens x 3 stages x ceil(cols / 512) slabs x rows fp32 partial sums (256-byte aligned)
+    # a 256-byte header, then per matrix: B tokens x 3 stages x ceil(cols / 512) slabs x rows fp32 partial sums
+    # (256-byte aligned)
     specs = [(2048, 7168, 0x10000, 0x20000)] * 16
     for B in (1, 4, 32):
         ws = lib.vq3r_gemv_workspace_size(_descs(specs), 16, B)
-        assert ws == 16 * B * 3 * 14 * 2048 * 4
+        assert ws == 256 + 16 * B * 3 * 14 * 2048 * 4
     specs = [(7168, 2048, 0x10000, 0x20000 + 0x10000 * i) for i in range(8)]
     ws = lib.vq3r_gemv_workspace_size(_descs(specs), 8, 1)
-    assert ws == 8 * 3 * 4 * 7168 * 4
+    assert ws == 256 + 8 * 3 * 4 * 7168 * 4
 
 
 def test_gemv_plane_stride_checks(lib):
@@ -108,7 +109,7 @@ def test_tiles_size_and_layout_checks(lib):
     arr[0].plane_stride = arr[1].plane_stride = 4 * 32768 + 16  # not a whole number of blocks
     assert lib.vq3r_gemv(arr, 2, 1, 1, 0x500000, 1 << 30, None) == 2
     arr[0].plane_stride = arr[1].plane_stride = 0
-    # one 64-bit (epoch, partial sum) slot per (token, stage, slab, row) in the tiled layout
-    assert lib.vq3r_gemv_workspace_size(arr, 2, 1) == 2 * 3 * 14 * 2048 * 8
+    # the header, then one 64-bit (tag, partial sum) slot per (token, stage, slab, row) in the tiled layout
+    assert lib.vq3r_gemv_workspace_size(arr, 2, 1) == 256 + 2 * 3 * 14 * 2048 * 8
     assert lib.vq3r_pack_tiles(None, 4, 16, 0, 0x100000, None) == 1
     assert lib.vq3r_pack_tiles(0x100000, 4, 12, 0, 0x100000, None) == 2

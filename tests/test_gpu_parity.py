@@ -260,6 +260,47 @@ def test_grouped_gemv_many_tokens(B):
         assert gemv_rel_err(y, ref) <= GEMV_TOL
 
 
+@pytest.mark.parametrize("B", [1, 3])
+def test_gemv_cuda_graph_replays(B):
+    """A tiled GEMV captured once in a CUDA graph and replayed with new inputs: every replay repeats the
+    captured call tag, so each must find the partial-sum slots cleared by the replay before it."""
+    rng = np.random.default_rng(90 + B)
+    cb = random_codebooks(400)
+    specs = [(1100, 1032), (70, 1032)]
+    mats, decoded = [], []
+    x_t = torch.zeros((B, 1032), dtype=torch.float32, device=DEV)
+    for rows, cols in specs:
+        W = rng.standard_normal((rows, cols)).astype(np.float32)
+        W_t, idx_t, sc_t, cb_t, idx_o, sc_o = check_encode_decode(W, "f32", cb)
+        mats.append(dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=x_t,
+                         y=torch.zeros((B, rows), dtype=torch.float32, device=DEV)))
+        decoded.append(oracle.decode(idx_o, sc_o, cb))
+    mats = as_layout(mats, "tiles")
+    ws = torch.zeros(max(vq.vq3r_gemv_workspace_size(mats, B), 16), dtype=torch.uint8, device=DEV)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        vq.vq3r_gemv(mats, B, workspace=ws)  # warm-up outside the capture (first-call device setup)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        vq.vq3r_gemv(mats, B, workspace=ws)
+    for rep in range(4):
+        x = rng.standard_normal((B, 1032)).astype(np.float32)
+        x_t.copy_(torch.from_numpy(x))
+        for m in mats:
+            m["y"].fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for m, Wd in zip(mats, decoded):
+            y = m["y"].cpu().numpy()
+            assert np.isfinite(y).all(), rep
+            assert gemv_rel_err(y, oracle.gemv(Wd, x, "f32")) <= GEMV_TOL, rep
+    assert vq.vq3r_device_error() == 0
+    del g
+
+
 # ------------------------------------------------------------------ error statuses
 
 def test_error_statuses():
