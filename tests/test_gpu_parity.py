@@ -429,3 +429,56 @@ def test_moe_decode_step_gemv_sampled_rows(B, layout):
         y = y_t.cpu().numpy()[:, sample]
         worst = max(worst, gemv_rel_err(y, y_ref))
     assert worst <= GEMV_TOL, worst
+
+
+@pytest.mark.parametrize("kind", [wl.W1, wl.W2])
+def test_sweep_256_experts_sampled_rows(kind):
+    """The 256-expert scale sweep (Student-t(3) rows with 0.1% outliers at 20 sigma): one stacked matrix of all
+    experts encoded in one call and bit-exact on 256 sampled rows; one expert's rel-Frobenius error consistent
+    with its decode; and the GEMV over all 256 experts at B = 1 (both layouts), 4 and 32 (tiled) within the
+    tolerance on the sampled rows."""
+    cfg = wl.SWEEP
+    cb = load_codebooks("sweep")
+    cb_t = torch.from_numpy(cb).to(DEV)
+    dist = wl.sweep_dist()
+    experts = list(range(cfg["experts"]))
+    rows, cols = wl.mat_shape(kind)
+    W_t = device_matrix(experts, kind, cfg["seed"], dist)
+    idx_t, sc_t = gpu_encode(W_t, cb)
+    rng = np.random.default_rng(500 + kind)
+    sample = np.sort(rng.choice(W_t.shape[0], 256, replace=False))
+    sel = torch.from_numpy(sample).to(DEV)
+    Wh = host_rows(experts, kind, cfg["seed"], dist, sample)
+    np.testing.assert_array_equal(host_bits(W_t[sel]), Wh)  # generators agree
+    idx_o, sc_o = oracle.encode(Wh, "bf16", cb)
+    np.testing.assert_array_equal(sc_t[sel].cpu().numpy().view(np.uint16), sc_o)
+    np.testing.assert_array_equal(idx_t[:, sel, :].cpu().numpy(), idx_o)
+
+    # one expert (the last) through the error kernel and the decode kernel, as a row range of the stacked arrays
+    e0 = (cfg["experts"] - 1) * rows
+    W_e, sc_e = W_t[e0:], sc_t[e0:]
+    idx_e = idx_t[:, e0:, :]
+    err = float(vq.vq3r_rel_frobenius_error(W_e, idx_e.contiguous(), sc_e, cb_t).cpu()[0])
+    Wd = vq.vq3r_decode(idx_e.contiguous(), sc_e, cb_t).double()
+    w = W_e.double()
+    err2 = float(torch.sqrt(((w - Wd) ** 2).sum() / (w ** 2).sum()))
+    assert abs(err - err2) <= 1e-9 * err2
+    assert 0.0 < err < 1.0
+    del W_t, W_e, Wd, w
+    torch.cuda.empty_cache()
+
+    W_ref = oracle.decode(idx_o, sc_o, cb)
+    tiles = vq.vq3r_pack_tiles(idx_t)
+    for B, layouts in ((1, ("planes", "tiles")), (4, ("tiles",)), (32, ("tiles",))):
+        x = synth.fill_rows(cols, 0, B, wl.ACT_SEED, wl.tag(900 + kind, wl.X_GATEUP), synth.normal())
+        y_ref = oracle.gemv(W_ref, x, "bf16")
+        for layout in layouts:
+            y_t = torch.full((B, idx_t.shape[1]), float("nan"), dtype=torch.float32, device=DEV)
+            m = dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=to_dev(x, "bf16"), y=y_t)
+            if layout == "tiles":
+                m.update(idx=tiles, layout="tiles", cols=cols)
+            vq.vq3r_gemv([m], B)
+            y = y_t[:, sel].cpu().numpy()
+            assert np.isfinite(y).all()
+            assert gemv_rel_err(y, y_ref) <= GEMV_TOL, (B, layout)
+    assert vq.vq3r_device_error() == 0

@@ -13,6 +13,7 @@ import pytest
 
 import oracle
 import synth
+from synth import workloads as wl
 
 K, D = 256, 8
 
@@ -43,6 +44,33 @@ def test_generator_moments_and_row_independence():
     t = synth.fill_rows(2048, 0, 64, 7, 3, synth.student_t(4), dtype="f32").astype(np.float64)
     # Student-t(4) variance = df / (df - 2) = 2
     assert abs(t.var() - 2.0) < 0.15
+
+
+def test_sweep_distribution_outliers_and_row_factors():
+    """The scale-sweep recipe: Student-t(3) values times a log-normal(0, 0.5) row factor, with 0.1% of the
+    positions replaced by +-20 sigma (sigma = sqrt(3), the t(3) standard deviation) times the row factor."""
+    rows, cols, seed, tag = 256, 4096, 4, 8
+    full = synth.fill_rows(cols, 0, rows, seed, tag, wl.sweep_dist(), dtype="f32").astype(np.float64)
+    plain = synth.fill_rows(cols, 0, rows, seed, tag, synth.student_t(3, row_sigma=0.5), dtype="f32")
+    unit = synth.fill_rows(cols, 0, rows, seed, tag, synth.student_t(3), dtype="f32").astype(np.float64)
+    rowf = plain.astype(np.float64) / unit
+    rowf_row = np.median(rowf, axis=1)
+    # one factor per row, log-normal with sigma 0.5
+    assert np.allclose(rowf, rowf_row[:, None], rtol=1e-6)
+    assert abs(np.log(rowf_row).std() - 0.5) < 0.08 and abs(np.log(rowf_row).mean()) < 0.1
+    # t(3) against its closed-form CDF, F(t) = 1/2 + (atan(u) + u / (1 + u^2)) / pi with u = t / sqrt(3):
+    # P(|t| <= a) = 2 F(a) - 1 (sd of the empirical fraction < 0.0005 at this size)
+    for a in (0.25, 0.7649, 1.5, 4.0, 10.0):
+        u = a / math.sqrt(3.0)
+        expect = 2.0 * (0.5 + (math.atan(u) + u / (1.0 + u * u)) / math.pi) - 1.0
+        assert abs((np.abs(unit) <= a).mean() - expect) < 0.003, a
+    # outliers: about 0.1% of the positions, exactly +-20 sqrt(3) x row factor, either sign
+    out = full != plain
+    n = out.sum()
+    assert 850 < n < 1250, n  # binomial(1 048 576, 1e-3): mean 1049, sd 32
+    mag = np.abs(full[out]) / np.broadcast_to(rowf_row[:, None], full.shape)[out]
+    assert np.allclose(mag, 20.0 * np.sqrt(3.0), rtol=1e-6)
+    assert 0.4 < (full[out] > 0).mean() < 0.6
 
 
 def test_sample_without_replacement():
