@@ -106,7 +106,11 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
  *   y[b][i] = sum_c w_hat[i][c] * x[b][c], fp32 accumulation, w_hat as in
  *   vq3r_decode.  Summation order is the library's own: results agree with
  *   an exact (binary64) product to about 1e-4 relative to rms(y), not bit
- *   for bit.
+ *   for bit.  TILES calls below 8 tokens (and all TILES calls with F32 or
+ *   F16 x) add each partial sum into y with an atomic add, in the order the
+ *   GPU schedules them, so two identical calls may differ in the last bits
+ *   of y; PLANES calls and TILES calls of 8 or more bf16 tokens give the
+ *   same bits every time.
  *
  * One descriptor per matrix; matrices may differ in shape, codebooks and x.
  * Matrices that share (codebooks, x, cols) share the x-projected tables the
@@ -114,18 +118,16 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
  * of all active experts builds each table once per SM that needs it.  y must
  * not overlap any input.
  *
- * Workspace: a 256-byte header, then one partial sum per (token, stage,
- * 64-column slab, row).  PLANES stores floats and adds them in a second
- * kernel; TILES stores 64-bit slots (call tag, float) and reduces them in the
- * same kernel, each SM waiting until the slots it adds carry this call's
- * tag.  The tag comes from a generation counter in the header that the last
- * CTA of each TILES call advances, so consecutive calls on one workspace,
- * replays of a captured CUDA graph included, never take each other's slots.
+ * Workspace: a 256-byte header, then, for PLANES, one float partial sum per
+ * (token, stage, 64-column slab, row), added in a second kernel.  TILES
+ * calls need the header only: the kernel zeroes y, and its CTAs meet on a
+ * grid barrier kept in the header (arrival counts) before the first add.
  * Fill a workspace with zeros once before its first call (e.g.
  * cudaMemsetAsync after allocating it); nothing needs clearing between
- * calls.  The TILES kernel runs one CTA per SM and needs all of them
- * resident together: if another workload holds SMs for more than about a
- * second, the call finishes with vq3r_device_error() = 2 and y undefined.
+ * calls, replays of a captured CUDA graph included.  The TILES kernel runs
+ * one CTA per SM and needs all of them resident together: if another
+ * workload holds SMs for more than about a second, the call finishes with
+ * vq3r_device_error() = 2 and y undefined.
  *   mats      HOST array of n_mats descriptors (copied before return)
  *   B         tokens, 1..32
  *   x_dtype   dtype of every x, {F32, BF16, F16}
@@ -213,9 +215,10 @@ vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const ui
  * exits.  The call allocates nothing (no cudaMalloc, cudaFree or allocating
  * library routine).
  *   - A call whose vq3r_gemv_workspace_size() exceeds 16 MiB returns
- *     VQ3R_ERR_WORKSPACE before launching anything (the 8-expert MoE decode
- *     step of 2048 x 7168 / 7168 x 2048 matrices in the TILES layout needs
- *     15.75 MiB at B = 1 as one call, 10.5 MiB for its gate/up half).
+ *     VQ3R_ERR_WORKSPACE before launching anything.  TILES calls need 256
+ *     bytes whatever their size; in the PLANES layout the 8-expert MoE
+ *     decode step of 2048 x 7168 / 7168 x 2048 matrices needs 7.9 MiB at
+ *     B = 1 as one call.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before capturing a stream into a graph.
@@ -234,8 +237,8 @@ const char* vq3r_status_string(vq3r_status s);
 int vq3r_last_cuda_error(void);
 
 /* Device-side error word, set by a kernel whose bounded wait gave up
- * (0 = none; 1 = a shared-memory bulk copy did not complete; 2 = vq3r_gemv
- * TILES partial sums did not all appear).  Synchronises the current device;
+ * (0 = none; 1 = a shared-memory bulk copy did not complete; 2 = not all
+ * CTAs of a vq3r_gemv TILES call reached its grid barrier).  Synchronises the current device;
  * reading it clears it. */
 vq3r_status vq3r_device_error(int* code);
 

@@ -14,14 +14,15 @@
 // pace with HBM (0.375 B of indices per weight).
 //
 // Work is split into units of (stage s, slab of 64 columns, token b, matrix,
-// tile of 256 rows).  A CTA builds the 64 KiB table T_s[slab][.] of its
-// current units in shared memory; two CTAs share an SM.  Each lane loads the
-// 16 index bytes of its two rows straight into registers and keeps the loads
-// of the next three units in flight (about 128 KiB per SM), so index bytes
+// row tile).  A CTA builds the 64 KiB table T_s[slab][.] of its current units
+// in shared memory.  Each lane loads the 16 index bytes of its rows straight
+// into registers and keeps the next units' loads in flight, so index bytes
 // never pass through shared memory, which is left to the lookups.
-// Per-(stage, slab, row) partial sums go to the workspace; the reduction
-// kernel adds them in a fixed order and applies the row scale, so results do
-// not depend on scheduling.
+// Two kernels: gemv_lut_kernel reads the encoder's plane layout (256-row
+// tiles, two CTAs per SM) and leaves per-(stage, slab, row) partial sums that
+// gemv_reduce_kernel adds in a fixed order, so its results do not depend on
+// scheduling; gemv_tiles_kernel reads the tiled layout (512-row tiles, one
+// CTA per SM) and adds each unit's scaled row sums straight into y.
 #pragma once
 
 #include "vq3r_common.cuh"
@@ -70,13 +71,13 @@ struct GvMat {
   const uint8_t* idx;
   const uint16_t* scales;
   float* y;
-  void* partial;         // [B][3][n_slabs][rows]: float (planes) or 64-bit slots (tiles)
+  void* partial;         // planes: [B][3][n_slabs][rows] float partial sums (unused by the tiled kernel)
   int64_t rows;
   int64_t plane_stride;  // bytes between index planes
   int32_t group;
   int32_t n_tiles;       // ceil(rows / kGvTileRows) >= 1
   int32_t tile_prefix;   // tiles of the earlier matrices of the same group
-  int32_t red_begin;     // first block (kRedRows rows) of this matrix in the tiled kernel's reduction
+  int32_t blk_begin;     // first row block of this matrix in the tensor-core kernel's grid
 };
 
 struct GvGroup {
@@ -100,8 +101,7 @@ struct GvParams {
   int64_t total_units;
   int32_t tile_rows;     // rows per work unit: kGvTileRows (planes) or kTileRows (tiles)
   int32_t layout;        // VQ3R_LAYOUT_PLANES or VQ3R_LAYOUT_TILES
-  uint32_t* hdr;         // workspace header: [0] slot tag generation, [1] CTAs of the tiled kernel counted
-  int32_t red_blocks;    // tiles: output blocks of kRedRows rows over all matrices
+  unsigned long long* hdr;  // workspace header: [0] arrival count at the start of the call, [1] arrival count
   int32_t n_split;       // tiles: entries of cta_begin in use minus one (0: equal split)
 };
 
@@ -335,12 +335,13 @@ __host__ __device__ __forceinline__ uint32_t table_key(int g, int slab, int s, i
   return (uint32_t)slab | ((uint32_t)s << 20) | ((uint32_t)b << 22) | ((uint32_t)g << 27);
 }
 
-// Position of the next unit to load: the index block, the partial sums of
-// its tile (row 0), the matrix rows from the tile's first row on, the table
-// key, and the coordinates needed for the carry to the next matrix or table.
+// Position of the next unit to load: the index block, y and the scales at the
+// tile's first row, the matrix rows from that row on, the table key, and the
+// coordinates needed for the carry to the next matrix or table.
 struct TileCursor {
   const uint8_t* p;
-  unsigned long long* q;
+  float* q;             // y of the unit's token, at the tile's first row
+  const uint16_t* sc;   // scales, at the tile's first row
   int32_t rows_left;
   uint32_t tkey;
   int32_t m, tile, ntiles;
@@ -353,8 +354,8 @@ __device__ __forceinline__ void tcur_fill(const GvParams& P, TileCursor& c) {
   const int64_t n_slabs = P.g[g].n_slabs;
   c.ntiles = M.n_tiles;
   c.p = M.idx + ((int64_t)s * n_slabs + slab) * M.plane_stride + (int64_t)c.tile * kTileBytes;
-  c.q = static_cast<unsigned long long*>(M.partial) + (((int64_t)b * kStages + s) * n_slabs + slab) * M.rows +
-        (int64_t)c.tile * kTileRows;
+  c.q = M.y + (int64_t)b * M.rows + (int64_t)c.tile * kTileRows;
+  c.sc = M.scales + (int64_t)c.tile * kTileRows;
   c.rows_left = (int32_t)(M.rows - (int64_t)c.tile * kTileRows);
 }
 
@@ -374,6 +375,7 @@ __device__ __forceinline__ void tcur_next(const GvParams& P, TileCursor& c) {
   if (++c.tile < c.ntiles) {
     c.p += kTileBytes;
     c.q += kTileRows;
+    c.sc += kTileRows;
     c.rows_left -= kTileRows;
     return;
   }
@@ -414,7 +416,6 @@ struct TilesSmem {
   float cb[2][kCodewords * kDim];                // 2 x 8 KiB
   unsigned char xraw[2][kSlabV * kDim * 4];      // 2 x 2 KiB (f32; 16-bit types use half)
   uint64_t mbar[2];
-  uint32_t tag;                                  // this call's slot tag (tag_issue / tag_take)
 };
 constexpr size_t kTilesSmemBytes = sizeof(TilesSmem);
 
@@ -507,115 +508,84 @@ __device__ __forceinline__ void build_piece(float* tab, const float* cb, const u
 }
 
 // ---------------------------------------------------------------------------
-// Stage reduction inside the tiled kernel.
+// Accumulation into y inside the tiled kernel.
 //
-// Each unit leaves one partial sum per row in a 64-bit slot: the high word is
-// the call's tag, the low word the float.  One aligned 64-bit store is
-// single-copy atomic, so a reader that sees this call's tag also sees the
-// value written with it.  The tag is 2 * generation + 1 (never 0), the
-// generation being a word of the workspace header that each call advances
-// once (tag_issue / tag_take): consecutive calls on one workspace carry different tags,
-// also when they are replays of one captured CUDA graph, and a slot repeats
-// its tag only after 2^31 calls.  After its own units,
-// each warp reduces output blocks of kRedRows rows of one matrix (block
-// numbers warp, warp + all warps of the grid, ...), one lane per row: it
-// waits, with a time bound, until every slot of its row carries the tag and
-// adds them in a fixed order.  No second kernel and no clearing of the slots
-// are needed.  Every CTA of the grid must be resident at once (one CTA per
-// SM, grid <= SMs), or the bound fires and the call reports
-// kDevErrSlotTimeout.
-constexpr int kRedRows = 32;  // rows per warp block: one lane per row
+// Each unit adds scale_i x (its partial sum of row i) to y[b][i] with one
+// fire-and-forget atomic add in L2 (red.add.f32), so no partial sums are
+// stored and no reduction pass follows the units; the order of the adds,
+// and so the rounding of y, depends on scheduling.  y must be zero before the
+// first add: every CTA zeroes a share of the outputs, then arrives on a grid
+// barrier that is waited for only after the first table build, by when it
+// has normally completed.  Every CTA of the grid must be resident at once
+// (one CTA per SM, grid <= SMs), or the wait's 1 s bound fires and the call
+// reports kDevErrBarrierTimeout.
+//
+// The barrier uses the workspace header: hdr[1] counts arrivals over all
+// calls on the workspace, hdr[0] holds its value at the start of the current
+// call, and the call's barrier is complete once hdr[1] - hdr[0] reaches the
+// grid size.  The last CTA to arrive moves hdr[0] on for the next call (which
+// starts after this grid has completed).  A zeroed header is a valid start.
 
-__device__ __forceinline__ void slot_store(unsigned long long* p, uint32_t epoch, float v) {
-  const unsigned long long w = ((unsigned long long)epoch << 32) | __float_as_uint(v);
-  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+// Zeroes this CTA's share of the outputs.  Zeroing jobs are (matrix, part)
+// pairs, parts = grid / n_mats pieces of a matrix's B x rows floats (at least
+// one); CTA c takes jobs c, c + grid, ...  A job touches one descriptor, so no
+// CTA walks the whole descriptor list.
+__device__ __forceinline__ void zero_y_share(const GvParams& P, int tid) {
+  const int n_mats = P.n_mats, grid = (int)gridDim.x;
+  const int parts = grid >= n_mats ? grid / n_mats : 1;
+  for (int j = blockIdx.x; j < n_mats * parts; j += grid) {
+    const int m = j % n_mats, part = j / n_mats;
+    const int64_t n = (int64_t)P.B * P.m[m].rows;
+    float* const y = P.m[m].y;
+    const int64_t lo = n * part / parts, hi = n * (part + 1) / parts;
+    for (int64_t i = lo + tid; i < hi; i += kGvThreads) y[i] = 0.0f;
+  }
 }
 
-// Tag of this call's slots, taken by one thread per CTA after griddep_wait
-// (the previous call on the workspace has completed) in two steps.
-// tag_issue reads the generation and counts the CTA on a counter that wraps
-// to 0 on the last CTA of the grid; tag_take, called once the two results
-// are needed, lets that last CTA (which comes after every CTA's read)
-// advance the generation for the next call.  Issued before the first table
-// build, the two accesses' latency is hidden behind it.
-struct TagTicket {
-  uint32_t gen, count;
+struct Arrival {
+  unsigned long long start, seq;  // count at the start of the call, this CTA's place in it
 };
 
-__device__ __forceinline__ TagTicket tag_issue(uint32_t* hdr) {
-  TagTicket t;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t.gen) : "l"(hdr) : "memory");
-  t.count = atomicInc(hdr + 1, gridDim.x - 1);
+// Arrival of this CTA, by one thread after a __syncthreads that follows the
+// CTA's zeros.  The add is acquire-release: it releases those zeros, and the
+// count it returns is used only later, so the thread does not wait for it.
+__device__ __forceinline__ Arrival barrier_arrive(unsigned long long* hdr) {
+  Arrival t;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(t.start) : "l"(hdr) : "memory");
+  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], 1;" : "=l"(t.seq) : "l"(hdr + 1) : "memory");
   return t;
 }
 
-__device__ __forceinline__ uint32_t tag_take(uint32_t* hdr, TagTicket t) {
-  if (t.count == gridDim.x - 1) asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(hdr) : "memory");
-  return 2u * t.gen + 1u;
+// The last CTA to arrive (every CTA read hdr[0] before its own arrival)
+// moves hdr[0] on for the next call.
+__device__ __forceinline__ void barrier_close(unsigned long long* hdr, Arrival t) {
+  if (t.seq - t.start == (unsigned long long)gridDim.x - 1)
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(hdr), "l"(t.start + gridDim.x) : "memory");
 }
 
-__device__ __forceinline__ unsigned long long slot_load(const unsigned long long* p) {
-  unsigned long long w;
-  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
-  return w;
-}
-
-// In-order sum of slots k0 .. k0 + N - 1 (those below np) of one output, once
-// all of them carry the epoch.  Past-the-end positions re-read the last slot
-// so that all N loads are issued together.
-template <int N>
-__device__ __forceinline__ float sum_slots(const unsigned long long* sp, int64_t stride, int np, int k0,
-                                           uint32_t epoch) {
-  unsigned long long w[N];
+// Waits, with a 1 s bound, until all CTAs of the grid have arrived; the
+// acquire load pairs with their releases.
+__device__ __forceinline__ void barrier_wait(unsigned long long* hdr, Arrival t) {
+  const unsigned long long grid = gridDim.x;
+  barrier_close(hdr, t);
   uint64_t t0 = 0;
   for (;;) {
-#pragma unroll
-    for (int j = 0; j < N; j++) w[j] = slot_load(sp + (int64_t)min(k0 + j, np - 1) * stride);
-    bool ready = true;
-#pragma unroll
-    for (int j = 0; j < N; j++) ready = ready && (uint32_t)(w[j] >> 32) == epoch;
-    if (ready) break;
+    unsigned long long n;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(n) : "l"(hdr + 1) : "memory");
+    if (n - t.start >= grid) break;
     const uint64_t now = global_timer_ns();
     if (t0 == 0) {
       t0 = now;
     } else if (now - t0 > 1000000000ull) {
-      set_device_error(kDevErrSlotTimeout);
+      set_device_error(kDevErrBarrierTimeout);
       break;
     }
-    __nanosleep(64);
+    __nanosleep(32);
   }
-  float acc = 0.0f;
-#pragma unroll
-  for (int j = 0; j < N; j++)
-    if (k0 + j < np) acc += __uint_as_float((uint32_t)w[j]);
-  return acc;
 }
 
-// y[b][i] = scale_i * sum over k = s * n_slabs + slab of the slots of row i,
-// added in k order by the row's lane, in load batches of up to 24 slots.
-// Work items are (output block, token) pairs dealt to warps round-robin.
-__device__ __forceinline__ void reduce_slots(const GvParams& P, int tid, uint32_t epoch) {
-  const int lane = tid & 31;
-  const int warps = gridDim.x * kGvWarps;
-  const int64_t items = (int64_t)P.red_blocks * P.B;  // (block, token) pairs
-  for (int64_t it = (int64_t)blockIdx.x * kGvWarps + (tid >> 5); it < items; it += warps) {
-    const int blk = (int)(it / P.B), b = (int)(it - (int64_t)blk * P.B);
-    int m = 0;
-    while (m + 1 < P.n_mats && P.m[m + 1].red_begin <= blk) m++;
-    const GvMat& M = P.m[m];
-    const int64_t row = (int64_t)(blk - M.red_begin) * kRedRows + lane;
-    if (row >= M.rows) continue;
-    const int np = kStages * P.g[M.group].n_slabs;
-    const unsigned long long* sp = static_cast<const unsigned long long*>(M.partial) + (int64_t)b * np * M.rows + row;
-    float acc;
-    if (np <= 12) {
-      acc = sum_slots<12>(sp, M.rows, np, 0, epoch);
-    } else {
-      acc = 0.0f;
-      for (int k0 = 0; k0 < np; k0 += 24) acc += sum_slots<24>(sp, M.rows, np, k0, epoch);
-    }
-    M.y[(int64_t)b * M.rows + row] = f16_bits_to_f32(__ldg(M.scales + row)) * acc;
-  }
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 
 // Table key of unit u (divisions; used once per CTA).
@@ -654,11 +624,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
     u1 = P.cta_begin[blockIdx.x + 1];
   }
   griddep_launch_dependents();
-  if (u0 >= u1) {  // no units: only the reduction share
+  if (u0 >= u1) {  // no units: only the share of y to zero
     griddep_wait();
-    if (tid == 0) S.tag = tag_take(P.hdr, tag_issue(P.hdr));
+    zero_y_share(P, tid);
     __syncthreads();
-    reduce_slots(P, tid, S.tag);
+    if (tid == 0) barrier_close(P.hdr, barrier_arrive(P.hdr));  // adds nothing, so it need not wait
     return;
   }
   TileCursor ci = tcur_at(P, u0);
@@ -672,18 +642,22 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
 
   // The first table's inputs arrive before the index stream is started (so
   // they do not queue behind it); its build then overlaps the first loads.
+  // The outputs are zeroed while they are in flight.
   uint32_t key_cur = ci.tkey;
   uint32_t key_next = key_cur == key_last ? kNoTable : next_table_key(P, key_cur);
-  TagTicket ticket = {0u, 0u};
   if (tid == 0) {
     stage_table<XDT>(P, key_cur, S, 0);
     if (key_next != kNoTable) stage_table<XDT>(P, key_next, S, 1);
-    ticket = tag_issue(P.hdr);
   }
+  zero_y_share(P, tid);
+  __syncthreads();  // the CTA's zeros precede its count
+  Arrival arrival = {0ull, 0ull};
+  if (tid == 0) arrival = barrier_arrive(P.hdr);
   bool ok = mbar_wait_bounded(&S.mbar[0], 0);
 
   uint4 r[NSLOT][4];
-  unsigned long long* sq[NSLOT];
+  float* sq[NSLOT];
+  uint32_t ssc[NSLOT];  // binary16 bits of the lane's row scale, converted when the unit's sum is added
   int32_t srows[NSLOT];
   uint32_t skey[NSLOT];
 #pragma unroll
@@ -692,11 +666,13 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
 #pragma unroll
       for (int t = 0; t < 4; t++) r[i][t] = ldg_stream16(ci.p + lane_off + t * 8 * kSlabV, pol);
       sq[i] = ci.q;
+      ssc[i] = out_row < ci.rows_left ? (uint32_t)__ldg(ci.sc + out_row) : 0u;
       srows[i] = ci.rows_left;
       skey[i] = ci.tkey;
       tcur_next(P, ci);
     } else {
       sq[i] = nullptr;
+      ssc[i] = 0u;
       srows[i] = 0;
       skey[i] = kNoTable;
     }
@@ -708,9 +684,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
 #pragma unroll 1
     for (int c = 0; c < kBuildChunks; c++) build_piece<XDT>(S.tab[0], S.cb[0], S.xraw[0], nv, c, warp, lane);
   }
-  if (tid == 0) S.tag = tag_take(P.hdr, ticket);
+  if (tid == 0) barrier_wait(P.hdr, arrival);  // every y is zeroed before the first add
   __syncthreads();
-  const uint32_t epoch = S.tag;
   int tno = 0;              // number of the current table within this CTA; it lives in tab[tno & 1]
   int pieces = 0;           // pieces of table tno + 1 this warp has built
   bool next_ready = false;  // the inputs of table tno + 1 have landed
@@ -746,7 +721,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
             pieces++;
           }
         }
-        unsigned long long* const q = sq[i];
+        float* const q = sq[i];
+        const uint32_t scale_bits = ssc[i];
         const int32_t rows_valid = srows[i];
         const bool refill = u + i + NSLOT < u1;
         const uint8_t* const pn = ci.p + lane_off;
@@ -765,6 +741,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
         }
         if (refill) {
           sq[i] = ci.q;
+          ssc[i] = out_row < ci.rows_left ? (uint32_t)__ldg(ci.sc + out_row) : 0u;
           srows[i] = ci.rows_left;
           skey[i] = ci.tkey;
           tcur_next(P, ci);
@@ -778,12 +755,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
         k1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
         float kk = hi1 ? k1 : k0;
         kk += __shfl_xor_sync(0xFFFFFFFFu, hi1 ? k0 : k1, 1);
-        if (out_row < rows_valid) slot_store(q + out_row, epoch, kk);
+        if (out_row < rows_valid) red_add_f32(q + out_row, f16_bits_to_f32((uint16_t)scale_bits) * kk);
       }
     }
   }
   (void)ok;  // a timed-out wait has recorded kDevErrMbarTimeout in the device error word
-  reduce_slots(P, tid, epoch);
 }
 
 // Repack the index planes [3][rows][cols/8] (plane_stride bytes apart) into

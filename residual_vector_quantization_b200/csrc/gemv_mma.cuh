@@ -122,7 +122,7 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int q) {
   return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
 }
 
-// Blocks of kMmaRows rows: matrix m owns blocks red_begin[m] .. (filled by the host for this kernel).
+// Blocks of kMmaRows rows: matrix m owns blocks blk_begin[m] .. (filled by the host for this kernel).
 template <int NT>
 __global__ void __launch_bounds__(kMmaThreads, 1) gemv_mma_kernel(const __grid_constant__ GvParams P) {
   extern __shared__ __align__(128) unsigned char mma_smem[];
@@ -130,10 +130,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1) gemv_mma_kernel(const __grid_c
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
   const int blk = blockIdx.x;
   int m = 0;
-  while (m + 1 < P.n_mats && P.m[m + 1].red_begin <= blk) m++;
+  while (m + 1 < P.n_mats && P.m[m + 1].blk_begin <= blk) m++;
   const GvMat& M = P.m[m];
   const GvGroup& G = P.g[M.group];
-  const int64_t row0 = (int64_t)(blk - M.red_begin) * kMmaRows + warp * 16;  // the warp's 16 rows
+  const int64_t row0 = (int64_t)(blk - M.blk_begin) * kMmaRows + warp * 16;  // the warp's 16 rows
   griddep_launch_dependents();
   griddep_wait();  // inputs may be written by the preceding kernel in the stream
 

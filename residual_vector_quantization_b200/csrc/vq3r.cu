@@ -155,10 +155,10 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
     P.g[g].mat_end = (int16_t)nm;
   }
   P.n_mats = nm;
-  // The workspace opens with a header (the tiled kernel's slot-tag
-  // generation and finished-CTA counter), kept out of every layout's
-  // partial sums so that calls of either layout may share a workspace.
-  P.hdr = reinterpret_cast<uint32_t*>(ws_base);
+  // The workspace opens with a header (the tiled kernel's grid-barrier
+  // arrival counts), kept apart from the planes kernel's partial sums so
+  // that calls of either layout may share a workspace.
+  P.hdr = reinterpret_cast<unsigned long long*>(ws_base);
   size_t off = kWsHeaderBytes;
   int64_t units = 0;
   for (int g = 0; g < n_groups; g++) {
@@ -166,19 +166,13 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
     G.unit_begin = units;
     units += (int64_t)G.n_slabs * kStages * B * G.tiles;
   }
-  // Partial sums: one float per (token, stage, slab, row) for the planes
-  // kernel, one 64-bit (epoch, float) slot for the tiled kernel.
-  const size_t part_bytes = tiles ? sizeof(unsigned long long) : sizeof(float);
-  int64_t red_blocks = 0;
+  // Partial sums of the planes kernel: one float per (token, stage, slab,
+  // row).  The tiled kernels add into y directly and need only the header.
   for (int i = 0; i < nm; i++) {
     GvMat& M = P.m[i];
-    M.partial = ws_base + off;
-    off = align_up(off + (size_t)B * kStages * P.g[M.group].n_slabs * (size_t)M.rows * part_bytes);
-    M.red_begin = (int32_t)red_blocks;
-    red_blocks += (M.rows + kRedRows - 1) / kRedRows;
+    M.partial = tiles ? nullptr : ws_base + off;
+    if (!tiles) off = align_up(off + (size_t)B * kStages * P.g[M.group].n_slabs * (size_t)M.rows * sizeof(float));
   }
-  if (red_blocks >= ((int64_t)1 << 31)) return VQ3R_ERR_SHAPE;
-  P.red_blocks = (int32_t)red_blocks;
   P.total_units = units;
   plan->ws_bytes = off;
   return VQ3R_OK;
@@ -355,10 +349,10 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   cfg.numAttrs = 1;
   if (P.layout == VQ3R_LAYOUT_TILES && x_dtype == VQ3R_BF16 && B >= kMmaMinB) {
     // Several tokens: rebuild the weights and contract on the tensor cores.
-    // One CTA per 128 rows of a matrix; red_begin numbers those blocks.
+    // One CTA per 128 rows of a matrix; blk_begin numbers those blocks.
     int64_t blocks = 0;
     for (int i = 0; i < P.n_mats; i++) {
-      plan.P.m[i].red_begin = (int32_t)blocks;
+      plan.P.m[i].blk_begin = (int32_t)blocks;
       blocks += (P.m[i].rows + kMmaRows - 1) / kMmaRows;
     }
     if (blocks >= ((int64_t)1 << 31)) return VQ3R_ERR_SHAPE;

@@ -19,7 +19,7 @@ constexpr int kCodebookBytes = kCodebookFloats * 4;           // 24 KiB
 
 // Error codes a kernel may leave in the device error word.
 constexpr int kDevErrMbarTimeout = 1;  // a bulk copy into shared memory did not complete within ~1 s
-constexpr int kDevErrSlotTimeout = 2;  // GEMV partial sums of this call did not all appear within ~1 s
+constexpr int kDevErrBarrierTimeout = 2;  // not all CTAs of a tiled GEMV reached its grid barrier within ~1 s
 
 // Device error word (one per GPU that loads the library).
 __device__ int g_device_error;

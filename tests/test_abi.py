@@ -109,7 +109,8 @@ def test_tiles_size_and_layout_checks(lib):
     arr[0].plane_stride = arr[1].plane_stride = 4 * 32768 + 16  # not a whole number of blocks
     assert lib.vq3r_gemv(arr, 2, 1, 1, 0x500000, 1 << 30, None) == 2
     arr[0].plane_stride = arr[1].plane_stride = 0
-    # the header, then one 64-bit (tag, partial sum) slot per (token, stage, slab, row) in the tiled layout
-    assert lib.vq3r_gemv_workspace_size(arr, 2, 1) == 256 + 2 * 3 * 14 * 2048 * 8
+    # the tiled layout adds into y directly: the workspace is only the 256-byte header
+    assert lib.vq3r_gemv_workspace_size(arr, 2, 1) == 256
+    assert lib.vq3r_gemv_workspace_size(arr, 2, 32) == 256
     assert lib.vq3r_pack_tiles(None, 4, 16, 0, 0x100000, None) == 1
     assert lib.vq3r_pack_tiles(0x100000, 4, 12, 0, 0x100000, None) == 2

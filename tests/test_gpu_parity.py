@@ -263,7 +263,8 @@ def test_grouped_gemv_many_tokens(B):
 @pytest.mark.parametrize("B", [1, 3])
 def test_gemv_cuda_graph_replays(B):
     """A tiled GEMV captured once in a CUDA graph and replayed with new inputs: every replay repeats the
-    captured call tag, so each must find the partial-sum slots cleared by the replay before it."""
+    captured kernel arguments, so the kernel's zeroing of y and its grid barrier (kept in the workspace
+    header) must work from the state the previous replay left."""
     rng = np.random.default_rng(90 + B)
     cb = random_codebooks(400)
     specs = [(1100, 1032), (70, 1032)]
