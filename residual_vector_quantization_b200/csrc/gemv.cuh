@@ -97,6 +97,11 @@ struct GvParams {
   GvMat m[VQ3R_GEMV_MAX_MATS];
   GvGroup g[VQ3R_GEMV_MAX_MATS];
   int64_t cta_begin[kMaxSplit + 1];  // tiles: CTA c takes units [cta_begin[c], cta_begin[c + 1]) when n_split == grid
+  // tiles, when n_split == grid: where CTA c starts (table key, matrix and
+  // tile of its first unit) and the table key of its last unit, so that a
+  // CTA need not search the descriptors for them
+  uint32_t cta_key0[kMaxSplit], cta_key_last[kMaxSplit];
+  int32_t cta_m0[kMaxSplit], cta_tile0[kMaxSplit];
   int32_t n_mats, n_groups, B, vec8;  // vec8: rows and planes 8-byte aligned (64-bit index loads)
   int64_t total_units;
   int32_t tile_rows;     // rows per work unit: kGvTileRows (planes) or kTileRows (tiles)
@@ -121,7 +126,7 @@ struct GvCursor {
   int g, slab, s, b, m, tile;
 };
 
-__device__ __forceinline__ GvCursor unit_cursor(const GvParams& P, int64_t u) {
+__host__ __device__ __forceinline__ GvCursor unit_cursor(const GvParams& P, int64_t u) {
   GvCursor c;
   int g = 0;
   while (g + 1 < P.n_groups && P.g[g + 1].unit_begin <= u) g++;
@@ -442,16 +447,36 @@ __device__ __forceinline__ int slab_columns(const GvParams& P, uint32_t k) {
 }
 
 // Issued by one thread: copy table k's inputs into staging buffer i.
+// Where a table's inputs come from: the x slab as stored (xbytes) and the
+// stage's codebook.  Kernel parameters only, so it may run before
+// griddep_wait.
+struct TableSrc {
+  const unsigned char* x;
+  const float* cb;
+  uint32_t xbytes;
+};
+
 template <int XDT>
-__device__ __forceinline__ void stage_table(const GvParams& P, uint32_t k, TilesSmem& S, int i) {
+__device__ __forceinline__ TableSrc table_src(const GvParams& P, uint32_t k) {
   const GvGroup& G = P.g[k >> 27];
   const int slab = (int)(k & 0xFFFFFu), s = (int)((k >> 20) & 3u), b = (int)((k >> 22) & 31u);
-  const uint32_t xbytes = (uint32_t)(slab_columns(P, k) * kDim * x_elt_bytes<XDT>());
-  const unsigned char* xsrc = static_cast<const unsigned char*>(G.x) +
-                              ((int64_t)b * G.cols + (int64_t)slab * kSlabV * kDim) * x_elt_bytes<XDT>();
-  mbar_arrive_expect_tx(&S.mbar[i], xbytes + (uint32_t)(kCodewords * kDim * 4));
-  bulk_copy_g2s(S.xraw[i], xsrc, xbytes, &S.mbar[i]);
-  bulk_copy_g2s(S.cb[i], G.codebooks + (size_t)s * kCodewords * kDim, kCodewords * kDim * 4, &S.mbar[i]);
+  TableSrc t;
+  t.xbytes = (uint32_t)(slab_columns(P, k) * kDim * x_elt_bytes<XDT>());
+  t.x = static_cast<const unsigned char*>(G.x) + ((int64_t)b * G.cols + (int64_t)slab * kSlabV * kDim) * x_elt_bytes<XDT>();
+  t.cb = G.codebooks + (size_t)s * kCodewords * kDim;
+  return t;
+}
+
+// Bulk copies of a table's inputs into xraw[i] / cb[i], completing on mbar[i].
+__device__ __forceinline__ void stage_src(const TableSrc& t, TilesSmem& S, int i) {
+  mbar_arrive_expect_tx(&S.mbar[i], t.xbytes + (uint32_t)(kCodewords * kDim * 4));
+  bulk_copy_g2s(S.xraw[i], t.x, t.xbytes, &S.mbar[i]);
+  bulk_copy_g2s(S.cb[i], t.cb, kCodewords * kDim * 4, &S.mbar[i]);
+}
+
+template <int XDT>
+__device__ __forceinline__ void stage_table(const GvParams& P, uint32_t k, TilesSmem& S, int i) {
+  stage_src(table_src<XDT>(P, k), S, i);
 }
 
 // The 8 x values of slab column v widened to float (zero for columns past the row end).
@@ -483,13 +508,10 @@ __device__ __forceinline__ void staged_x(const unsigned char* xr, int v, int nv,
 }
 
 // Piece c of a table: warp w computes codewords 32c + w and 32c + w + 16 for
-// slab columns lane and lane + 32, T[v][j] = C[j] . x[v] in k order.
-template <int XDT>
-__device__ __forceinline__ void build_piece(float* tab, const float* cb, const unsigned char* xr, int nv, int c,
-                                            int warp, int lane) {
-  float xa[8], xb[8];
-  staged_x<XDT>(xr, lane, nv, xa);
-  staged_x<XDT>(xr, lane + 32, nv, xb);
+// slab columns lane and lane + 32 (x values xa, xb), T[v][j] = C[j] . x[v] in
+// k order.
+__device__ __forceinline__ void build_piece_x(float* tab, const float* cb, const float xa[8], const float xb[8],
+                                              int c, int warp, int lane) {
   const float4* c4 = reinterpret_cast<const float4*>(cb);
 #pragma unroll
   for (int h = 0; h < 2; h++) {
@@ -505,6 +527,27 @@ __device__ __forceinline__ void build_piece(float* tab, const float* cb, const u
     tab[tab_word(lane, j)] = ta;
     tab[tab_word(lane + 32, j)] = tb;
   }
+}
+
+template <int XDT>
+__device__ __forceinline__ void build_piece(float* tab, const float* cb, const unsigned char* xr, int nv, int c,
+                                            int warp, int lane) {
+  float xa[8], xb[8];
+  staged_x<XDT>(xr, lane, nv, xa);
+  staged_x<XDT>(xr, lane + 32, nv, xb);
+  build_piece_x(tab, cb, xa, xb, c, warp, lane);
+}
+
+// Pieces c0 .. kBuildChunks - 1 of a table, the lane's x values read once.
+template <int XDT>
+__device__ __forceinline__ void build_pieces_from(float* tab, const float* cb, const unsigned char* xr, int nv,
+                                                  int c0, int warp, int lane) {
+  if (c0 >= kBuildChunks) return;
+  float xa[8], xb[8];
+  staged_x<XDT>(xr, lane, nv, xa);
+  staged_x<XDT>(xr, lane + 32, nv, xb);
+#pragma unroll 2
+  for (int c = c0; c < kBuildChunks; c++) build_piece_x(tab, cb, xa, xb, c, warp, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -526,20 +569,38 @@ __device__ __forceinline__ void build_piece(float* tab, const float* cb, const u
 // grid size.  The last CTA to arrive moves hdr[0] on for the next call (which
 // starts after this grid has completed).  A zeroed header is a valid start.
 
-// Zeroes this CTA's share of the outputs.  Zeroing jobs are (matrix, part)
+// This CTA's share of the outputs to zero.  Zeroing jobs are (matrix, part)
 // pairs, parts = grid / n_mats pieces of a matrix's B x rows floats (at least
 // one); CTA c takes jobs c, c + grid, ...  A job touches one descriptor, so no
-// CTA walks the whole descriptor list.
-__device__ __forceinline__ void zero_y_share(const GvParams& P, int tid) {
+// CTA walks the whole descriptor list.  When the grid has at least as many
+// CTAs as matrices (the usual case) a CTA has at most one job, which zero_job
+// describes from the kernel parameters alone (so before griddep_wait);
+// zero_rest does any further jobs.
+struct ZeroJob {
+  float* y;
+  int64_t lo, hi;
+};
+
+__device__ __forceinline__ ZeroJob zero_job(const GvParams& P, int j) {
   const int n_mats = P.n_mats, grid = (int)gridDim.x;
   const int parts = grid >= n_mats ? grid / n_mats : 1;
-  for (int j = blockIdx.x; j < n_mats * parts; j += grid) {
+  ZeroJob z = {nullptr, 0, 0};
+  if (j < n_mats * parts) {
     const int m = j % n_mats, part = j / n_mats;
     const int64_t n = (int64_t)P.B * P.m[m].rows;
-    float* const y = P.m[m].y;
-    const int64_t lo = n * part / parts, hi = n * (part + 1) / parts;
-    for (int64_t i = lo + tid; i < hi; i += kGvThreads) y[i] = 0.0f;
+    z.y = P.m[m].y;
+    z.lo = n * part / parts;
+    z.hi = n * (part + 1) / parts;
   }
+  return z;
+}
+
+__device__ __forceinline__ void zero_run(const ZeroJob& z, int tid) {
+  for (int64_t i = z.lo + tid; i < z.hi; i += kGvThreads) z.y[i] = 0.0f;
+}
+
+__device__ __forceinline__ void zero_rest(const GvParams& P, int tid) {
+  for (int j = blockIdx.x + gridDim.x; j < P.n_mats; j += gridDim.x) zero_run(zero_job(P, j), tid);
 }
 
 struct Arrival {
@@ -624,18 +685,37 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
     u1 = P.cta_begin[blockIdx.x + 1];
   }
   griddep_launch_dependents();
+  const ZeroJob zj = zero_job(P, blockIdx.x);
   if (u0 >= u1) {  // no units: only the share of y to zero
     griddep_wait();
-    zero_y_share(P, tid);
+    zero_run(zj, tid);
+    zero_rest(P, tid);
     __syncthreads();
     if (tid == 0) barrier_close(P.hdr, barrier_arrive(P.hdr));  // adds nothing, so it need not wait
     return;
   }
-  TileCursor ci = tcur_at(P, u0);
-  const uint32_t key_last = unit_table_key(P, u1 - 1);
+  TileCursor ci;
+  uint32_t key_last;
+  if (P.n_split == (int)gridDim.x) {  // start position precomputed by the host
+    ci.tkey = P.cta_key0[blockIdx.x];
+    ci.m = P.cta_m0[blockIdx.x];
+    ci.tile = P.cta_tile0[blockIdx.x];
+    tcur_fill(P, ci);
+    key_last = P.cta_key_last[blockIdx.x];
+  } else {
+    ci = tcur_at(P, u0);
+    key_last = unit_table_key(P, u1 - 1);
+  }
+  uint32_t key_cur = ci.tkey;
+  uint32_t key_next = key_cur == key_last ? kNoTable : next_table_key(P, key_cur);
+  // Everything that reads only the kernel parameters is done before
+  // griddep_wait, while the preceding kernel drains.
+  TableSrc src0 = {nullptr, nullptr, 0u}, src1 = {nullptr, nullptr, 0u};
   if (tid == 0) {
     mbar_init(&S.mbar[0], 1);
     mbar_init(&S.mbar[1], 1);
+    src0 = table_src<XDT>(P, key_cur);
+    if (key_next != kNoTable) src1 = table_src<XDT>(P, key_next);
   }
   __syncthreads();
   griddep_wait();  // inputs may be written by the preceding kernel in the stream
@@ -643,13 +723,12 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   // The first table's inputs arrive before the index stream is started (so
   // they do not queue behind it); its build then overlaps the first loads.
   // The outputs are zeroed while they are in flight.
-  uint32_t key_cur = ci.tkey;
-  uint32_t key_next = key_cur == key_last ? kNoTable : next_table_key(P, key_cur);
   if (tid == 0) {
-    stage_table<XDT>(P, key_cur, S, 0);
-    if (key_next != kNoTable) stage_table<XDT>(P, key_next, S, 1);
+    stage_src(src0, S, 0);
+    if (key_next != kNoTable) stage_src(src1, S, 1);
   }
-  zero_y_share(P, tid);
+  zero_run(zj, tid);
+  zero_rest(P, tid);
   __syncthreads();  // the CTA's zeros precede its count
   Arrival arrival = {0ull, 0ull};
   if (tid == 0) arrival = barrier_arrive(P.hdr);
@@ -679,11 +758,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   }
 
   // The first table is built at once, while the first index loads are in flight.
-  {
-    const int nv = slab_columns(P, key_cur);
-#pragma unroll 1
-    for (int c = 0; c < kBuildChunks; c++) build_piece<XDT>(S.tab[0], S.cb[0], S.xraw[0], nv, c, warp, lane);
-  }
+  build_pieces_from<XDT>(S.tab[0], S.cb[0], S.xraw[0], slab_columns(P, key_cur), 0, warp, lane);
   if (tid == 0) barrier_wait(P.hdr, arrival);  // every y is zeroed before the first add
   __syncthreads();
   int tno = 0;              // number of the current table within this CTA; it lives in tab[tno & 1]
@@ -699,9 +774,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
         const uint32_t nparity = (uint32_t)((tno + 1) >> 1) & 1u;
         if (skey[i] != key_cur) {  // switch to table tno + 1 (= key_next)
           if (!next_ready) ok = mbar_wait_bounded(&S.mbar[nb], nparity) && ok;
-          const int nv = slab_columns(P, key_next);
-#pragma unroll 1
-          for (; pieces < kBuildChunks; pieces++) build_piece<XDT>(S.tab[nb], S.cb[nb], S.xraw[nb], nv, pieces, warp, lane);
+          build_pieces_from<XDT>(S.tab[nb], S.cb[nb], S.xraw[nb], slab_columns(P, key_next), pieces, warp, lane);
           __syncthreads();  // table complete; every warp is done with table tno - 1's buffers
           tno++;
           key_cur = key_next;

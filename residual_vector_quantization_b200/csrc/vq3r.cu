@@ -184,7 +184,7 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
 // largest range cost; for a given budget, ranges are filled greedily table by
 // table.  Writes P.cta_begin[0..n] and P.n_split = n (ranges past the last
 // unit are empty).
-constexpr int64_t kTableCost = 2;  // one table build costs about two units of streaming and lookups
+constexpr int64_t kTableCost = 4;  // a table build, and the stall at a switch, cost about four units
 
 int64_t split_ranges(const GvParams& P, int64_t budget, int n, int64_t* begin) {
   int used = 0;
@@ -230,6 +230,17 @@ void balance_split(GvParams& P, int n) {
   }
   const int64_t used = split_ranges(P, lo, n, P.cta_begin);
   for (int64_t c = used; c <= n; c++) P.cta_begin[c] = P.total_units;
+  for (int c = 0; c < n; c++) {
+    P.cta_key0[c] = P.cta_key_last[c] = 0;
+    P.cta_m0[c] = P.cta_tile0[c] = 0;
+    if (P.cta_begin[c] >= P.cta_begin[c + 1]) continue;  // no units
+    const GvCursor first = unit_cursor(P, P.cta_begin[c]);
+    const GvCursor last = unit_cursor(P, P.cta_begin[c + 1] - 1);
+    P.cta_key0[c] = table_key(first.g, first.slab, first.s, first.b);
+    P.cta_m0[c] = first.m;
+    P.cta_tile0[c] = first.tile;
+    P.cta_key_last[c] = table_key(last.g, last.slab, last.s, last.b);
+  }
   P.n_split = n;
 }
 
