@@ -47,6 +47,8 @@ def lib():
         L.orc_fp16_to_double.restype = D_
         L.orc_bf16_to_float.argtypes = [ctypes.c_uint16]
         L.orc_bf16_to_float.restype = ctypes.c_float
+        L.orc_bf16_from_float.argtypes = [ctypes.c_float]
+        L.orc_bf16_from_float.restype = ctypes.c_uint16
         L.orc_row_sumsq.argtypes = [P, I32, I64, I64]
         L.orc_row_sumsq.restype = D_
         L.orc_row_scales.argtypes = [P, I32, I64, I64, P]
@@ -157,6 +159,15 @@ def decode(idx, scales, codebooks, out="f32"):
     if rc:
         raise ValueError("orc_decode: bad shape")
     return o
+
+
+def gemm(idx, scales, codebooks, x):
+    """Prefill product Y[t][i] = sum_c bf16(w_hat[i][c]) * x[t][c] in binary64 for bf16 x [T][cols]: the
+    weights as decode writes them, rounded to bfloat16 (RNE), the operand type of a bf16 tensor-core product.
+    The pages define no batched product; this reading keeps decode's arithmetic and adds one rounding."""
+    Wb = decode(idx, scales, codebooks, out="bf16")
+    W = (Wb.astype(np.uint32) << 16).view(np.float32)
+    return gemv(W, x, "bf16")
 
 
 def rel_frobenius(W, dtype, What):

@@ -109,6 +109,17 @@ float orc_bf16_to_float(uint16_t b) {
   return f;
 }
 
+/* binary32 -> bfloat16 bits by round to nearest, ties to even on the 16
+ * dropped bits (a NaN stays a quiet NaN). */
+uint16_t orc_bf16_from_float(float x) {
+  uint32_t u;
+  memcpy(&u, &x, 4);
+  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return (uint16_t)((u >> 16) | 0x0040u);
+  const uint32_t rest = u & 0xFFFFu, keep = u >> 16;
+  if (rest > 0x8000u || (rest == 0x8000u && (keep & 1u))) return (uint16_t)(keep + 1u);
+  return (uint16_t)keep;
+}
+
 static float load_w(const void* W, int dtype, int64_t i) {
   if (dtype == ORC_BF16) return orc_bf16_to_float(((const uint16_t*)W)[i]);
   if (dtype == ORC_F16) return (float)orc_fp16_to_double(((const uint16_t*)W)[i]);
@@ -243,8 +254,9 @@ int orc_encode_rows(const void* Wrows, int dtype, int64_t n, int64_t cols, const
 /* ---------------- decode (§2 reconstruction rule) ---------------- */
 
 /* w_hat = (float)scale * ((C1[i1] + C2[i2]) + C3[i3]) in binary32 (fewer
- * terms for nstages < 3).  out_dtype ORC_F32 or ORC_F16 (RNE of the binary32
- * value, overflow to inf). */
+ * terms for nstages < 3).  out_dtype ORC_F32, ORC_F16 (RNE of the binary32
+ * value, overflow to inf) or ORC_BF16 (RNE of the binary32 value; the
+ * weights a bf16 tensor-core product consumes). */
 int orc_decode(const uint8_t* idx, const uint16_t* scales, const float* codebooks, int64_t rows, int64_t cols,
                int nstages, void* out, int out_dtype) {
   if (rows < 0 || cols < ORC_D || cols % ORC_D || nstages < 1 || nstages > 3) return 2;
@@ -262,6 +274,7 @@ int orc_decode(const uint8_t* idx, const uint16_t* scales, const float* codebook
         float w = sf * acc;
         int64_t o = i * cols + v * ORC_D + k;
         if (out_dtype == ORC_F16) ((uint16_t*)out)[o] = orc_fp16_from_float(w);
+        else if (out_dtype == ORC_BF16) ((uint16_t*)out)[o] = orc_bf16_from_float(w);
         else ((float*)out)[o] = w;
       }
     }

@@ -330,6 +330,39 @@ def test_gemv_matches_float64_matmul():
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
 
 
+def test_bf16_rounding_matches_torch():
+    """binary32 -> bfloat16 (RNE) against torch's CPU conversion: random values, exact ties either way,
+    signed zeros, infinities, the largest finite values (overflow to inf) and subnormals."""
+    import torch
+    rng = np.random.default_rng(14)
+    vals = [rng.standard_normal(3000) * 10.0 ** rng.integers(-38, 38, 3000)]
+    ties = (np.arange(1, 200, dtype=np.uint32) << 16) | 0x8000  # exactly half-way, even and odd kept parts
+    vals.append(ties.view(np.float32))
+    vals.append(np.array([0.0, -0.0, np.inf, -np.inf, 3.3895314e38, -3.3895314e38, 1e-40, -1e-45], np.float64))
+    xs = np.concatenate([v.astype(np.float32) for v in vals])
+    ref = torch.from_numpy(xs).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.lib().orc_bf16_from_float(float(x)) for x in xs], dtype=np.uint16)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_gemm_is_bf16_decoded_weights_times_x():
+    """The prefill oracle: decode to bf16 equals torch's RNE of the binary32 decode, and the product equals
+    numpy's float64 matmul of those weights with x."""
+    import torch
+    rng = np.random.default_rng(15)
+    cb = rng.standard_normal((3, K, D)).astype(np.float32)
+    idx = rng.integers(0, K, size=(3, 40, 24), dtype=np.uint8)
+    sc = np.array([oracle.fp16_from_double_sat(v) for v in np.exp(rng.standard_normal(40))], np.uint16)
+    w32 = oracle.decode(idx, sc, cb)
+    wb = oracle.decode(idx, sc, cb, out="bf16")
+    np.testing.assert_array_equal(wb, torch.from_numpy(w32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    xb = (rng.standard_normal((7, 192)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    y = oracle.gemm(idx, sc, cb, xb)
+    W = (wb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    x = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    np.testing.assert_allclose(y, x @ W.T, rtol=1e-12, atol=1e-12)
+
+
 def test_rtn4_row_exact_grid_and_clamp():
     rng = np.random.default_rng(13)
     s = np.float32(0.375)
