@@ -38,7 +38,7 @@ FLOPS_PER_WEIGHT = 2304  # 3 stages x 256 codewords x 8 dims x (sub, mul, add) /
 # DRAM bytes (read + write) per weight of the encode kernel, from an ncu capture
 # of this kernel (dram__bytes_read.sum + dram__bytes_write.sum over 117.4 M
 # weights); None once the kernel changes and until it is captured again.
-ENCODE_DRAM_BYTES_PER_WEIGHT = (235124480 + 7574784) / 117440512
+ENCODE_DRAM_BYTES_PER_WEIGHT = (235084544 + 7774976) / 117440512
 SM_COUNT_NOMINAL = 148
 FP32_LANES_PER_SM = 128
 
@@ -396,7 +396,9 @@ def main():
     hbm_gbs, sm_max_mhz, peak_src = peaks()
     props = torch.cuda.get_device_properties(dev)
     sms = props.multi_processor_count
-    fp32_peak_tflops = sms * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
+    # The distance is defined with every operation rounded (no fused multiply-add), so each FP32 lane does one
+    # operation per clock: the attainable ceiling is half the FMA-counted figure.
+    fp32_peak_tflops = sms * FP32_LANES_PER_SM * 1 * sm_max_mhz * 1e6 / 1e12
 
     def barrier():
         if world > 1:
@@ -538,9 +540,9 @@ def main():
                                      else ENCODE_DRAM_BYTES_PER_WEIGHT * layer.weights / 3),
                          "kernel": "vq3r_encode (row scale + greedy assignment; per launch = one stacked matrix "
                                    "kind, 3 per step), %d algorithmic flops/weight; peak = %d SMs x 128 FP32 lanes x "
-                                   "2 (FMA-counted) x %.0f MHz; traffic = DRAM bytes per launch" %
-                                   (FLOPS_PER_WEIGHT, sms, sm_max_mhz),
-                         "frac_of_non_fma_ceiling": 2 * enc_tflops / fp32_peak_tflops * 23 / 24},
+                                   "1 operation (no fused multiply-add in the distance) x %.0f MHz; traffic = DRAM "
+                                   "bytes per launch" % (FLOPS_PER_WEIGHT, sms, sm_max_mhz),
+                         "frac_of_fma_counted_peak": enc_tflops / (2 * fp32_peak_tflops)},
             "kernels": {
                 "encode": {"ms": enc_ms, "Gweights/s": layer.weights / enc_ms / 1e6, "TFLOP/s": enc_tflops},
                 "pack_tiles": {"ms": pack_ms, "GB/s": 2 * 0.375 * layer.weights / pack_ms / 1e6},

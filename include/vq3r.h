@@ -230,6 +230,50 @@ vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const ui
 #define VQ3R_GEMV_NOALLOC_BYTES (16u << 20)
 vq3r_status vq3r_gemv_noalloc(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype x_dtype, vq3r_stream stream);
 
+/*
+ * vq3r_gemm -- the many-token product for prompts (prefill), on the tensor
+ * cores:  Y[t][i] = sum_c bf16(w_hat[i][c]) * x[t][c],  fp32 accumulation.
+ * w_hat is the binary32 value vq3r_decode writes (page §2 reconstruction
+ * rule); bf16() rounds it to nearest even, the operand type of the bf16
+ * tensor-core product.  The pages define no batched product (their
+ * measurements are per token, page §1); this call is the prefill counterpart
+ * of vq3r_gemv and reuses its TILES layout.  Summation order is the
+ * library's: results agree with a binary64 product of the same bf16 weights
+ * to about 1e-5 relative to rms(Y), not bit for bit.
+ *
+ * One descriptor per matrix (up to VQ3R_GEMV_MAX_MATS), each with its own
+ * tokens, e.g. the experts of an MoE layer and the tokens routed to each.
+ *   idx       first TILES block (see vq3r_pack_tiles); plane_stride as in
+ *             vq3r_gemv_desc (0 = ceil(rows / 512) * 32768, else a multiple
+ *             of 32768 and at least that)
+ *   scales, codebooks as written by / given to vq3r_encode
+ *   x         [tokens][cols] bf16, row-major, DEVICE
+ *   y         [tokens][rows] fp32, row-major, DEVICE, written (not added to);
+ *             must not overlap any input
+ *   tokens    number of rows of x and y; 0 (or rows == 0) is a no-op for the
+ *             matrix (its pointers may then be NULL)
+ * x_dtype must be VQ3R_BF16 (VQ3R_ERR_DTYPE otherwise).  rows and tokens
+ * below 2^31, cols a multiple of 8 and cols / 8 at most 2^26
+ * (VQ3R_ERR_SHAPE); all pointers 16-byte aligned (VQ3R_ERR_ALIGN).  Needs no
+ * workspace.  One CTA per 128 rows x 256 tokens of a matrix; each uses 256
+ * columns of tensor memory and about 153 KiB of shared memory, so one runs
+ * per SM.  A bounded wait that gives up (about one second) sets
+ * vq3r_device_error() = 1 and leaves y undefined.
+ */
+typedef struct {
+  const uint8_t* idx;
+  const uint16_t* scales;
+  const float* codebooks;
+  int64_t rows, cols;
+  const void* x;
+  float* y;
+  int64_t plane_stride;
+  int64_t tokens;
+  int64_t reserved;         /* must be 0 */
+} vq3r_gemm_desc;
+
+vq3r_status vq3r_gemm(const vq3r_gemm_desc* mats, int n_mats, vq3r_dtype x_dtype, vq3r_stream stream);
+
 /* Human-readable name of a status code (static string). */
 const char* vq3r_status_string(vq3r_status s);
 

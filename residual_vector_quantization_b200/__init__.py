@@ -24,7 +24,7 @@ TILE_ROWS, TILE_BYTES, SLAB_COLS = 512, 32768, 512
 
 EXPORTED = ["vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_gemv_workspace_size", "vq3r_rel_frobenius_error",
             "vq3r_rel_frobenius_workspace_size", "vq3r_status_string", "vq3r_last_cuda_error",
-            "vq3r_device_error", "vq3r_gemv_noalloc", "vq3r_tiles_size", "vq3r_pack_tiles"]
+            "vq3r_device_error", "vq3r_gemv_noalloc", "vq3r_tiles_size", "vq3r_pack_tiles", "vq3r_gemm"]
 
 
 class VQ3RError(RuntimeError):
@@ -40,6 +40,12 @@ class GemvDesc(ctypes.Structure):
     _fields_ = [("idx", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("codebooks", ctypes.c_void_p),
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
                 ("plane_stride", ctypes.c_int64), ("layout", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class GemmDesc(ctypes.Structure):
+    _fields_ = [("idx", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("codebooks", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("plane_stride", ctypes.c_int64), ("tokens", ctypes.c_int64), ("reserved", ctypes.c_int64)]
 
 
 _L = None
@@ -68,8 +74,9 @@ def _lib():
         L.vq3r_status_string.restype = ctypes.c_char_p
         L.vq3r_last_cuda_error.restype = I32
         L.vq3r_device_error.argtypes = [P]
+        L.vq3r_gemm.argtypes = [P, I32, I32, P]
         for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error",
-                  "vq3r_gemv_noalloc", "vq3r_pack_tiles"):
+                  "vq3r_gemv_noalloc", "vq3r_pack_tiles", "vq3r_gemm"):
             getattr(L, f).restype = I32
         _L = L
     return _L
@@ -153,6 +160,36 @@ def _descs(mats):
             arr[i] = GemvDesc(_dev(idx, "idx"), _dev(scales, "scales"), _dev(cb, "codebooks"), idx.shape[1],
                               idx.shape[2] * DIM, _dev(x, "x"), _dev(y, "y"), 0, LAYOUT_PLANES, 0)
     return arr
+
+
+def _gemm_descs(mats):
+    """ctypes descriptor array for vq3r_gemm.  Each entry is a dict with idx (a tiled tensor from
+    vq3r_pack_tiles), scales, codebooks, cols, x [T][cols] bf16, y [T][rows] float32 and optionally row0, rows
+    (a row range of a larger packed matrix, row0 a multiple of 512)."""
+    arr = (GemmDesc * len(mats))()
+    for i, m in enumerate(mats):
+        idx, scales, cb, x, y = m["idx"], m["scales"], m["codebooks"], m["x"], m["y"]
+        if not (idx.is_cuda and idx.is_contiguous() and scales.is_cuda and scales.is_contiguous()):
+            raise ValueError("idx and scales must be contiguous CUDA tensors")
+        if x.dtype != torch.bfloat16:
+            raise ValueError("x must be bfloat16")
+        total_rows = scales.shape[0]
+        r0, rows = m.get("row0", 0), m.get("rows", total_rows)
+        if r0 % TILE_ROWS:
+            raise ValueError("row0 of a tiled matrix must be a multiple of 512")
+        n_tiles = (total_rows + TILE_ROWS - 1) // TILE_ROWS
+        arr[i] = GemmDesc(idx.data_ptr() + (r0 // TILE_ROWS) * TILE_BYTES, scales.data_ptr() + 2 * r0,
+                          _dev(cb, "codebooks"), rows, m["cols"], _dev(x, "x"), _dev(y, "y"), n_tiles * TILE_BYTES,
+                          x.shape[0], 0)
+    return arr
+
+
+def vq3r_gemm(mats, stream=None):
+    """Prefill product on the tensor cores: y[t][i] = sum_c bf16(w_hat[i][c]) x[t][c] for each descriptor
+    dict {idx (tiled), scales, codebooks, cols, x [T][cols] bf16, y [T][rows] float32} (see _gemm_descs)."""
+    arr = _gemm_descs(mats)
+    _check(_lib().vq3r_gemm(arr, len(mats), _DT[torch.bfloat16], _stream(stream)), "vq3r_gemm")
+    return [m["y"] for m in mats]
 
 
 def vq3r_tiles_size(rows, cols):

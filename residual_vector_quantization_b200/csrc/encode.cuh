@@ -71,13 +71,43 @@ struct __align__(16) EncSmem {
   uint64_t mbar;
 };
 
-__device__ __forceinline__ float2 f2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 f2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
+// Paired binary32 arithmetic for the distances, d = sum_k (r_k - c_k)^2 with
+// every operation rounded to nearest even (no fused multiply-add).  A paired
+// multiply followed by a paired add is contracted into a fused multiply-add
+// even when both carry an explicit rounding modifier (measured: a vector
+// whose two best codewords tie under the definition came out with the higher
+// index ahead).  So each square is a paired fused multiply-add whose addend
+// is a zero the compiler cannot see (a kernel argument): fma(e, e, +0) rounds
+// e * e once, exactly like a rounded multiply, and a fused multiply-add's
+// result cannot be fused into the add that follows.
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+// e * e rounded once (z holds +0 in both lanes).
+__device__ __forceinline__ float2 f2sq(float2 e, float2 z) {
+  float2 d;
+  asm("{\n\t.reg .b64 re, rz, rd;\n\t"
+      "mov.b64 re, {%2, %3};\n\t"
+      "mov.b64 rz, {%4, %5};\n\t"
+      "fma.rn.f32x2 rd, re, re, rz;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(e.x), "f"(e.y), "f"(z.x), "f"(z.y));
+  return d;
+}
 
 template <int DT>
 __global__ void __launch_bounds__(kEncThreads, 2)
     encode_kernel(const void* __restrict__ W, int64_t cols, int64_t nvec, const float* __restrict__ codebooks,
-                  const uint16_t* __restrict__ scales, uint8_t* __restrict__ idx) {
+                  const uint16_t* __restrict__ scales, uint8_t* __restrict__ idx, float zero) {
   extern __shared__ __align__(16) unsigned char enc_smem_raw[];
   EncSmem& sm = *reinterpret_cast<EncSmem*>(enc_smem_raw);
   const int tid = threadIdx.x;
@@ -99,6 +129,7 @@ __global__ void __launch_bounds__(kEncThreads, 2)
 
   const int64_t V = cols / kDim;
   const int64_t ntiles = (nvec + kEncTile - 1) / kEncTile;
+  const float2 z2 = make_float2(zero, zero);  // +0, unknown to the compiler
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     // Vector q of this thread: g = tile * kEncTile + q * kEncThreads + tid.
     float2 r[kEncPairs][kDim];
@@ -146,11 +177,11 @@ __global__ void __launch_bounds__(kEncThreads, 2)
 #pragma unroll
         for (int pr = 0; pr < kEncPairs; pr++) {
           float2 e = f2add(r[pr][0], c[0]);
-          float2 d = f2mul(e, e);
+          float2 d = f2sq(e, z2);
 #pragma unroll
           for (int k = 1; k < kDim; k++) {
             e = f2add(r[pr][k], c[k]);
-            d = f2add(d, f2mul(e, e));
+            d = f2add(d, f2sq(e, z2));
           }
           if (d.x < best[2 * pr]) { best[2 * pr] = d.x; bi[2 * pr] = j; }
           if (d.y < best[2 * pr + 1]) { best[2 * pr + 1] = d.y; bi[2 * pr + 1] = j; }

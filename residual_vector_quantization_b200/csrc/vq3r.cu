@@ -5,6 +5,7 @@
 
 #include "decode.cuh"
 #include "encode.cuh"
+#include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_mma.cuh"
 #include "vq3r_common.cuh"
@@ -71,6 +72,7 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes);
     g_dev_err[dev] = r;
   });
   *sms = g_dev_sms[dev];
@@ -252,7 +254,7 @@ vq3r_status launch_encode(const void* W, int64_t rows, int64_t cols, const float
   row_scale_kernel<DT><<<g1, kScaleThreads, 0, s>>>(W, rows, cols, scales);
   const int64_t ntiles = (nvec + kEncTile - 1) / kEncTile;
   const int g2 = (int)(ntiles < (int64_t)sms * 2 ? ntiles : (int64_t)sms * 2);
-  encode_kernel<DT><<<g2, kEncThreads, sizeof(EncSmem), s>>>(W, cols, nvec, cb, scales, idx);
+  encode_kernel<DT><<<g2, kEncThreads, sizeof(EncSmem), s>>>(W, cols, nvec, cb, scales, idx, 0.0f);
   return check_launch();
 }
 
@@ -408,6 +410,64 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   cfg.blockDim = dim3(2 * kPlanesRedRows);
   cfg.dynamicSmemBytes = 0;
   e = cudaLaunchKernelEx(&cfg, gemv_reduce_kernel, P);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return check_launch();
+}
+
+vq3r_status vq3r_gemm(const vq3r_gemm_desc* mats, int n_mats, vq3r_dtype x_dtype, vq3r_stream stream) {
+  if (!mats) return VQ3R_ERR_NULL;
+  if (n_mats < 1 || n_mats > VQ3R_GEMV_MAX_MATS) return VQ3R_ERR_BATCH;
+  if (x_dtype != VQ3R_BF16) return VQ3R_ERR_DTYPE;  // the tensor-core product takes bf16 x
+  GemmParams P;
+  memset(&P, 0, sizeof(P));
+  int64_t ctas = 0;
+  int nm = 0;
+  for (int i = 0; i < n_mats; i++) {
+    const vq3r_gemm_desc& d = mats[i];
+    vq3r_status st = check_shape(d.rows, d.cols, 0);
+    if (st != VQ3R_OK) return st;
+    if (d.tokens < 0 || d.tokens >= ((int64_t)1 << 31) || d.rows >= ((int64_t)1 << 31) ||
+        d.cols / kDim > (int64_t)kSlabV * (1 << 20) || d.reserved != 0)
+      return VQ3R_ERR_SHAPE;
+    const int64_t plane = (d.rows + kTileRows - 1) / kTileRows * kTileBytes;
+    if (d.plane_stride != 0 && (d.plane_stride < plane || d.plane_stride % kTileBytes)) return VQ3R_ERR_SHAPE;
+    if (d.rows == 0 || d.tokens == 0) continue;  // nothing to compute; pointers may be NULL
+    if (!d.idx || !d.scales || !d.codebooks || !d.x || !d.y) return VQ3R_ERR_NULL;
+    if (!aligned16(d.idx) || !aligned16(d.scales) || !aligned16(d.codebooks) || !aligned16(d.x) || !aligned16(d.y))
+      return VQ3R_ERR_ALIGN;
+    GmMat& M = P.m[nm++];
+    M.idx = d.idx;
+    M.scales = d.scales;
+    M.codebooks = d.codebooks;
+    M.x = static_cast<const uint16_t*>(d.x);
+    M.y = d.y;
+    M.rows = d.rows;
+    M.cols = d.cols;
+    M.tokens = d.tokens;
+    M.plane_stride = d.plane_stride ? d.plane_stride : plane;
+    M.n_slabs = (int32_t)((d.cols / kDim + kSlabV - 1) / kSlabV);
+    M.tok_tiles = (int32_t)((d.tokens + kTcTokens - 1) / kTcTokens);
+    M.cta_begin = ctas;
+    ctas += (d.rows + kTcRows - 1) / kTcRows * M.tok_tiles;
+  }
+  if (nm == 0) return VQ3R_OK;
+  if (ctas >= ((int64_t)1 << 31)) return VQ3R_ERR_SHAPE;
+  P.n_mats = nm;
+  P.total_ctas = ctas;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = kTcSmemBytes;
+  e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel, P);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }

@@ -114,3 +114,42 @@ def test_tiles_size_and_layout_checks(lib):
     assert lib.vq3r_gemv_workspace_size(arr, 2, 32) == 256
     assert lib.vq3r_pack_tiles(None, 4, 16, 0, 0x100000, None) == 1
     assert lib.vq3r_pack_tiles(0x100000, 4, 12, 0, 0x100000, None) == 2
+
+
+def _gemm_descs(specs):
+    arr = (vq.GemmDesc * len(specs))()
+    for i, (rows, cols, tokens) in enumerate(specs):
+        arr[i] = vq.GemmDesc(0x200000 + 0x1000 * i, 0x300000 + 0x1000 * i, 0x10000, rows, cols, 0x20000,
+                             0x400000 + 0x1000 * i, 0, tokens, 0)
+    return arr
+
+
+def test_gemm_argument_checks(lib):
+    """vq3r_gemm's host checks, all before any launch (the pointers are never dereferenced)."""
+    arr = _gemm_descs([(2048, 7168, 512)])
+    assert lib.vq3r_gemm(None, 1, 1, None) == 1
+    assert lib.vq3r_gemm(arr, 0, 1, None) == 5
+    assert lib.vq3r_gemm(arr, 33, 1, None) == 5
+    assert lib.vq3r_gemm(arr, 1, 0, None) == 4   # f32 x: the tensor-core product takes bf16
+    assert lib.vq3r_gemm(arr, 1, 2, None) == 4
+    bad = _gemm_descs([(2048, 7164, 512)])        # cols not a multiple of 8
+    assert lib.vq3r_gemm(bad, 1, 1, None) == 2
+    bad = _gemm_descs([(2048, 7168, -1)])
+    assert lib.vq3r_gemm(bad, 1, 1, None) == 2
+    bad = _gemm_descs([(2048, 7168, 512)])
+    bad[0].plane_stride = 4 * 32768 + 16          # not a whole number of blocks
+    assert lib.vq3r_gemm(bad, 1, 1, None) == 2
+    bad[0].plane_stride = 2 * 32768               # below ceil(2048 / 512) blocks
+    assert lib.vq3r_gemm(bad, 1, 1, None) == 2
+    bad = _gemm_descs([(2048, 7168, 512)])
+    bad[0].reserved = 1
+    assert lib.vq3r_gemm(bad, 1, 1, None) == 2
+    bad = _gemm_descs([(2048, 7168, 512)])
+    bad[0].x = 0x20008                            # not 16-byte aligned
+    assert lib.vq3r_gemm(bad, 1, 1, None) == 3
+    bad = _gemm_descs([(2048, 7168, 512)])
+    bad[0].y = None
+    assert lib.vq3r_gemm(bad, 1, 1, None) == 1
+    empty = _gemm_descs([(2048, 7168, 0), (0, 7168, 64)])  # nothing to compute: no launch, pointers unused
+    empty[1].idx = None
+    assert lib.vq3r_gemm(empty, 2, 1, None) == 0

@@ -12,7 +12,7 @@ import torch
 import oracle
 import synth
 from synth import workloads as wl
-from vq3r_cases import (GEMV_TOL, RELFRO_TOL, energy8_vectors, f32_to_bf16_bits, gemv_rel_err, random_codebooks,
+from vq3r_cases import (GEMM_TOL, GEMV_TOL, RELFRO_TOL, energy8_vectors, f32_to_bf16_bits, gemv_rel_err, random_codebooks,
                         sign_pattern_codebooks)
 
 pytestmark = pytest.mark.gpu
@@ -160,6 +160,30 @@ def test_ties_take_the_lowest_index():
     check_encode_decode(W, "f32", cb)
     perm = rng.permutation(256)
     check_encode_decode(W, "f32", np.ascontiguousarray(cb[:, perm, :]))
+
+
+def test_encode_tie_that_a_fused_multiply_add_would_break():
+    """A vector whose two best stage-1 codewords (37 and 61) tie exactly under the distance definition (every
+    binary32 operation rounded, k ascending) while a fused d + e * e accumulation makes 61 strictly closer.
+    The lowest index must win, as in the oracle.  (Found as a mismatch in a seeded 513 x 2048 matrix: the
+    paired add and multiply of the encoder had been contracted into fused multiply-adds.)"""
+    rng = np.random.default_rng(513 * 7 + 2048 + 300)
+    cb = random_codebooks(513 + 2048)
+    W = f32_to_bf16_bits(rng.standard_normal((513, 2048)).astype(np.float32))[500:501]
+    # the tie, checked on the host: equal with per-operation rounding, 61 first with fused accumulation
+    s = np.float32(oracle.fp16_to_double(int(oracle.row_scales(W, "bf16")[0])))
+    r = ((W[0, 160:168].astype(np.uint32) << 16).view(np.float32) / s).astype(np.float32)
+
+    def dist(c, fused):
+        acc = np.float32(0.0)
+        for k in range(8):
+            e = np.float32(r[k] - c[k])
+            acc = np.float32(np.float64(e) * np.float64(e) + np.float64(acc)) if fused else np.float32(acc + np.float32(e * e))
+        return acc
+    assert dist(cb[0, 37], False) == dist(cb[0, 61], False)
+    assert dist(cb[0, 61], True) < dist(cb[0, 37], True)
+    W_t, idx_t, sc_t, cb_t, idx_o, sc_o = check_encode_decode(W, "bf16", cb)
+    assert idx_o[0, 0, 20] == 37
 
 
 def test_scale_limits_zero_rows_and_subnormals():
@@ -483,3 +507,81 @@ def test_sweep_256_experts_sampled_rows(kind):
             assert np.isfinite(y).all()
             assert gemv_rel_err(y, y_ref) <= GEMV_TOL, (B, layout)
     assert vq.vq3r_device_error() == 0
+
+
+# ------------------------------------------------------------------ prefill product on the tensor cores
+
+@pytest.mark.parametrize("specs", [
+    [(128, 64, 1)],                        # one tile, one token, one step
+    [(130, 72, 5)],                        # ragged rows (2 blocks), ragged last step (9 vectors)
+    [(300, 1032, 257)],                    # 3 row blocks, two token tiles (one of a single token)
+    [(513, 2048, 300)],                    # a row block past a 512-row tile, 32 steps
+    [(64, 520, 600), (200, 512, 40), (0, 64, 7), (96, 128, 0)],  # one call, several matrices, empty ones
+])
+def test_gemm_parity(specs):
+    """The prefill product against the binary64 product of the bf16-rounded decoded weights (the oracle), on
+    ragged rows, columns and token counts."""
+    rng = np.random.default_rng(sum(r * 7 + c + t for r, c, t in specs))
+    mats, refs = [], []
+    for rows, cols, T in specs:
+        cb = random_codebooks(rows + cols)
+        W = f32_to_bf16_bits(rng.standard_normal((max(rows, 1), cols)).astype(np.float32))[:rows]
+        W_t = to_dev(W, "bf16")
+        idx_t, sc_t = gpu_encode(W_t, cb) if rows else (torch.zeros((3, 0, cols // 8), dtype=torch.uint8, device=DEV),
+                                                      torch.zeros(0, dtype=torch.int16, device=DEV))
+        x = f32_to_bf16_bits(rng.standard_normal((T, cols)).astype(np.float32))
+        y_t = torch.full((T, rows), float("nan"), dtype=torch.float32, device=DEV)
+        tiles = vq.vq3r_pack_tiles(idx_t) if rows else torch.zeros(16, dtype=torch.uint8, device=DEV)
+        mats.append(dict(idx=tiles, scales=sc_t, codebooks=torch.from_numpy(cb).to(DEV), cols=cols,
+                         x=to_dev(x, "bf16"), y=y_t))
+        if rows and T:
+            idx_o, sc_o = oracle.encode(W, "bf16", cb)
+            refs.append(oracle.gemm(idx_o, sc_o, cb, x))
+        else:
+            refs.append(None)
+    vq.vq3r_gemm(mats)
+    torch.cuda.synchronize()
+    assert vq.vq3r_device_error() == 0
+    for m, ref in zip(mats, refs):
+        if ref is None:
+            continue
+        y = m["y"].cpu().numpy()
+        assert np.isfinite(y).all()  # every output written
+        assert gemv_rel_err(y, ref) <= GEMM_TOL
+
+
+def test_gemm_moe_prefill_sampled_rows():
+    """Prefill of 8 experts' gate projections (2048 x 7168 each, rows of one packed stacked matrix) with a
+    different number of routed tokens per expert, in one call; 24 sampled rows of every expert against the
+    oracle."""
+    cfg = wl.LAYER
+    cb = load_codebooks("layer")
+    cb_t = torch.from_numpy(cb).to(DEV)
+    experts = list(range(8))
+    rows, cols = wl.mat_shape(wl.W1)
+    W_t = device_matrix(experts, wl.W1, cfg["seed"], wl.expert_dist())
+    idx_t, sc_t = gpu_encode(W_t, cb)
+    del W_t
+    tiles = vq.vq3r_pack_tiles(idx_t)
+    rng = np.random.default_rng(33)
+    mats, checks = [], []
+    for e in experts:
+        T = 64 + 97 * e  # 64 .. 743 tokens
+        x = synth.fill_rows(cols, 0, T, wl.ACT_SEED, wl.tag(100 + e, wl.X_GATEUP), synth.normal())
+        y_t = torch.full((T, rows), float("nan"), dtype=torch.float32, device=DEV)
+        mats.append(dict(idx=tiles, scales=sc_t, codebooks=cb_t, cols=cols, row0=e * rows, rows=rows,
+                         x=to_dev(x, "bf16"), y=y_t))
+        checks.append((e, x, y_t, np.sort(rng.choice(rows, 24, replace=False))))
+    vq.vq3r_gemm(mats)
+    torch.cuda.synchronize()
+    assert vq.vq3r_device_error() == 0
+    worst = 0.0
+    for e, x, y_t, sample in checks:
+        Wh = host_rows([e], wl.W1, cfg["seed"], wl.expert_dist(), sample)
+        idx_o, sc_o = oracle.encode(Wh, "bf16", cb)
+        ref = oracle.gemm(idx_o, sc_o, cb, x)
+        y = y_t.cpu().numpy()
+        assert np.isfinite(y).all()
+        # the per-token rms floor is taken over the sampled rows
+        worst = max(worst, gemv_rel_err(y[:, sample], ref))
+    assert worst <= GEMM_TOL, worst

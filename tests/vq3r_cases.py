@@ -59,3 +59,8 @@ def gemv_rel_err(y, y_ref):
 
 GEMV_TOL = 2e-3       # max relative error of the GEMV (fp32 accumulation vs binary64)
 RELFRO_TOL = 1e-9     # relative agreement of the binary64 error sums
+# The prefill product multiplies bf16 weights by bf16 x: each product is exact in fp32, so only the fp32
+# additions round.  Adding K terms of random sign, each addition errs by at most 2^-24 of a partial sum of
+# size ~ sqrt(k) rms(term), so the error is at most ~ (2/3) 2^-24 K^1.5 rms(term) against |y| ~ sqrt(K)
+# rms(term): (2/3) 2^-24 K = 3e-4 relative to rms(y) at K = 7168 in the worst case, about 1e-6 typically.
+GEMM_TOL = 3e-4
