@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--impl", default="vq3r", choices=["vq3r", "reference"])
     ap.add_argument("--experts", type=int, default=64)
     ap.add_argument("--gemv-iters", type=int, default=40)
+    ap.add_argument("--gemm-iters", type=int, default=10,
+                    help="timed calls of the prefill product (8 experts' w1, 512 tokens each); 0 skips it")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -75,6 +77,15 @@ def peaks():
         return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", 1965.0)), "measured"
     except Exception:
         return 6650.0, 1965.0, "fallback"
+
+
+def bf16_peak():
+    """Measured dense bf16 tensor throughput (burst), else the fallback figure."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 class ClockSampler:
@@ -481,6 +492,35 @@ def main():
         layer_sweep[str(B)] = {"us_per_call": 1e3 * ms, "GB/s": nbytes / ms / 1e6, "frac_hbm": nbytes / ms / 1e6 / hbm_gbs}
         del plan
 
+    # the prefill product on the tensor cores: the gate projections of 8 experts, 512 seeded random tokens each,
+    # in one vq3r_gemm call (weights rebuilt from the tiled indices, bf16, fp32 accumulation)
+    prefill = None
+    if args.gemm_iters > 0:
+        T, E8 = 512, min(8, layer.E)
+        rows, cols = wl.mat_shape(wl.W1)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(wl.ACT_SEED)
+        xs = torch.randn((E8, T, cols), generator=gen, device=dev).to(torch.bfloat16)
+        ys = torch.empty((E8, T, rows), dtype=torch.float32, device=dev)
+        mats = [dict(idx=layer.tiles[wl.W1], scales=layer.sc[wl.W1], codebooks=layer.cb, cols=cols, row0=e * rows,
+                     rows=rows, x=xs[e], y=ys[e]) for e in range(E8)]
+        for i in range(3):
+            vq.vq3r_gemm(mats)
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record()
+        for i in range(args.gemm_iters):
+            vq.vq3r_gemm(mats)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / args.gemm_iters
+        tflops = 2.0 * E8 * T * rows * cols / ms / 1e9
+        peak_tc, peak_tc_src = bf16_peak()
+        prefill = {"config": "%d experts x w1 %dx%d, %d tokens each, one call" % (E8, rows, cols, T), "ms": ms,
+                   "TFLOP/s": tflops, "frac_bf16_peak": tflops / peak_tc, "bf16_peak_tflops": peak_tc,
+                   "peak_source": peak_tc_src}
+        del xs, ys, mats
+
     # end to end through the public API with host buffers: H2D of the layer, the step, D2H of the results
     e2e = None
     if args.e2e_steps > 0:
@@ -554,6 +594,7 @@ def main():
                                     "frac_hbm": moe_step_bytes(1) / gv1_ms / 1e6 / hbm_gbs},
                 "gemv_sweep": gemv,
                 "gemv_layer_sweep": layer_sweep,
+                "gemm_prefill": prefill,
                 "hbm_peak_gbs": hbm_gbs, "peak_source": peak_src},
             "e2e": e2e,
             "gpu_launches": Layer.LAUNCHES_PER_STEP * args.steps,

@@ -256,7 +256,7 @@ vq3r_status vq3r_gemv_noalloc(const vq3r_gemv_desc* mats, int n_mats, int B, vq3
  * below 2^31, cols a multiple of 8 and cols / 8 at most 2^26
  * (VQ3R_ERR_SHAPE); all pointers 16-byte aligned (VQ3R_ERR_ALIGN).  Needs no
  * workspace.  One CTA per 128 rows x 256 tokens of a matrix; each uses 256
- * columns of tensor memory and about 153 KiB of shared memory, so one runs
+ * columns of tensor memory and about 225 KiB of shared memory, so one runs
  * per SM.  A bounded wait that gives up (about one second) sets
  * vq3r_device_error() = 1 and leaves y undefined.
  */

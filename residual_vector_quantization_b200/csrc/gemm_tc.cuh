@@ -11,7 +11,7 @@
 //
 // One CTA computes 128 weight rows x 256 tokens over all columns, in steps
 // of 64 columns (one 128-byte swizzle atom of bf16 per row):
-//   - all 256 threads rebuild the step's 128 x 64 weights from the tiled
+//   - all 512 threads rebuild the step's 128 x 64 weights from the tiled
 //     indices and the shared-memory codebooks, round them to bf16 and store
 //     them in the K-major 128-byte-swizzled layout the tensor core reads
 //     (operand A, two buffers);
@@ -21,7 +21,7 @@
 //   - one thread issues four tcgen05.mma (M = 128, N = 256, K = 16, bf16 in,
 //     fp32 accumulate) into tensor memory and commits them to the buffer's
 //     mbarrier, which the rebuild of the step after next waits for;
-//   - at the end, eight warps read the accumulators back (tcgen05.ld) and
+//   - at the end, sixteen warps read the accumulators back (tcgen05.ld) and
 //     store Y, one token per store instruction across 32 consecutive rows.
 #pragma once
 
@@ -35,7 +35,9 @@ namespace vq3r {
 constexpr int kTcRows = 128;     // M: weight rows per CTA
 constexpr int kTcTokens = 256;   // N: tokens per CTA
 constexpr int kTcK = 64;         // columns per step
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 512;
+constexpr int kTcParts = kTcThreads / kTcRows;   // threads per weight row: 4
+constexpr int kTcVecs = 8 / kTcParts;            // 8-vectors per thread and step: 2
 constexpr int kTcBStages = 3;
 constexpr int kTcTmemCols = 256;  // fp32 accumulator columns (one per token)
 
@@ -60,7 +62,7 @@ struct GemmParams {
 struct TcSmem {
   uint8_t a[2][kTcRows * 128];            // 2 x 16 KiB, rebuilt weights
   uint8_t b[kTcBStages][kTcTokens * 128];  // 3 x 32 KiB, x tiles
-  float cb[kStages * kCodewords * kDim];   // 24 KiB
+  float cbr[kStages * kCodewords * 4 * kDim];  // 96 KiB: each codeword 4 times side by side (128-byte rows)
   uint64_t mma_done[2];
   uint32_t tmem_base;
 };
@@ -148,8 +150,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
   const int64_t V = M.cols / kDim;
   const int n_steps = (int)((M.cols + kTcK - 1) / kTcK);
 
-  // Rebuild role: row r of the block, vectors 4h .. 4h + 3 of each step.
-  const int r = tid & (kTcRows - 1), h = tid >> 7;
+  // Rebuild role: row r of the block, vectors kTcVecs * part .. of each step.
+  const int r = tid & (kTcRows - 1), part = tid >> 7;
   const int64_t row = row0 + r;
   const int64_t rr = row & (kTileRows - 1), tile = row / kTileRows;
   const uint32_t rowsel = (uint32_t)((rr >> 2) & 1);
@@ -166,23 +168,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
   griddep_launch_dependents();
   griddep_wait();  // inputs may be written by the preceding kernel in the stream
 
-  for (int i = tid; i < kStages * kCodewords * kDim / 4; i += kTcThreads)
-    reinterpret_cast<float4*>(S.cb)[i] = __ldg(reinterpret_cast<const float4*>(M.codebooks) + i);
+  // Codeword (s, j) occupies the 128-byte row s * 256 + j, four copies of its
+  // 32 bytes.  Lane l reads copy l & 3, first the half (l >> 2) & 1, so the 8
+  // lanes of a quarter-warp touch 8 distinct 16-byte bank groups whatever
+  // codewords they gather (one copy left random rows conflicting).
+  for (int i = tid; i < kStages * kCodewords * 4 * 2; i += kTcThreads) {
+    const int half = i & 1, row = i >> 3;  // i = (row * 4 + copy) * 2 + half
+    reinterpret_cast<float4*>(S.cbr)[i] = __ldg(reinterpret_cast<const float4*>(M.codebooks) + 2 * row + half);
+  }
   const float scale = row < M.rows ? f16_bits_to_f32(__ldg(M.scales + row)) : 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
 
-  // Index words of step k: 4 bytes (vectors 4h .. 4h + 3) of each stage.
+  // Index bytes of step k: the thread's kTcVecs vectors (2 bytes) of each stage.
   auto load_idx = [&](int k, uint32_t ib[kStages]) {
     const int slab = k >> 3, kc = k & 7;
-    const int64_t off = tile * kTileBytes + rr * kSlabV + 16 * (kc >> 1) + 8 * ((uint32_t)(kc & 1) ^ rowsel) + 4 * h;
+    const int64_t off =
+        tile * kTileBytes + rr * kSlabV + 16 * (kc >> 1) + 8 * ((uint32_t)(kc & 1) ^ rowsel) + kTcVecs * part;
 #pragma unroll
     for (int s = 0; s < kStages; s++)
-      ib[s] = __ldg(reinterpret_cast<const uint32_t*>(M.idx + ((int64_t)s * M.n_slabs + slab) * M.plane_stride + off));
+      ib[s] = __ldg(reinterpret_cast<const uint16_t*>(M.idx + ((int64_t)s * M.n_slabs + slab) * M.plane_stride + off));
   };
-  // x tile of step k into b[stage]: 256 tokens x 8 chunks of 16 bytes, 8 chunks per thread.
+  // x tile of step k into b[stage]: 256 tokens x 8 chunks of 16 bytes, 4 chunks per thread.
   auto load_x = [&](int k, int stage) {
     const uint32_t base = smem_u32(S.b[stage]);
 #pragma unroll
@@ -200,7 +209,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
   load_idx(0, ib);
   load_x(0, 0);
   bool ok = true;
-  const float4* cbv = reinterpret_cast<const float4*>(S.cb);
+  const float4* cbv = reinterpret_cast<const float4*>(S.cbr) + 2 * (lane & 3);  // this lane's copy
+  const int h0 = (lane >> 2) & 1;                                                // its first half
   for (int k = 0; k < n_steps; k++) {
     const int ab = k & 1, bs = k % kTcBStages;
     if (k >= 2)  // the MMAs of step k - 2 are done with a[ab] and b[(k + 1) % 3]
@@ -210,24 +220,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
     // Rebuild: w = scale * ((C1 + C2) + C3) in binary32, rounded to bf16.
     const uint32_t abase = smem_u32(S.a[ab]);
 #pragma unroll
-    for (int e = 0; e < 4; e++) {
-      const int64_t v = (int64_t)k * 8 + 4 * h + e;
+    for (int e = 0; e < kTcVecs; e++) {
+      const int c = kTcVecs * part + e;  // the vector's 16-byte chunk in the row
+      const int64_t v = (int64_t)k * 8 + c;
       const uint32_t j1 = (ib[0] >> (8 * e)) & 0xFFu, j2 = (ib[1] >> (8 * e)) & 0xFFu, j3 = (ib[2] >> (8 * e)) & 0xFFu;
-      const float4 a0 = cbv[(0 * kCodewords + j1) * 2], a1 = cbv[(0 * kCodewords + j1) * 2 + 1];
-      const float4 b0 = cbv[(1 * kCodewords + j2) * 2], b1 = cbv[(1 * kCodewords + j2) * 2 + 1];
-      const float4 c0 = cbv[(2 * kCodewords + j3) * 2], c1 = cbv[(2 * kCodewords + j3) * 2 + 1];
+      // p: the half this lane reads first (h0), q: the other one
+      const float4 ap = cbv[(0 * kCodewords + j1) * 8 + h0], aq = cbv[(0 * kCodewords + j1) * 8 + (h0 ^ 1)];
+      const float4 bp = cbv[(1 * kCodewords + j2) * 8 + h0], bq = cbv[(1 * kCodewords + j2) * 8 + (h0 ^ 1)];
+      const float4 cp = cbv[(2 * kCodewords + j3) * 8 + h0], cq = cbv[(2 * kCodewords + j3) * 8 + (h0 ^ 1)];
       const float sv = v < V ? scale : 0.0f;
-      const float w0 = __fmul_rn(sv, __fadd_rn(__fadd_rn(a0.x, b0.x), c0.x));
-      const float w1 = __fmul_rn(sv, __fadd_rn(__fadd_rn(a0.y, b0.y), c0.y));
-      const float w2 = __fmul_rn(sv, __fadd_rn(__fadd_rn(a0.z, b0.z), c0.z));
-      const float w3 = __fmul_rn(sv, __fadd_rn(__fadd_rn(a0.w, b0.w), c0.w));
-      const float w4 = __fmul_rn(sv, __fadd_rn(__fadd_rn(a1.x, b1.x), c1.x));
-      const float w5 = __fmul_rn(sv, __fadd_rn(__fadd_rn(a1.y, b1.y), c1.y));
-      const float w6 = __fmul_rn(sv, __fadd_rn(__fadd_rn(a1.z, b1.z), c1.z));
-      const float w7 = __fmul_rn(sv, __fadd_rn(__fadd_rn(a1.w, b1.w), c1.w));
-      const uint4 pk = make_uint4(pack_bf16x2_rn(w0, w1), pack_bf16x2_rn(w2, w3), pack_bf16x2_rn(w4, w5),
-                                  pack_bf16x2_rn(w6, w7));
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(abase + sw128_offset(r, 4 * h + e)), "r"(pk.x),
+      const uint32_t p01 = pack_bf16x2_rn(__fmul_rn(sv, __fadd_rn(__fadd_rn(ap.x, bp.x), cp.x)),
+                                          __fmul_rn(sv, __fadd_rn(__fadd_rn(ap.y, bp.y), cp.y)));
+      const uint32_t p23 = pack_bf16x2_rn(__fmul_rn(sv, __fadd_rn(__fadd_rn(ap.z, bp.z), cp.z)),
+                                          __fmul_rn(sv, __fadd_rn(__fadd_rn(ap.w, bp.w), cp.w)));
+      const uint32_t q01 = pack_bf16x2_rn(__fmul_rn(sv, __fadd_rn(__fadd_rn(aq.x, bq.x), cq.x)),
+                                          __fmul_rn(sv, __fadd_rn(__fadd_rn(aq.y, bq.y), cq.y)));
+      const uint32_t q23 = pack_bf16x2_rn(__fmul_rn(sv, __fadd_rn(__fadd_rn(aq.z, bq.z), cq.z)),
+                                          __fmul_rn(sv, __fadd_rn(__fadd_rn(aq.w, bq.w), cq.w)));
+      // weights 0..3 are the half-0 values, 4..7 the half-1 values
+      const uint4 pk = h0 ? make_uint4(q01, q23, p01, p23) : make_uint4(p01, p23, q01, q23);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(abase + sw128_offset(r, c)), "r"(pk.x),
                    "r"(pk.y), "r"(pk.z), "r"(pk.w)
                    : "memory");
     }
@@ -250,12 +262,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const __grid_con
   tc_fence_after();
 
   // Epilogue: warp w reads lanes 32 (w mod 4) .. (its rows) and columns
-  // 128 (w / 4) .. (its tokens), 32 at a time.
-  const int q = warp & 3, half = warp >> 2;
+  // 64 (w / 4) .. (its tokens), 32 at a time.
+  const int q = warp & 3, cgrp = warp >> 2;
   const int64_t orow = row0 + q * 32 + lane;
 #pragma unroll 1
-  for (int cc = 0; cc < kTcTokens / 2 / 32; cc++) {
-    const int col = half * (kTcTokens / 2) + cc * 32;
+  for (int cc = 0; cc < kTcTokens / (kTcThreads / 128) / 32; cc++) {
+    const int col = cgrp * (kTcTokens / (kTcThreads / 128)) + cc * 32;
     uint32_t v[32];
     tc_load32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col, v);
     if (orow < M.rows) {
