@@ -521,6 +521,26 @@ def main():
                    "peak_source": peak_tc_src}
         del xs, ys, mats
 
+    # codebook training on the GPU: Lloyd, 3 stages x 20 iterations on 65536 seeded random 8-vectors (the size of
+    # the layer's training sample)
+    train = None
+    if args.gemm_iters > 0:
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(wl.LAYER_SEED)
+        vecs = torch.randn((65536, 8), generator=gen, device=dev)
+        cbk = torch.empty((3, 256, 8), dtype=torch.float32, device=dev)
+        trc = torch.empty((3, 21), dtype=torch.float64, device=dev)
+        wst = torch.empty(vq.vq3r_train_workspace_size(65536), dtype=torch.uint8, device=dev)
+        vq.vq3r_train(vecs, 20, codebooks=cbk, trace=trc, workspace=wst)
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record()
+        vq.vq3r_train(vecs, 20, codebooks=cbk, trace=trc, workspace=wst)
+        b.record()
+        torch.cuda.synchronize()
+        train = {"vectors": 65536, "stages": 3, "iters": 20, "ms": a.elapsed_time(b)}
+        del vecs, wst
+
     # end to end through the public API with host buffers: H2D of the layer, the step, D2H of the results
     e2e = None
     if args.e2e_steps > 0:
@@ -595,6 +615,7 @@ def main():
                 "gemv_sweep": gemv,
                 "gemv_layer_sweep": layer_sweep,
                 "gemm_prefill": prefill,
+                "train_lloyd": train,
                 "hbm_peak_gbs": hbm_gbs, "peak_source": peak_src},
             "e2e": e2e,
             "gpu_launches": Layer.LAUNCHES_PER_STEP * args.steps,

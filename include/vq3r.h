@@ -231,6 +231,32 @@ vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const ui
 vq3r_status vq3r_gemv_noalloc(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype x_dtype, vq3r_stream stream);
 
 /*
+ * vq3r_train -- fit the three codebooks (page §2: per-layer codebooks by
+ * Lloyd k-means on sampled vectors; stage s is trained on the residuals left
+ * by stage s - 1).  Readings where the page is silent: the initial
+ * centroids are the first 256 training vectors (of the stage's residuals);
+ * assignment uses vq3r_encode's distance and tie rule; a centroid is the
+ * binary64 sum of its members' components in training order, divided by
+ * their count and rounded to binary32; an empty cluster keeps its centroid;
+ * `iters` updates, then a final assignment from which the residuals
+ * r - C[a] (binary32) of the next stage are taken.  Results are bit-identical
+ * to that definition.
+ *   vecs       [n][8] float, DEVICE, the training vectors (already divided by
+ *              their rows' scales), n >= 256 (VQ3R_ERR_SHAPE)
+ *   iters      Lloyd updates per stage, >= 0
+ *   nstages    1..3
+ *   codebooks  out, [nstages][256][8] float, DEVICE
+ *   trace      out, DEVICE or NULL: [nstages][iters + 1] binary64 total
+ *              squared distance after each assignment (summed in the
+ *              library's order: equal to the sequential sum to ~1e-12)
+ *   workspace  at least vq3r_train_workspace_size(n) bytes, DEVICE
+ * Launches about nstages * (2 * iters + 3) small kernels.
+ */
+size_t vq3r_train_workspace_size(int64_t n);
+vq3r_status vq3r_train(const float* vecs, int64_t n, int iters, int nstages, float* codebooks, double* trace,
+                       void* workspace, size_t ws_bytes, vq3r_stream stream);
+
+/*
  * vq3r_gemm -- the many-token product for prompts (prefill), on the tensor
  * cores:  Y[t][i] = sum_c bf16(w_hat[i][c]) * x[t][c],  fp32 accumulation.
  * w_hat is the binary32 value vq3r_decode writes (page §2 reconstruction

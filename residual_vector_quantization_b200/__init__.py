@@ -24,7 +24,8 @@ TILE_ROWS, TILE_BYTES, SLAB_COLS = 512, 32768, 512
 
 EXPORTED = ["vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_gemv_workspace_size", "vq3r_rel_frobenius_error",
             "vq3r_rel_frobenius_workspace_size", "vq3r_status_string", "vq3r_last_cuda_error",
-            "vq3r_device_error", "vq3r_gemv_noalloc", "vq3r_tiles_size", "vq3r_pack_tiles", "vq3r_gemm"]
+            "vq3r_device_error", "vq3r_gemv_noalloc", "vq3r_tiles_size", "vq3r_pack_tiles", "vq3r_gemm",
+            "vq3r_train", "vq3r_train_workspace_size"]
 
 
 class VQ3RError(RuntimeError):
@@ -75,8 +76,11 @@ def _lib():
         L.vq3r_last_cuda_error.restype = I32
         L.vq3r_device_error.argtypes = [P]
         L.vq3r_gemm.argtypes = [P, I32, I32, P]
+        L.vq3r_train.argtypes = [P, I64, I32, I32, P, P, P, SZ, P]
+        L.vq3r_train_workspace_size.argtypes = [I64]
+        L.vq3r_train_workspace_size.restype = SZ
         for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error",
-                  "vq3r_gemv_noalloc", "vq3r_pack_tiles", "vq3r_gemm"):
+                  "vq3r_gemv_noalloc", "vq3r_pack_tiles", "vq3r_gemm", "vq3r_train"):
             getattr(L, f).restype = I32
         _L = L
     return _L
@@ -190,6 +194,27 @@ def vq3r_gemm(mats, stream=None):
     arr = _gemm_descs(mats)
     _check(_lib().vq3r_gemm(arr, len(mats), _DT[torch.bfloat16], _stream(stream)), "vq3r_gemm")
     return [m["y"] for m in mats]
+
+
+def vq3r_train_workspace_size(n):
+    return _lib().vq3r_train_workspace_size(n)
+
+
+def vq3r_train(vecs, iters, nstages=STAGES, codebooks=None, trace=None, workspace=None, stream=None):
+    """Lloyd codebooks from training vectors [n][8] float32 -> (codebooks [nstages][256][8] float32,
+    trace [nstages][iters + 1] float64: the total squared distance after each assignment)."""
+    n = vecs.shape[0]
+    if vecs.dtype != torch.float32 or vecs.dim() != 2 or vecs.shape[1] != DIM:
+        raise ValueError("vecs must be a float32 [n][8] tensor")
+    if codebooks is None:
+        codebooks = torch.empty((nstages, CODEWORDS, DIM), dtype=torch.float32, device=vecs.device)
+    if trace is None:
+        trace = torch.empty((nstages, iters + 1), dtype=torch.float64, device=vecs.device)
+    if workspace is None:
+        workspace = torch.empty(max(vq3r_train_workspace_size(n), 16), dtype=torch.uint8, device=vecs.device)
+    _check(_lib().vq3r_train(_dev(vecs, "vecs"), n, iters, nstages, _dev(codebooks, "codebooks"), _dev(trace, "trace"),
+                             _dev(workspace, "workspace"), workspace.numel(), _stream(stream)), "vq3r_train")
+    return codebooks, trace
 
 
 def vq3r_tiles_size(rows, cols):

@@ -8,6 +8,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_mma.cuh"
+#include "train.cuh"
 #include "vq3r_common.cuh"
 
 using namespace vq3r;
@@ -469,6 +470,51 @@ vq3r_status vq3r_gemm(const vq3r_gemm_desc* mats, int n_mats, vq3r_dtype x_dtype
   cfg.dynamicSmemBytes = kTcSmemBytes;
   e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel, P);
   if (e != cudaSuccess) return cuda_fail(e);
+  return check_launch();
+}
+
+int train_grid(int64_t n, int sms) {
+  const int64_t need = (n + kTrainThreads - 1) / kTrainThreads;
+  return (int)(need < 2 * (int64_t)sms ? need : 2 * (int64_t)sms);
+}
+
+size_t vq3r_train_workspace_size(int64_t n) {
+  if (n < kCodewords || n > ((int64_t)1 << 40)) return 0;
+  // residuals [n][8] float, assignments [n] int32, per-CTA trace partials (at most 2 per SM, 1024 SMs)
+  return align_up((size_t)n * kDim * sizeof(float)) + align_up((size_t)n * sizeof(int32_t)) + 2048 * sizeof(double);
+}
+
+vq3r_status vq3r_train(const float* vecs, int64_t n, int iters, int nstages, float* codebooks, double* trace,
+                       void* workspace, size_t ws_bytes, vq3r_stream stream) {
+  if (!vecs || !codebooks) return VQ3R_ERR_NULL;
+  if (n < kCodewords || n > ((int64_t)1 << 40) || iters < 0 || nstages < 1 || nstages > kStages) return VQ3R_ERR_SHAPE;
+  if (!workspace || ws_bytes < vq3r_train_workspace_size(n)) return VQ3R_ERR_WORKSPACE;
+  if (!aligned16(vecs) || !aligned16(codebooks) || !aligned16(workspace) || (trace && !aligned16(trace)))
+    return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (sms > 1024) return VQ3R_ERR_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(workspace);
+  float* R = reinterpret_cast<float*>(w);
+  int32_t* a = reinterpret_cast<int32_t*>(w + align_up((size_t)n * kDim * sizeof(float)));
+  double* part = reinterpret_cast<double*>(w + align_up((size_t)n * kDim * sizeof(float)) + align_up((size_t)n * sizeof(int32_t)));
+  const int grid = train_grid(n, sms);
+  e = cudaMemcpyAsync(R, vecs, (size_t)n * kDim * sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  for (int st = 0; st < nstages; st++) {
+    float* C = codebooks + (size_t)st * kCodewords * kDim;
+    e = cudaMemcpyAsync(C, R, (size_t)kCodewords * kDim * sizeof(float), cudaMemcpyDeviceToDevice, s);  // first 256
+    if (e != cudaSuccess) return cuda_fail(e);
+    for (int it = 0; it <= iters; it++) {
+      train_assign_kernel<<<grid, kTrainThreads, 0, s>>>(R, n, C, a, part);
+      if (trace) train_trace_kernel<<<1, 32, 0, s>>>(part, grid, trace + (size_t)st * (iters + 1) + it);
+      if (it == iters) break;
+      train_update_kernel<<<kCodewords / kTrainUpdateWarps, kTrainUpdateWarps * 32, 0, s>>>(R, n, a, C);
+    }
+    if (st + 1 < nstages) train_residual_kernel<<<grid, kTrainThreads, 0, s>>>(R, n, C, a);
+  }
   return check_launch();
 }
 

@@ -153,3 +153,20 @@ def test_gemm_argument_checks(lib):
     empty = _gemm_descs([(2048, 7168, 0), (0, 7168, 64)])  # nothing to compute: no launch, pointers unused
     empty[1].idx = None
     assert lib.vq3r_gemm(empty, 2, 1, None) == 0
+
+
+def test_train_argument_checks(lib):
+    fake = 0x100000
+    need = lib.vq3r_train_workspace_size(1000)
+    assert need >= 1000 * 32 + 1000 * 4
+    assert lib.vq3r_train_workspace_size(255) == 0
+    assert lib.vq3r_train(None, 1000, 5, 3, fake, None, fake, need, None) == 1
+    assert lib.vq3r_train(fake, 1000, 5, 3, None, None, fake, need, None) == 1
+    assert lib.vq3r_train(fake, 255, 5, 3, fake, None, fake, need, None) == 2   # fewer vectors than centroids
+    assert lib.vq3r_train(fake, 1000, -1, 3, fake, None, fake, need, None) == 2
+    assert lib.vq3r_train(fake, 1000, 5, 0, fake, None, fake, need, None) == 2
+    assert lib.vq3r_train(fake, 1000, 5, 4, fake, None, fake, need, None) == 2
+    assert lib.vq3r_train(fake, 1000, 5, 3, fake, None, fake, need - 1, None) == 7
+    assert lib.vq3r_train(fake, 1000, 5, 3, fake, None, None, need, None) == 7
+    assert lib.vq3r_train(fake + 4, 1000, 5, 3, fake, None, fake, need, None) == 3
+    assert lib.vq3r_train(fake, 1000, 5, 3, fake, fake + 8, fake, need, None) == 3

@@ -585,3 +585,48 @@ def test_gemm_moe_prefill_sampled_rows():
         # the per-token rms floor is taken over the sampled rows
         worst = max(worst, gemv_rel_err(y[:, sample], ref))
     assert worst <= GEMM_TOL, worst
+
+
+# ------------------------------------------------------------------ codebook training (Lloyd) on the GPU
+
+def test_train_tiny_workload_bit_exact(tiny):
+    """The tiny workload's codebooks (10 Lloyd iterations on all 16384 vectors) trained on the GPU equal the
+    oracle's bit for bit; the distortion trace agrees to 1e-12."""
+    W, cb = tiny
+    cfg = wl.TINY
+    vecs = oracle.normalize_rows(W, "f32", oracle.row_scales(W, "f32")).reshape(-1, 8)
+    _, tr_o = oracle.lloyd_train(vecs, cfg["lloyd_iters"])
+    cb_t, tr_t = vq.vq3r_train(torch.from_numpy(np.ascontiguousarray(vecs)).to(DEV), cfg["lloyd_iters"])
+    np.testing.assert_array_equal(cb_t.cpu().numpy().view(np.uint32), cb.view(np.uint32))
+    np.testing.assert_allclose(tr_t.cpu().numpy(), tr_o, rtol=1e-12)
+
+
+@pytest.mark.parametrize("n,iters,nstages,dup", [(256, 3, 3, False), (1000, 5, 3, True), (4099, 0, 2, False),
+                                                 (3000, 7, 1, True)])
+def test_train_small_cases_bit_exact(n, iters, nstages, dup):
+    """n = 256 (every vector its own centroid), duplicated vectors (empty clusters keep their centroid), no
+    iterations, fewer stages, a ragged vector count."""
+    rng = np.random.default_rng(n + iters)
+    vecs = (rng.standard_normal((n, 8)) * np.exp(rng.standard_normal((n, 1)))).astype(np.float32)
+    if dup:  # only 100 distinct vectors after the first 256: most clusters end up empty
+        vecs[256:] = vecs[rng.integers(0, 100, n - 256)]
+        vecs[:256] = vecs[rng.integers(0, 100, 256)]
+    cb_o, tr_o = oracle.lloyd_train(vecs, iters, nstages)
+    cb_t, tr_t = vq.vq3r_train(torch.from_numpy(vecs).to(DEV), iters, nstages)
+    np.testing.assert_array_equal(cb_t.cpu().numpy().view(np.uint32), cb_o.view(np.uint32))
+    np.testing.assert_allclose(tr_t.cpu().numpy(), tr_o, rtol=1e-12, atol=1e-300)
+
+
+def test_train_reproduces_the_expert_codebooks():
+    """The single-expert workload's stored codebooks (tests/golden/codebooks_expert.txt, written by the oracle:
+    65536 sampled normalised vectors, 20 iterations, 3 stages) retrained on the GPU, bit for bit."""
+    import importlib.util
+    import os
+    p = os.path.join(os.path.dirname(__file__), "golden", "make_codebooks.py")
+    spec = importlib.util.spec_from_file_location("make_codebooks", p)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    cfg = wl.EXPERT
+    vecs = mod.training_vectors(cfg["seed"], wl.expert_dist(), [0], cfg["train_vectors"])
+    cb_t, tr_t = vq.vq3r_train(torch.from_numpy(vecs).to(DEV), cfg["lloyd_iters"])
+    np.testing.assert_array_equal(cb_t.cpu().numpy().view(np.uint32), mod.load("expert").view(np.uint32))
