@@ -67,6 +67,16 @@ def lib():
         L.orc_rtn4_row.argtypes = [P, I32, I64, I64, P, P]
         L.orc_rtn4_row.restype = I32
         L.orc_bruteforce_joint.argtypes = [P, I64, P, P, P]
+        L.orc_vq4p_pack.argtypes = [P, I64, P]
+        L.orc_vq4p_unpack.argtypes = [P, I64, P]
+        L.orc_vq4p_encode_vectors.argtypes = [P, I64, P, P, P]
+        L.orc_vq4p_encode.argtypes = [P, I32, I64, I64, P, P, P]
+        L.orc_vq4p_encode.restype = I32
+        L.orc_vq4p_decode.argtypes = [P, P, P, I64, I64, P, I32]
+        L.orc_vq4p_decode.restype = I32
+        L.orc_vq4p_train.argtypes = [P, I64, I32, P, P]
+        L.orc_vq4p_train.restype = I32
+        L.orc_vq4p_bruteforce.argtypes = [P, I64, P, P, P]
         _lib = L
     return _lib
 
@@ -217,3 +227,91 @@ def bruteforce_joint(r, codebooks):
     err = np.empty(r.shape[0], dtype=np.float64)
     lib().orc_bruteforce_joint(r.ctypes.data, r.shape[0], cb.ctypes.data, idx.ctypes.data, err.ctypes.data)
     return idx, err
+
+
+# ---------------------------------------------------------------- VQ3R's sibling VQ4P (page §5)
+# 4 stages x 64-entry codebooks [4][64][8]; the 4 six-bit indices of a vector packed into the 24-bit word
+# i1 | i2 << 6 | i3 << 12 | i4 << 18, stored as three byte planes [3][rows][cols/8].
+
+K4, S4 = 64, 4
+
+
+def vq4p_pack(idx4):
+    """[4][...] indices (< 64) -> [3][...] byte planes."""
+    idx4 = _c(idx4, np.uint8)
+    shape = idx4.shape[1:]
+    n = int(np.prod(shape))
+    planes = np.empty((3,) + shape, dtype=np.uint8)
+    lib().orc_vq4p_pack(idx4.ctypes.data, n, planes.ctypes.data)
+    return planes
+
+
+def vq4p_unpack(planes):
+    planes = _c(planes, np.uint8)
+    shape = planes.shape[1:]
+    n = int(np.prod(shape))
+    idx4 = np.empty((4,) + shape, dtype=np.uint8)
+    lib().orc_vq4p_unpack(planes.ctypes.data, n, idx4.ctypes.data)
+    return idx4
+
+
+def vq4p_encode_vectors(r, codebooks):
+    """Greedy 4-stage assignment of normalised vectors -> (idx [n][4], final residuals [n][8])."""
+    r = _c(r, np.float32).reshape(-1, D)
+    cb = _c(codebooks, np.float32)
+    idx = np.empty((r.shape[0], S4), dtype=np.uint8)
+    res = np.empty_like(r)
+    lib().orc_vq4p_encode_vectors(r.ctypes.data, r.shape[0], cb.ctypes.data, idx.ctypes.data, res.ctypes.data)
+    return idx, res
+
+
+def vq4p_encode(W, dtype, codebooks):
+    """-> (planes uint8 [3][rows][cols/8], scales uint16 [rows] binary16 bits)."""
+    W = _w(W, dtype)
+    rows, cols = W.shape
+    cb = _c(codebooks, np.float32)
+    planes = np.empty((3, rows, cols // D), dtype=np.uint8)
+    sc = np.empty(rows, dtype=np.uint16)
+    rc = lib().orc_vq4p_encode(W.ctypes.data, DTYPES[dtype], rows, cols, cb.ctypes.data, planes.ctypes.data,
+                               sc.ctypes.data)
+    if rc:
+        raise ValueError("orc_vq4p_encode: bad shape")
+    return planes, sc
+
+
+def vq4p_decode(planes, scales, codebooks, out="f32"):
+    planes = _c(planes, np.uint8)
+    _, rows, V = planes.shape
+    scales = _c(scales, np.uint16)
+    cb = _c(codebooks, np.float32)
+    o = np.empty((rows, V * D), dtype=np.float32 if out == "f32" else np.uint16)
+    rc = lib().orc_vq4p_decode(planes.ctypes.data, scales.ctypes.data, cb.ctypes.data, rows, V * D, o.ctypes.data,
+                               DTYPES[out])
+    if rc:
+        raise ValueError("orc_vq4p_decode: bad shape")
+    return o
+
+
+def vq4p_train(vecs, iters):
+    """-> (codebooks float32 [4][64][8], trace float64 [4][iters+1])."""
+    v = _c(vecs, np.float32).reshape(-1, D)
+    cb = np.empty((S4, K4, D), dtype=np.float32)
+    tr = np.empty((S4, iters + 1), dtype=np.float64)
+    rc = lib().orc_vq4p_train(v.ctypes.data, v.shape[0], iters, cb.ctypes.data, tr.ctypes.data)
+    if rc:
+        raise ValueError("orc_vq4p_train failed (%d)" % rc)
+    return cb, tr
+
+
+def vq4p_bruteforce(r, codebooks):
+    r = _c(r, np.float32).reshape(-1, D)
+    cb = _c(codebooks, np.float32)
+    idx = np.empty((r.shape[0], 4), dtype=np.int32)
+    err = np.empty(r.shape[0], dtype=np.float64)
+    lib().orc_vq4p_bruteforce(r.ctypes.data, r.shape[0], cb.ctypes.data, idx.ctypes.data, err.ctypes.data)
+    return idx, err
+
+
+def vq4p_gemv(planes, scales, codebooks, x, x_dtype):
+    """y[b][i] = sum_c w_hat[i][c] x[b][c] in binary64 with the VQ4P decoded weights."""
+    return gemv(vq4p_decode(planes, scales, codebooks), x, x_dtype)

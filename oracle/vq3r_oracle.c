@@ -435,3 +435,217 @@ void orc_bruteforce_joint(const float* r, int64_t n, const float* codebooks, int
     best_err[i] = best;
   }
 }
+
+/* ---------------- VQ4P (page §5): 4 stages x 64 entries, 6-bit packed indices ---------------- */
+/*
+ * The page names VQ4P as VQ3R's sibling at the same 3.00 bits/weight: four
+ * stages of 64-entry codebooks, 6-bit indices packed so that the container is
+ * byte-for-byte the size of VQ3R's.  The page gives no packing, scale or
+ * arithmetic details; the readings taken here keep everything of VQ3R that
+ * applies and add the packing:
+ *   - the same per-row binary16 RMS scale and normalisation;
+ *   - stage s (s = 1..4) picks the nearest of 64 codewords to the running
+ *     residual with VQ3R's distance (binary32, every operation rounded, k
+ *     ascending) and tie rule (lowest index); r -= C_s[i_s];
+ *   - the four indices of a vector form the 24-bit word
+ *     i1 | i2 << 6 | i3 << 12 | i4 << 18, stored as three byte planes:
+ *     plane p of [3][rows][cols/8] holds byte p of each vector's word;
+ *   - decode: (float)scale * (((C1 + C2) + C3) + C4) in binary32;
+ *   - Lloyd per stage as for VQ3R with 64 centroids (init = first 64
+ *     vectors).
+ */
+#define ORC_K4 64
+#define ORC_S4 4
+
+static int nearest_k(const float* r, const float* C, int K) {
+  float best = INFINITY;
+  int bi = 0;
+  for (int j = 0; j < K; j++) {
+    const float* c = C + ORC_D * j;
+    float e = r[0] - c[0];
+    float d = e * e;
+    for (int k = 1; k < ORC_D; k++) {
+      float ek = r[k] - c[k];
+      float sq = ek * ek;
+      d = d + sq;
+    }
+    if (d < best) { best = d; bi = j; }
+  }
+  return bi;
+}
+
+/* idx4 [4][n] (one byte per index, values < 64) <-> planes [3][n]. */
+void orc_vq4p_pack(const uint8_t* idx4, int64_t n, uint8_t* planes) {
+  for (int64_t i = 0; i < n; i++) {
+    uint32_t w = (uint32_t)(idx4[i] & 63) | ((uint32_t)(idx4[n + i] & 63) << 6) |
+                 ((uint32_t)(idx4[2 * n + i] & 63) << 12) | ((uint32_t)(idx4[3 * n + i] & 63) << 18);
+    planes[i] = (uint8_t)(w & 0xFF);
+    planes[n + i] = (uint8_t)((w >> 8) & 0xFF);
+    planes[2 * n + i] = (uint8_t)((w >> 16) & 0xFF);
+  }
+}
+
+void orc_vq4p_unpack(const uint8_t* planes, int64_t n, uint8_t* idx4) {
+  for (int64_t i = 0; i < n; i++) {
+    uint32_t w = (uint32_t)planes[i] | ((uint32_t)planes[n + i] << 8) | ((uint32_t)planes[2 * n + i] << 16);
+    for (int s = 0; s < ORC_S4; s++) idx4[(int64_t)s * n + i] = (uint8_t)((w >> (6 * s)) & 63);
+  }
+}
+
+/* Greedy 4-stage assignment of n normalised vectors: idx4 [n][4] (vector-major),
+ * resid_out (optional) the final residuals. */
+void orc_vq4p_encode_vectors(const float* r_in, int64_t n, const float* codebooks, uint8_t* idx4, float* resid_out) {
+  #pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; i++) {
+    float r[ORC_D];
+    for (int k = 0; k < ORC_D; k++) r[k] = r_in[i * ORC_D + k];
+    for (int s = 0; s < ORC_S4; s++) {
+      const float* C = codebooks + (int64_t)s * ORC_K4 * ORC_D;
+      int j = nearest_k(r, C, ORC_K4);
+      idx4[i * ORC_S4 + s] = (uint8_t)j;
+      for (int k = 0; k < ORC_D; k++) r[k] = r[k] - C[ORC_D * j + k];
+    }
+    if (resid_out)
+      for (int k = 0; k < ORC_D; k++) resid_out[i * ORC_D + k] = r[k];
+  }
+}
+
+/* Encode a rows x cols matrix: scales[rows] and the packed planes [3][rows][cols/8]. */
+int orc_vq4p_encode(const void* W, int dtype, int64_t rows, int64_t cols, const float* codebooks, uint8_t* planes,
+                    uint16_t* scales) {
+  if (rows < 0 || cols < ORC_D || cols % ORC_D) return 2;
+  int64_t V = cols / ORC_D, n = rows * V;
+  #pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < rows; i++) {
+    uint16_t s = orc_row_scale(W, dtype, i, cols);
+    scales[i] = s;
+    for (int64_t v = 0; v < V; v++) {
+      float r[ORC_D];
+      normalise(W, dtype, cols, i, v, s, r);
+      uint32_t w = 0;
+      for (int st = 0; st < ORC_S4; st++) {
+        const float* C = codebooks + (int64_t)st * ORC_K4 * ORC_D;
+        int j = nearest_k(r, C, ORC_K4);
+        w |= (uint32_t)j << (6 * st);
+        for (int k = 0; k < ORC_D; k++) r[k] = r[k] - C[ORC_D * j + k];
+      }
+      planes[i * V + v] = (uint8_t)(w & 0xFF);
+      planes[n + i * V + v] = (uint8_t)((w >> 8) & 0xFF);
+      planes[2 * n + i * V + v] = (uint8_t)((w >> 16) & 0xFF);
+    }
+  }
+  return 0;
+}
+
+/* w_hat = (float)scale * (((C1 + C2) + C3) + C4), binary32; out_dtype as orc_decode. */
+int orc_vq4p_decode(const uint8_t* planes, const uint16_t* scales, const float* codebooks, int64_t rows, int64_t cols,
+                    void* out, int out_dtype) {
+  if (rows < 0 || cols < ORC_D || cols % ORC_D) return 2;
+  int64_t V = cols / ORC_D, n = rows * V;
+  #pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < rows; i++) {
+    float sf = (float)orc_fp16_to_double(scales[i]);
+    for (int64_t v = 0; v < V; v++) {
+      int64_t e = i * V + v;
+      uint32_t w = (uint32_t)planes[e] | ((uint32_t)planes[n + e] << 8) | ((uint32_t)planes[2 * n + e] << 16);
+      for (int k = 0; k < ORC_D; k++) {
+        float acc = codebooks[(int64_t)(w & 63) * ORC_D + k];
+        for (int st = 1; st < ORC_S4; st++) {
+          int j = (int)((w >> (6 * st)) & 63);
+          acc = acc + codebooks[((int64_t)st * ORC_K4 + j) * ORC_D + k];
+        }
+        float x = sf * acc;
+        int64_t o = i * cols + v * ORC_D + k;
+        if (out_dtype == ORC_F16) ((uint16_t*)out)[o] = orc_fp16_from_float(x);
+        else if (out_dtype == ORC_BF16) ((uint16_t*)out)[o] = orc_bf16_from_float(x);
+        else ((float*)out)[o] = x;
+      }
+    }
+  }
+  return 0;
+}
+
+/* Lloyd per stage with 64 centroids; as orc_lloyd_train otherwise. */
+int orc_vq4p_train(const float* vecs, int64_t n, int iters, float* codebooks, double* trace) {
+  if (n < ORC_K4 || iters < 0) return 2;
+  float* R = (float*)malloc(sizeof(float) * (size_t)n * ORC_D);
+  int* a = (int*)malloc(sizeof(int) * (size_t)n);
+  double* sum = (double*)malloc(sizeof(double) * ORC_K4 * ORC_D);
+  int64_t* cnt = (int64_t*)malloc(sizeof(int64_t) * ORC_K4);
+  if (!R || !a || !sum || !cnt) { free(R); free(a); free(sum); free(cnt); return 3; }
+  memcpy(R, vecs, sizeof(float) * (size_t)n * ORC_D);
+  for (int s = 0; s < ORC_S4; s++) {
+    float* C = codebooks + (int64_t)s * ORC_K4 * ORC_D;
+    memcpy(C, R, sizeof(float) * ORC_K4 * ORC_D);
+    for (int it = 0; it <= iters; it++) {
+      double dist = 0.0;
+      #pragma omp parallel for schedule(static)
+      for (int64_t i = 0; i < n; i++) a[i] = nearest_k(R + i * ORC_D, C, ORC_K4);
+      for (int64_t i = 0; i < n; i++)
+        for (int k = 0; k < ORC_D; k++) {
+          double e = (double)R[i * ORC_D + k] - (double)C[a[i] * ORC_D + k];
+          dist = dist + e * e;
+        }
+      if (trace) trace[(int64_t)s * (iters + 1) + it] = dist;
+      if (it == iters) break;
+      memset(sum, 0, sizeof(double) * ORC_K4 * ORC_D);
+      memset(cnt, 0, sizeof(int64_t) * ORC_K4);
+      for (int64_t i = 0; i < n; i++) {
+        cnt[a[i]]++;
+        for (int k = 0; k < ORC_D; k++) sum[a[i] * ORC_D + k] = sum[a[i] * ORC_D + k] + (double)R[i * ORC_D + k];
+      }
+      for (int j = 0; j < ORC_K4; j++)
+        if (cnt[j] > 0)
+          for (int k = 0; k < ORC_D; k++) C[j * ORC_D + k] = (float)(sum[j * ORC_D + k] / (double)cnt[j]);
+    }
+    for (int64_t i = 0; i < n; i++)
+      for (int k = 0; k < ORC_D; k++) R[i * ORC_D + k] = R[i * ORC_D + k] - C[a[i] * ORC_D + k];
+  }
+  free(R); free(a); free(sum); free(cnt);
+  return 0;
+}
+
+/* Exhaustive joint search over all 64^4 quadruples (binary64), per vector. */
+void orc_vq4p_bruteforce(const float* r, int64_t n, const float* codebooks, int32_t* best_idx, double* best_err) {
+  const float* C = codebooks;
+  for (int64_t i = 0; i < n; i++) {
+    double best = INFINITY;
+    int32_t bb[4] = {0, 0, 0, 0};
+    #pragma omp parallel
+    {
+      double lbest = INFINITY;
+      int32_t lb[4] = {0, 0, 0, 0};
+      #pragma omp for schedule(static)
+      for (int a = 0; a < ORC_K4; a++)
+        for (int b = 0; b < ORC_K4; b++)
+          for (int c = 0; c < ORC_K4; c++) {
+            double p[ORC_D];
+            for (int k = 0; k < ORC_D; k++)
+              p[k] = (double)r[i * ORC_D + k] - (((double)C[a * ORC_D + k] + (double)C[(ORC_K4 + b) * ORC_D + k]) +
+                                                 (double)C[(2 * ORC_K4 + c) * ORC_D + k]);
+            for (int d = 0; d < ORC_K4; d++) {
+              double e = 0.0;
+              for (int k = 0; k < ORC_D; k++) {
+                double t = p[k] - (double)C[(3 * ORC_K4 + d) * ORC_D + k];
+                e = e + t * t;
+              }
+              if (e < lbest) { lbest = e; lb[0] = a; lb[1] = b; lb[2] = c; lb[3] = d; }
+            }
+          }
+      #pragma omp critical
+      {
+        int better = lbest < best;
+        if (lbest == best)
+          for (int q = 0; q < 4; q++) {
+            if (lb[q] != bb[q]) { better = lb[q] < bb[q]; break; }
+          }
+        if (better) {
+          best = lbest;
+          for (int q = 0; q < 4; q++) bb[q] = lb[q];
+        }
+      }
+    }
+    for (int q = 0; q < 4; q++) best_idx[i * 4 + q] = bb[q];
+    best_err[i] = best;
+  }
+}

@@ -3,7 +3,8 @@ fix, independent of the oracle's own code.
 
 Page: "3比特逼近4比特精度？WARP残差向量量化VQ3R的完整测量实验"
 (xdnf.cn/news/289497), §2 (format, reconstruction rule, Lloyd codebooks),
-§3.1 (relative Frobenius error, rtn4-row, vq2), §4 (greedy single pass).
+§3.1 (relative Frobenius error, rtn4-row, vq2), §4 (greedy single pass),
+§5 (the VQ4P sibling: 4 stages x 64 entries, 6-bit packed indices).
 """
 import math
 from fractions import Fraction
@@ -398,3 +399,110 @@ def test_tiny_pipeline_sanity_bands():
     rt, _ = oracle.rtn4_row(W, "f32")
     e4 = oracle.rel_frobenius(W, "f32", rt)
     assert 0.10 < e3 < 0.26 and e2 > e3 and 0.10 < e4 < 0.18, (e4, e3, e2)
+
+
+# ---------------------------------------------------------------- VQ4P, VQ3R's sibling (§5)
+
+K4 = 64
+
+
+def test_vq4p_packing_layout():
+    """Four 6-bit indices per vector in the 24-bit word i1 | i2 << 6 | i3 << 12 | i4 << 18, stored as three
+    byte planes: exactly the bytes of VQ3R's three index planes (3.00 bits/weight)."""
+    idx = np.array([[1], [2], [4], [8]], dtype=np.uint8)  # word 0x204081
+    np.testing.assert_array_equal(oracle.vq4p_pack(idx)[:, 0], [0x81, 0x40, 0x20])
+    np.testing.assert_array_equal(oracle.vq4p_pack(np.full((4, 1), 63, np.uint8))[:, 0], [0xFF, 0xFF, 0xFF])
+    np.testing.assert_array_equal(oracle.vq4p_pack(np.array([[0], [0], [0], [63]], np.uint8))[:, 0], [0, 0, 0xFC])
+    rng = np.random.default_rng(40)
+    idx = rng.integers(0, K4, size=(4, 7, 33), dtype=np.uint8)
+    planes = oracle.vq4p_pack(idx)
+    assert planes.shape == (3, 7, 33)
+    np.testing.assert_array_equal(oracle.vq4p_unpack(planes), idx)
+
+
+def _vq4p_sign_codebooks():
+    """Stage s codeword j: dims 0..5 = -step if bit k of j is set else +step (step = 1, 1/2, 1/4, 1/8),
+    dims 6 and 7 zero."""
+    cb = np.zeros((4, K4, D), np.float32)
+    for s, step in enumerate([1.0, 0.5, 0.25, 0.125]):
+        for j in range(K4):
+            for k in range(6):
+                cb[s, j, k] = -step if (j >> k) & 1 else step
+    return cb
+
+
+def test_vq4p_sign_codebooks_equal_16_level_scalar_quantizer():
+    """With those codebooks greedy VQ4P quantises dims 0..5 independently by sign at each stage (the 16-level
+    uniform scalar quantizer), a zero residual taking the positive codeword (the lower index); inputs on a
+    1/64 grid keep all binary32 arithmetic exact, so the expected indices follow in rationals."""
+    rng = np.random.default_rng(41)
+    cb = _vq4p_sign_codebooks()
+    r = np.zeros((300, D), np.float32)
+    r[:, :6] = rng.integers(-128, 129, size=(300, 6)) / 64.0
+    r[:5, :6] = 0.0  # ties everywhere at stage 1
+    idx, res = oracle.vq4p_encode_vectors(r, cb)
+    for i in range(300):
+        e = [Fraction(float(v)) for v in r[i, :6]]
+        for s, step in enumerate([Fraction(1), Fraction(1, 2), Fraction(1, 4), Fraction(1, 8)]):
+            bits = [1 if ek < 0 else 0 for ek in e]
+            assert idx[i, s] == sum(b << k for k, b in enumerate(bits)), (i, s)
+            e = [ek + step if b else ek - step for ek, b in zip(e, bits)]
+        np.testing.assert_array_equal(res[i, :6], np.array([float(v) for v in e], np.float32))
+        assert not res[i, 6:].any()
+
+
+def test_vq4p_planted_exact_reconstruction():
+    """Rows s * C1[pi(v)] with 64 distinct +-1 patterns as C1 and a zero codeword 0 in C2..C4: scale s exactly,
+    indices (pi(v), 0, 0, 0), decode exact, error 0."""
+    rng = np.random.default_rng(42)
+    cb = (rng.standard_normal((4, K4, D)) * np.array([1.0, 0.3, 0.1, 0.03])[:, None, None]).astype(np.float32)
+    for j in range(K4):
+        cb[0, j] = [-1.0 if (j >> k) & 1 else 1.0 for k in range(6)] + [-1.0 if bin(j).count("1") & 1 else 1.0, 1.0]
+    cb[0] = cb[0][rng.permutation(K4)]
+    cb[1:, 0] = 0.0
+    rows, V = 6, 16
+    pi = rng.integers(0, K4, size=(rows, V))
+    svals = np.array([0.75, 3.0, 2.0 ** -6, 1.5, 40.0, 0.125], dtype=np.float32)
+    W = (cb[0][pi].reshape(rows, V * D) * svals[:, None]).astype(np.float32)
+    planes, sc = oracle.vq4p_encode(W, "f32", cb)
+    np.testing.assert_array_equal([oracle.fp16_to_double(s) for s in sc], svals.astype(np.float64))
+    idx = oracle.vq4p_unpack(planes)
+    np.testing.assert_array_equal(idx[0], pi)
+    assert not idx[1:].any()
+    What = oracle.vq4p_decode(planes, sc, cb)
+    np.testing.assert_array_equal(What, W)
+    assert oracle.rel_frobenius(W, "f32", What) == 0.0
+
+
+def test_vq4p_exhaustive_joint_search_lower_bounds_greedy():
+    rng = np.random.default_rng(43)
+    cb = (rng.standard_normal((4, K4, D)) * np.array([1.0, 0.5, 0.25, 0.125])[:, None, None]).astype(np.float32)
+    r = rng.standard_normal((2, D)).astype(np.float32)
+    idx, _ = oracle.vq4p_encode_vectors(r, cb)
+    g = sum(cb[s][idx[:, s]].astype(np.float64) for s in range(4))
+    greedy_err = ((r.astype(np.float64) - g) ** 2).sum(1)
+    bidx, berr = oracle.vq4p_bruteforce(r, cb)
+    assert np.all(berr <= greedy_err + 1e-12)
+    bj = sum(cb[s][bidx[:, s]].astype(np.float64) for s in range(4))
+    np.testing.assert_allclose(((r.astype(np.float64) - bj) ** 2).sum(1), berr, rtol=1e-12)
+
+
+def test_vq4p_lloyd_matches_sklearn_and_stages_reduce_error():
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(44)
+    X = rng.standard_normal((4096, D)).astype(np.float32)
+    cb, tr = oracle.vq4p_train(X, 4)
+    km = KMeans(n_clusters=K4, init=X[:K4].astype(np.float64), n_init=1, max_iter=4, tol=0.0,
+                algorithm="lloyd").fit(X.astype(np.float64))
+    close = np.all(np.abs(km.cluster_centers_ - cb[0]) < 1e-5, axis=1)
+    assert close.mean() > 0.95
+    for s in range(4):
+        assert np.all(np.diff(tr[s]) <= 1e-6 * tr[s][0])
+    idx, res = oracle.vq4p_encode_vectors(X, cb)
+    np.testing.assert_allclose(tr[3, -1], float((res.astype(np.float64) ** 2).sum()), rtol=1e-6)
+    # each added stage lowers the training error
+    errs = []
+    for ns in range(1, 5):
+        g = sum(cb[s][idx[:, s]].astype(np.float64) for s in range(ns))
+        errs.append(float(((X.astype(np.float64) - g) ** 2).sum()))
+    assert errs[0] > errs[1] > errs[2] > errs[3]
