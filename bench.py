@@ -35,6 +35,7 @@ from synth import workloads as wl  # noqa: E402
 
 METRIC = "VQ3R encode Gweights/s (vs fp32 peak); decode-GEMV GB/s vs HBM roofline, 1 B200"
 FLOPS_PER_WEIGHT = 2304  # 3 stages x 256 codewords x 8 dims x (sub, mul, add) / 8 weights
+VQ4P_FLOPS_PER_WEIGHT = 768  # 4 stages x 64 codewords x 8 dims x (sub, mul, add) / 8 weights
 # DRAM bytes (read + write) per weight of the encode kernel, from an ncu capture
 # of this kernel (dram__bytes_read.sum + dram__bytes_write.sum over 117.4 M
 # weights); None once the kernel changes and until it is captured again.
@@ -67,7 +68,7 @@ def load_codebooks(name):
             if line.startswith("#") or not line.strip():
                 continue
             rows.append([int(t, 16) for t in line.split()])
-    return np.array(rows, dtype=np.uint32).view(np.float32).reshape(3, 256, 8)
+    return np.array(rows, dtype=np.uint32).view(np.float32).reshape((4, 64, 8) if name.startswith("vq4p_") else (3, 256, 8))
 
 
 def peaks():
@@ -541,6 +542,42 @@ def main():
         train = {"vectors": 65536, "stages": 3, "iters": 20, "ms": a.elapsed_time(b)}
         del vecs, wst
 
+    # VQ4P (page §5: 4 stages x 64 codewords, packed 6-bit indices, the same 3.00 bits/weight) on the layer's
+    # stacked gate matrix, beside VQ3R's decode of the same matrix: encode, decode to fp32, error
+    vq4p = None
+    if args.gemm_iters > 0:
+        k = wl.W1
+        cb4 = torch.from_numpy(load_codebooks("vq4p_layer")).to(dev)
+        pl = torch.empty_like(layer.idx[k])
+        sc4 = torch.empty_like(layer.sc[k])
+        e4 = torch.empty(1, dtype=torch.float64, device=dev)
+        n_w = layer.W[k].numel()
+
+        def timed(fn, reps):
+            fn()
+            torch.cuda.synchronize()
+            a, b = ev(), ev()
+            a.record()
+            for _ in range(reps):
+                fn()
+            b.record()
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / reps
+
+        enc4_ms = timed(lambda: vq.vq4p_encode(layer.W[k], cb4, pl, sc4), 2)
+        dec4_ms = timed(lambda: vq.vq4p_decode(pl, sc4, cb4, out=layer.dec[k]), 3)
+        dec3_ms = timed(lambda: vq.vq3r_decode(layer.idx[k], layer.sc[k], layer.cb, out=layer.dec[k]), 3)
+        err4_ms = timed(lambda: vq.vq4p_rel_frobenius_error(layer.W[k], pl, sc4, cb4, out=e4,
+                                                            workspace=layer.err_ws[k]), 3)
+        vq4p = {"matrix": "w1 of the layer, %d x %d stacked" % tuple(layer.W[k].shape),
+                "encode_ms": enc4_ms, "encode_TFLOP/s": VQ4P_FLOPS_PER_WEIGHT * n_w / enc4_ms / 1e9,
+                "encode_frac_alu": VQ4P_FLOPS_PER_WEIGHT * n_w / enc4_ms / 1e9 / fp32_peak_tflops,
+                "decode_f32_ms": dec4_ms, "decode_f32_frac_hbm": n_w * 4.375 / dec4_ms / 1e6 / hbm_gbs,
+                "vq3r_decode_f32_ms": dec3_ms, "decode_speedup_vs_vq3r": dec3_ms / dec4_ms,
+                "rel_frobenius_ms": err4_ms, "rel_frobenius_frac_hbm": n_w * 2.375 / err4_ms / 1e6 / hbm_gbs,
+                "error": float(e4.item()), "vq3r_error": float(layer.err[k].item())}
+        del pl, sc4, cb4
+
     # end to end through the public API with host buffers: H2D of the layer, the step, D2H of the results
     e2e = None
     if args.e2e_steps > 0:
@@ -616,6 +653,7 @@ def main():
                 "gemv_layer_sweep": layer_sweep,
                 "gemm_prefill": prefill,
                 "train_lloyd": train,
+                "vq4p": vq4p,
                 "hbm_peak_gbs": hbm_gbs, "peak_source": peak_src},
             "e2e": e2e,
             "gpu_launches": Layer.LAUNCHES_PER_STEP * args.steps,

@@ -300,6 +300,35 @@ typedef struct {
 
 vq3r_status vq3r_gemm(const vq3r_gemm_desc* mats, int n_mats, vq3r_dtype x_dtype, vq3r_stream stream);
 
+/*
+ * VQ4P -- the sibling format of page §5 at the same 3.00 bits/weight: four
+ * stages of 64-entry codebooks (6-bit indices) instead of three of 256.
+ * Readings where the page names the format but gives no layout: the
+ * encoder, scale, distance, tie rule and stage order are vq3r_encode's with
+ * S = 4 stages and K = 64 codewords; the four indices of a vector form the
+ * 24-bit word  w = i1 | i2 << 6 | i3 << 12 | i4 << 18  whose byte p (p = 0,
+ * 1, 2) is stored in byte plane p, so the index storage is byte for byte
+ * that of VQ3R.
+ *   codebooks  [4][64][8] float, stage-major, 8 KiB
+ *   planes     [3][rows][cols/8] uint8, plane p = byte p of w
+ *   w_hat[i][8v+k] = (float)scale_i * (((C1[i1][k] + C2[i2][k]) + C3[i3][k]) + C4[i4][k])
+ * in binary32, every operation rounded.  Arguments, conventions, errors and
+ * bit-exactness are those of the VQ3R call of the same name.
+ */
+vq3r_status vq4p_encode(const void* W, vq3r_dtype w_dtype, int64_t rows, int64_t cols, const float* codebooks,
+                        uint8_t* planes, uint16_t* scales, vq3r_stream stream);
+vq3r_status vq4p_decode(const uint8_t* planes, const uint16_t* scales, const float* codebooks, int64_t rows,
+                        int64_t cols, void* out, vq3r_dtype out_dtype, vq3r_stream stream);
+/* workspace: at least vq3r_rel_frobenius_workspace_size(rows, cols) bytes */
+vq3r_status vq4p_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const uint8_t* planes, const uint16_t* scales,
+                                     const float* codebooks, int64_t rows, int64_t cols, double* err_out,
+                                     void* workspace, size_t ws_bytes, vq3r_stream stream);
+/* vq3r_train's Lloyd reading with 64 centroids per stage (initial centroids:
+ * the first 64 vectors); n >= 64, nstages 1..4, codebooks [nstages][64][8]. */
+size_t vq4p_train_workspace_size(int64_t n);
+vq3r_status vq4p_train(const float* vecs, int64_t n, int iters, int nstages, float* codebooks, double* trace,
+                       void* workspace, size_t ws_bytes, vq3r_stream stream);
+
 /* Human-readable name of a status code (static string). */
 const char* vq3r_status_string(vq3r_status s);
 

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_DIR, "csrc", "libvq3r.so")
 VQ3R_F32, VQ3R_BF16, VQ3R_F16 = 0, 1, 2
 _DT = {torch.float32: VQ3R_F32, torch.bfloat16: VQ3R_BF16, torch.float16: VQ3R_F16}
 STAGES, CODEWORDS, DIM = 3, 256, 8
+VQ4P_STAGES, VQ4P_CODEWORDS = 4, 64  # VQ4P: 4 stages x 64 codewords, indices packed in 3 byte planes
 GEMV_MAX_B = 32
 GEMV_MAX_MATS = 32
 LAYOUT_PLANES, LAYOUT_TILES = 0, 1
@@ -25,7 +26,8 @@ TILE_ROWS, TILE_BYTES, SLAB_COLS = 512, 32768, 512
 EXPORTED = ["vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_gemv_workspace_size", "vq3r_rel_frobenius_error",
             "vq3r_rel_frobenius_workspace_size", "vq3r_status_string", "vq3r_last_cuda_error",
             "vq3r_device_error", "vq3r_gemv_noalloc", "vq3r_tiles_size", "vq3r_pack_tiles", "vq3r_gemm",
-            "vq3r_train", "vq3r_train_workspace_size"]
+            "vq3r_train", "vq3r_train_workspace_size", "vq4p_encode", "vq4p_decode", "vq4p_rel_frobenius_error",
+            "vq4p_train", "vq4p_train_workspace_size"]
 
 
 class VQ3RError(RuntimeError):
@@ -79,8 +81,15 @@ def _lib():
         L.vq3r_train.argtypes = [P, I64, I32, I32, P, P, P, SZ, P]
         L.vq3r_train_workspace_size.argtypes = [I64]
         L.vq3r_train_workspace_size.restype = SZ
+        L.vq4p_encode.argtypes = L.vq3r_encode.argtypes
+        L.vq4p_decode.argtypes = L.vq3r_decode.argtypes
+        L.vq4p_rel_frobenius_error.argtypes = L.vq3r_rel_frobenius_error.argtypes
+        L.vq4p_train.argtypes = L.vq3r_train.argtypes
+        L.vq4p_train_workspace_size.argtypes = [I64]
+        L.vq4p_train_workspace_size.restype = SZ
         for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error",
-                  "vq3r_gemv_noalloc", "vq3r_pack_tiles", "vq3r_gemm", "vq3r_train"):
+                  "vq3r_gemv_noalloc", "vq3r_pack_tiles", "vq3r_gemm", "vq3r_train", "vq4p_encode", "vq4p_decode",
+                  "vq4p_rel_frobenius_error", "vq4p_train"):
             getattr(L, f).restype = I32
         _L = L
     return _L
@@ -108,8 +117,7 @@ def _dev(t, name):
     return t.data_ptr()
 
 
-def vq3r_encode(W, codebooks, idx=None, scales=None, stream=None):
-    """Encode W [rows][cols] (f32/bf16/f16) -> (idx uint8 [3][rows][cols/8], scales int16 [rows] fp16 bits)."""
+def _encode(fn, W, codebooks, idx, scales, stream):
     rows, cols = W.shape
     if idx is None:
         idx = torch.empty((STAGES, rows, cols // DIM), dtype=torch.uint8, device=W.device)
@@ -117,19 +125,39 @@ def vq3r_encode(W, codebooks, idx=None, scales=None, stream=None):
         scales = torch.empty(rows, dtype=torch.int16, device=W.device)
     if W.dtype not in _DT:
         raise ValueError("W dtype must be float32, bfloat16 or float16")
-    _check(_lib().vq3r_encode(_dev(W, "W"), _DT[W.dtype], rows, cols, _dev(codebooks, "codebooks"),
-                              _dev(idx, "idx"), _dev(scales, "scales"), _stream(stream)), "vq3r_encode")
+    _check(getattr(_lib(), fn)(_dev(W, "W"), _DT[W.dtype], rows, cols, _dev(codebooks, "codebooks"),
+                               _dev(idx, "idx"), _dev(scales, "scales"), _stream(stream)), fn)
     return idx, scales
+
+
+def _decode(fn, idx, scales, codebooks, out_dtype, out, stream):
+    _, rows, V = idx.shape
+    if out is None:
+        out = torch.empty((rows, V * DIM), dtype=out_dtype, device=idx.device)
+    _check(getattr(_lib(), fn)(_dev(idx, "idx"), _dev(scales, "scales"), _dev(codebooks, "codebooks"), rows,
+                               V * DIM, _dev(out, "out"), _DT[out.dtype], _stream(stream)), fn)
+    return out
+
+
+def vq3r_encode(W, codebooks, idx=None, scales=None, stream=None):
+    """Encode W [rows][cols] (f32/bf16/f16) -> (idx uint8 [3][rows][cols/8], scales int16 [rows] fp16 bits)."""
+    return _encode("vq3r_encode", W, codebooks, idx, scales, stream)
 
 
 def vq3r_decode(idx, scales, codebooks, out_dtype=torch.float32, out=None, stream=None):
     """Reconstruct W_hat [rows][cols] as float32 or float16."""
-    _, rows, V = idx.shape
-    if out is None:
-        out = torch.empty((rows, V * DIM), dtype=out_dtype, device=idx.device)
-    _check(_lib().vq3r_decode(_dev(idx, "idx"), _dev(scales, "scales"), _dev(codebooks, "codebooks"), rows,
-                              V * DIM, _dev(out, "out"), _DT[out.dtype], _stream(stream)), "vq3r_decode")
-    return out
+    return _decode("vq3r_decode", idx, scales, codebooks, out_dtype, out, stream)
+
+
+def vq4p_encode(W, codebooks, planes=None, scales=None, stream=None):
+    """VQ4P encode with codebooks [4][64][8] -> (planes uint8 [3][rows][cols/8] holding the packed 24-bit
+    index words, scales int16 [rows] fp16 bits)."""
+    return _encode("vq4p_encode", W, codebooks, planes, scales, stream)
+
+
+def vq4p_decode(planes, scales, codebooks, out_dtype=torch.float32, out=None, stream=None):
+    """Reconstruct W_hat [rows][cols] from VQ4P planes as float32 or float16."""
+    return _decode("vq4p_decode", planes, scales, codebooks, out_dtype, out, stream)
 
 
 def _descs(mats):
@@ -200,21 +228,36 @@ def vq3r_train_workspace_size(n):
     return _lib().vq3r_train_workspace_size(n)
 
 
-def vq3r_train(vecs, iters, nstages=STAGES, codebooks=None, trace=None, workspace=None, stream=None):
-    """Lloyd codebooks from training vectors [n][8] float32 -> (codebooks [nstages][256][8] float32,
-    trace [nstages][iters + 1] float64: the total squared distance after each assignment)."""
+def vq4p_train_workspace_size(n):
+    return _lib().vq4p_train_workspace_size(n)
+
+
+def _train(fn, K, vecs, iters, nstages, codebooks, trace, workspace, stream):
     n = vecs.shape[0]
     if vecs.dtype != torch.float32 or vecs.dim() != 2 or vecs.shape[1] != DIM:
         raise ValueError("vecs must be a float32 [n][8] tensor")
     if codebooks is None:
-        codebooks = torch.empty((nstages, CODEWORDS, DIM), dtype=torch.float32, device=vecs.device)
+        codebooks = torch.empty((nstages, K, DIM), dtype=torch.float32, device=vecs.device)
     if trace is None:
         trace = torch.empty((nstages, iters + 1), dtype=torch.float64, device=vecs.device)
     if workspace is None:
-        workspace = torch.empty(max(vq3r_train_workspace_size(n), 16), dtype=torch.uint8, device=vecs.device)
-    _check(_lib().vq3r_train(_dev(vecs, "vecs"), n, iters, nstages, _dev(codebooks, "codebooks"), _dev(trace, "trace"),
-                             _dev(workspace, "workspace"), workspace.numel(), _stream(stream)), "vq3r_train")
+        ws = getattr(_lib(), fn + "_workspace_size")(n)
+        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=vecs.device)
+    _check(getattr(_lib(), fn)(_dev(vecs, "vecs"), n, iters, nstages, _dev(codebooks, "codebooks"),
+                               _dev(trace, "trace"), _dev(workspace, "workspace"), workspace.numel(),
+                               _stream(stream)), fn)
     return codebooks, trace
+
+
+def vq3r_train(vecs, iters, nstages=STAGES, codebooks=None, trace=None, workspace=None, stream=None):
+    """Lloyd codebooks from training vectors [n][8] float32 -> (codebooks [nstages][256][8] float32,
+    trace [nstages][iters + 1] float64: the total squared distance after each assignment)."""
+    return _train("vq3r_train", CODEWORDS, vecs, iters, nstages, codebooks, trace, workspace, stream)
+
+
+def vq4p_train(vecs, iters, nstages=VQ4P_STAGES, codebooks=None, trace=None, workspace=None, stream=None):
+    """VQ4P Lloyd codebooks [nstages][64][8] float32 and the distortion trace, as vq3r_train."""
+    return _train("vq4p_train", VQ4P_CODEWORDS, vecs, iters, nstages, codebooks, trace, workspace, stream)
 
 
 def vq3r_tiles_size(rows, cols):
@@ -266,18 +309,26 @@ def vq3r_rel_frobenius_workspace_size(rows, cols):
     return _lib().vq3r_rel_frobenius_workspace_size(rows, cols)
 
 
-def vq3r_rel_frobenius_error(W, idx, scales, codebooks, out=None, workspace=None, stream=None):
-    """Device float64 tensor [1] holding sqrt(sum (w - w_hat)^2 / sum w^2)."""
+def _relfro(fn, W, idx, scales, codebooks, out, workspace, stream):
     rows, cols = W.shape
     if out is None:
         out = torch.empty(1, dtype=torch.float64, device=W.device)
     if workspace is None:
         workspace = torch.empty(vq3r_rel_frobenius_workspace_size(rows, cols), dtype=torch.uint8, device=W.device)
-    _check(_lib().vq3r_rel_frobenius_error(_dev(W, "W"), _DT[W.dtype], _dev(idx, "idx"), _dev(scales, "scales"),
-                                           _dev(codebooks, "codebooks"), rows, cols, _dev(out, "out"),
-                                           _dev(workspace, "workspace"), workspace.numel(), _stream(stream)),
-           "vq3r_rel_frobenius_error")
+    _check(getattr(_lib(), fn)(_dev(W, "W"), _DT[W.dtype], _dev(idx, "idx"), _dev(scales, "scales"),
+                               _dev(codebooks, "codebooks"), rows, cols, _dev(out, "out"),
+                               _dev(workspace, "workspace"), workspace.numel(), _stream(stream)), fn)
     return out
+
+
+def vq3r_rel_frobenius_error(W, idx, scales, codebooks, out=None, workspace=None, stream=None):
+    """Device float64 tensor [1] holding sqrt(sum (w - w_hat)^2 / sum w^2)."""
+    return _relfro("vq3r_rel_frobenius_error", W, idx, scales, codebooks, out, workspace, stream)
+
+
+def vq4p_rel_frobenius_error(W, planes, scales, codebooks, out=None, workspace=None, stream=None):
+    """vq3r_rel_frobenius_error for VQ4P planes and codebooks [4][64][8]."""
+    return _relfro("vq4p_rel_frobenius_error", W, planes, scales, codebooks, out, workspace, stream)
 
 
 def vq3r_device_error():

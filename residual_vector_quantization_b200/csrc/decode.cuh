@@ -17,15 +17,32 @@ namespace vq3r {
 
 constexpr int kDecThreads = 512;
 
+// Index formats.  FMT_VQ3R: three 1-byte indices into 256-entry codebooks
+// [3][256][8], one byte plane per stage.  FMT_VQ4P (page §5, VQ3R's sibling at
+// the same 3.00 bits/weight): four 6-bit indices into 64-entry codebooks
+// [4][64][8], packed into the 24-bit word i1 | i2 << 6 | i3 << 12 | i4 << 18
+// whose byte p is stored in plane p.  Both read three byte planes per vector.
+constexpr int FMT_VQ3R = 0, FMT_VQ4P = 1;
+template <int FMT>
+__host__ __device__ constexpr int fmt_codewords_total() {
+  return FMT == FMT_VQ4P ? 4 * 64 : kStages * kCodewords;
+}
+
 // Codebooks for gathers by 32 lanes: every codeword stored four times side by
-// side in a 128-byte row, cbr[s][j][copy][8].  Lane L reads copy (L >> 1) & 3,
-// half L & 1, so the eight lanes of a quarter-warp hit eight distinct 16-byte
-// bank groups whatever the indices are.  96 KiB.
-constexpr int kCbrFloats = kStages * kCodewords * 4 * kDim;
+// side in a 128-byte row, cbr[row][copy][8] with row = stage * K + j.  Lane L
+// reads copy (L >> 1) & 3, half L & 1, so the eight lanes of a quarter-warp
+// hit eight distinct 16-byte bank groups whatever the indices are.  96 KiB
+// for VQ3R, 32 KiB for VQ4P.
+template <int FMT>
+__host__ __device__ constexpr int fmt_cbr_floats() {
+  return fmt_codewords_total<FMT>() * 4 * kDim;
+}
+constexpr int kCbrFloats = fmt_cbr_floats<FMT_VQ3R>();
+template <int FMT>
 __device__ __forceinline__ void load_codebooks_replicated(float* cbr, const float* __restrict__ codebooks) {
   const float4* src = reinterpret_cast<const float4*>(codebooks);
   float4* dst = reinterpret_cast<float4*>(cbr);
-  for (int i = threadIdx.x; i < kCodebookFloats / 4; i += blockDim.x) {  // i: half of codeword i >> 1
+  for (int i = threadIdx.x; i < fmt_codewords_total<FMT>() * kDim / 4; i += blockDim.x) {  // i: half of codeword i >> 1
     const float4 v = __ldg(src + i);
 #pragma unroll
     for (int c = 0; c < 4; c++) dst[((i >> 1) * 4 + c) * 2 + (i & 1)] = v;
@@ -33,16 +50,52 @@ __device__ __forceinline__ void load_codebooks_replicated(float* cbr, const floa
   __syncthreads();
 }
 
+// Codebook rows of a vector from its three plane bytes e0, e1, e2.
+template <int FMT>
+__device__ __forceinline__ void fmt_rows(uint32_t e0, uint32_t e1, uint32_t e2, uint32_t r[4]) {
+  if constexpr (FMT == FMT_VQ4P) {
+    const uint32_t w = e0 | (e1 << 8) | (e2 << 16);
+    r[0] = w & 63u;
+    r[1] = 64u + ((w >> 6) & 63u);
+    r[2] = 128u + ((w >> 12) & 63u);
+    r[3] = 192u + (w >> 18);
+  } else {
+    r[0] = e0;
+    r[1] = kCodewords + e1;
+    r[2] = 2 * kCodewords + e2;
+    r[3] = 0;
+  }
+}
+
+// scale * (sum of the stage codewords, added in stage order), each operation rounded.
+template <int FMT>
+__device__ __forceinline__ float4 combine4(float s, const float4& a, const float4& b, const float4& c, const float4& d) {
+  if constexpr (FMT == FMT_VQ4P) {
+    return make_float4(__fmul_rn(s, __fadd_rn(__fadd_rn(__fadd_rn(a.x, b.x), c.x), d.x)),
+                       __fmul_rn(s, __fadd_rn(__fadd_rn(__fadd_rn(a.y, b.y), c.y), d.y)),
+                       __fmul_rn(s, __fadd_rn(__fadd_rn(__fadd_rn(a.z, b.z), c.z), d.z)),
+                       __fmul_rn(s, __fadd_rn(__fadd_rn(__fadd_rn(a.w, b.w), c.w), d.w)));
+  } else {
+    return make_float4(__fmul_rn(s, __fadd_rn(__fadd_rn(a.x, b.x), c.x)), __fmul_rn(s, __fadd_rn(__fadd_rn(a.y, b.y), c.y)),
+                       __fmul_rn(s, __fadd_rn(__fadd_rn(a.z, b.z), c.z)), __fmul_rn(s, __fadd_rn(__fadd_rn(a.w, b.w), c.w)));
+  }
+}
+
 // Half h = L & 1 (elements 4h .. 4h + 3) of w_hat for one vector:
-// (float)scale * ((C1 + C2) + C3), each operation rounded.
-__device__ __forceinline__ float4 decode_half_r(const float* cbr, uint32_t i1, uint32_t i2, uint32_t i3, float s,
+// (float)scale * ((C1 + C2) + C3) (VQ3R) or (((C1 + C2) + C3) + C4) (VQ4P),
+// each operation rounded.
+template <int FMT>
+__device__ __forceinline__ float4 decode_half_r(const float* cbr, uint32_t e0, uint32_t e1, uint32_t e2, float s,
                                                 int lane) {
   const int off = ((lane >> 1) & 3) * kDim + 4 * (lane & 1);
-  const float4 a = *reinterpret_cast<const float4*>(cbr + (0 * kCodewords + i1) * 4 * kDim + off);
-  const float4 b = *reinterpret_cast<const float4*>(cbr + (1 * kCodewords + i2) * 4 * kDim + off);
-  const float4 c = *reinterpret_cast<const float4*>(cbr + (2 * kCodewords + i3) * 4 * kDim + off);
-  return make_float4(__fmul_rn(s, __fadd_rn(__fadd_rn(a.x, b.x), c.x)), __fmul_rn(s, __fadd_rn(__fadd_rn(a.y, b.y), c.y)),
-                     __fmul_rn(s, __fadd_rn(__fadd_rn(a.z, b.z), c.z)), __fmul_rn(s, __fadd_rn(__fadd_rn(a.w, b.w), c.w)));
+  uint32_t r[4];
+  fmt_rows<FMT>(e0, e1, e2, r);
+  const float4 a = *reinterpret_cast<const float4*>(cbr + r[0] * 4 * kDim + off);
+  const float4 b = *reinterpret_cast<const float4*>(cbr + r[1] * 4 * kDim + off);
+  const float4 c = *reinterpret_cast<const float4*>(cbr + r[2] * 4 * kDim + off);
+  float4 d = make_float4(0.f, 0.f, 0.f, 0.f);
+  if constexpr (FMT == FMT_VQ4P) d = *reinterpret_cast<const float4*>(cbr + r[3] * 4 * kDim + off);
+  return combine4<FMT>(s, a, b, c, d);
 }
 
 // Traversal shared by decode and the error kernel.  Rows are split evenly over
@@ -98,13 +151,13 @@ __device__ __forceinline__ bool walk_batch(RowWalk& it, int64_t r1, const uint8_
   return true;
 }
 
-template <int OUT_DT>
+template <int OUT_DT, int FMT>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const uint8_t* __restrict__ idx,
                                                                  const uint16_t* __restrict__ scales,
                                                                  const float* __restrict__ codebooks, int64_t rows,
                                                                  int64_t cols, void* __restrict__ out) {
   extern __shared__ __align__(16) float cbr[];
-  load_codebooks_replicated(cbr, codebooks);
+  load_codebooks_replicated<FMT>(cbr, codebooks);
   const int lane = threadIdx.x & 31, h = lane & 1;
   const int64_t V = cols / kDim, nvec = rows * V;
   const int64_t r0 = (int64_t)blockIdx.x * rows / gridDim.x, r1 = (int64_t)(blockIdx.x + 1) * rows / gridDim.x;
@@ -116,7 +169,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const uint8_t* _
     for (int u = 0; u < kWalkUnroll; u++) {
       if (!wb.ok[u]) continue;
       const int64_t g = wb.g[u];
-      const float4 o = decode_half_r(cbr, wb.e[u][0], wb.e[u][1], wb.e[u][2], wb.s[u], lane);
+      const float4 o = decode_half_r<FMT>(cbr, wb.e[u][0], wb.e[u][1], wb.e[u][2], wb.s[u], lane);
       if constexpr (OUT_DT == VQ3R_F32) {
         __stcs(reinterpret_cast<float4*>(static_cast<float*>(out) + g * kDim + 4 * h), o);
       } else {
@@ -142,18 +195,19 @@ __device__ __forceinline__ double warp_sum_f64(double v) {
 
 // Whole w_hat vector for one lane: both halves, the lane's copy of each
 // codeword, half L & 1 first (conflict-free order for a quarter-warp).
-__device__ __forceinline__ void decode_vector_r(const float* cbr, uint32_t i1, uint32_t i2, uint32_t i3, float s,
+template <int FMT>
+__device__ __forceinline__ void decode_vector_r(const float* cbr, uint32_t e0, uint32_t e1, uint32_t e2, float s,
                                                 int lane, float4& lo, float4& hi) {
   const int copy = (lane >> 1) & 3, h0 = lane & 1;
-  const float4* c1 = reinterpret_cast<const float4*>(cbr + ((0 * kCodewords + i1) * 4 + copy) * kDim);
-  const float4* c2 = reinterpret_cast<const float4*>(cbr + ((1 * kCodewords + i2) * 4 + copy) * kDim);
-  const float4* c3 = reinterpret_cast<const float4*>(cbr + ((2 * kCodewords + i3) * 4 + copy) * kDim);
-  const float4 a0 = c1[h0], b0 = c2[h0], d0 = c3[h0];
-  const float4 a1 = c1[h0 ^ 1], b1 = c2[h0 ^ 1], d1 = c3[h0 ^ 1];
-  const float4 first = make_float4(__fmul_rn(s, __fadd_rn(__fadd_rn(a0.x, b0.x), d0.x)), __fmul_rn(s, __fadd_rn(__fadd_rn(a0.y, b0.y), d0.y)),
-                                   __fmul_rn(s, __fadd_rn(__fadd_rn(a0.z, b0.z), d0.z)), __fmul_rn(s, __fadd_rn(__fadd_rn(a0.w, b0.w), d0.w)));
-  const float4 second = make_float4(__fmul_rn(s, __fadd_rn(__fadd_rn(a1.x, b1.x), d1.x)), __fmul_rn(s, __fadd_rn(__fadd_rn(a1.y, b1.y), d1.y)),
-                                    __fmul_rn(s, __fadd_rn(__fadd_rn(a1.z, b1.z), d1.z)), __fmul_rn(s, __fadd_rn(__fadd_rn(a1.w, b1.w), d1.w)));
+  uint32_t r[4];
+  fmt_rows<FMT>(e0, e1, e2, r);
+  const float4* c1 = reinterpret_cast<const float4*>(cbr + (r[0] * 4 + copy) * kDim);
+  const float4* c2 = reinterpret_cast<const float4*>(cbr + (r[1] * 4 + copy) * kDim);
+  const float4* c3 = reinterpret_cast<const float4*>(cbr + (r[2] * 4 + copy) * kDim);
+  const float4* c4 = reinterpret_cast<const float4*>(cbr + (r[3] * 4 + copy) * kDim);
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4 first = combine4<FMT>(s, c1[h0], c2[h0], c3[h0], FMT == FMT_VQ4P ? c4[h0] : z);
+  const float4 second = combine4<FMT>(s, c1[h0 ^ 1], c2[h0 ^ 1], c3[h0 ^ 1], FMT == FMT_VQ4P ? c4[h0 ^ 1] : z);
   lo = h0 ? second : first;
   hi = h0 ? first : second;
 }
@@ -171,7 +225,7 @@ constexpr int kErrVecs = 4;  // consecutive vectors per thread and step
 // groups t, t + 512, ...: the index bytes of a group are one 32-bit word per
 // plane when V is a multiple of 4, and a warp's 16-byte W loads are 512
 // contiguous bytes.  Each thread keeps two binary64 sums, reduced per CTA.
-template <int DT>
+template <int DT, int FMT>
 __global__ void __launch_bounds__(kErrThreads, 2) relfro_partial_kernel(const void* __restrict__ W,
                                                                          const uint8_t* __restrict__ idx,
                                                                          const uint16_t* __restrict__ scales,
@@ -180,7 +234,7 @@ __global__ void __launch_bounds__(kErrThreads, 2) relfro_partial_kernel(const vo
                                                                          double* __restrict__ partial) {
   extern __shared__ __align__(16) float cbr[];
   __shared__ double red[2][kErrThreads / 32];
-  load_codebooks_replicated(cbr, codebooks);
+  load_codebooks_replicated<FMT>(cbr, codebooks);
   const int lane = threadIdx.x & 31;
   const int64_t V = cols / kDim, nvec = rows * V;
   const uint32_t gpr = (uint32_t)((V + kErrVecs - 1) / kErrVecs);  // groups per row
@@ -209,7 +263,7 @@ __global__ void __launch_bounds__(kErrThreads, 2) relfro_partial_kernel(const vo
     for (int i = 0; i < kErrVecs; i++) {
       if (i < n) {
         float4 lo, hi;
-        decode_vector_r(cbr, (w3[0] >> (8 * i)) & 0xFFu, (w3[1] >> (8 * i)) & 0xFFu, (w3[2] >> (8 * i)) & 0xFFu, s, lane,
+        decode_vector_r<FMT>(cbr, (w3[0] >> (8 * i)) & 0xFFu, (w3[1] >> (8 * i)) & 0xFFu, (w3[2] >> (8 * i)) & 0xFFu, s, lane,
                         lo, hi);
         float wv[8];
         load8<DT>(W, (g + i) * kDim, wv);

@@ -104,26 +104,32 @@ __device__ __forceinline__ float2 f2sq(float2 e, float2 z) {
   return d;
 }
 
-template <int DT>
+// FMT 0 (VQ3R): 3 stages x 256 codewords, index byte of stage s in plane s.
+// FMT 1 (VQ4P, page §5): 4 stages x 64 codewords, the 6-bit indices packed
+// into the 24-bit word i1 | i2 << 6 | i3 << 12 | i4 << 18, byte p in plane p.
+template <int DT, int FMT>
 __global__ void __launch_bounds__(kEncThreads, 2)
     encode_kernel(const void* __restrict__ W, int64_t cols, int64_t nvec, const float* __restrict__ codebooks,
                   const uint16_t* __restrict__ scales, uint8_t* __restrict__ idx, float zero) {
+  constexpr int S = FMT ? 4 : kStages, K = FMT ? 64 : kCodewords;
+  constexpr int kFloats = S * K * kDim;  // the caller's codebooks: 24 KiB (VQ3R), 8 KiB (VQ4P)
   extern __shared__ __align__(16) unsigned char enc_smem_raw[];
   EncSmem& sm = *reinterpret_cast<EncSmem*>(enc_smem_raw);
+  float2* const ncb = &sm.ncb[0][0][0];  // [S][K][8]
   const int tid = threadIdx.x;
 
-  // Stage the 24 KiB codebooks with one bulk asynchronous copy, then expand
-  // to negated, lane-duplicated pairs.
+  // Stage the codebooks with one bulk asynchronous copy, then expand to
+  // negated, lane-duplicated pairs.
   if (tid == 0) {
     mbar_init(&sm.mbar, 1);
-    mbar_arrive_expect_tx(&sm.mbar, kCodebookBytes);
-    bulk_copy_g2s(sm.raw, codebooks, kCodebookBytes, &sm.mbar);
+    mbar_arrive_expect_tx(&sm.mbar, kFloats * 4);
+    bulk_copy_g2s(sm.raw, codebooks, kFloats * 4, &sm.mbar);
   }
   __syncthreads();
   if (!mbar_wait_bounded(&sm.mbar, 0)) return;
-  for (int i = tid; i < kCodebookFloats; i += kEncThreads) {
+  for (int i = tid; i < kFloats; i += kEncThreads) {
     const float c = -sm.raw[i];
-    (&sm.ncb[0][0][0])[i] = make_float2(c, c);
+    ncb[i] = make_float2(c, c);
   }
   __syncthreads();
 
@@ -157,15 +163,16 @@ __global__ void __launch_bounds__(kEncThreads, 2)
       }
     }
 
+    uint32_t word[kEncVecPerThread] = {0u, 0u, 0u, 0u};  // VQ4P: packed indices
 #pragma unroll 1
-    for (int s = 0; s < kStages; s++) {
+    for (int s = 0; s < S; s++) {
       float best[kEncVecPerThread];
       int bi[kEncVecPerThread];
 #pragma unroll
       for (int q = 0; q < kEncVecPerThread; q++) { best[q] = __int_as_float(0x7F800000); bi[q] = 0; }
-      const float4* cw = reinterpret_cast<const float4*>(&sm.ncb[s][0][0]);
+      const float4* cw = reinterpret_cast<const float4*>(ncb + (size_t)s * K * kDim);
 #pragma unroll 4
-      for (int j = 0; j < kCodewords; j++) {
+      for (int j = 0; j < K; j++) {
         // (-c_k, -c_k) for k = 0..7: four broadcast 16-byte shared loads
         float2 c[kDim];
 #pragma unroll
@@ -190,12 +197,26 @@ __global__ void __launch_bounds__(kEncThreads, 2)
       // write the winning indices and update the residuals
 #pragma unroll
       for (int q = 0; q < kEncVecPerThread; q++) {
-        if (g[q] < nvec) idx[(int64_t)s * nvec + g[q]] = (uint8_t)bi[q];
-        const float2* cwin = &sm.ncb[s][bi[q]][0];
+        if constexpr (FMT == 0) {
+          if (g[q] < nvec) idx[(int64_t)s * nvec + g[q]] = (uint8_t)bi[q];
+        } else {
+          word[q] |= (uint32_t)bi[q] << (6 * s);
+        }
+        const float2* cwin = ncb + ((size_t)s * K + bi[q]) * kDim;
 #pragma unroll
         for (int k = 0; k < kDim; k++) {
           if (q & 1) r[q >> 1][k].y = __fadd_rn(r[q >> 1][k].y, cwin[k].x);
           else r[q >> 1][k].x = __fadd_rn(r[q >> 1][k].x, cwin[k].x);
+        }
+      }
+    }
+    if constexpr (FMT != 0) {  // the packed word's three bytes, one per plane
+#pragma unroll
+      for (int q = 0; q < kEncVecPerThread; q++) {
+        if (g[q] < nvec) {
+          idx[g[q]] = (uint8_t)(word[q] & 0xFFu);
+          idx[nvec + g[q]] = (uint8_t)((word[q] >> 8) & 0xFFu);
+          idx[2 * nvec + g[q]] = (uint8_t)(word[q] >> 16);
         }
       }
     }

@@ -30,14 +30,16 @@ namespace vq3r {
 constexpr int kTrainThreads = 256;
 constexpr int kTrainUpdateWarps = 8;  // centroids per CTA of the update kernel
 
-// a[i] = nearest centroid of vector i; part[blockIdx.x] = binary64 sum over the
-// CTA's vectors of their squared distance to it (for the trace).
+// a[i] = nearest of the K centroids to vector i; part[blockIdx.x] = binary64
+// sum over the CTA's vectors of their squared distance to it (for the trace).
+// K = 256 (VQ3R) or 64 (VQ4P).
+template <int K>
 __global__ void __launch_bounds__(kTrainThreads) train_assign_kernel(const float* __restrict__ R, int64_t n,
                                                                      const float* __restrict__ C,
                                                                      int32_t* __restrict__ a, double* __restrict__ part) {
-  __shared__ float cs[kCodewords * kDim];
+  __shared__ float cs[K * kDim];
   __shared__ double red[kTrainThreads / 32];
-  for (int i = threadIdx.x; i < kCodewords * kDim; i += kTrainThreads) cs[i] = C[i];
+  for (int i = threadIdx.x; i < K * kDim; i += kTrainThreads) cs[i] = C[i];
   __syncthreads();
   double acc = 0.0;
   for (int64_t i = (int64_t)blockIdx.x * kTrainThreads + threadIdx.x; i < n; i += (int64_t)gridDim.x * kTrainThreads) {
@@ -49,7 +51,7 @@ __global__ void __launch_bounds__(kTrainThreads) train_assign_kernel(const float
     float best = __int_as_float(0x7F800000);
     int bi = 0;
 #pragma unroll 4
-    for (int j = 0; j < kCodewords; j++) {
+    for (int j = 0; j < K; j++) {
       const float* c = cs + j * kDim;  // broadcast reads
       float e = __fsub_rn(r[0], c[0]);
       float d = __fmul_rn(e, e);
@@ -85,11 +87,12 @@ __global__ void __launch_bounds__(kTrainThreads) train_assign_kernel(const float
 
 // Centroid j = blockIdx.x * kTrainUpdateWarps + warp: the binary64 mean of its
 // members in training order, rounded to binary32 (unchanged when empty).
+template <int K>
 __global__ void __launch_bounds__(kTrainUpdateWarps * 32) train_update_kernel(const float* __restrict__ R, int64_t n,
                                                                               const int32_t* __restrict__ a,
                                                                               float* __restrict__ C) {
   const int lane = threadIdx.x & 31, j = blockIdx.x * kTrainUpdateWarps + (threadIdx.x >> 5);
-  if (j >= kCodewords) return;
+  if (j >= K) return;
   double sum = 0.0;  // component k = lane (lanes 0..7)
   int64_t cnt = 0;
   constexpr int kChunks = 8;  // 256 assignments per round, their loads all in flight

@@ -53,9 +53,12 @@ cudaError_t device_setup(int* sms) {
     const int enc = (int)sizeof(EncSmem);
     const int gv = (int)kGvSmemBytes;
     const int gt = (int)kTilesSmemBytes;
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F32, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_BF16, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F16, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F32, FMT_VQ4P>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_BF16, FMT_VQ4P>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(encode_kernel<VQ3R_F16, FMT_VQ4P>, cudaFuncAttributeMaxDynamicSharedMemorySize, enc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
@@ -64,11 +67,11 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
     const int gm = (int)kMmaSmemBytes;
     const int gc = (int)(kCbrFloats * sizeof(float));
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_kernel<VQ3R_F32, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_kernel<VQ3R_F16, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F32, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_BF16, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F16, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
@@ -247,7 +250,7 @@ void balance_split(GvParams& P, int n) {
   P.n_split = n;
 }
 
-template <int DT>
+template <int DT, int FMT>
 vq3r_status launch_encode(const void* W, int64_t rows, int64_t cols, const float* cb, uint8_t* idx,
                           uint16_t* scales, cudaStream_t s, int sms) {
   const int64_t nvec = rows * (cols / kDim);
@@ -255,7 +258,7 @@ vq3r_status launch_encode(const void* W, int64_t rows, int64_t cols, const float
   row_scale_kernel<DT><<<g1, kScaleThreads, 0, s>>>(W, rows, cols, scales);
   const int64_t ntiles = (nvec + kEncTile - 1) / kEncTile;
   const int g2 = (int)(ntiles < (int64_t)sms * 2 ? ntiles : (int64_t)sms * 2);
-  encode_kernel<DT><<<g2, kEncThreads, sizeof(EncSmem), s>>>(W, cols, nvec, cb, scales, idx, 0.0f);
+  encode_kernel<DT, FMT><<<g2, kEncThreads, sizeof(EncSmem), s>>>(W, cols, nvec, cb, scales, idx, 0.0f);
   return check_launch();
 }
 
@@ -272,22 +275,19 @@ int64_t rowsplit_blocks(int64_t rows, int64_t cols, int sms, int64_t cap) {
   return blocks;
 }
 
-template <int DT>
+template <int DT, int FMT>
 vq3r_status launch_relfro(const void* W, const uint8_t* idx, const uint16_t* scales, const float* cb, int64_t rows,
                           int64_t cols, double* err_out, double* partial, cudaStream_t s, int sms) {
   const int64_t blocks = rowsplit_blocks(rows, cols, sms, kErrMaxBlocks);
-  relfro_partial_kernel<DT><<<(int)blocks, kErrThreads, kCbrFloats * sizeof(float), s>>>(W, idx, scales, cb, rows,
-                                                                                          cols, partial);
+  relfro_partial_kernel<DT, FMT><<<(int)blocks, kErrThreads, fmt_cbr_floats<FMT>() * sizeof(float), s>>>(
+      W, idx, scales, cb, rows, cols, partial);
   relfro_final_kernel<<<1, 256, 0, s>>>(partial, (int)blocks, err_out);
   return check_launch();
 }
 
-}  // namespace
-
-extern "C" {
-
-vq3r_status vq3r_encode(const void* W, vq3r_dtype w_dtype, int64_t rows, int64_t cols, const float* codebooks,
-                        uint8_t* idx, uint16_t* scales, vq3r_stream stream) {
+template <int FMT>
+vq3r_status encode_entry(const void* W, vq3r_dtype w_dtype, int64_t rows, int64_t cols, const float* codebooks,
+                         uint8_t* idx, uint16_t* scales, vq3r_stream stream) {
   vq3r_status st = check_shape(rows, cols, 0);
   if (st != VQ3R_OK) return st;
   if (!valid_dtype(w_dtype)) return VQ3R_ERR_DTYPE;
@@ -299,14 +299,15 @@ vq3r_status vq3r_encode(const void* W, vq3r_dtype w_dtype, int64_t rows, int64_t
   if (e != cudaSuccess) return cuda_fail(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (w_dtype) {
-    case VQ3R_F32: return launch_encode<VQ3R_F32>(W, rows, cols, codebooks, idx, scales, s, sms);
-    case VQ3R_BF16: return launch_encode<VQ3R_BF16>(W, rows, cols, codebooks, idx, scales, s, sms);
-    default: return launch_encode<VQ3R_F16>(W, rows, cols, codebooks, idx, scales, s, sms);
+    case VQ3R_F32: return launch_encode<VQ3R_F32, FMT>(W, rows, cols, codebooks, idx, scales, s, sms);
+    case VQ3R_BF16: return launch_encode<VQ3R_BF16, FMT>(W, rows, cols, codebooks, idx, scales, s, sms);
+    default: return launch_encode<VQ3R_F16, FMT>(W, rows, cols, codebooks, idx, scales, s, sms);
   }
 }
 
-vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float* codebooks, int64_t rows,
-                        int64_t cols, void* out, vq3r_dtype out_dtype, vq3r_stream stream) {
+template <int FMT>
+vq3r_status decode_entry(const uint8_t* idx, const uint16_t* scales, const float* codebooks, int64_t rows,
+                         int64_t cols, void* out, vq3r_dtype out_dtype, vq3r_stream stream) {
   vq3r_status st = check_shape(rows, cols, 0);
   if (st != VQ3R_OK) return st;
   if (out_dtype != VQ3R_F32 && out_dtype != VQ3R_F16) return VQ3R_ERR_DTYPE;
@@ -318,12 +319,96 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
   if (e != cudaSuccess) return cuda_fail(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t blocks = rowsplit_blocks(rows, cols, sms, (int64_t)1 << 30);
-  const size_t smem = kCbrFloats * sizeof(float);
+  const size_t smem = fmt_cbr_floats<FMT>() * sizeof(float);
   if (out_dtype == VQ3R_F32)
-    decode_kernel<VQ3R_F32><<<(int)blocks, kDecThreads, smem, s>>>(idx, scales, codebooks, rows, cols, out);
+    decode_kernel<VQ3R_F32, FMT><<<(int)blocks, kDecThreads, smem, s>>>(idx, scales, codebooks, rows, cols, out);
   else
-    decode_kernel<VQ3R_F16><<<(int)blocks, kDecThreads, smem, s>>>(idx, scales, codebooks, rows, cols, out);
+    decode_kernel<VQ3R_F16, FMT><<<(int)blocks, kDecThreads, smem, s>>>(idx, scales, codebooks, rows, cols, out);
   return check_launch();
+}
+
+template <int FMT>
+vq3r_status relfro_entry(const void* W, vq3r_dtype w_dtype, const uint8_t* idx, const uint16_t* scales,
+                         const float* codebooks, int64_t rows, int64_t cols, double* err_out, void* workspace,
+                         size_t ws_bytes, vq3r_stream stream) {
+  if (!W || !idx || !scales || !codebooks || !err_out) return VQ3R_ERR_NULL;
+  vq3r_status st = check_shape(rows, cols, 1);
+  if (st != VQ3R_OK) return st;
+  if (!valid_dtype(w_dtype)) return VQ3R_ERR_DTYPE;
+  if (!workspace || ws_bytes < vq3r_rel_frobenius_workspace_size(rows, cols)) return VQ3R_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(idx) || !aligned16(scales) || !aligned16(codebooks) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(err_out) & 7u))
+    return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double* partial = static_cast<double*>(workspace);
+  switch (w_dtype) {
+    case VQ3R_F32: return launch_relfro<VQ3R_F32, FMT>(W, idx, scales, codebooks, rows, cols, err_out, partial, s, sms);
+    case VQ3R_BF16: return launch_relfro<VQ3R_BF16, FMT>(W, idx, scales, codebooks, rows, cols, err_out, partial, s, sms);
+    default: return launch_relfro<VQ3R_F16, FMT>(W, idx, scales, codebooks, rows, cols, err_out, partial, s, sms);
+  }
+}
+
+int train_grid(int64_t n, int sms) {
+  const int64_t need = (n + kTrainThreads - 1) / kTrainThreads;
+  return (int)(need < 2 * (int64_t)sms ? need : 2 * (int64_t)sms);
+}
+
+// residuals [n][8] float, assignments [n] int32, per-CTA trace partials (at most 2 per SM, 1024 SMs)
+size_t train_ws_bytes(int64_t n) {
+  return align_up((size_t)n * kDim * sizeof(float)) + align_up((size_t)n * sizeof(int32_t)) + 2048 * sizeof(double);
+}
+
+// Lloyd training of S stages of K codewords (VQ3R: 3 x 256, VQ4P: 4 x 64).
+template <int S, int K>
+vq3r_status train_entry(const float* vecs, int64_t n, int iters, int nstages, float* codebooks, double* trace,
+                        void* workspace, size_t ws_bytes, vq3r_stream stream) {
+  if (!vecs || !codebooks) return VQ3R_ERR_NULL;
+  if (n < K || n > ((int64_t)1 << 40) || iters < 0 || nstages < 1 || nstages > S) return VQ3R_ERR_SHAPE;
+  if (!workspace || ws_bytes < train_ws_bytes(n)) return VQ3R_ERR_WORKSPACE;
+  if (!aligned16(vecs) || !aligned16(codebooks) || !aligned16(workspace) || (trace && !aligned16(trace)))
+    return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (sms > 1024) return VQ3R_ERR_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(workspace);
+  float* R = reinterpret_cast<float*>(w);
+  int32_t* a = reinterpret_cast<int32_t*>(w + align_up((size_t)n * kDim * sizeof(float)));
+  double* part = reinterpret_cast<double*>(w + align_up((size_t)n * kDim * sizeof(float)) + align_up((size_t)n * sizeof(int32_t)));
+  const int grid = train_grid(n, sms);
+  e = cudaMemcpyAsync(R, vecs, (size_t)n * kDim * sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  for (int st = 0; st < nstages; st++) {
+    float* C = codebooks + (size_t)st * K * kDim;
+    e = cudaMemcpyAsync(C, R, (size_t)K * kDim * sizeof(float), cudaMemcpyDeviceToDevice, s);  // first K
+    if (e != cudaSuccess) return cuda_fail(e);
+    for (int it = 0; it <= iters; it++) {
+      train_assign_kernel<K><<<grid, kTrainThreads, 0, s>>>(R, n, C, a, part);
+      if (trace) train_trace_kernel<<<1, 32, 0, s>>>(part, grid, trace + (size_t)st * (iters + 1) + it);
+      if (it == iters) break;
+      train_update_kernel<K><<<K / kTrainUpdateWarps, kTrainUpdateWarps * 32, 0, s>>>(R, n, a, C);
+    }
+    if (st + 1 < nstages) train_residual_kernel<<<grid, kTrainThreads, 0, s>>>(R, n, C, a);
+  }
+  return check_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+vq3r_status vq3r_encode(const void* W, vq3r_dtype w_dtype, int64_t rows, int64_t cols, const float* codebooks,
+                        uint8_t* idx, uint16_t* scales, vq3r_stream stream) {
+  return encode_entry<FMT_VQ3R>(W, w_dtype, rows, cols, codebooks, idx, scales, stream);
+}
+
+vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float* codebooks, int64_t rows,
+                        int64_t cols, void* out, vq3r_dtype out_dtype, vq3r_stream stream) {
+  return decode_entry<FMT_VQ3R>(idx, scales, codebooks, rows, cols, out, out_dtype, stream);
 }
 
 size_t vq3r_gemv_workspace_size(const vq3r_gemv_desc* mats, int n_mats, int B) {
@@ -473,49 +558,24 @@ vq3r_status vq3r_gemm(const vq3r_gemm_desc* mats, int n_mats, vq3r_dtype x_dtype
   return check_launch();
 }
 
-int train_grid(int64_t n, int sms) {
-  const int64_t need = (n + kTrainThreads - 1) / kTrainThreads;
-  return (int)(need < 2 * (int64_t)sms ? need : 2 * (int64_t)sms);
-}
-
 size_t vq3r_train_workspace_size(int64_t n) {
   if (n < kCodewords || n > ((int64_t)1 << 40)) return 0;
-  // residuals [n][8] float, assignments [n] int32, per-CTA trace partials (at most 2 per SM, 1024 SMs)
-  return align_up((size_t)n * kDim * sizeof(float)) + align_up((size_t)n * sizeof(int32_t)) + 2048 * sizeof(double);
+  return train_ws_bytes(n);
+}
+
+size_t vq4p_train_workspace_size(int64_t n) {
+  if (n < 64 || n > ((int64_t)1 << 40)) return 0;
+  return train_ws_bytes(n);
 }
 
 vq3r_status vq3r_train(const float* vecs, int64_t n, int iters, int nstages, float* codebooks, double* trace,
                        void* workspace, size_t ws_bytes, vq3r_stream stream) {
-  if (!vecs || !codebooks) return VQ3R_ERR_NULL;
-  if (n < kCodewords || n > ((int64_t)1 << 40) || iters < 0 || nstages < 1 || nstages > kStages) return VQ3R_ERR_SHAPE;
-  if (!workspace || ws_bytes < vq3r_train_workspace_size(n)) return VQ3R_ERR_WORKSPACE;
-  if (!aligned16(vecs) || !aligned16(codebooks) || !aligned16(workspace) || (trace && !aligned16(trace)))
-    return VQ3R_ERR_ALIGN;
-  int sms = 0;
-  cudaError_t e = device_setup(&sms);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (sms > 1024) return VQ3R_ERR_SHAPE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  char* w = static_cast<char*>(workspace);
-  float* R = reinterpret_cast<float*>(w);
-  int32_t* a = reinterpret_cast<int32_t*>(w + align_up((size_t)n * kDim * sizeof(float)));
-  double* part = reinterpret_cast<double*>(w + align_up((size_t)n * kDim * sizeof(float)) + align_up((size_t)n * sizeof(int32_t)));
-  const int grid = train_grid(n, sms);
-  e = cudaMemcpyAsync(R, vecs, (size_t)n * kDim * sizeof(float), cudaMemcpyDeviceToDevice, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  for (int st = 0; st < nstages; st++) {
-    float* C = codebooks + (size_t)st * kCodewords * kDim;
-    e = cudaMemcpyAsync(C, R, (size_t)kCodewords * kDim * sizeof(float), cudaMemcpyDeviceToDevice, s);  // first 256
-    if (e != cudaSuccess) return cuda_fail(e);
-    for (int it = 0; it <= iters; it++) {
-      train_assign_kernel<<<grid, kTrainThreads, 0, s>>>(R, n, C, a, part);
-      if (trace) train_trace_kernel<<<1, 32, 0, s>>>(part, grid, trace + (size_t)st * (iters + 1) + it);
-      if (it == iters) break;
-      train_update_kernel<<<kCodewords / kTrainUpdateWarps, kTrainUpdateWarps * 32, 0, s>>>(R, n, a, C);
-    }
-    if (st + 1 < nstages) train_residual_kernel<<<grid, kTrainThreads, 0, s>>>(R, n, C, a);
-  }
-  return check_launch();
+  return train_entry<kStages, kCodewords>(vecs, n, iters, nstages, codebooks, trace, workspace, ws_bytes, stream);
+}
+
+vq3r_status vq4p_train(const float* vecs, int64_t n, int iters, int nstages, float* codebooks, double* trace,
+                       void* workspace, size_t ws_bytes, vq3r_stream stream) {
+  return train_entry<4, 64>(vecs, n, iters, nstages, codebooks, trace, workspace, ws_bytes, stream);
 }
 
 size_t vq3r_tiles_size(int64_t rows, int64_t cols) {
@@ -558,24 +618,24 @@ size_t vq3r_rel_frobenius_workspace_size(int64_t rows, int64_t cols) {
 vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const uint8_t* idx, const uint16_t* scales,
                                      const float* codebooks, int64_t rows, int64_t cols, double* err_out,
                                      void* workspace, size_t ws_bytes, vq3r_stream stream) {
-  if (!W || !idx || !scales || !codebooks || !err_out) return VQ3R_ERR_NULL;
-  vq3r_status st = check_shape(rows, cols, 1);
-  if (st != VQ3R_OK) return st;
-  if (!valid_dtype(w_dtype)) return VQ3R_ERR_DTYPE;
-  if (!workspace || ws_bytes < vq3r_rel_frobenius_workspace_size(rows, cols)) return VQ3R_ERR_WORKSPACE;
-  if (!aligned16(W) || !aligned16(idx) || !aligned16(scales) || !aligned16(codebooks) || !aligned16(workspace) ||
-      (reinterpret_cast<uintptr_t>(err_out) & 7u))
-    return VQ3R_ERR_ALIGN;
-  int sms = 0;
-  cudaError_t e = device_setup(&sms);
-  if (e != cudaSuccess) return cuda_fail(e);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  double* partial = static_cast<double*>(workspace);
-  switch (w_dtype) {
-    case VQ3R_F32: return launch_relfro<VQ3R_F32>(W, idx, scales, codebooks, rows, cols, err_out, partial, s, sms);
-    case VQ3R_BF16: return launch_relfro<VQ3R_BF16>(W, idx, scales, codebooks, rows, cols, err_out, partial, s, sms);
-    default: return launch_relfro<VQ3R_F16>(W, idx, scales, codebooks, rows, cols, err_out, partial, s, sms);
-  }
+  return relfro_entry<FMT_VQ3R>(W, w_dtype, idx, scales, codebooks, rows, cols, err_out, workspace, ws_bytes, stream);
+}
+
+vq3r_status vq4p_encode(const void* W, vq3r_dtype w_dtype, int64_t rows, int64_t cols, const float* codebooks,
+                        uint8_t* planes, uint16_t* scales, vq3r_stream stream) {
+  return encode_entry<FMT_VQ4P>(W, w_dtype, rows, cols, codebooks, planes, scales, stream);
+}
+
+vq3r_status vq4p_decode(const uint8_t* planes, const uint16_t* scales, const float* codebooks, int64_t rows,
+                        int64_t cols, void* out, vq3r_dtype out_dtype, vq3r_stream stream) {
+  return decode_entry<FMT_VQ4P>(planes, scales, codebooks, rows, cols, out, out_dtype, stream);
+}
+
+vq3r_status vq4p_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const uint8_t* planes, const uint16_t* scales,
+                                     const float* codebooks, int64_t rows, int64_t cols, double* err_out,
+                                     void* workspace, size_t ws_bytes, vq3r_stream stream) {
+  return relfro_entry<FMT_VQ4P>(W, w_dtype, planes, scales, codebooks, rows, cols, err_out, workspace, ws_bytes,
+                                stream);
 }
 
 }  // extern "C"

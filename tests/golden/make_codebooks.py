@@ -1,4 +1,4 @@
-"""Write the per-layer VQ3R codebooks of the synthetic workloads.
+"""Write the per-layer VQ3R (and VQ4P) codebooks of the synthetic workloads.
 
 Page "3比特逼近4比特精度？WARP残差向量量化VQ3R的完整测量实验"
 (xdnf.cn/news/289497), §2 and §4: codebooks are fitted per layer by Lloyd
@@ -11,10 +11,12 @@ Workloads (synth/workloads.py):
   expert: the single expert (w1, w3, w2), 65536 vectors sampled uniformly
           without replacement from all of its vectors, 20 iterations;
   layer:  64 experts; 12 experts drawn, 65536 vectors from their matrices;
-  sweep:  256 experts, Student-t(3) with outliers; same sampling.
+  sweep:  256 experts, Student-t(3) with outliers; same sampling;
+  vq4p_layer: the layer workload's training vectors, VQ4P codebooks
+          [4][64][8] (page §5) from oracle.vq4p_train, 20 iterations.
 Training vectors are normalised by their row's FP16 scale first.
 
-Usage: python tests/golden/make_codebooks.py [expert|layer|sweep ...]
+Usage: python tests/golden/make_codebooks.py [expert|layer|sweep|vq4p_layer ...]
 """
 import os
 import sys
@@ -71,7 +73,7 @@ def training_vectors(seed, dist, experts, n_vec):
 def make(name):
     if name == "expert":
         cfg, dist, experts = wl.EXPERT, wl.expert_dist(), [0]
-    elif name == "layer":
+    elif name in ("layer", "vq4p_layer"):
         cfg, dist = wl.LAYER, wl.expert_dist()
         experts = synth.sample(cfg["seed"], wl.SAMPLE_EXPERTS, cfg["experts"], cfg["train_experts"])
     elif name == "sweep":
@@ -80,8 +82,15 @@ def make(name):
     else:
         raise ValueError(name)
     vecs = training_vectors(cfg["seed"], dist, list(experts), cfg["train_vectors"])
-    cb, trace = oracle.lloyd_train(vecs, cfg["lloyd_iters"])
+    if name.startswith("vq4p_"):
+        cb, trace = oracle.vq4p_train(vecs, cfg["lloyd_iters"])
+    else:
+        cb, trace = oracle.lloyd_train(vecs, cfg["lloyd_iters"])
     return cb, trace, list(int(e) for e in experts)
+
+
+def shape(name):
+    return (4, 64, 8) if name.startswith("vq4p_") else (3, 256, 8)
 
 
 def path(name):
@@ -90,9 +99,11 @@ def path(name):
 
 def write(name, cb, trace, experts):
     with open(path(name), "w") as f:
-        f.write("# VQ3R codebooks [3][256][8] float32 (hex bit patterns, one codeword per line)\n")
+        S, K, _ = shape(name)
+        fmt, fn = ("VQ4P", "oracle.vq4p_train") if S == 4 else ("VQ3R", "oracle.lloyd_train")
+        f.write("# %s codebooks [%d][%d][8] float32 (hex bit patterns, one codeword per line)\n" % (fmt, S, K))
         f.write("# workload: %s; Lloyd on sampled normalised vectors (page §2, §4); experts %s\n" % (name, experts))
-        f.write("# written by tests/golden/make_codebooks.py with oracle.lloyd_train only\n")
+        f.write("# written by tests/golden/make_codebooks.py with %s only\n" % fn)
         f.write("# final training distortion per stage: %s\n" % " ".join("%.6e" % t for t in trace[:, -1]))
         u = cb.reshape(-1, 8).view(np.uint32)
         for row in u:
@@ -106,7 +117,7 @@ def load(name):
             if line.startswith("#") or not line.strip():
                 continue
             rows.append([int(t, 16) for t in line.split()])
-    return np.array(rows, dtype=np.uint32).view(np.float32).reshape(3, 256, 8)
+    return np.array(rows, dtype=np.uint32).view(np.float32).reshape(shape(name))
 
 
 if __name__ == "__main__":

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "vq3r.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(vq3r_[a-z0-9_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b((?:vq3r|vq4p)_[a-z0-9_]+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
@@ -28,7 +28,8 @@ def lib():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error"):
+    for n in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq4p_encode", "vq4p_decode",
+              "vq4p_rel_frobenius_error", "vq4p_train"):
         assert n in names
 
 
@@ -170,3 +171,24 @@ def test_train_argument_checks(lib):
     assert lib.vq3r_train(fake, 1000, 5, 3, fake, None, None, need, None) == 7
     assert lib.vq3r_train(fake + 4, 1000, 5, 3, fake, None, fake, need, None) == 3
     assert lib.vq3r_train(fake, 1000, 5, 3, fake, fake + 8, fake, need, None) == 3
+
+
+def test_vq4p_argument_checks(lib):
+    fake = 0x100000
+    assert lib.vq4p_encode(None, 1, 4, 16, fake, fake, fake, None) == 1
+    assert lib.vq4p_encode(fake, 1, 4, 12, fake, fake, fake, None) == 2
+    assert lib.vq4p_encode(fake, 7, 4, 16, fake, fake, fake, None) == 4
+    assert lib.vq4p_encode(fake, 1, 4, 16, fake + 8, fake, fake, None) == 3
+    assert lib.vq4p_encode(fake, 1, 0, 16, fake, fake, fake, None) == 0
+    assert lib.vq4p_decode(fake, fake, fake, 4, 16, fake, 1, None) == 4
+    assert lib.vq4p_decode(fake, fake, None, 4, 16, fake, 0, None) == 1
+    assert lib.vq4p_rel_frobenius_error(fake, 1, fake, fake, fake, 0, 16, fake, fake, 1 << 20, None) == 2
+    assert lib.vq4p_rel_frobenius_error(fake, 1, fake, fake, fake, 4, 16, fake, fake, 16, None) == 7
+    need = lib.vq4p_train_workspace_size(100)
+    assert need >= 100 * 36 and lib.vq4p_train_workspace_size(63) == 0
+    assert lib.vq4p_train_workspace_size(1000) == lib.vq3r_train_workspace_size(1000)
+    assert lib.vq4p_train(fake, 63, 5, 4, fake, None, fake, need, None) == 2    # fewer vectors than centroids
+    assert lib.vq4p_train(fake, 100, 5, 5, fake, None, fake, need, None) == 2   # at most 4 stages
+    assert lib.vq4p_train(fake, 100, 5, 0, fake, None, fake, need, None) == 2
+    assert lib.vq4p_train(fake, 100, 5, 4, fake, None, fake, need - 1, None) == 7
+    assert lib.vq4p_train(None, 100, 5, 4, fake, None, fake, need, None) == 1
