@@ -34,12 +34,19 @@ import synth  # noqa: E402
 from synth import workloads as wl  # noqa: E402
 
 METRIC = "VQ3R encode Gweights/s (vs fp32 peak); decode-GEMV GB/s vs HBM roofline, 1 B200"
-FLOPS_PER_WEIGHT = 2304  # 3 stages x 256 codewords x 8 dims x (sub, mul, add) / 8 weights
+# The definition's work: 3 stages x 256 codewords x 8 dims x (sub, mul, add) / 8 weights.
+FLOPS_PER_WEIGHT = 2304
 VQ4P_FLOPS_PER_WEIGHT = 768  # 4 stages x 64 codewords x 8 dims x (sub, mul, add) / 8 weights
+# What the encoder executes: a screening pass per (vector, codeword) of 8 fused multiply-adds on the FP32 pipe
+# and 5 ALU-pipe operations of bookkeeping (max and min for the second smallest, a compare, two selects), plus
+# the definition's scan for the rare vectors whose margin test fails.  The ALU pipe (64 lanes per SM) bounds it.
+ALU_OPS_PER_VEC_CODEWORD = 5
+ENC_ALU_OPS_PER_WEIGHT = 3 * 256 * ALU_OPS_PER_VEC_CODEWORD / 8  # 480
+ALU_LANES_PER_SM = 64
 # DRAM bytes (read + write) per weight of the encode kernel, from an ncu capture
 # of this kernel (dram__bytes_read.sum + dram__bytes_write.sum over 117.4 M
 # weights); None once the kernel changes and until it is captured again.
-ENCODE_DRAM_BYTES_PER_WEIGHT = (235084544 + 7774976) / 117440512
+ENCODE_DRAM_BYTES_PER_WEIGHT = (235268096 + 8084736) / 117440512
 SM_COUNT_NOMINAL = 148
 FP32_LANES_PER_SM = 128
 
@@ -408,9 +415,10 @@ def main():
     hbm_gbs, sm_max_mhz, peak_src = peaks()
     props = torch.cuda.get_device_properties(dev)
     sms = props.multi_processor_count
-    # The distance is defined with every operation rounded (no fused multiply-add), so each FP32 lane does one
-    # operation per clock: the attainable ceiling is half the FMA-counted figure.
+    # The definition's distance has every operation rounded (no fused multiply-add): one operation per FP32
+    # lane and clock.  The screened encoder is bound by the ALU pipe instead.
     fp32_peak_tflops = sms * FP32_LANES_PER_SM * 1 * sm_max_mhz * 1e6 / 1e12
+    alu_peak_tops = sms * ALU_LANES_PER_SM * sm_max_mhz * 1e6 / 1e12
 
     def barrier():
         if world > 1:
@@ -493,6 +501,29 @@ def main():
         layer_sweep[str(B)] = {"us_per_call": 1e3 * ms, "GB/s": nbytes / ms / 1e6, "frac_hbm": nbytes / ms / 1e6 / hbm_gbs}
         del plan
 
+    # achievable streaming bandwidth of this GPU, for context beside the copy-bandwidth fractions: a read-only
+    # reduction and a write-only fill of 4 GiB (torch's kernels; not part of the path)
+    stream_bw = None
+    if args.gemm_iters > 0:
+        buf = torch.empty(1 << 30, dtype=torch.float32, device=dev)
+        buf.fill_(1.0)
+        acc = torch.empty((), dtype=torch.float32, device=dev)
+        rd, wr = [], []
+        for _ in range(4):
+            a, b, c = ev(), ev(), ev()
+            a.record()
+            torch.sum(buf, dim=0, out=acc)
+            b.record()
+            buf.fill_(2.0)
+            c.record()
+            torch.cuda.synchronize()
+            rd.append(a.elapsed_time(b))
+            wr.append(b.elapsed_time(c))
+        nbytes = buf.numel() * 4
+        stream_bw = {"read_GB/s": nbytes / min(rd[1:]) / 1e6, "write_GB/s": nbytes / min(wr[1:]) / 1e6,
+                     "bytes": nbytes, "how": "torch.sum and Tensor.fill_ over a 4 GiB float32 buffer, best of 3"}
+        del buf, acc
+
     # the prefill product on the tensor cores: the gate projections of 8 experts, 512 seeded random tokens each,
     # in one vq3r_gemm call (weights rebuilt from the tiled indices, bf16, fp32 accumulation)
     prefill = None
@@ -570,8 +601,9 @@ def main():
         err4_ms = timed(lambda: vq.vq4p_rel_frobenius_error(layer.W[k], pl, sc4, cb4, out=e4,
                                                             workspace=layer.err_ws[k]), 3)
         vq4p = {"matrix": "w1 of the layer, %d x %d stacked" % tuple(layer.W[k].shape),
-                "encode_ms": enc4_ms, "encode_TFLOP/s": VQ4P_FLOPS_PER_WEIGHT * n_w / enc4_ms / 1e9,
-                "encode_frac_alu": VQ4P_FLOPS_PER_WEIGHT * n_w / enc4_ms / 1e9 / fp32_peak_tflops,
+                "encode_ms": enc4_ms, "encode_Gweights/s": n_w / enc4_ms / 1e6,
+                "encode_definition_equivalent_tflops": VQ4P_FLOPS_PER_WEIGHT * n_w / enc4_ms / 1e9,
+                "encode_frac_alu": 4 * 64 * ALU_OPS_PER_VEC_CODEWORD / 8 * n_w / enc4_ms / 1e9 / alu_peak_tops,
                 "decode_f32_ms": dec4_ms, "decode_f32_frac_hbm": n_w * 4.375 / dec4_ms / 1e6 / hbm_gbs,
                 "vq3r_decode_f32_ms": dec3_ms, "decode_speedup_vs_vq3r": dec3_ms / dec4_ms,
                 "rel_frobenius_ms": err4_ms, "rel_frobenius_frac_hbm": n_w * 2.375 / err4_ms / 1e6 / hbm_gbs,
@@ -619,6 +651,7 @@ def main():
     ms_step = total_ms / args.steps
     value = whole_job_rate(world, layer.weights, ms_step)  # Gweights/s over the whole path
     enc_tflops = FLOPS_PER_WEIGHT * layer.weights / enc_ms / 1e9
+    enc_tops = ENC_ALU_OPS_PER_WEIGHT * layer.weights / enc_ms / 1e9
     dev_err = vq.vq3r_device_error()
     if rank == 0:
         out = {
@@ -631,15 +664,20 @@ def main():
                        "matrices": "w1,w3 2048x7168; w2 7168x2048 per expert, stacked per kind",
                        "l2": "inputs larger than L2 (5.6 GB layer); GEMV rotates 8 disjoint 8-expert groups "
                              "(1.06 GB of indices)"},
-            "roofline": {"bound": "alu", "achieved": enc_tflops, "peak": fp32_peak_tflops, "unit": "TFLOP/s",
-                         "frac": enc_tflops / fp32_peak_tflops,
+            "roofline": {"bound": "alu", "achieved": enc_tflops, "peak": 2 * fp32_peak_tflops, "unit": "TFLOP/s",
+                         "frac": enc_tflops / (2 * fp32_peak_tflops),
                          "traffic": (None if ENCODE_DRAM_BYTES_PER_WEIGHT is None
                                      else ENCODE_DRAM_BYTES_PER_WEIGHT * layer.weights / 3),
-                         "kernel": "vq3r_encode (row scale + greedy assignment; per launch = one stacked matrix "
-                                   "kind, 3 per step), %d algorithmic flops/weight; peak = %d SMs x 128 FP32 lanes x "
-                                   "1 operation (no fused multiply-add in the distance) x %.0f MHz; traffic = DRAM "
-                                   "bytes per launch" % (FLOPS_PER_WEIGHT, sms, sm_max_mhz),
-                         "frac_of_fma_counted_peak": enc_tflops / (2 * fp32_peak_tflops)},
+                         "kernel": "vq3r_encode (row scale + screened greedy assignment; per launch = one stacked "
+                                   "matrix kind, 3 per step): the definition's %d flops per weight (3 stages x 256 "
+                                   "codewords x 8 dims x 3 / 8) per second; peak = FMA-counted FP32 peak, %d SMs x "
+                                   "128 lanes x 2 x %.0f MHz; traffic = DRAM bytes per launch"
+                                   % (FLOPS_PER_WEIGHT, sms, sm_max_mhz),
+                         "executed": {"bound": "ALU pipe (screening bookkeeping)",
+                                      "alu_ops_per_weight": ENC_ALU_OPS_PER_WEIGHT, "achieved_tops": enc_tops,
+                                      "peak_tops": alu_peak_tops, "frac": enc_tops / alu_peak_tops,
+                                      "peak": "%d SMs x %d ALU lanes x %.0f MHz" % (sms, ALU_LANES_PER_SM,
+                                                                                     sm_max_mhz)}},
             "kernels": {
                 "encode": {"ms": enc_ms, "Gweights/s": layer.weights / enc_ms / 1e6, "TFLOP/s": enc_tflops},
                 "pack_tiles": {"ms": pack_ms, "GB/s": 2 * 0.375 * layer.weights / pack_ms / 1e6},
@@ -654,6 +692,7 @@ def main():
                 "gemm_prefill": prefill,
                 "train_lloyd": train,
                 "vq4p": vq4p,
+                "stream_bandwidth": stream_bw,
                 "hbm_peak_gbs": hbm_gbs, "peak_source": peak_src},
             "e2e": e2e,
             "gpu_launches": Layer.LAUNCHES_PER_STEP * args.steps,

@@ -186,6 +186,31 @@ def test_encode_tie_that_a_fused_multiply_add_would_break():
     assert idx_o[0, 0, 20] == 37
 
 
+def test_encode_near_twin_codewords():
+    """Every codeword of every stage has a twin (index + 128) perturbed in one coordinate by 0 ulps (an exact tie)
+    up to 2^-12 relative, so the two best screening values of most vectors lie on either side of the encoder's
+    margin: the winners it accepts without the definition's scan and the ones it re-scans must both equal the
+    oracle's indices."""
+    rng = np.random.default_rng(41)
+    cb = random_codebooks(41)
+    for s in range(3):
+        for j in range(128):
+            k = j % 8
+            c = cb[s, j].copy()
+            if j % 4 == 0:
+                pass                                             # exact duplicate
+            elif j % 4 == 1:
+                c[k] = np.nextafter(c[k], np.float32(np.inf))    # 1 ulp
+            else:
+                c[k] = np.float32(c[k] * (1 + 2.0 ** -rng.integers(12, 24)))
+            cb[s, 128 + j] = c
+    W = rng.standard_normal((192, 1024)).astype(np.float32)
+    # every third row is made of stage-1 codewords (close to a codeword and its twin after the row's scaling)
+    W[::3, :] = cb[0][rng.integers(0, 256, size=(64, 128))].reshape(64, 1024)
+    check_encode_decode(W, "f32", cb)
+    check_encode_decode(f32_to_bf16_bits(W), "bf16", cb)
+
+
 def test_scale_limits_zero_rows_and_subnormals():
     rng = np.random.default_rng(22)
     cb = random_codebooks(5)
