@@ -77,6 +77,10 @@ def lib():
         L.orc_vq4p_train.argtypes = [P, I64, I32, P, P]
         L.orc_vq4p_train.restype = I32
         L.orc_vq4p_bruteforce.argtypes = [P, I64, P, P, P]
+        L.orc_outliers_select.argtypes = [P, I32, P, I64, I64, I64, P, P]
+        L.orc_outliers_select.restype = I32
+        L.orc_outliers_apply.argtypes = [P, I64, I64, I64, P, P]
+        L.orc_outliers_apply.restype = I32
         _lib = L
     return _lib
 
@@ -315,3 +319,31 @@ def vq4p_bruteforce(r, codebooks):
 def vq4p_gemv(planes, scales, codebooks, x, x_dtype):
     """y[b][i] = sum_c w_hat[i][c] x[b][c] in binary64 with the VQ4P decoded weights."""
     return gemv(vq4p_decode(planes, scales, codebooks), x, x_dtype)
+
+
+def outliers_select(W, dtype, What, k):
+    """Sparse FP16 outlier residual of W over its decode What: the k largest |(double)w - (double)w_hat| per
+    row (ties to the lower column) -> (columns uint16 [rows][k] ascending, fp16 bits uint16 [rows][k])."""
+    W = _w(W, dtype)
+    What = _c(What, np.float32)
+    rows, cols = W.shape
+    oc = np.zeros((rows, k), dtype=np.uint16)
+    ov = np.zeros((rows, k), dtype=np.uint16)
+    rc = lib().orc_outliers_select(W.ctypes.data, DTYPES[dtype], What.ctypes.data, rows, cols, k, oc.ctypes.data,
+                                   ov.ctypes.data)
+    if rc:
+        raise ValueError("orc_outliers_select: bad shape")
+    return oc, ov
+
+
+def outliers_apply(What, ocols, ovals):
+    """What with (float)o added at each stored outlier (binary32); returns a new array."""
+    out = np.array(What, dtype=np.float32, copy=True, order="C")
+    ocols = _c(ocols, np.uint16)
+    ovals = _c(ovals, np.uint16)
+    rows, cols = out.shape
+    k = ocols.shape[1] if ocols.ndim == 2 else 0
+    rc = lib().orc_outliers_apply(out.ctypes.data, rows, cols, k, ocols.ctypes.data, ovals.ctypes.data)
+    if rc:
+        raise ValueError("orc_outliers_apply: bad arguments")
+    return out

@@ -649,3 +649,81 @@ void orc_vq4p_bruteforce(const float* r, int64_t n, const float* codebooks, int3
     best_err[i] = best;
   }
 }
+
+/* ---------------- outlier-aware variant: sparse FP16 residual on top of VQ3R ---------------- */
+/*
+ * Page "XFP：质量目标驱动的自适应码本量化" (zingnex.cn/forum/thread/xfp-llm),
+ * 技术实现 / 权重分解: a weight matrix is split into a dense index tensor
+ * into learned codebooks and a sparse FP16 outlier residual kept at full
+ * precision; the outlier budget is a parameter of the format.  The page
+ * gives no selection rule, layout or combination order; readings:
+ *   - the dense part is the VQ3R encoding of W and w_hat its binary32 decode;
+ *   - e = (double)w - (double)w_hat (one binary64 subtraction);
+ *   - per row, the k positions with the largest |e| are the outliers (|e|
+ *     ordered by its binary64 bit pattern, so a NaN ranks first), ties to
+ *     the lower column;
+ *   - each outlier stores its column (uint16) and o = fp16(e) (round to
+ *     nearest even, saturating at +-65504), the k entries of a row in
+ *     ascending column order;
+ *   - the decode adds (float)o to w_hat in binary32.
+ */
+typedef struct { uint64_t key; int64_t col; } orc_outlier_cand;
+
+static int orc_outlier_rank(const void* a, const void* b) {
+  const orc_outlier_cand* x = (const orc_outlier_cand*)a;
+  const orc_outlier_cand* y = (const orc_outlier_cand*)b;
+  if (x->key != y->key) return x->key > y->key ? -1 : 1; /* larger |e| first */
+  return x->col < y->col ? -1 : (x->col > y->col);       /* then lower column */
+}
+
+static int orc_col_order(const void* a, const void* b) {
+  const orc_outlier_cand* x = (const orc_outlier_cand*)a;
+  const orc_outlier_cand* y = (const orc_outlier_cand*)b;
+  return x->col < y->col ? -1 : (x->col > y->col);
+}
+
+/* ocols, ovals: [rows][k].  Returns 2 on a bad shape (cols > 65536, k > cols). */
+int orc_outliers_select(const void* W, int dtype, const float* What, int64_t rows, int64_t cols, int64_t k,
+                        uint16_t* ocols, uint16_t* ovals) {
+  if (rows < 0 || cols < 1 || cols > 65536 || k < 0 || k > cols) return 2;
+  if (k == 0) return 0;
+  #pragma omp parallel
+  {
+    orc_outlier_cand* c = (orc_outlier_cand*)malloc(sizeof(orc_outlier_cand) * (size_t)cols);
+    #pragma omp for schedule(dynamic, 16)
+    for (int64_t i = 0; i < rows; i++) {
+      for (int64_t j = 0; j < cols; j++) {
+        double e = (double)load_w(W, dtype, i * cols + j) - (double)What[i * cols + j];
+        double a = fabs(e);
+        uint64_t bits;
+        memcpy(&bits, &a, sizeof bits);
+        c[j].key = bits;
+        c[j].col = j;
+      }
+      qsort(c, (size_t)cols, sizeof *c, orc_outlier_rank);
+      qsort(c, (size_t)k, sizeof *c, orc_col_order);
+      for (int64_t q = 0; q < k; q++) {
+        int64_t j = c[q].col;
+        double e = (double)load_w(W, dtype, i * cols + j) - (double)What[i * cols + j];
+        ocols[i * k + q] = (uint16_t)j;
+        ovals[i * k + q] = fp16_from_double(e, 1);
+      }
+    }
+    free(c);
+  }
+  return 0;
+}
+
+/* What[i][col] += (float)o for each stored outlier, in binary32. */
+int orc_outliers_apply(float* What, int64_t rows, int64_t cols, int64_t k, const uint16_t* ocols,
+                       const uint16_t* ovals) {
+  if (rows < 0 || cols < 1 || k < 0 || k > cols) return 2;
+  for (int64_t i = 0; i < rows; i++)
+    for (int64_t q = 0; q < k; q++) {
+      int64_t j = ocols[i * k + q];
+      if (j >= cols) return 3;
+      float o = (float)orc_fp16_to_double(ovals[i * k + q]);
+      What[i * cols + j] = What[i * cols + j] + o;
+    }
+  return 0;
+}

@@ -506,3 +506,87 @@ def test_vq4p_lloyd_matches_sklearn_and_stages_reduce_error():
         g = sum(cb[s][idx[:, s]].astype(np.float64) for s in range(ns))
         errs.append(float(((X.astype(np.float64) - g) ** 2).sum()))
     assert errs[0] > errs[1] > errs[2] > errs[3]
+
+
+# ---------------------------------------------------------------- outlier-aware variant (page "XFP", 权重分解)
+
+def _vq3r_roundtrip(W, dtype, cb):
+    idx, sc = oracle.encode(W, dtype, cb)
+    return oracle.decode(idx, sc, cb)
+
+
+def _widened(W, dtype):
+    if dtype == "f32":
+        return np.asarray(W, dtype=np.float64)
+    if dtype == "bf16":
+        return (np.asarray(W, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+    return np.asarray(W, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_outliers_are_the_k_largest_errors_ties_to_lower_columns(dtype):
+    """The stored set is the k largest |w - w_hat| of each row, lower columns first on ties, stored in column
+    order with fp16(e) values: checked against numpy's own sort and float16 conversion."""
+    from vq3r_cases import f32_to_bf16_bits, random_codebooks
+    rng = np.random.default_rng(5)
+    Wf = rng.standard_normal((24, 256)).astype(np.float32)
+    Wf[:4] = rng.choice([-2.0, -1.0, 1.0, 2.0], size=(4, 256))  # many exact ties among the |e| of these rows
+    W = Wf if dtype == "f32" else f32_to_bf16_bits(Wf)
+    cb = random_codebooks(3)
+    What = _vq3r_roundtrip(W, dtype, cb)
+    What[:4] = 0.0  # so e = w exactly on the tie rows
+    for k in (1, 7, 40, 256):
+        oc, ov = oracle.outliers_select(W, dtype, What, k)
+        e = _widened(W, dtype) - What.astype(np.float64)
+        for i in range(W.shape[0]):
+            order = np.lexsort((np.arange(256), -np.abs(e[i])))[:k]
+            sel = np.sort(order)
+            np.testing.assert_array_equal(oc[i], sel)
+            np.testing.assert_array_equal(ov[i], e[i][sel].astype(np.float16).view(np.uint16))
+
+
+def test_outliers_with_zero_codebooks_and_full_budget_reconstruct_exactly():
+    """Zero codebooks decode to 0, so e = w; with every position an outlier and fp16-representable weights the
+    decode plus outliers is W itself and the relative Frobenius error is exactly 0."""
+    rng = np.random.default_rng(6)
+    W = (rng.integers(-2048, 2048, size=(16, 128)) / 64.0).astype(np.float32)
+    cb = np.zeros((3, 256, 8), dtype=np.float32)
+    What = _vq3r_roundtrip(W, "f32", cb)
+    assert not What.any()
+    oc, ov = oracle.outliers_select(W, "f32", What, 128)
+    W2 = oracle.outliers_apply(What, oc, ov)
+    np.testing.assert_array_equal(W2, W)
+    assert oracle.rel_frobenius(W, "f32", W2) == 0.0
+
+
+def test_outlier_budget_never_increases_the_error():
+    """Each added outlier replaces |e| by |e - fp16(e)| (plus one binary32 rounding), so the error is
+    non-increasing in k; with every position an outlier it falls by about 2^-11."""
+    cfg = wl.TINY
+    W = synth.fill_rows(cfg["cols"], 0, cfg["rows"], cfg["seed"], wl.tag(0, wl.W1), synth.normal(), dtype="f32")
+    cb, _ = oracle.lloyd_train(oracle.normalize_rows(W, "f32", oracle.row_scales(W, "f32")), 3)
+    What = _vq3r_roundtrip(W, "f32", cb)
+    errs = []
+    for k in (0, 1, 2, 4, 8, 32, 128, 512):
+        oc, ov = oracle.outliers_select(W, "f32", What, k)
+        errs.append(oracle.rel_frobenius(W, "f32", oracle.outliers_apply(What, oc, ov)))
+    assert all(b <= a for a, b in zip(errs, errs[1:])), errs
+    assert errs[-1] < 1e-3 * errs[0]
+
+
+def test_outliers_pick_planted_spikes():
+    """Rows of N(0,1) weights with three 20-sigma spikes: the codebooks cannot follow a spike, so with k = 3 the
+    spikes are exactly the stored outliers, and the error falls well below the plain VQ3R error."""
+    from vq3r_cases import random_codebooks
+    rng = np.random.default_rng(7)
+    W = rng.standard_normal((32, 512)).astype(np.float32)
+    spikes = np.stack([np.sort(rng.choice(512, 3, replace=False)) for _ in range(32)])
+    for i in range(32):
+        W[i, spikes[i]] = 20.0 * rng.choice([-1.0, 1.0], size=3)
+    cb = random_codebooks(8)
+    What = _vq3r_roundtrip(W, "f32", cb)
+    oc, ov = oracle.outliers_select(W, "f32", What, 3)
+    np.testing.assert_array_equal(oc, spikes)
+    e0 = oracle.rel_frobenius(W, "f32", What)
+    e3 = oracle.rel_frobenius(W, "f32", oracle.outliers_apply(What, oc, ov))
+    assert e3 < 0.9 * e0
