@@ -280,6 +280,10 @@ class Layer:
     LAUNCHES_PER_STEP = 3 * 2 + 3 + 3 * 1 + 3 * 2 + 1  # encode, pack, decode, error, gemv (kernels)
 
 
+def errs_plain_w1(layer):
+    return float(layer.err[wl.W1].item())
+
+
 # ----------------------------------------------------------------------------- CPU oracle sample
 
 def cpu_oracle_sample(seconds, experts=64):
@@ -610,6 +614,93 @@ def main():
                 "error": float(e4.item()), "vq3r_error": float(layer.err[k].item())}
         del pl, sc4, cb4
 
+    # outlier-aware variant (page "XFP", 权重分解): a sparse FP16 residual of cols/512 entries per row on top of
+    # the layer's VQ3R encoding: selection, decode and error with outliers, the MoE decode step with the sparse add,
+    # and the error gain on the sweep distribution (Student-t(3) with 0.1% of weights at 20 sigma)
+    outl = None
+    if args.gemm_iters > 0:
+        def timed_ms(fn, reps):
+            fn()
+            torch.cuda.synchronize()
+            a, b = ev(), ev()
+            a.record()
+            for _ in range(reps):
+                fn()
+            b.record()
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / reps
+
+        oc, ov, sel = {}, {}, {}
+        for k in layer.kinds:
+            rows_t, cols = layer.W[k].shape
+            kk = cols // 512
+            oc[k] = torch.empty((rows_t, kk), dtype=torch.int16, device=dev)
+            ov[k] = torch.empty((rows_t, kk), dtype=torch.int16, device=dev)
+            sel[k] = timed_ms(lambda: vq.vq3r_outliers(layer.W[k], layer.idx[k], layer.sc[k], layer.cb, kk, oc[k],
+                                                        ov[k]), 2)
+        k1 = wl.W1
+        n1 = layer.W[k1].numel()
+        e1 = torch.empty(1, dtype=torch.float64, device=dev)
+        dec_o = timed_ms(lambda: vq.vq3r_decode_outliers(layer.idx[k1], layer.sc[k1], layer.cb, oc[k1], ov[k1],
+                                                         out=layer.dec[k1]), 3)
+        dec_p = timed_ms(lambda: vq.vq3r_decode(layer.idx[k1], layer.sc[k1], layer.cb, out=layer.dec[k1]), 3)
+        err_o = timed_ms(lambda: vq.vq3r_rel_frobenius_error_outliers(layer.W[k1], layer.idx[k1], layer.sc[k1],
+                                                                      layer.cb, oc[k1], ov[k1], out=e1,
+                                                                      workspace=layer.err_ws[k1]), 3)
+        err_with = float(e1.item())
+        # the MoE decode step (B = 1) with the sparse add: one extra grouped launch over the same 24 matrices
+        plans, _, xu, xd = layer.moe[1]
+        odescs = []
+        for g in range(layer.groups):
+            mats = plans[g][2]
+            om = []
+            for j in range(min(8, layer.E)):
+                e = g * 8 + j
+                for slot, kind in ((2 * j, wl.W1), (2 * j + 1, wl.W3), (16 + j, wl.W2)):
+                    rows, cols = wl.mat_shape(kind)
+                    om.append(dict(ocols=oc[kind], ovals=ov[kind], cols=cols, row0=e * rows, rows=rows,
+                                   x=xu if kind != wl.W2 else xd[j], y=mats[slot]["y"]))
+            odescs.append(vq._outlier_descs(om))
+        L = vq.lib()
+
+        def step_plain(i):
+            layer.gemv(1, i)
+
+        def step_out(i):
+            layer.gemv(1, i)
+            d = odescs[i % layer.groups]
+            st = L.vq3r_gemv_outliers(d, len(d), 1, 1, torch.cuda.current_stream().cuda_stream)
+            if st:
+                raise vq.VQ3RError(st, "vq3r_gemv_outliers")
+
+        reps = max(8, args.gemv_iters)
+        t_plain = timed_ms(lambda: [step_plain(i) for i in range(reps)], 1) / reps
+        t_out = timed_ms(lambda: [step_out(i) for i in range(reps)], 1) / reps
+        # error gain on 8 experts' w1 of the sweep distribution
+        rows, cols = wl.mat_shape(wl.W1)
+        Ws = torch.empty((8 * rows, cols), dtype=torch.bfloat16, device=dev)
+        for e in range(8):
+            synth.fill_rows_device(Ws[e * rows:(e + 1) * rows].data_ptr(), cols, 0, rows, wl.SWEEP["seed"],
+                                   wl.tag(e, wl.W1), wl.sweep_dist(), stream=torch.cuda.current_stream().cuda_stream)
+        cbs = torch.from_numpy(load_codebooks("sweep")).to(dev)
+        idx_s, sc_s = vq.vq3r_encode(Ws, cbs)
+        es0 = float(vq.vq3r_rel_frobenius_error(Ws, idx_s, sc_s, cbs).item())
+        sweep_gain = {}
+        for kk in (cols // 512, cols // 128):
+            ocs, ovs = vq.vq3r_outliers(Ws, idx_s, sc_s, cbs, kk)
+            sweep_gain[str(kk)] = float(vq.vq3r_rel_frobenius_error_outliers(Ws, idx_s, sc_s, cbs, ocs, ovs).item())
+        del Ws, idx_s, sc_s, ocs, ovs
+        outl = {"budget": "cols/512 per row (14 for 7168 columns, 4 for 2048): %.4f extra bits/weight"
+                          % (32.0 / 512),
+                "select_ms": {str(k): sel[k] for k in layer.kinds},
+                "select_Gweights/s": sum(layer.W[k].numel() for k in layer.kinds) / sum(sel.values()) / 1e6,
+                "decode_f32_w1_ms": dec_o, "decode_f32_w1_plain_ms": dec_p,
+                "rel_frobenius_w1_ms": err_o, "rel_frobenius_w1_frac_hbm": n1 * 2.375 / err_o / 1e6 / hbm_gbs,
+                "error_w1": err_with, "error_w1_plain": errs_plain_w1(layer),
+                "moe_step_B1_us": 1e3 * t_out, "moe_step_B1_plain_us": 1e3 * t_plain,
+                "sweep_8x_w1_error_plain": es0, "sweep_8x_w1_error_with_outliers": sweep_gain}
+        del oc, ov, odescs
+
     # end to end through the public API with host buffers: H2D of the layer, the step, D2H of the results
     e2e = None
     if args.e2e_steps > 0:
@@ -692,6 +783,7 @@ def main():
                 "gemm_prefill": prefill,
                 "train_lloyd": train,
                 "vq4p": vq4p,
+                "outliers": outl,
                 "stream_bandwidth": stream_bw,
                 "hbm_peak_gbs": hbm_gbs, "peak_source": peak_src},
             "e2e": e2e,

@@ -329,6 +329,58 @@ size_t vq4p_train_workspace_size(int64_t n);
 vq3r_status vq4p_train(const float* vecs, int64_t n, int iters, int nstages, float* codebooks, double* trace,
                        void* workspace, size_t ws_bytes, vq3r_stream stream);
 
+/*
+ * Outlier-aware variant -- a sparse FP16 residual on top of the VQ3R
+ * encoding (page "XFP：质量目标驱动的自适应码本量化",
+ * zingnex.cn/forum/thread/xfp-llm, 技术实现 / 权重分解: a weight matrix is a
+ * dense index tensor into learned codebooks plus a sparse FP16 outlier
+ * residual kept at full precision, with an outlier budget).  The page gives
+ * no selection rule or layout; readings:
+ *   e = (double)w - (double)w_hat, w_hat the binary32 decode of vq3r_decode;
+ *   per row, the k positions with the largest |e| (ordered by the binary64
+ *   bit pattern of |e|; a NaN ranks first), ties to the lower column;
+ *   each stores its column and o = fp16(e) (nearest even, saturating at
+ *   +-65504); the decode adds (float)o to w_hat in binary32.
+ * Layout: ocols [rows][k] uint16 (ascending within a row), ovals [rows][k]
+ * uint16 binary16 bits: 4 bytes per outlier, 32 k / cols bits per weight.
+ * cols <= 16384 (VQ3R_ERR_SHAPE otherwise), 0 <= k <= cols.
+ *
+ * vq3r_outliers: the outliers of W given its VQ3R encoding (idx, scales,
+ *   codebooks as written by vq3r_encode).  Bit-identical to the reading.
+ *   k == 0 or rows == 0 is a no-op.
+ * vq3r_decode_outliers: vq3r_decode to binary32 followed by the outlier
+ *   additions (out [rows][cols] float).
+ * vq3r_rel_frobenius_error_outliers: vq3r_rel_frobenius_error of the decode
+ *   with outliers; workspace of vq3r_rel_frobenius_outliers_workspace_size.
+ * vq3r_gemv_outliers: y[b][i] += sum_q (float)o_iq * x[b][c_iq] (binary32,
+ *   q ascending) for each descriptor, in one launch: enqueue it after the
+ *   vq3r_gemv call that wrote y to get the product with the outliers.
+ *   1 <= n_mats <= 32, 1 <= B <= 32.
+ */
+typedef struct {
+  const uint16_t* ocols;
+  const uint16_t* ovals;
+  int64_t rows, cols, k;
+  const void* x;            /* [B][cols], x_dtype */
+  float* y;                 /* [B][rows] */
+  int64_t reserved;         /* must be 0 */
+} vq3r_outlier_desc;
+
+vq3r_status vq3r_outliers(const void* W, vq3r_dtype w_dtype, const uint8_t* idx, const uint16_t* scales,
+                          const float* codebooks, int64_t rows, int64_t cols, int64_t k, uint16_t* ocols,
+                          uint16_t* ovals, vq3r_stream stream);
+vq3r_status vq3r_decode_outliers(const uint8_t* idx, const uint16_t* scales, const float* codebooks,
+                                 const uint16_t* ocols, const uint16_t* ovals, int64_t rows, int64_t cols, int64_t k,
+                                 float* out, vq3r_stream stream);
+size_t vq3r_rel_frobenius_outliers_workspace_size(int64_t rows, int64_t cols, int64_t k);
+vq3r_status vq3r_rel_frobenius_error_outliers(const void* W, vq3r_dtype w_dtype, const uint8_t* idx,
+                                              const uint16_t* scales, const float* codebooks, const uint16_t* ocols,
+                                              const uint16_t* ovals, int64_t rows, int64_t cols, int64_t k,
+                                              double* err_out, void* workspace, size_t ws_bytes,
+                                              vq3r_stream stream);
+vq3r_status vq3r_gemv_outliers(const vq3r_outlier_desc* mats, int n_mats, int B, vq3r_dtype x_dtype,
+                               vq3r_stream stream);
+
 /* Human-readable name of a status code (static string). */
 const char* vq3r_status_string(vq3r_status s);
 

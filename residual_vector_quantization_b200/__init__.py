@@ -27,7 +27,8 @@ EXPORTED = ["vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_gemv_workspace_size
             "vq3r_rel_frobenius_workspace_size", "vq3r_status_string", "vq3r_last_cuda_error",
             "vq3r_device_error", "vq3r_gemv_noalloc", "vq3r_tiles_size", "vq3r_pack_tiles", "vq3r_gemm",
             "vq3r_train", "vq3r_train_workspace_size", "vq4p_encode", "vq4p_decode", "vq4p_rel_frobenius_error",
-            "vq4p_train", "vq4p_train_workspace_size"]
+            "vq4p_train", "vq4p_train_workspace_size", "vq3r_outliers", "vq3r_decode_outliers",
+            "vq3r_rel_frobenius_error_outliers", "vq3r_rel_frobenius_outliers_workspace_size", "vq3r_gemv_outliers"]
 
 
 class VQ3RError(RuntimeError):
@@ -49,6 +50,12 @@ class GemmDesc(ctypes.Structure):
     _fields_ = [("idx", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("codebooks", ctypes.c_void_p),
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
                 ("plane_stride", ctypes.c_int64), ("tokens", ctypes.c_int64), ("reserved", ctypes.c_int64)]
+
+
+class OutlierDesc(ctypes.Structure):
+    _fields_ = [("ocols", ctypes.c_void_p), ("ovals", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64), ("k", ctypes.c_int64), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("reserved", ctypes.c_int64)]
 
 
 _L = None
@@ -87,9 +94,16 @@ def _lib():
         L.vq4p_train.argtypes = L.vq3r_train.argtypes
         L.vq4p_train_workspace_size.argtypes = [I64]
         L.vq4p_train_workspace_size.restype = SZ
+        L.vq3r_outliers.argtypes = [P, I32, P, P, P, I64, I64, I64, P, P, P]
+        L.vq3r_decode_outliers.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
+        L.vq3r_rel_frobenius_outliers_workspace_size.argtypes = [I64, I64, I64]
+        L.vq3r_rel_frobenius_outliers_workspace_size.restype = SZ
+        L.vq3r_rel_frobenius_error_outliers.argtypes = [P, I32, P, P, P, P, P, I64, I64, I64, P, P, SZ, P]
+        L.vq3r_gemv_outliers.argtypes = [P, I32, I32, I32, P]
         for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error",
                   "vq3r_gemv_noalloc", "vq3r_pack_tiles", "vq3r_gemm", "vq3r_train", "vq4p_encode", "vq4p_decode",
-                  "vq4p_rel_frobenius_error", "vq4p_train"):
+                  "vq4p_rel_frobenius_error", "vq4p_train", "vq3r_outliers", "vq3r_decode_outliers",
+                  "vq3r_rel_frobenius_error_outliers", "vq3r_gemv_outliers"):
             getattr(L, f).restype = I32
         _L = L
     return _L
@@ -329,6 +343,78 @@ def vq3r_rel_frobenius_error(W, idx, scales, codebooks, out=None, workspace=None
 def vq4p_rel_frobenius_error(W, planes, scales, codebooks, out=None, workspace=None, stream=None):
     """vq3r_rel_frobenius_error for VQ4P planes and codebooks [4][64][8]."""
     return _relfro("vq4p_rel_frobenius_error", W, planes, scales, codebooks, out, workspace, stream)
+
+
+def vq3r_outliers(W, idx, scales, codebooks, k, ocols=None, ovals=None, stream=None):
+    """Sparse FP16 outlier residual of W over its VQ3R encoding: the k largest |w - w_hat| per row ->
+    (ocols uint16-as-int16 [rows][k], ovals int16 [rows][k] binary16 bits)."""
+    rows, cols = W.shape
+    if W.dtype not in _DT:
+        raise ValueError("W dtype must be float32, bfloat16 or float16")
+    if ocols is None:
+        ocols = torch.empty((rows, k), dtype=torch.int16, device=W.device)
+    if ovals is None:
+        ovals = torch.empty((rows, k), dtype=torch.int16, device=W.device)
+    _check(_lib().vq3r_outliers(_dev(W, "W"), _DT[W.dtype], _dev(idx, "idx"), _dev(scales, "scales"),
+                                _dev(codebooks, "codebooks"), rows, cols, k, _dev(ocols, "ocols"),
+                                _dev(ovals, "ovals"), _stream(stream)), "vq3r_outliers")
+    return ocols, ovals
+
+
+def vq3r_decode_outliers(idx, scales, codebooks, ocols, ovals, out=None, stream=None):
+    """W_hat [rows][cols] float32 with the outliers added."""
+    _, rows, V = idx.shape
+    k = ocols.shape[1]
+    if out is None:
+        out = torch.empty((rows, V * DIM), dtype=torch.float32, device=idx.device)
+    _check(_lib().vq3r_decode_outliers(_dev(idx, "idx"), _dev(scales, "scales"), _dev(codebooks, "codebooks"),
+                                       _dev(ocols, "ocols"), _dev(ovals, "ovals"), rows, V * DIM, k,
+                                       _dev(out, "out"), _stream(stream)), "vq3r_decode_outliers")
+    return out
+
+
+def vq3r_rel_frobenius_outliers_workspace_size(rows, cols, k):
+    return _lib().vq3r_rel_frobenius_outliers_workspace_size(rows, cols, k)
+
+
+def vq3r_rel_frobenius_error_outliers(W, idx, scales, codebooks, ocols, ovals, out=None, workspace=None,
+                                      stream=None):
+    """Device float64 tensor [1]: the relative Frobenius error of the decode with outliers."""
+    rows, cols = W.shape
+    k = ocols.shape[1]
+    if out is None:
+        out = torch.empty(1, dtype=torch.float64, device=W.device)
+    if workspace is None:
+        workspace = torch.empty(vq3r_rel_frobenius_outliers_workspace_size(rows, cols, k), dtype=torch.uint8,
+                                device=W.device)
+    _check(_lib().vq3r_rel_frobenius_error_outliers(
+        _dev(W, "W"), _DT[W.dtype], _dev(idx, "idx"), _dev(scales, "scales"), _dev(codebooks, "codebooks"),
+        _dev(ocols, "ocols"), _dev(ovals, "ovals"), rows, cols, k, _dev(out, "out"), _dev(workspace, "workspace"),
+        workspace.numel(), _stream(stream)), "vq3r_rel_frobenius_error_outliers")
+    return out
+
+
+def _outlier_descs(mats):
+    arr = (OutlierDesc * len(mats))()
+    for i, m in enumerate(mats):
+        oc, ov, x, y = m["ocols"], m["ovals"], m["x"], m["y"]
+        r0 = m.get("row0", 0)
+        rows = m.get("rows", oc.shape[0])
+        k = oc.shape[1]
+        if not (oc.is_cuda and oc.is_contiguous() and ov.is_cuda and ov.is_contiguous()):
+            raise ValueError("ocols and ovals must be contiguous CUDA tensors")
+        arr[i] = OutlierDesc(oc.data_ptr() + 2 * r0 * k, ov.data_ptr() + 2 * r0 * k, rows, m["cols"], k,
+                             _dev(x, "x"), _dev(y, "y"), 0)
+    return arr
+
+
+def vq3r_gemv_outliers(mats, B, stream=None):
+    """y += the outliers' product for each dict {ocols, ovals, cols, x [B][cols], y [B][rows]} (optionally
+    row0, rows: a row range of a larger matrix's outliers), in one launch; enqueue after vq3r_gemv."""
+    arr = _outlier_descs(mats)
+    xdt = _DT[mats[0]["x"].dtype]
+    _check(_lib().vq3r_gemv_outliers(arr, len(mats), B, xdt, _stream(stream)), "vq3r_gemv_outliers")
+    return [m["y"] for m in mats]
 
 
 def vq3r_device_error():

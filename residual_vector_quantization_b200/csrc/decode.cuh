@@ -225,13 +225,22 @@ constexpr int kErrVecs = 4;  // consecutive vectors per thread and step
 // groups t, t + 512, ...: the index bytes of a group are one 32-bit word per
 // plane when V is a multiple of 4, and a warp's 16-byte W loads are 512
 // contiguous bytes.  Each thread keeps two binary64 sums, reduced per CTA.
-template <int DT, int FMT>
+//
+// OUT: the decode carries a sparse outlier residual (ocols / ovals [rows][k],
+// columns ascending per row): each outlier's (float)o is added to its
+// decoded value in binary32 before the sums, so the numerator is summed
+// directly.  A thread finds the first outlier of its 32 columns by binary
+// search in the row's columns.
+template <int DT, int FMT, bool OUT = false>
 __global__ void __launch_bounds__(kErrThreads, 2) relfro_partial_kernel(const void* __restrict__ W,
                                                                          const uint8_t* __restrict__ idx,
                                                                          const uint16_t* __restrict__ scales,
                                                                          const float* __restrict__ codebooks,
                                                                          int64_t rows, int64_t cols,
-                                                                         double* __restrict__ partial) {
+                                                                         double* __restrict__ partial,
+                                                                         const uint16_t* __restrict__ ocols = nullptr,
+                                                                         const uint16_t* __restrict__ ovals = nullptr,
+                                                                         int k = 0) {
   extern __shared__ __align__(16) float cbr[];
   __shared__ double red[2][kErrThreads / 32];
   load_codebooks_replicated<FMT>(cbr, codebooks);
@@ -259,22 +268,42 @@ __global__ void __launch_bounds__(kErrThreads, 2) relfro_partial_kernel(const vo
         w3[st] = x;
       }
     }
+    int oq = 0;  // OUT: first outlier of the row at or after this group's first column
+    const uint16_t* orow = nullptr;
+    if constexpr (OUT) {
+      orow = ocols + row * k;
+      const int c_lo = q * kErrVecs * kDim;
+      int lo = 0, hi = k;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((int)__ldg(orow + mid) < c_lo) lo = mid + 1;
+        else hi = mid;
+      }
+      oq = lo;
+    }
 #pragma unroll
     for (int i = 0; i < kErrVecs; i++) {
       if (i < n) {
         float4 lo, hi;
         decode_vector_r<FMT>(cbr, (w3[0] >> (8 * i)) & 0xFFu, (w3[1] >> (8 * i)) & 0xFFu, (w3[2] >> (8 * i)) & 0xFFu, s, lane,
                         lo, hi);
+        float wh[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        if constexpr (OUT) {
+          const int cv = (q * kErrVecs + i) * kDim;
+          while (oq < k) {
+            const int c = (int)__ldg(orow + oq);
+            if (c >= cv + kDim) break;
+            const float o = f16_bits_to_f32(__ldg(ovals + row * k + oq));
+#pragma unroll
+            for (int j = 0; j < kDim; j++)
+              if (c == cv + j) wh[j] = __fadd_rn(wh[j], o);
+            oq++;
+          }
+        }
         float wv[8];
         load8<DT>(W, (g + i) * kDim, wv);
-        acc_err(num, den, wv[0], lo.x);
-        acc_err(num, den, wv[1], lo.y);
-        acc_err(num, den, wv[2], lo.z);
-        acc_err(num, den, wv[3], lo.w);
-        acc_err(num, den, wv[4], hi.x);
-        acc_err(num, den, wv[5], hi.y);
-        acc_err(num, den, wv[6], hi.z);
-        acc_err(num, den, wv[7], hi.w);
+#pragma unroll
+        for (int j = 0; j < kDim; j++) acc_err(num, den, wv[j], wh[j]);
       }
     }
   }

@@ -9,6 +9,7 @@
 #include "gemv.cuh"
 #include "gemv_mma.cuh"
 #include "train.cuh"
+#include "outliers.cuh"
 #include "vq3r_common.cuh"
 
 using namespace vq3r;
@@ -72,11 +73,18 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F32, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_BF16, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F16, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F32, FMT_VQ3R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_BF16, FMT_VQ3R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F16, FMT_VQ3R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes);
+    const int go = (int)outlier_select_smem(kOutMaxCols);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
     g_dev_err[dev] = r;
   });
   *sms = g_dev_sms[dev];
@@ -636,6 +644,153 @@ vq3r_status vq4p_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const ui
                                      void* workspace, size_t ws_bytes, vq3r_stream stream) {
   return relfro_entry<FMT_VQ4P>(W, w_dtype, planes, scales, codebooks, rows, cols, err_out, workspace, ws_bytes,
                                 stream);
+}
+
+// ---- outlier-aware variant ----
+
+static vq3r_status check_outliers(int64_t rows, int64_t cols, int64_t k) {
+  vq3r_status st = check_shape(rows, cols, 0);
+  if (st != VQ3R_OK) return st;
+  if (cols > kOutMaxCols || k < 0 || k > cols) return VQ3R_ERR_SHAPE;
+  return VQ3R_OK;
+}
+
+vq3r_status vq3r_outliers(const void* W, vq3r_dtype w_dtype, const uint8_t* idx, const uint16_t* scales,
+                          const float* codebooks, int64_t rows, int64_t cols, int64_t k, uint16_t* ocols,
+                          uint16_t* ovals, vq3r_stream stream) {
+  vq3r_status st = check_outliers(rows, cols, k);
+  if (st != VQ3R_OK) return st;
+  if (!valid_dtype(w_dtype)) return VQ3R_ERR_DTYPE;
+  if (rows == 0 || k == 0) return VQ3R_OK;
+  if (!W || !idx || !scales || !codebooks || !ocols || !ovals) return VQ3R_ERR_NULL;
+  if (!aligned16(W) || !aligned16(idx) || !aligned16(scales) || !aligned16(codebooks) || !aligned16(ocols) ||
+      !aligned16(ovals))
+    return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t smem = outlier_select_smem(cols);
+  const int per_sm = smem <= 100 * 1024 ? 2 : 1;
+  const int grid = (int)(rows < (int64_t)sms * per_sm ? rows : (int64_t)sms * per_sm);
+  switch (w_dtype) {
+    case VQ3R_F32:
+      outlier_select_kernel<VQ3R_F32><<<grid, kOutThreads, smem, s>>>(W, idx, scales, codebooks, rows, cols, (int)k, ocols, ovals);
+      break;
+    case VQ3R_BF16:
+      outlier_select_kernel<VQ3R_BF16><<<grid, kOutThreads, smem, s>>>(W, idx, scales, codebooks, rows, cols, (int)k, ocols, ovals);
+      break;
+    default:
+      outlier_select_kernel<VQ3R_F16><<<grid, kOutThreads, smem, s>>>(W, idx, scales, codebooks, rows, cols, (int)k, ocols, ovals);
+  }
+  return check_launch();
+}
+
+vq3r_status vq3r_decode_outliers(const uint8_t* idx, const uint16_t* scales, const float* codebooks,
+                                 const uint16_t* ocols, const uint16_t* ovals, int64_t rows, int64_t cols, int64_t k,
+                                 float* out, vq3r_stream stream) {
+  vq3r_status st = check_outliers(rows, cols, k);
+  if (st != VQ3R_OK) return st;
+  if (rows > 0 && k > 0 && (!ocols || !ovals)) return VQ3R_ERR_NULL;
+  st = decode_entry<FMT_VQ3R>(idx, scales, codebooks, rows, cols, out, VQ3R_F32, stream);
+  if (st != VQ3R_OK || rows == 0 || k == 0) return st;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int64_t n = rows * k, need = (n + 255) / 256;
+  const int grid = (int)(need < ((int64_t)1 << 30) ? need : ((int64_t)1 << 30));
+  outlier_apply_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(out, rows, cols, k, ocols, ovals);
+  return check_launch();
+}
+
+size_t vq3r_rel_frobenius_outliers_workspace_size(int64_t rows, int64_t cols, int64_t k) {
+  (void)k;
+  return vq3r_rel_frobenius_workspace_size(rows, cols);
+}
+
+vq3r_status vq3r_rel_frobenius_error_outliers(const void* W, vq3r_dtype w_dtype, const uint8_t* idx,
+                                              const uint16_t* scales, const float* codebooks, const uint16_t* ocols,
+                                              const uint16_t* ovals, int64_t rows, int64_t cols, int64_t k,
+                                              double* err_out, void* workspace, size_t ws_bytes,
+                                              vq3r_stream stream) {
+  if (!W || !idx || !scales || !codebooks || !err_out) return VQ3R_ERR_NULL;
+  vq3r_status st = check_outliers(rows, cols, k);
+  if (st != VQ3R_OK) return st;
+  if (rows < 1) return VQ3R_ERR_SHAPE;
+  if (k > 0 && (!ocols || !ovals)) return VQ3R_ERR_NULL;
+  if (!valid_dtype(w_dtype)) return VQ3R_ERR_DTYPE;
+  if (!workspace || ws_bytes < vq3r_rel_frobenius_outliers_workspace_size(rows, cols, k)) return VQ3R_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(idx) || !aligned16(scales) || !aligned16(codebooks) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(err_out) & 7u) || (k > 0 && (!aligned16(ocols) || !aligned16(ovals))))
+    return VQ3R_ERR_ALIGN;
+  if (k == 0) return relfro_entry<FMT_VQ3R>(W, w_dtype, idx, scales, codebooks, rows, cols, err_out, workspace,
+                                            ws_bytes, stream);
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double* partial = static_cast<double*>(workspace);
+  const int64_t blocks = rowsplit_blocks(rows, cols, sms, kErrMaxBlocks);
+  const size_t smem = kCbrFloats * sizeof(float);
+  const int kk = (int)k;
+  switch (w_dtype) {
+    case VQ3R_F32:
+      relfro_partial_kernel<VQ3R_F32, FMT_VQ3R, true><<<(int)blocks, kErrThreads, smem, s>>>(W, idx, scales, codebooks, rows, cols, partial, ocols, ovals, kk);
+      break;
+    case VQ3R_BF16:
+      relfro_partial_kernel<VQ3R_BF16, FMT_VQ3R, true><<<(int)blocks, kErrThreads, smem, s>>>(W, idx, scales, codebooks, rows, cols, partial, ocols, ovals, kk);
+      break;
+    default:
+      relfro_partial_kernel<VQ3R_F16, FMT_VQ3R, true><<<(int)blocks, kErrThreads, smem, s>>>(W, idx, scales, codebooks, rows, cols, partial, ocols, ovals, kk);
+  }
+  relfro_final_kernel<<<1, 256, 0, s>>>(partial, (int)blocks, err_out);
+  return check_launch();
+}
+
+vq3r_status vq3r_gemv_outliers(const vq3r_outlier_desc* mats, int n_mats, int B, vq3r_dtype x_dtype,
+                               vq3r_stream stream) {
+  if (!mats) return VQ3R_ERR_NULL;
+  if (n_mats < 1 || n_mats > kOutGemvMaxMats || B < 1 || B > VQ3R_GEMV_MAX_B) return VQ3R_ERR_BATCH;
+  if (!valid_dtype(x_dtype)) return VQ3R_ERR_DTYPE;
+  OutGemvParams P;
+  memset(&P, 0, sizeof(P));
+  int m = 0;
+  int64_t total = 0;
+  for (int i = 0; i < n_mats; i++) {
+    const vq3r_outlier_desc& d = mats[i];
+    vq3r_status st = check_outliers(d.rows, d.cols, d.k);
+    if (st != VQ3R_OK) return st;
+    if (d.reserved != 0) return VQ3R_ERR_SHAPE;
+    if (d.rows == 0 || d.k == 0) continue;
+    if (!d.ocols || !d.ovals || !d.x || !d.y) return VQ3R_ERR_NULL;
+    if (!aligned16(d.ocols) || !aligned16(d.ovals) || !aligned16(d.x) || !aligned16(d.y)) return VQ3R_ERR_ALIGN;
+    P.ocols[m] = d.ocols;
+    P.ovals[m] = d.ovals;
+    P.x[m] = d.x;
+    P.y[m] = d.y;
+    P.rows[m] = d.rows;
+    P.k[m] = d.k;
+    P.cols[m] = d.cols;
+    P.row_begin[m] = total;
+    total += d.rows;
+    m++;
+  }
+  if (m == 0) return VQ3R_OK;
+  P.row_begin[m] = total;
+  P.n_mats = m;
+  P.B = B;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int64_t grid = (total + 255) / 256;
+  if (grid > INT32_MAX) return VQ3R_ERR_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (x_dtype) {
+    case VQ3R_F32: outlier_gemv_kernel<VQ3R_F32><<<(int)grid, 256, 0, s>>>(P); break;
+    case VQ3R_BF16: outlier_gemv_kernel<VQ3R_BF16><<<(int)grid, 256, 0, s>>>(P); break;
+    default: outlier_gemv_kernel<VQ3R_F16><<<(int)grid, 256, 0, s>>>(P);
+  }
+  return check_launch();
 }
 
 }  // extern "C"

@@ -192,3 +192,23 @@ def test_vq4p_argument_checks(lib):
     assert lib.vq4p_train(fake, 100, 5, 0, fake, None, fake, need, None) == 2
     assert lib.vq4p_train(fake, 100, 5, 4, fake, None, fake, need - 1, None) == 7
     assert lib.vq4p_train(None, 100, 5, 4, fake, None, fake, need, None) == 1
+
+
+def test_outlier_argument_checks(lib):
+    fake = 0x100000
+    assert lib.vq3r_outliers(fake, 1, fake, fake, fake, 4, 16392, 3, fake, fake, None) == 2   # cols > 16384
+    assert lib.vq3r_outliers(fake, 1, fake, fake, fake, 4, 64, 65, fake, fake, None) == 2     # k > cols
+    assert lib.vq3r_outliers(fake, 1, fake, fake, fake, 4, 64, -1, fake, fake, None) == 2
+    assert lib.vq3r_outliers(fake, 1, fake, fake, fake, 4, 64, 0, None, None, None) == 0      # no budget: no-op
+    assert lib.vq3r_outliers(fake, 9, fake, fake, fake, 4, 64, 3, fake, fake, None) == 4
+    assert lib.vq3r_outliers(fake, 1, fake, fake, fake, 4, 64, 3, None, fake, None) == 1
+    assert lib.vq3r_outliers(fake, 1, fake, fake, fake, 4, 64, 3, fake + 2, fake, None) == 3
+    assert lib.vq3r_decode_outliers(fake, fake, fake, None, fake, 4, 64, 3, fake, None) == 1
+    need = lib.vq3r_rel_frobenius_outliers_workspace_size(4, 64, 3)
+    assert need > lib.vq3r_rel_frobenius_workspace_size(4, 64)
+    assert lib.vq3r_rel_frobenius_error_outliers(fake, 1, fake, fake, fake, fake, fake, 4, 64, 3, fake, fake,
+                                                 need - 8, None) == 7
+    d = (vq.OutlierDesc * 1)(vq.OutlierDesc(fake, fake, 4, 64, 3, fake, fake, 1))
+    assert lib.vq3r_gemv_outliers(d, 1, 1, 1, None) == 2   # reserved must be 0
+    assert lib.vq3r_gemv_outliers(d, 0, 1, 1, None) == 5
+    assert lib.vq3r_gemv_outliers(d, 1, 33, 1, None) == 5

@@ -1,0 +1,133 @@
+"""Outlier-aware variant (sparse FP16 residual over VQ3R, page "XFP", 权重分解) on the CUDA path vs the oracle,
+through the C ABI.
+
+Bars: outlier columns and values bit-exact (integer selection work), the decode with outliers bit-exact, the
+relative Frobenius error within 1e-9 relative, the GEMV with outliers within 2e-3 (rms floor).  Oracle inputs
+come from the host generator or the oracle itself.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import workloads as wl
+from vq3r_cases import GEMV_TOL, RELFRO_TOL, f32_to_bf16_bits, gemv_rel_err, random_codebooks
+
+pytestmark = pytest.mark.gpu
+
+vq = pytest.importorskip("residual_vector_quantization_b200")
+DEV = "cuda"
+
+
+def to_dev(a, dtype):
+    if dtype == "f32":
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(DEV)
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).to(DEV)
+    return t.view(torch.bfloat16 if dtype == "bf16" else torch.float16)
+
+
+def u16(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+def check(W, dtype, cb, ks, B=2, seed=0):
+    """Encode on the GPU (bit-exact with the oracle, checked elsewhere), then for each budget k: outliers, decode
+    with outliers, error with outliers and the GEMV with outliers against the oracle."""
+    W_t = to_dev(W, dtype)
+    cb_t = torch.from_numpy(np.ascontiguousarray(cb)).to(DEV)
+    idx_t, sc_t = vq.vq3r_encode(W_t, cb_t)
+    idx_o, sc_o = oracle.encode(W, dtype, cb)
+    np.testing.assert_array_equal(idx_t.cpu().numpy(), idx_o)
+    What = oracle.decode(idx_o, sc_o, cb)
+    rows, cols = What.shape
+    rng = np.random.default_rng(seed)
+    xb = f32_to_bf16_bits(rng.standard_normal((B, cols)).astype(np.float32))
+    results = {}
+    for k in ks:
+        oc_t, ov_t = vq.vq3r_outliers(W_t, idx_t, sc_t, cb_t, k)
+        oc_o, ov_o = oracle.outliers_select(W, dtype, What, k)
+        np.testing.assert_array_equal(u16(oc_t), oc_o)
+        np.testing.assert_array_equal(u16(ov_t), ov_o)
+        W2 = oracle.outliers_apply(What, oc_o, ov_o)
+        d = vq.vq3r_decode_outliers(idx_t, sc_t, cb_t, oc_t, ov_t).cpu().numpy()
+        np.testing.assert_array_equal(d.view(np.uint32), W2.view(np.uint32))
+        e_gpu = float(vq.vq3r_rel_frobenius_error_outliers(W_t, idx_t, sc_t, cb_t, oc_t, ov_t).cpu()[0])
+        e_ref = oracle.rel_frobenius(W, dtype, W2)
+        assert abs(e_gpu - e_ref) <= RELFRO_TOL * e_ref + 1e-300, (k, e_gpu, e_ref)
+        y = torch.empty((B, rows), dtype=torch.float32, device=DEV)
+        x_t = to_dev(xb, "bf16")
+        vq.vq3r_gemv([dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=x_t, y=y)], B)
+        vq.vq3r_gemv_outliers([dict(ocols=oc_t, ovals=ov_t, cols=cols, x=x_t, y=y)], B)
+        assert gemv_rel_err(y.cpu().numpy(), oracle.gemv(W2, xb, "bf16")) <= GEMV_TOL
+        results[k] = e_ref
+    return results
+
+
+def test_tiny_workload_budgets():
+    cfg = wl.TINY
+    W = synth.fill_rows(cfg["cols"], 0, cfg["rows"], cfg["seed"], wl.tag(0, wl.W1), synth.normal(), dtype="f32")
+    cb, _ = oracle.lloyd_train(oracle.normalize_rows(W, "f32", oracle.row_scales(W, "f32")), cfg["lloyd_iters"])
+    errs = check(W, "f32", cb, (1, 5, 64, 512))
+    assert errs[512] < errs[64] < errs[5] < errs[1]
+
+
+def test_exact_ties_go_to_lower_columns():
+    """Zero codebooks decode to 0, so e = w; weights drawn from {-2, -1, 1, 2} tie in blocks, and budgets that
+    end inside a block must take its lowest columns."""
+    rng = np.random.default_rng(11)
+    W = rng.choice([-2.0, -1.0, 1.0, 2.0], size=(40, 1024)).astype(np.float32)
+    cb = np.zeros((3, 256, 8), dtype=np.float32)
+    n2 = (np.abs(W) == 2).sum(axis=1)
+    check(W, "f32", cb, (1, 100, int(n2.min()), int(n2.max()) + 3, 1024))
+
+
+@pytest.mark.parametrize("rows,cols,dtype,ks", [(3, 40, "bf16", (1, 40)), (130, 800, "f16", (7, 33)),
+                                                (257, 1032, "f32", (2, 129)), (5, 16384, "bf16", (1, 37, 700))])
+def test_shapes_dtypes_and_the_column_limit(rows, cols, dtype, ks):
+    rng = np.random.default_rng(rows + cols)
+    Wf = (rng.standard_normal((rows, cols)) * np.exp(rng.standard_normal((rows, 1)))).astype(np.float32)
+    W = Wf if dtype == "f32" else (f32_to_bf16_bits(Wf) if dtype == "bf16" else Wf.astype(np.float16).view(np.uint16))
+    check(W, dtype, random_codebooks(rows), ks)
+
+
+def test_sweep_distribution_outliers_reduce_the_error():
+    """Rows of the 256-expert sweep distribution (Student-t(3), 0.1% of weights at +-20 sigma): with a budget of
+    cols/512 the outliers are bit-exact and cut the relative error well below plain VQ3R's."""
+    import importlib.util
+    import os
+    p = os.path.join(os.path.dirname(__file__), "golden", "make_codebooks.py")
+    spec = importlib.util.spec_from_file_location("make_codebooks", p)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    cb = mod.load("sweep")
+    rows, cols = wl.mat_shape(wl.W1)
+    W = synth.fill_rows(cols, 0, 256, wl.SWEEP["seed"], wl.tag(3, wl.W1), wl.sweep_dist(), dtype="bf16")
+    errs = check(W, "bf16", cb, (0, cols // 512, cols // 128))
+    assert errs[cols // 512] < 0.9 * errs[0], errs
+
+
+def test_grouped_sparse_add_over_expert_row_ranges():
+    """One vq3r_gemv_outliers call over row ranges of two stacked matrices (as for experts), B = 3."""
+    rng = np.random.default_rng(12)
+    cb = random_codebooks(12)
+    W = rng.standard_normal((1024, 256)).astype(np.float32)
+    W_t = to_dev(W, "f32")
+    cb_t = torch.from_numpy(cb).to(DEV)
+    idx_t, sc_t = vq.vq3r_encode(W_t, cb_t)
+    oc_t, ov_t = vq.vq3r_outliers(W_t, idx_t, sc_t, cb_t, 9)
+    What = oracle.decode(*oracle.encode(W, "f32", cb), cb)
+    W2 = oracle.outliers_apply(What, *oracle.outliers_select(W, "f32", What, 9))
+    B = 3
+    x = rng.standard_normal((2, B, 256)).astype(np.float32)
+    mats, outs = [], []
+    for j, (r0, n) in enumerate(((0, 512), (512, 512))):
+        y = torch.empty((B, n), dtype=torch.float32, device=DEV)
+        xt = to_dev(x[j], "f32")
+        vq.vq3r_gemv([dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=xt, y=y, row0=r0, rows=n)], B)
+        mats.append(dict(ocols=oc_t, ovals=ov_t, cols=256, x=xt, y=y, row0=r0, rows=n))
+        outs.append((r0, n, y))
+    vq.vq3r_gemv_outliers(mats, B)
+    for j, (r0, n, y) in enumerate(outs):
+        ref = oracle.gemv(W2[r0:r0 + n], x[j], "f32")
+        assert gemv_rel_err(y.cpu().numpy(), ref) <= GEMV_TOL
