@@ -205,7 +205,7 @@ def test_outlier_argument_checks(lib):
     assert lib.vq3r_outliers(fake, 1, fake, fake, fake, 4, 64, 3, fake + 2, fake, None) == 3
     assert lib.vq3r_decode_outliers(fake, fake, fake, None, fake, 4, 64, 3, fake, None) == 1
     need = lib.vq3r_rel_frobenius_outliers_workspace_size(4, 64, 3)
-    assert need > lib.vq3r_rel_frobenius_workspace_size(4, 64)
+    assert need >= lib.vq3r_rel_frobenius_workspace_size(4, 64)
     assert lib.vq3r_rel_frobenius_error_outliers(fake, 1, fake, fake, fake, fake, fake, 4, 64, 3, fake, fake,
                                                  need - 8, None) == 7
     d = (vq.OutlierDesc * 1)(vq.OutlierDesc(fake, fake, 4, 64, 3, fake, fake, 1))
