@@ -315,9 +315,17 @@ def cpu_oracle_sample(seconds, experts=64):
     per_w = t / n
     nrows = max(16, int(seconds / (per_w * (2 * 7168 + 2048))))
     t, n = run(nrows)
-    return {"value": n / t / 1e9, "unit": "Gweights/s", "cores": oracle.max_threads(), "kind": "oracle",
+    cores = oracle.max_threads()
+    # the same work on one core, on a tenth of the rows (reported beside the all-core figure)
+    oracle.set_threads(1)
+    try:
+        t1, n1 = run(max(4, nrows // 10))
+    finally:
+        oracle.set_threads(cores)
+    return {"value": n / t / 1e9, "unit": "Gweights/s", "cores": cores, "kind": "oracle",
             "sample": "%d sampled rows of each of w1, w3, w2 of the 64-expert layer (%d weights): encode + decode + "
-                      "rel-Frobenius + binary64 GEMV, %.1f s" % (nrows, n, t)}
+                      "rel-Frobenius + binary64 GEMV, %.1f s" % (nrows, n, t),
+            "one_core": {"value": n1 / t1 / 1e9, "unit": "Gweights/s", "weights": n1, "seconds": t1}}
 
 
 def run_reference(args, rank, world):
