@@ -349,13 +349,17 @@ vq3r_status vq4p_train(const float* vecs, int64_t n, int iters, int nstages, flo
  *   codebooks as written by vq3r_encode).  Bit-identical to the reading.
  *   k == 0 or rows == 0 is a no-op.
  * vq3r_decode_outliers: vq3r_decode to binary32 followed by the outlier
- *   additions (out [rows][cols] float).
+ *   additions (out [rows][cols] float).  A row's columns must be distinct
+ *   (as vq3r_outliers writes them); a repeated column is a data race.
  * vq3r_rel_frobenius_error_outliers: vq3r_rel_frobenius_error of the decode
  *   with outliers; workspace of vq3r_rel_frobenius_outliers_workspace_size.
  * vq3r_gemv_outliers: y[b][i] += sum_q (float)o_iq * x[b][c_iq] (binary32,
  *   q ascending) for each descriptor, in one launch: enqueue it after the
  *   vq3r_gemv call that wrote y to get the product with the outliers.
- *   1 <= n_mats <= 32, 1 <= B <= 32.
+ *   1 <= n_mats <= 32, 1 <= B <= 32.  No two descriptors may write the same
+ *   elements of y (each y element is updated by one thread, without atomics).
+ * The error call and the sparse add read a row's columns as sorted
+ * ascending, as vq3r_outliers writes them.
  */
 typedef struct {
   const uint16_t* ocols;
