@@ -28,7 +28,7 @@
 
 namespace vq3r {
 
-constexpr int kOutThreads = 256;
+constexpr int kOutThreads = 512;  // >= 256: one histogram bin per thread for the clearing
 constexpr int64_t kOutMaxCols = 16384;  // a row's binary64 errors live in shared memory
 constexpr int kOutGemvMaxMats = 32;
 
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kOutThreads) outlier_select_kernel(const void*
     uint32_t remaining = (uint32_t)k;
     for (int pass = 0; pass < 8; pass++) {
       const int shift = 56 - 8 * pass;
-      hist[tid] = 0u;  // kOutThreads == 256 bins
+      if (tid < 256) hist[tid] = 0u;
       __syncthreads();
       for (int64_t c = tid; c < cols; c += kOutThreads) {
         const uint64_t key = abs_key(ev[c]);
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kOutThreads) outlier_select_kernel(const void*
           neq += key == T;
         }
       }
-      // block exclusive scan of (gt << 16 | eq); each count <= 2048
+      // block exclusive scan of (gt << 16 | eq); each count <= 8 * kOutThreads
       const uint32_t packed = (ngt << 16) | neq;
       uint32_t incl = packed;
 #pragma unroll
