@@ -280,6 +280,17 @@ class Layer:
     LAUNCHES_PER_STEP = 3 * 2 + 3 + 3 * 1 + 3 * 2 + 1  # encode, pack, decode, error, gemv (kernels)
 
 
+def bench_config(experts):
+    """The workload both arms report (the reference arm times bounded row samples of it)."""
+    rows_w13, cols_w13 = wl.mat_shape(wl.W1)
+    rows_w2, cols_w2 = wl.mat_shape(wl.W2)
+    return {"workload": "moe-layer-64x3-bf16: encode + tile repack + decode(fp32) + rel-Frobenius of the layer, "
+                        "then moe-decode-step-8-experts GEMV (B=1)",
+            "experts_per_gpu": experts, "weights_per_gpu": experts * (2 * rows_w13 * cols_w13 + rows_w2 * cols_w2),
+            "matrices": "w1,w3 2048x7168; w2 7168x2048 per expert, stacked per kind",
+            "l2": "inputs larger than L2 (5.6 GB layer); GEMV rotates 8 disjoint 8-expert groups (1.06 GB of indices)"}
+
+
 def errs_plain_w1(layer):
     return float(layer.err[wl.W1].item())
 
@@ -365,7 +376,7 @@ def run_reference(args, rank, world):
     out = {"metric": METRIC, "value": v, "unit": "Gweights/s", "impl": "reference", "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / len(samples),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-           "config": {"workload": "moe-layer-64x3-bf16 (sampled rows) + moe-decode-step", "experts": args.experts},
+           "config": bench_config(args.experts),
            "cpu_baseline": {"value": v, "unit": "Gweights/s", "cores": oracle.max_threads(), "kind": "oracle",
                             "sample": desc},
            "e2e": {"value": v, "unit": "Gweights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -789,12 +800,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "Gweights/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "moe-layer-64x3-bf16: encode + tile repack + decode(fp32) + rel-Frobenius of "
-                                   "the layer, then moe-decode-step-8-experts GEMV (B=1)",
-                       "experts_per_gpu": args.experts, "weights_per_gpu": layer.weights,
-                       "matrices": "w1,w3 2048x7168; w2 7168x2048 per expert, stacked per kind",
-                       "l2": "inputs larger than L2 (5.6 GB layer); GEMV rotates 8 disjoint 8-expert groups "
-                             "(1.06 GB of indices)"},
+            "config": bench_config(args.experts),
             "roofline": {"bound": "alu", "achieved": enc_tflops, "peak": 2 * fp32_peak_tflops, "unit": "TFLOP/s",
                          "frac": enc_tflops / (2 * fp32_peak_tflops),
                          "traffic": (None if ENCODE_DRAM_BYTES_PER_WEIGHT is None
