@@ -14,7 +14,8 @@
 // Kernels:
 //   outlier_select_kernel  one CTA per row: the row's e values in shared
 //                          memory, an exact radix select of the k-th largest
-//                          |e| (8 passes of 8 bits over the 64-bit pattern),
+//                          |e| (up to 8 passes of 8 bits over the 64-bit
+//                          pattern, stopping once the bucket is decided),
 //                          then a column-ordered compaction that takes every
 //                          larger key and the lowest-column equal keys;
 //   outlier_apply_kernel   adds the outliers onto a binary32 decode;

@@ -131,3 +131,42 @@ def test_grouped_sparse_add_over_expert_row_ranges():
     for j, (r0, n, y) in enumerate(outs):
         ref = oracle.gemv(W2[r0:r0 + n], x[j], "f32")
         assert gemv_rel_err(y.cpu().numpy(), ref) <= GEMV_TOL
+
+
+def test_layer_stacked_outliers_sampled_rows():
+    """Outliers of the 64-expert layer's stacked w1 (131072 x 7168 bf16, budget cols/512 = 14 per row, the
+    benchmark's launch), bit-exact against the oracle on 256 sampled rows; the error with outliers of the whole
+    matrix agrees with the decode-with-outliers kernel's output summed in binary64."""
+    import importlib.util
+    import os
+    p = os.path.join(os.path.dirname(__file__), "golden", "make_codebooks.py")
+    spec = importlib.util.spec_from_file_location("make_codebooks", p)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    cb = np.ascontiguousarray(mod.load("layer"))
+    cfg = wl.LAYER
+    rows, cols = wl.mat_shape(wl.W1)
+    E, k = cfg["experts"], cols // 512
+    W_t = torch.empty((E * rows, cols), dtype=torch.bfloat16, device=DEV)
+    for e in range(E):
+        synth.fill_rows_device(W_t[e * rows:(e + 1) * rows].data_ptr(), cols, 0, rows, cfg["seed"], wl.tag(e, wl.W1),
+                               wl.expert_dist(), stream=torch.cuda.current_stream().cuda_stream)
+    cb_t = torch.from_numpy(cb).to(DEV)
+    idx_t, sc_t = vq.vq3r_encode(W_t, cb_t)
+    oc_t, ov_t = vq.vq3r_outliers(W_t, idx_t, sc_t, cb_t, k)
+    rng = np.random.default_rng(45)
+    sample = np.sort(rng.choice(E * rows, 256, replace=False))
+    Wh = np.stack([synth.fill_row_list(cols, [r % rows], cfg["seed"], wl.tag(int(r // rows), wl.W1),
+                                       wl.expert_dist())[0] for r in sample])
+    idx_o, sc_o = oracle.encode(Wh, "bf16", cb)
+    sel = torch.from_numpy(sample).to(DEV)
+    np.testing.assert_array_equal(idx_t[:, sel, :].cpu().numpy(), idx_o)
+    oc_o, ov_o = oracle.outliers_select(Wh, "bf16", oracle.decode(idx_o, sc_o, cb), k)
+    np.testing.assert_array_equal(u16(oc_t[sel]), oc_o)
+    np.testing.assert_array_equal(u16(ov_t[sel]), ov_o)
+    d = vq.vq3r_decode_outliers(idx_t, sc_t, cb_t, oc_t, ov_t)
+    w = W_t.double()
+    e2 = float(torch.sqrt(((w - d.double()) ** 2).sum() / (w ** 2).sum()))
+    del d
+    e = float(vq.vq3r_rel_frobenius_error_outliers(W_t, idx_t, sc_t, cb_t, oc_t, ov_t).cpu()[0])
+    assert abs(e - e2) <= 1e-9 * e2

@@ -164,3 +164,36 @@ def test_expert_w2_full_matrix_bit_exact():
     idx3, sc3 = vq.vq3r_encode(W_t, cb3_t)
     e3 = float(vq.vq3r_rel_frobenius_error(W_t, idx3, sc3, cb3_t).cpu()[0])
     assert 0.1 < e3 < e4 < 0.4, (e3, e4)
+
+
+def test_layer_stacked_encode_sampled_rows():
+    """VQ4P encode of the 64-expert layer's stacked w1 (131072 x 7168 bf16, the benchmark's launch), bit-exact
+    against the oracle on 256 sampled rows (planes and scales); decode of those rows bit-exact."""
+    import importlib.util
+    import os
+    p = os.path.join(os.path.dirname(__file__), "golden", "make_codebooks.py")
+    spec = importlib.util.spec_from_file_location("make_codebooks", p)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    cb = np.ascontiguousarray(mod.load("vq4p_layer"))
+    cfg = wl.LAYER
+    rows, cols = wl.mat_shape(wl.W1)
+    E = cfg["experts"]
+    W_t = torch.empty((E * rows, cols), dtype=torch.bfloat16, device=DEV)
+    for e in range(E):
+        synth.fill_rows_device(W_t[e * rows:(e + 1) * rows].data_ptr(), cols, 0, rows, cfg["seed"], wl.tag(e, wl.W1),
+                               wl.expert_dist(), stream=torch.cuda.current_stream().cuda_stream)
+    cb_t = torch.from_numpy(cb).to(DEV)
+    pl_t, sc_t = vq.vq4p_encode(W_t, cb_t)
+    d_t = vq.vq4p_decode(pl_t, sc_t, cb_t)
+    rng = np.random.default_rng(44)
+    sample = np.sort(rng.choice(E * rows, 256, replace=False))
+    Wh = np.stack([synth.fill_row_list(cols, [r % rows], cfg["seed"], wl.tag(int(r // rows), wl.W1),
+                                       wl.expert_dist())[0] for r in sample])
+    sel = torch.from_numpy(sample).to(DEV)
+    np.testing.assert_array_equal(host_bits(W_t[sel]), Wh)  # the two generators agree
+    pl_o, sc_o = oracle.vq4p_encode(Wh, "bf16", cb)
+    np.testing.assert_array_equal(sc_t[sel].cpu().numpy().view(np.uint16), sc_o)
+    np.testing.assert_array_equal(pl_t[:, sel, :].cpu().numpy(), pl_o)
+    np.testing.assert_array_equal(d_t[sel].cpu().numpy().view(np.uint32),
+                                  oracle.vq4p_decode(pl_o, sc_o, cb).view(np.uint32))
