@@ -1,0 +1,98 @@
+"""The encoder's screening certificate, checked on the CPU against the distance definition.
+
+The GPU encoder screens every codeword with a fused form
+    L(c) = fl32((1/2 - 16u) |c|^2), then acc = fma(r_k, -c_k, acc), k = 0..7   (u = 2^-24)
+and accepts the smallest L without the definition's scan when the second smallest exceeds it by
+    M = fma(fl(fl(|c_best|^2 + R2) + |L_best|), 2^-19, 2^-126),   R2 = sum_k r_k^2 by fused multiply-adds.
+These tests emulate that arithmetic in numpy (binary32 products are exact in binary64, so a fused multiply-add is
+the binary64 sum rounded once to binary32) and assert that whenever the test accepts, the screened winner is the
+definition's winner: d_j = sum_k (r_k - c_jk)^2 with every binary32 operation rounded, lowest index on ties.
+They also check that the test accepts nearly every vector of ordinary data.
+"""
+import numpy as np
+
+F32 = np.float32
+
+
+def fma32(a, b, c):
+    return (a.astype(np.float64) * b.astype(np.float64) + c.astype(np.float64)).astype(F32)
+
+
+def definition_argmin(r, C):
+    """d_j in binary32 with every operation rounded, k ascending; argmin with the lowest index on ties."""
+    e = (r[:, None, 0] - C[None, :, 0]).astype(F32)
+    d = (e * e).astype(F32)
+    for k in range(1, 8):
+        e = (r[:, None, k] - C[None, :, k]).astype(F32)
+        d = (d + (e * e).astype(F32)).astype(F32)
+    return np.argmin(d, axis=1)  # first minimum = lowest index
+
+
+def screen(r, C):
+    """(index of the smallest L, accepted?) per vector, as the kernel computes them."""
+    n = (C.astype(np.float64) ** 2).sum(axis=1)
+    start = ((0.5 - 2.0 ** -20) * n).astype(F32)
+    c2 = n.astype(F32)
+    c2 = np.where(c2.astype(np.float64) < n, np.nextafter(c2, F32(np.inf)), c2)  # rounded up
+    acc = np.broadcast_to(start, (r.shape[0], C.shape[0])).astype(F32)
+    for k in range(8):
+        acc = fma32(np.broadcast_to(r[:, None, k], acc.shape), np.broadcast_to(-C[None, :, k], acc.shape), acc)
+    bi = np.argmin(acc, axis=1)  # strict < tracking keeps the first minimum
+    best = acc[np.arange(len(r)), bi]
+    part = np.partition(acc, 1, axis=1)
+    second = part[:, 1]
+    r2 = fma32(r[:, 0], r[:, 0], np.zeros(len(r), F32))
+    for k in range(1, 8):
+        r2 = fma32(r[:, k], r[:, k], r2)
+    s = ((c2[bi] + r2).astype(F32) + np.abs(best)).astype(F32)
+    m = fma32(s, np.full_like(s, F32(2.0 ** -19)), np.full_like(s, F32(2.0 ** -126)))
+    ok = ((second - best).astype(F32) > m) & (m < F32(2.0 ** 100))
+    return bi, ok
+
+
+def near_twin_codebook(rng, K=256, scale=1.0):
+    C = (rng.standard_normal((K, 8)) * scale).astype(F32)
+    half = K // 2
+    for j in range(half):
+        c = C[j].copy()
+        k = j % 8
+        kind = j % 4
+        if kind == 1:
+            c[k] = np.nextafter(c[k], F32(np.inf))
+        elif kind >= 2:
+            c[k] = F32(c[k] * (1 + 2.0 ** -int(rng.integers(10, 24))))
+        C[half + j] = c
+    return C
+
+
+def test_no_false_accept_on_near_twins_and_near_codeword_vectors():
+    rng = np.random.default_rng(2024)
+    for trial in range(6):
+        C = near_twin_codebook(rng, scale=float(0.25 * (trial + 1)))
+        # residuals close to codewords (tiny gaps between a codeword and its twin), plus plain random ones
+        j = rng.integers(0, 256, 6000)
+        near = (C[j] + rng.standard_normal((6000, 8)).astype(F32) * F32(10.0 ** -rng.integers(1, 7))).astype(F32)
+        plain = (rng.standard_normal((6000, 8)) * rng.uniform(0.1, 4.0)).astype(F32)
+        r = np.concatenate([near, plain]).astype(F32)
+        bi, ok = screen(r, C)
+        want = definition_argmin(r, C)
+        assert np.array_equal(bi[ok], want[ok]), "certificate accepted a wrong winner"
+        assert ok.sum() > 0
+
+
+def test_certificate_accepts_almost_all_ordinary_vectors():
+    rng = np.random.default_rng(7)
+    C = (rng.standard_normal((256, 8)) * 0.8).astype(F32)
+    r = (rng.standard_normal((20000, 8))).astype(F32)
+    bi, ok = screen(r, C)
+    assert np.array_equal(bi[ok], definition_argmin(r, C)[ok])
+    assert ok.mean() > 0.995, ok.mean()
+
+
+def test_exact_ties_are_never_accepted():
+    rng = np.random.default_rng(9)
+    C = (rng.standard_normal((128, 8))).astype(F32)
+    C = np.concatenate([C, C]).astype(F32)  # every codeword twice: every screen has a tie
+    r = (rng.standard_normal((4000, 8))).astype(F32)
+    _, ok = screen(r, C)
+    assert not ok.any()
