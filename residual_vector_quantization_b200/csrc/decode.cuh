@@ -183,6 +183,84 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const uint8_t* _
   }
 }
 
+// Decode with the index bytes staged per tile: a CTA takes tiles of
+// kDecTileV consecutive vectors (t = blockIdx.x, + gridDim.x, ...); thread 0
+// copies a tile's three index planes into shared memory with bulk
+// asynchronous copies (no multicast), two tiles in flight, and the threads
+// decode from there.  Plane p of a tile starts at idx + p * nvec + t *
+// kDecTileV: the host uses this kernel when nvec is a multiple of 16, so
+// every copy starts on a 16-byte boundary and moves a multiple of 16 bytes.
+constexpr int kDecTileV = 2048;
+template <int FMT>
+__host__ __device__ constexpr size_t decode_bulk_smem() {
+  return fmt_cbr_floats<FMT>() * sizeof(float) + 2 * 3 * kDecTileV;
+}
+
+template <int OUT_DT, int FMT>
+__global__ void __launch_bounds__(kDecThreads, 2) decode_bulk_kernel(const uint8_t* __restrict__ idx,
+                                                                      const uint16_t* __restrict__ scales,
+                                                                      const float* __restrict__ codebooks,
+                                                                      int64_t rows, int64_t cols,
+                                                                      void* __restrict__ out) {
+  extern __shared__ __align__(16) float cbr[];
+  uint8_t* const tiles = reinterpret_cast<uint8_t*>(cbr + fmt_cbr_floats<FMT>());  // [2][3][kDecTileV]
+  __shared__ uint64_t mbar[2];
+  const int tid = threadIdx.x, lane = tid & 31, h = lane & 1;
+  const int64_t V = cols / kDim, nvec = rows * V;
+  const int64_t ntiles = (nvec + kDecTileV - 1) / kDecTileV;
+  auto issue = [&](int64_t t, int b) {  // thread 0: tile t into buffer b
+    const int64_t g0 = t * kDecTileV;
+    const uint32_t n = (uint32_t)(nvec - g0 < kDecTileV ? nvec - g0 : kDecTileV);
+    mbar_arrive_expect_tx(&mbar[b], 3 * n);
+#pragma unroll
+    for (int p = 0; p < 3; p++) bulk_copy_g2s(tiles + (b * 3 + p) * kDecTileV, idx + p * nvec + g0, n, &mbar[b]);
+  };
+  if (tid == 0) {
+    mbar_init(&mbar[0], 1);
+    mbar_init(&mbar[1], 1);
+    if (blockIdx.x < ntiles) issue(blockIdx.x, 0);
+    if (blockIdx.x + gridDim.x < ntiles) issue(blockIdx.x + gridDim.x, 1);
+  }
+  load_codebooks_replicated<FMT>(cbr, codebooks);  // ends with a barrier: the barriers are initialised too
+  const int64_t step = kDecThreads / 2, dq = step / V, dr = step - dq * V;
+  bool ok = true;
+  int it = 0;
+  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, it++) {
+    const int b = it & 1;
+    ok = mbar_wait_bounded(&mbar[b], (uint32_t)(it >> 1) & 1u) && ok;
+    const int64_t g0 = t * kDecTileV;
+    const int n = (int)(nvec - g0 < kDecTileV ? nvec - g0 : kDecTileV);
+    const uint8_t* tp = tiles + b * 3 * kDecTileV;
+    int64_t row = (g0 + (tid >> 1)) / V, v = g0 + (tid >> 1) - row * V;
+    for (int j = tid >> 1; j < n; j += (int)step) {
+      const float s = f16_bits_to_f32(__ldg(scales + row));
+      const float4 o = decode_half_r<FMT>(cbr, tp[j], tp[kDecTileV + j], tp[2 * kDecTileV + j], s, lane);
+      const int64_t g = g0 + j;
+      if constexpr (OUT_DT == VQ3R_F32) {
+        __stcs(reinterpret_cast<float4*>(static_cast<float*>(out) + g * kDim + 4 * h), o);
+      } else {
+        const uint32_t u0 = (uint32_t)__half_as_ushort(__float2half_rn(o.x)) |
+                            ((uint32_t)__half_as_ushort(__float2half_rn(o.y)) << 16);
+        const uint32_t u1 = (uint32_t)__half_as_ushort(__float2half_rn(o.z)) |
+                            ((uint32_t)__half_as_ushort(__float2half_rn(o.w)) << 16);
+        __stcs(reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + g * kDim + 4 * h), make_uint2(u0, u1));
+      }
+      row += dq;
+      v += dr;
+      if (v >= V) {
+        v -= V;
+        row++;
+      }
+    }
+    __syncthreads();  // every thread is done with buffer b
+    if (tid == 0 && t + 2 * (int64_t)gridDim.x < ntiles) {
+      fence_proxy_async_smem();  // generic reads of the buffer precede its async refill
+      issue(t + 2 * (int64_t)gridDim.x, b);
+    }
+  }
+  (void)ok;  // a timed-out wait has recorded the device error word
+}
+
 // ---- relative Frobenius error: per-CTA binary64 partials, then one CTA ----
 
 constexpr int kErrThreads = 512;

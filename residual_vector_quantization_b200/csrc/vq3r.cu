@@ -68,6 +68,10 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
     const int gm = (int)kMmaSmemBytes;
     const int gc = (int)(kCbrFloats * sizeof(float));
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_bulk_kernel<VQ3R_F32, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_bulk_smem<FMT_VQ3R>());
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_bulk_kernel<VQ3R_F16, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_bulk_smem<FMT_VQ3R>());
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_bulk_kernel<VQ3R_F32, FMT_VQ4P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_bulk_smem<FMT_VQ4P>());
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_bulk_kernel<VQ3R_F16, FMT_VQ4P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_bulk_smem<FMT_VQ4P>());
     if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_kernel<VQ3R_F32, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_kernel<VQ3R_F16, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(relfro_partial_kernel<VQ3R_F32, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, gc);
@@ -326,6 +330,17 @@ vq3r_status decode_entry(const uint8_t* idx, const uint16_t* scales, const float
   cudaError_t e = device_setup(&sms);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nvec = rows * (cols / kDim);
+  if (nvec % 16 == 0) {  // index tiles staged by bulk copies (16-byte aligned planes)
+    const int64_t ntiles = (nvec + kDecTileV - 1) / kDecTileV;
+    const int grid = (int)(ntiles < 2 * (int64_t)sms ? ntiles : 2 * (int64_t)sms);
+    const size_t smem = decode_bulk_smem<FMT>();
+    if (out_dtype == VQ3R_F32)
+      decode_bulk_kernel<VQ3R_F32, FMT><<<grid, kDecThreads, smem, s>>>(idx, scales, codebooks, rows, cols, out);
+    else
+      decode_bulk_kernel<VQ3R_F16, FMT><<<grid, kDecThreads, smem, s>>>(idx, scales, codebooks, rows, cols, out);
+    return check_launch();
+  }
   const int64_t blocks = rowsplit_blocks(rows, cols, sms, (int64_t)1 << 30);
   const size_t smem = fmt_cbr_floats<FMT>() * sizeof(float);
   if (out_dtype == VQ3R_F32)
