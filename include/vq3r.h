@@ -397,6 +397,12 @@ int vq3r_last_cuda_error(void);
  * reading it clears it. */
 vq3r_status vq3r_device_error(int* code);
 
+/* Failure-path self-test: launches one warp that waits on a shared-memory
+ * barrier nothing completes.  After about one second the bounded wait gives
+ * up and records device error 1 (read it with vq3r_device_error); the kernel
+ * returns and the context stays usable.  Takes about one second. */
+vq3r_status vq3r_selftest_wait_timeout(vq3r_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

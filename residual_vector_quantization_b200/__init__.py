@@ -28,7 +28,8 @@ EXPORTED = ["vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_gemv_workspace_size
             "vq3r_device_error", "vq3r_gemv_noalloc", "vq3r_tiles_size", "vq3r_pack_tiles", "vq3r_gemm",
             "vq3r_train", "vq3r_train_workspace_size", "vq4p_encode", "vq4p_decode", "vq4p_rel_frobenius_error",
             "vq4p_train", "vq4p_train_workspace_size", "vq3r_outliers", "vq3r_decode_outliers",
-            "vq3r_rel_frobenius_error_outliers", "vq3r_rel_frobenius_outliers_workspace_size", "vq3r_gemv_outliers"]
+            "vq3r_rel_frobenius_error_outliers", "vq3r_rel_frobenius_outliers_workspace_size", "vq3r_gemv_outliers",
+            "vq3r_selftest_wait_timeout"]
 
 
 class VQ3RError(RuntimeError):
@@ -100,6 +101,8 @@ def _lib():
         L.vq3r_rel_frobenius_outliers_workspace_size.restype = SZ
         L.vq3r_rel_frobenius_error_outliers.argtypes = [P, I32, P, P, P, P, P, I64, I64, I64, P, P, SZ, P]
         L.vq3r_gemv_outliers.argtypes = [P, I32, I32, I32, P]
+        L.vq3r_selftest_wait_timeout.argtypes = [P]
+        L.vq3r_selftest_wait_timeout.restype = I32
         for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error",
                   "vq3r_gemv_noalloc", "vq3r_pack_tiles", "vq3r_gemm", "vq3r_train", "vq4p_encode", "vq4p_decode",
                   "vq4p_rel_frobenius_error", "vq4p_train", "vq3r_outliers", "vq3r_decode_outliers",
@@ -415,6 +418,11 @@ def vq3r_gemv_outliers(mats, B, stream=None):
     xdt = _DT[mats[0]["x"].dtype]
     _check(_lib().vq3r_gemv_outliers(arr, len(mats), B, xdt, _stream(stream)), "vq3r_gemv_outliers")
     return [m["y"] for m in mats]
+
+
+def vq3r_selftest_wait_timeout(stream=None):
+    """Launch the failure-path self-test (a bounded wait that runs out after about one second)."""
+    _check(_lib().vq3r_selftest_wait_timeout(_stream(stream)), "vq3r_selftest_wait_timeout")
 
 
 def vq3r_device_error():

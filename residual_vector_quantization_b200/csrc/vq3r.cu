@@ -869,6 +869,14 @@ const char* vq3r_status_string(vq3r_status s) {
 
 int vq3r_last_cuda_error(void) { return t_last_cuda_error; }
 
+vq3r_status vq3r_selftest_wait_timeout(vq3r_stream stream) {
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return check_launch();
+}
+
 vq3r_status vq3r_device_error(int* code) {
   if (!code) return VQ3R_ERR_NULL;
   cudaError_t e = cudaDeviceSynchronize();

@@ -188,4 +188,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* mbar, uint32_t parit
   }
 }
 
+// Self-test of the failure path: one warp initialises a shared-memory barrier
+// that nothing arrives at and waits on it.  The bounded wait gives up after
+// about one second, records kDevErrMbarTimeout, and the kernel returns.
+__global__ void __launch_bounds__(32) selftest_wait_kernel() {
+  __shared__ uint64_t mbar;
+  if (threadIdx.x == 0) mbar_init(&mbar, 1);
+  __syncwarp();
+  (void)mbar_wait_bounded(&mbar, 0);
+}
+
 }  // namespace vq3r
