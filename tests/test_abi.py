@@ -212,3 +212,28 @@ def test_outlier_argument_checks(lib):
     assert lib.vq3r_gemv_outliers(d, 1, 1, 1, None) == 2   # reserved must be 0
     assert lib.vq3r_gemv_outliers(d, 0, 1, 1, None) == 5
     assert lib.vq3r_gemv_outliers(d, 1, 33, 1, None) == 5
+
+
+def test_outlier_descriptor_and_budget_checks(lib):
+    fake = 0x100000
+    ok_desc = vq.OutlierDesc(fake, fake, 4, 64, 3, fake, fake, 0)
+    null_y = vq.OutlierDesc(fake, fake, 4, 64, 3, fake, None, 0)
+    bad_align = vq.OutlierDesc(fake + 2, fake, 4, 64, 3, fake, fake, 0)
+    too_many = vq.OutlierDesc(fake, fake, 4, 64, 65, fake, fake, 0)
+    empty = vq.OutlierDesc(None, None, 4, 64, 0, None, None, 0)   # k = 0: skipped, no pointers needed
+    for d, want in ((null_y, 1), (bad_align, 3), (too_many, 2)):
+        arr = (vq.OutlierDesc * 2)(ok_desc, d)
+        assert lib.vq3r_gemv_outliers(arr, 2, 1, 1, None) == want
+    assert lib.vq3r_gemv_outliers((vq.OutlierDesc * 1)(empty), 1, 1, 1, None) == 0
+    assert lib.vq3r_gemv_outliers((vq.OutlierDesc * 1)(ok_desc), 1, 1, 9, None) == 4   # bad x dtype
+    assert lib.vq3r_decode_outliers(fake, fake, fake, fake, fake, 4, 64, 65, fake, None) == 2
+    assert lib.vq3r_decode_outliers(fake, fake, fake, fake, fake, 4, 16392, 3, fake, None) == 2
+    assert lib.vq3r_rel_frobenius_error_outliers(fake, 1, fake, fake, fake, None, fake, 4, 64, 3, fake, fake,
+                                                 1 << 20, None) == 1
+    assert lib.vq3r_rel_frobenius_error_outliers(fake, 1, fake, fake, fake, fake, fake, 0, 64, 3, fake, fake,
+                                                 1 << 20, None) == 2   # rows >= 1
+
+
+def test_selftest_symbol_is_exported(lib):
+    assert hasattr(lib, "vq3r_selftest_wait_timeout")
+    assert "vq3r_selftest_wait_timeout" in vq.EXPORTED
