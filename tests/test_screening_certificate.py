@@ -96,3 +96,52 @@ def test_exact_ties_are_never_accepted():
     r = (rng.standard_normal((4000, 8))).astype(F32)
     _, ok = screen(r, C)
     assert not ok.any()
+
+
+def test_vq4p_sized_codebooks_near_twins():
+    rng = np.random.default_rng(64)
+    for trial in range(4):
+        C = near_twin_codebook(rng, K=64, scale=float(0.5 * (trial + 1)))
+        j = rng.integers(0, 64, 8000)
+        r = (C[j] + rng.standard_normal((8000, 8)).astype(F32) * F32(10.0 ** -rng.integers(1, 7))).astype(F32)
+        bi, ok = screen(r, C)
+        assert np.array_equal(bi[ok], definition_argmin(r, C)[ok])
+
+
+def test_mixed_norm_codebooks():
+    """A few codewords of norm ~1e3 among ordinary ones: the margin uses the chosen codeword's own norm."""
+    rng = np.random.default_rng(65)
+    C = (rng.standard_normal((256, 8)) * 0.7).astype(F32)
+    C[rng.choice(256, 8, replace=False)] *= F32(1500.0)
+    r = np.concatenate([(rng.standard_normal((8000, 8))).astype(F32),
+                        (C[rng.integers(0, 256, 2000)] * F32(1.0001)).astype(F32)])
+    bi, ok = screen(r, C)
+    assert np.array_equal(bi[ok], definition_argmin(r, C)[ok])
+    assert ok[:8000].mean() > 0.99
+
+
+def test_tiny_and_subnormal_scale_residuals():
+    """Residuals and codewords around 1e-20 (squares near the binary32 subnormal range)."""
+    rng = np.random.default_rng(66)
+    for s in (1e-12, 1e-18, 1e-20):
+        C = (rng.standard_normal((256, 8)) * s).astype(F32)
+        r = (rng.standard_normal((6000, 8)) * s).astype(F32)
+        bi, ok = screen(r, C)
+        assert np.array_equal(bi[ok], definition_argmin(r, C)[ok])
+
+
+def test_large_values_and_overflow():
+    """Large values whose squares stay finite (1e17): accepted winners are right.  Values whose squares overflow
+    binary32 (1e19 and up): the margin is infinite or at least 2^100 and the test refuses, so those vectors go to
+    the definition's scan."""
+    rng = np.random.default_rng(67)
+    with np.errstate(over="ignore", invalid="ignore"):
+        C = (rng.standard_normal((256, 8)) * 1e17).astype(F32)
+        r = (rng.standard_normal((2000, 8)) * 1e17).astype(F32)
+        bi, ok = screen(r, C)
+        assert np.array_equal(bi[ok], definition_argmin(r, C)[ok])
+        for s in (1e19, 1e30):
+            C = (rng.standard_normal((256, 8)) * s).astype(F32)
+            r = (rng.standard_normal((2000, 8)) * s).astype(F32)
+            _, ok = screen(r, C)
+            assert not ok.any()
