@@ -257,6 +257,41 @@ def test_exhaustive_joint_search_lower_bounds_greedy():
     np.testing.assert_allclose(((r.astype(np.float64) - bj) ** 2).sum(1), berr, rtol=1e-12)
 
 
+def test_exhaustive_finds_a_planted_joint_optimum_that_greedy_misses():
+    """Codebooks built so that each test vector r = e_m (unit vector of dim m) has exactly one triple summing to
+    it, C1[b] + C2[p] + C3[z3] = 0.5 e_m + 0.5 e_m + 0, while greedy is lured by C1[a] = 0.875 e_m (distance
+    1/64 against 1/4 for C1[b]) and then takes the zero codewords, ending at error exactly 1/64.  Every other
+    codeword sits at 64 + j on dimension 7 (all positive, so no two of them cancel).  The planted indices sit at
+    the ends and the middle of each range (b = 255 for one vector, p = 255 for another, z3 = 255 for all), so a
+    search that skipped any part of a range, or mixed up which stage a codebook belongs to, returns another
+    triple or a non-zero error.  All values are dyadic: the expected errors are exact in binary64."""
+    cb = np.zeros((3, K, D), np.float32)
+    for s in range(3):
+        cb[s, :, 7] = 64.0 + np.arange(K)
+    z2, z3 = 7, 255
+    cb[1, z2] = 0.0
+    cb[2, z3] = 0.0
+    plants = [(0, 0, 255, 17), (1, 1, 3, 255), (2, 2, 128, 129), (3, 254, 200, 0), (4, 100, 5, 254)]
+    for m, a, b, p in plants:
+        cb[0, a] = 0.0
+        cb[0, a, m] = 0.875
+        cb[0, b] = 0.0
+        cb[0, b, m] = 0.5
+        cb[1, p] = 0.0
+        cb[1, p, m] = 0.5
+    r = np.zeros((len(plants), D), np.float32)
+    for i, (m, _, _, _) in enumerate(plants):
+        r[i, m] = 1.0
+    # greedy: the lure, then the zero codewords; error 1/64
+    idx, res = oracle.encode_vectors(r, cb)
+    np.testing.assert_array_equal(idx, [[a, z2, z3] for _, a, _, _ in plants])
+    np.testing.assert_array_equal((res.astype(np.float64) ** 2).sum(1), np.full(len(plants), 1.0 / 64))
+    # exhaustive: the planted triple, error exactly zero
+    bidx, berr = oracle.bruteforce_joint(r, cb)
+    np.testing.assert_array_equal(bidx, [[b, p, z3] for _, _, b, p in plants])
+    np.testing.assert_array_equal(berr, np.zeros(len(plants)))
+
+
 def test_exhaustive_equals_greedy_when_later_stages_are_zero():
     rng = np.random.default_rng(7)
     cb = np.zeros((3, K, D), np.float32)

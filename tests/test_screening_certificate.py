@@ -4,18 +4,73 @@ The GPU encoder screens every codeword with a fused form
     L(c) = fl32((1/2 - 16u) |c|^2), then acc = fma(r_k, -c_k, acc), k = 0..7   (u = 2^-24)
 and accepts the smallest L without the definition's scan when the second smallest exceeds it by
     M = fma(fl(fl(|c_best|^2 + R2) + |L_best|), 2^-19, 2^-126),   R2 = sum_k r_k^2 by fused multiply-adds.
-These tests emulate that arithmetic in numpy (binary32 products are exact in binary64, so a fused multiply-add is
-the binary64 sum rounded once to binary32) and assert that whenever the test accepts, the screened winner is the
+These tests emulate that arithmetic in numpy and assert that whenever the test accepts, the screened winner is the
 definition's winner: d_j = sum_k (r_k - c_jk)^2 with every binary32 operation rounded, lowest index on ties.
 They also check that the test accepts nearly every vector of ordinary data.
+
+The fused multiply-add is emulated exactly.  A binary32 product is exact in binary64, but the binary64 sum p + c
+may round, and rounding that sum again to binary32 can differ from one rounding of the exact value: this happens
+exactly when the binary64 sum lands on a binary32 rounding midpoint while the exact sum does not.  TwoSum gives
+the rounding error of the binary64 sum, and its sign settles those midpoints.
 """
+from fractions import Fraction
+
 import numpy as np
 
 F32 = np.float32
 
 
 def fma32(a, b, c):
-    return (a.astype(np.float64) * b.astype(np.float64) + c.astype(np.float64)).astype(F32)
+    """binary32 fused multiply-add fl32(a*b + c) with a single rounding (round to nearest even), elementwise."""
+    a, b, c = np.broadcast_arrays(np.asarray(a, F32), np.asarray(b, F32), np.asarray(c, F32))
+    p = a.astype(np.float64) * b.astype(np.float64)  # exact: 24 + 24 bits fit in 53
+    c64 = c.astype(np.float64)
+    s = p + c64
+    bb = s - p
+    err = (p - (s - bb)) + (c64 - bb)  # TwoSum: p + c = s + err exactly
+    out = s.astype(F32)
+    # binary32 neighbours around s, and the midpoint between them (exact in binary64)
+    lo = np.where(out.astype(np.float64) <= s, out, np.nextafter(out, F32(-np.inf)))
+    hi = np.nextafter(lo, F32(np.inf))
+    mid = (lo.astype(np.float64) + hi.astype(np.float64)) * 0.5
+    on_mid = np.isfinite(mid) & (s == mid) & (err != 0)
+    return np.where(on_mid, np.where(err > 0, hi, lo), out).astype(F32)
+
+
+def _fma32_exact(a, b, c):
+    """Reference for fma32: the exact rational a*b + c rounded once to binary32 (nearest, ties to even)."""
+    v = Fraction(float(a)) * Fraction(float(b)) + Fraction(float(c))
+    x = F32(float(v))  # float(v) rounds once to binary64; correct it below when that lands on a midpoint
+    lo = x if Fraction(float(x)) <= v else np.nextafter(x, F32(-np.inf))
+    hi = np.nextafter(lo, F32(np.inf))
+    dl, dh = v - Fraction(float(lo)), Fraction(float(hi)) - v
+    if dl < dh:
+        return lo
+    if dh < dl:
+        return hi
+    return lo if (int(lo.view(np.uint32)) & 1) == 0 else hi
+
+
+def test_fma32_rounds_once():
+    """The emulation against exact rational arithmetic, on a constructed double-rounding case and on random and
+    cancelling inputs.  The constructed case: c = 1 + 2^-23 (odd last bit), a*b = 2^-24 - 2^-70; the exact sum
+    lies just below the midpoint 1 + 3 * 2^-24 and rounds down to c, while its binary64 rounding is the midpoint
+    itself, which rounds to even, up to 1 + 2^-22."""
+    a = np.array([2.0 ** -24 * (1 + 2.0 ** -23)], F32)
+    b = np.array([1 - 2.0 ** -23], F32)
+    c = np.array([1 + 2.0 ** -23], F32)
+    naive = (a.astype(np.float64) * b.astype(np.float64) + c.astype(np.float64)).astype(F32)
+    assert naive[0] == F32(1 + 2.0 ** -22)
+    assert fma32(a, b, c)[0] == F32(1 + 2.0 ** -23) == _fma32_exact(a[0], b[0], c[0])
+    rng = np.random.default_rng(11)
+    n = 4000
+    a = (rng.standard_normal(n) * 2.0 ** rng.integers(-30, 30, n)).astype(F32)
+    b = (rng.standard_normal(n) * 2.0 ** rng.integers(-30, 30, n)).astype(F32)
+    c = (rng.standard_normal(n) * 2.0 ** rng.integers(-60, 60, n)).astype(F32)
+    c[: n // 4] = (-(a[: n // 4].astype(np.float64) * b[: n // 4])).astype(F32)  # near-total cancellation
+    got = fma32(a, b, c)
+    for i in range(n):
+        assert got[i] == _fma32_exact(a[i], b[i], c[i]), (a[i], b[i], c[i])
 
 
 def definition_argmin(r, C):
