@@ -1,6 +1,7 @@
 // C ABI of the VQ3R library (declared in include/vq3r.h): argument checks,
 // launch configuration and status codes.  All arithmetic runs in the
 // kernels of encode.cuh, decode.cuh and gemv.cuh.
+#include <atomic>
 #include <mutex>
 
 #include "decode.cuh"
@@ -40,16 +41,21 @@ vq3r_status check_shape(int64_t rows, int64_t cols, int64_t min_rows) {
 
 // Per-device launch setup: SM count and the dynamic shared-memory opt-ins.
 constexpr int kMaxDevices = 64;
-std::once_flag g_dev_once[kMaxDevices];
+std::mutex g_dev_mu;
+std::atomic<bool> g_dev_ready[kMaxDevices];  // set once a setup has succeeded; a failed one is retried
 int g_dev_sms[kMaxDevices];
-cudaError_t g_dev_err[kMaxDevices];
 
 cudaError_t device_setup(int* sms) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_dev_once[dev], [dev]() {
+  if (g_dev_ready[dev].load(std::memory_order_acquire)) {
+    *sms = g_dev_sms[dev];
+    return cudaSuccess;
+  }
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  {
     cudaError_t r = cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev);
     const int enc = (int)sizeof(EncSmem);
     const int gv = (int)kGvSmemBytes;
@@ -89,10 +95,11 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
-    g_dev_err[dev] = r;
-  });
+    if (r != cudaSuccess) return r;
+  }
+  g_dev_ready[dev].store(true, std::memory_order_release);
   *sms = g_dev_sms[dev];
-  return g_dev_err[dev];
+  return cudaSuccess;
 }
 
 constexpr size_t kWsAlign = 256;
@@ -819,22 +826,25 @@ namespace {
 // current.
 static __device__ __align__(256) unsigned char g_gemv_noalloc_scratch[VQ3R_GEMV_NOALLOC_BYTES];
 
-std::once_flag g_noalloc_once[kMaxDevices];
+// Looked-up addresses, per device; null until a lookup has succeeded.  A
+// failed lookup is not remembered, so the next call tries again.
+std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices];
-cudaError_t g_noalloc_err[kMaxDevices];
 
 cudaError_t noalloc_scratch(void** ptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_noalloc_once[dev], [dev]() {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
     void* p = nullptr;
-    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_gemv_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_gemv_noalloc_scratch);
+    if (e != cudaSuccess) return e;
     g_noalloc_ptr[dev] = p;
-  });
+  }
   *ptr = g_noalloc_ptr[dev];
-  return g_noalloc_err[dev];
+  return cudaSuccess;
 }
 
 }  // namespace
