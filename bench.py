@@ -43,9 +43,9 @@ VQ4P_FLOPS_PER_WEIGHT = 768  # 4 stages x 64 codewords x 8 dims x (sub, mul, add
 ALU_OPS_PER_VEC_CODEWORD = 5
 ENC_ALU_OPS_PER_WEIGHT = 3 * 256 * ALU_OPS_PER_VEC_CODEWORD / 8  # 480
 ALU_LANES_PER_SM = 64
-# DRAM bytes (read + write) per weight of the encode kernel, from an ncu capture
-# of this kernel (dram__bytes_read.sum + dram__bytes_write.sum over 117.4 M
-# weights); None once the kernel changes and until it is captured again.
+# DRAM bytes (read + write) per weight of the encode kernel: dram__bytes_read.sum + dram__bytes_write.sum of the
+# ncu capture in profiles/encode_kernel_moe-layer-8-experts.md (117.4 M weights).  Set to None when the encode
+# kernel changes, until it is captured again.
 ENCODE_DRAM_BYTES_PER_WEIGHT = (235268096 + 8084736) / 117440512
 SM_COUNT_NOMINAL = 148
 FP32_LANES_PER_SM = 128
@@ -64,6 +64,11 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep-experts", type=int, default=256,
+                    help="experts of the scale-sweep workload (Student-t(3) with 0.1%% outliers at 20 sigma) whose "
+                         "encode and decode-GEMV are measured after the timed step; 0 skips it")
+    ap.add_argument("--no-expert-quality", action="store_true",
+                    help="skip the single-expert quality table (VQ3R beside the oracle's rtn4-row)")
     return ap.parse_args()
 
 
@@ -339,6 +344,23 @@ def cpu_oracle_sample(seconds, experts=64):
             "one_core": {"value": n1 / t1 / 1e9, "unit": "Gweights/s", "weights": n1, "seconds": t1}}
 
 
+def expert_rtn4_quality():
+    """The single-expert workload (w1, w3: 2048 x 7168, w2: 7168 x 2048, Student-t(4) x log-normal rows, seed 1):
+    the oracle's rtn4-row baseline error of each matrix (symmetric per-row int4, fp16 scale, 4.01 bits/weight).
+    Part of the CPU leg: the oracle on host cores, before CUDA starts."""
+    import oracle
+    cfg, dist = wl.EXPERT, wl.expert_dist()
+    out = {}
+    t0 = time.perf_counter()
+    for k, name in ((wl.W1, "w1"), (wl.W3, "w3"), (wl.W2, "w2")):
+        rows, cols = wl.mat_shape(k)
+        W = synth.fill_rows(cols, 0, rows, cfg["seed"], wl.tag(0, k), dist)
+        Wq, _ = oracle.rtn4_row(W, "bf16")
+        out[name] = oracle.rel_frobenius(W, "bf16", Wq)
+    out["seconds"] = time.perf_counter() - t0
+    return out
+
+
 def run_reference(args, rank, world):
     """--impl reference: the CPU oracle on a bounded sample, same metric and config."""
     if rank != 0:
@@ -400,6 +422,19 @@ def max_over_ranks(torch, value, world, device):
     return float(t.item())
 
 
+def timed_region(torch, fn, reps):
+    """Mean ms of reps calls of fn (after one untimed call), CUDA events on the current stream."""
+    fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
 def whole_job_rate(world, weights_per_rank, ms):
     """Gweights/s of the whole job: every rank's weights over the slowest rank's time."""
     return world * weights_per_rank / ms / 1e6
@@ -420,8 +455,11 @@ def main():
 
     # CPU baseline first (the oracle on host cores, before CUDA starts)
     cpu = None
+    rtn4 = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(args.cpu_seconds, args.experts)
+        if not args.no_expert_quality:
+            rtn4 = expert_rtn4_quality()
 
     import torch
     import residual_vector_quantization_b200 as vq
@@ -720,6 +758,115 @@ def main():
                 "sweep_8x_w1_error_plain": es0, "sweep_8x_w1_error_with_outliers": sweep_gain}
         del oc, ov, odescs
 
+    # the single-expert workload's quality table: VQ3R error of w1, w3, w2 (this library, expert codebooks) beside
+    # the oracle's rtn4-row error of the same matrices (computed in the CPU leg), outside the timed region
+    quality = None
+    if rtn4 is not None:
+        cbe = torch.from_numpy(load_codebooks("expert")).to(dev)
+        vq3 = {}
+        for k, name in ((wl.W1, "w1"), (wl.W3, "w3"), (wl.W2, "w2")):
+            rows, cols = wl.mat_shape(k)
+            We = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+            synth.fill_rows_device(We.data_ptr(), cols, 0, rows, wl.EXPERT["seed"], wl.tag(0, k), wl.expert_dist(),
+                                   stream=torch.cuda.current_stream().cuda_stream)
+            ie, se = vq.vq3r_encode(We, cbe)
+            vq3[name] = float(vq.vq3r_rel_frobenius_error(We, ie, se, cbe).item())
+            del We, ie, se
+        quality = {"workload": wl.EXPERT["name"] + ", seed %d" % wl.EXPERT["seed"],
+                   "vq3r_3.00bpw": vq3, "rtn4_row_4.01bpw_oracle": {n: rtn4[n] for n in ("w1", "w3", "w2")},
+                   "bits_per_weight": {"vq3r": {"w1": 3 + 16 / 7168, "w3": 3 + 16 / 7168, "w2": 3 + 16 / 2048},
+                                       "rtn4_row": {"w1": 4 + 16 / 7168, "w3": 4 + 16 / 7168, "w2": 4 + 16 / 2048}}}
+
+    # the scale-sweep workload: 256 experts x {w1, w3: 2048 x 7168; w2: 7168 x 2048}, Student-t(3) rows with 0.1%
+    # of the weights at +-20 sigma, seed 4 (11.27 G weights, 22.5 GB of bf16): encode of each stacked matrix kind,
+    # then the decode-GEMV at B = 1, 4, 8, 32 over all experts, as one call over the three stacked matrices and as
+    # 8-expert decode steps rotating over all 32 disjoint groups
+    sweep = None
+    if args.sweep_experts > 0:
+        E5 = args.sweep_experts
+        st5 = torch.cuda.current_stream().cuda_stream
+        cb5 = torch.from_numpy(load_codebooks("sweep")).to(dev)
+        W5, I5, S5 = {}, {}, {}
+        for k in layer.kinds:
+            rows, cols = wl.mat_shape(k)
+            W5[k] = torch.empty((E5 * rows, cols), dtype=torch.bfloat16, device=dev)
+            for e in range(E5):
+                synth.fill_rows_device(W5[k][e * rows:(e + 1) * rows].data_ptr(), cols, 0, rows, wl.SWEEP["seed"],
+                                       wl.tag(e, k), wl.sweep_dist(), stream=st5)
+            I5[k] = torch.empty((3, E5 * rows, cols // 8), dtype=torch.uint8, device=dev)
+            S5[k] = torch.empty(E5 * rows, dtype=torch.int16, device=dev)
+        n5 = sum(W5[k].numel() for k in layer.kinds)
+
+        def enc5():
+            for k in layer.kinds:
+                vq.vq3r_encode(W5[k], cb5, I5[k], S5[k])
+
+        enc5_ms = timed_region(torch, enc5, 2)
+        del W5
+        torch.cuda.empty_cache()
+        T5 = {k: vq.vq3r_pack_tiles(I5[k]) for k in layer.kinds}
+        del I5
+        enc5_tflops = FLOPS_PER_WEIGHT * n5 / enc5_ms / 1e9
+        gv_all, gv_steps = {}, {}
+        for B in B_list:
+            _, _, xu, xd = layer.moe[B]
+            mats = []
+            for k in layer.kinds:
+                rows, cols = wl.mat_shape(k)
+                mats.append(dict(idx=T5[k], scales=S5[k], codebooks=cb5, x=xu if cols == wl.HIDDEN else xd[0],
+                                 rows=E5 * rows, layout="tiles", cols=cols,
+                                 y=torch.empty((B, E5 * rows), dtype=torch.float32, device=dev)))
+            d = vq._descs(mats)
+            ws5 = torch.zeros(max(256, vq.lib().vq3r_gemv_workspace_size(d, 3, B)), dtype=torch.uint8, device=dev)
+            def call():
+                st = vq.lib().vq3r_gemv(d, 3, B, 1, ws5.data_ptr(), ws5.numel(), st5)
+                if st:
+                    raise vq.VQ3RError(st, "vq3r_gemv")
+
+            ms = timed_region(torch, call, 3 if B <= 8 else 2)
+            nbytes = layer_gemv_bytes(B, E5)
+            gv_all[str(B)] = {"us_per_call": 1e3 * ms, "GB/s": nbytes / ms / 1e6,
+                              "frac_hbm": nbytes / ms / 1e6 / hbm_gbs}
+            del mats, d
+            groups = []
+            for g in range(E5 // 8):
+                ms_ = []
+                for j in range(8):
+                    e = g * 8 + j
+                    for k in (wl.W1, wl.W3):
+                        rows, cols = wl.mat_shape(k)
+                        ms_.append(dict(idx=T5[k], scales=S5[k], codebooks=cb5, x=xu, row0=e * rows, rows=rows,
+                                        layout="tiles", cols=cols,
+                                        y=torch.empty((B, rows), dtype=torch.float32, device=dev)))
+                for j in range(8):
+                    e = g * 8 + j
+                    rows, cols = wl.mat_shape(wl.W2)
+                    ms_.append(dict(idx=T5[wl.W2], scales=S5[wl.W2], codebooks=cb5, x=xd[j], row0=e * rows,
+                                    rows=rows, layout="tiles", cols=cols,
+                                    y=torch.empty((B, rows), dtype=torch.float32, device=dev)))
+                groups.append((vq._descs(ms_), ms_))
+
+            def steps():
+                for dg, _ in groups:
+                    st = vq.lib().vq3r_gemv(dg, 24, B, 1, ws5.data_ptr(), ws5.numel(), st5)
+                    if st:
+                        raise vq.VQ3RError(st, "vq3r_gemv")
+
+            ms = timed_region(torch, steps, 2) / len(groups)
+            gv_steps[str(B)] = {"us_per_step": 1e3 * ms, "GB/s": moe_step_bytes(B) / ms / 1e6,
+                                "frac_hbm": moe_step_bytes(B) / ms / 1e6 / hbm_gbs, "tokens_per_s": B / ms * 1e3}
+            del groups, ws5
+        sweep = {"workload": wl.SWEEP["name"] + ", seed %d, %d experts" % (wl.SWEEP["seed"], E5), "weights": n5,
+                 "index_bytes": 3 * n5 // 8,
+                 "encode": {"ms": enc5_ms, "Gweights/s": n5 / enc5_ms / 1e6,
+                            "definition_equivalent_tflops": enc5_tflops,
+                            "definition_equivalent_frac_fma_counted_fp32_peak": enc5_tflops / (2 * fp32_peak_tflops),
+                            "executed_alu_frac": ENC_ALU_OPS_PER_WEIGHT * n5 / enc5_ms / 1e9 / alu_peak_tops},
+                 "gemv_all_experts_one_call": gv_all,
+                 "gemv_decode_steps_8_experts_rotating_32_groups": gv_steps}
+        del T5, S5
+        torch.cuda.empty_cache()
+
     # end to end through the public API with host buffers: every step uploads the layer from pinned host memory
     # and reads its results back (indices, scales, errors, y).  The device inputs and index outputs are double
     # buffered, so step i + 1's upload (its own copy stream) and step i's index read-back (a third stream) overlap
@@ -801,20 +948,27 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": bench_config(args.experts),
-            "roofline": {"bound": "alu", "achieved": enc_tflops, "peak": 2 * fp32_peak_tflops, "unit": "TFLOP/s",
-                         "frac": enc_tflops / (2 * fp32_peak_tflops),
+            "roofline": {"bound": "alu", "achieved": enc_tops, "peak": alu_peak_tops, "unit": "Top/s",
+                         "frac": enc_tops / alu_peak_tops,
                          "traffic": (None if ENCODE_DRAM_BYTES_PER_WEIGHT is None
                                      else ENCODE_DRAM_BYTES_PER_WEIGHT * layer.weights / 3),
                          "kernel": "vq3r_encode (row scale + screened greedy assignment; per launch = one stacked "
-                                   "matrix kind, 3 per step): the definition's %d flops per weight (3 stages x 256 "
-                                   "codewords x 8 dims x 3 / 8) per second; peak = FMA-counted FP32 peak, %d SMs x "
-                                   "128 lanes x 2 x %.0f MHz; traffic = DRAM bytes per launch"
-                                   % (FLOPS_PER_WEIGHT, sms, sm_max_mhz),
-                         "executed": {"bound": "ALU pipe (screening bookkeeping)",
-                                      "alu_ops_per_weight": ENC_ALU_OPS_PER_WEIGHT, "achieved_tops": enc_tops,
-                                      "peak_tops": alu_peak_tops, "frac": enc_tops / alu_peak_tops,
-                                      "peak": "%d SMs x %d ALU lanes x %.0f MHz" % (sms, ALU_LANES_PER_SM,
-                                                                                     sm_max_mhz)}},
+                                   "matrix kind, 3 per step).  achieved = the ALU-pipe operations the screened "
+                                   "encoder executes, %d per weight (3 stages x 256 codewords x %d bookkeeping "
+                                   "operations / 8), per second; peak = %d SMs x %d ALU lanes x %.0f MHz; traffic = "
+                                   "DRAM bytes per launch from the committed ncu capture"
+                                   % (ENC_ALU_OPS_PER_WEIGHT, ALU_OPS_PER_VEC_CODEWORD, sms, ALU_LANES_PER_SM,
+                                      sm_max_mhz),
+                         "definition_equivalent": {
+                             "flops_per_weight": FLOPS_PER_WEIGHT, "achieved_tflops": enc_tflops,
+                             "frac_of_fma_counted_fp32_peak": enc_tflops / (2 * fp32_peak_tflops),
+                             "fma_counted_fp32_peak_tflops": 2 * fp32_peak_tflops,
+                             "frac_of_non_fma_fp32_ceiling": enc_tflops / fp32_peak_tflops,
+                             "non_fma_fp32_ceiling_tflops": fp32_peak_tflops,
+                             "note": "the definition's arithmetic (3 x 256 x 8 x (sub, mul, add) per 8 weights) "
+                                     "credited at the kernel's rate; the kernel reaches the same indices with a "
+                                     "screen and runs the definition's scan only where the screen's margin fails, "
+                                     "so the rate can exceed the non-FMA ceiling of the operations it credits"}},
             "kernels": {
                 "encode": {"ms": enc_ms, "Gweights/s": layer.weights / enc_ms / 1e6, "TFLOP/s": enc_tflops},
                 "pack_tiles": {"ms": pack_ms, "GB/s": 2 * 0.375 * layer.weights / pack_ms / 1e6},
@@ -830,6 +984,8 @@ def main():
                 "train_lloyd": train,
                 "vq4p": vq4p,
                 "outliers": outl,
+                "expert_quality": quality,
+                "sweep_256_experts": sweep,
                 "stream_bandwidth": stream_bw,
                 "hbm_peak_gbs": hbm_gbs, "peak_source": peak_src},
             "e2e": e2e,
