@@ -405,24 +405,33 @@ __device__ __forceinline__ void tcur_next(const GvParams& P, TileCursor& c) {
 }
 
 // Table pipeline of the tiled kernel.  A CTA walks its units table by table
-// (table = group, slab, stage, token).  Table t lives in tab[t & 1]; its
-// inputs (the x slab as stored and the stage's 8 KiB codebook) are brought
-// into xraw[t & 1] / cb[t & 1] by bulk asynchronous copies completing on
-// mbar[t & 1], issued one table ahead, so they never wait behind the index
-// stream.  While the units of table t run, table t + 1 is computed in
-// kBuildChunks pieces, one piece per unit; the switch only finishes what is
-// left.
+// (table = group, slab, stage, token).  Table t lives in table buffer t & 1;
+// its inputs (the x slab as stored and the stage's 8 KiB codebook) are
+// brought into xraw[t & 1] / cb[t & 1] by bulk asynchronous copies
+// completing on mbar[t & 1], issued one table ahead, so they never wait
+// behind the index stream.  At the switch to table t + 1 all warps build it
+// at once (each its share of the codewords, kBuildChunks pieces): spread over
+// the units of table t instead, one piece per unit, the build's dependent
+// chains held every warp back at the same time and cost about three times
+// as much.
 constexpr int kBuildChunks = 8;
 constexpr int kChunkCw = kCodewords / kBuildChunks;  // 32 codewords per piece
 constexpr uint32_t kNoTable = 0xFFFFFFFFu;           // no key has all bits set (group < 32, s < 3)
 
+// Staging area of the tiled kernel's tables (inputs and barriers).
 struct TilesSmem {
-  float tab[2][kTabWords];                       // 2 x 64 KiB
   float cb[2][kCodewords * kDim];                // 2 x 8 KiB
   unsigned char xraw[2][kSlabV * kDim * 4];      // 2 x 2 KiB (f32; 16-bit types use half)
   uint64_t mbar[2];
 };
-constexpr size_t kTilesSmemBytes = sizeof(TilesSmem);
+// The two 64 KiB table buffers start on a 64 KiB boundary of the shared
+// address space, so that a lookup's byte permute (index byte in byte 1, bank
+// offset in byte 0, table number in byte 2) is its full shared address.  The
+// staging area sits below the tables when it fits there, else after them;
+// 64 KiB of slack covers any placement of the dynamic shared memory.
+constexpr size_t kTilesSmemBytes = 0x10000 + 2 * (size_t)kTabBytes;
+// Index blocks prefetched into L2 ahead of the register ring.
+constexpr int kPrefetchUnits = 2;
 
 template <int XDT>
 __host__ __device__ constexpr int x_elt_bytes() {
@@ -529,15 +538,6 @@ __device__ __forceinline__ void build_piece_x(float* tab, const float* cb, const
   }
 }
 
-template <int XDT>
-__device__ __forceinline__ void build_piece(float* tab, const float* cb, const unsigned char* xr, int nv, int c,
-                                            int warp, int lane) {
-  float xa[8], xb[8];
-  staged_x<XDT>(xr, lane, nv, xa);
-  staged_x<XDT>(xr, lane + 32, nv, xb);
-  build_piece_x(tab, cb, xa, xb, c, warp, lane);
-}
-
 // Pieces c0 .. kBuildChunks - 1 of a table, the lane's x values read once.
 template <int XDT>
 __device__ __forceinline__ void build_pieces_from(float* tab, const float* cb, const unsigned char* xr, int nv,
@@ -608,12 +608,13 @@ struct Arrival {
 };
 
 // Arrival of this CTA, by one thread after a __syncthreads that follows the
-// CTA's zeros.  The add is acquire-release: it releases those zeros, and the
-// count it returns is used only later, so the thread does not wait for it.
+// CTA's zeros.  The add is a release (it publishes those zeros; the acquire
+// is the waiter's load), so the thread goes on without waiting for it; the
+// count it returns is used only later.
 __device__ __forceinline__ Arrival barrier_arrive(unsigned long long* hdr) {
   Arrival t;
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(t.start) : "l"(hdr) : "memory");
-  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], 1;" : "=l"(t.seq) : "l"(hdr + 1) : "memory");
+  asm volatile("atom.release.gpu.global.add.u64 %0, [%1], 1;" : "=l"(t.seq) : "l"(hdr + 1) : "memory");
   return t;
 }
 
@@ -645,6 +646,25 @@ __device__ __forceinline__ void barrier_wait(unsigned long long* hdr, Arrival t)
   }
 }
 
+// One table entry at a 32-bit shared address (plus 128 bytes for the second
+// column slot).
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_f32_128(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1+128];" : "=f"(v) : "r"(a));
+  return v;
+}
+
+// Bulk prefetch of one 32 KiB index block into L2 (a hint: it reads, writes
+// nothing, and may be issued before the inputs are final).
+__device__ __forceinline__ void prefetch_block_l2(const void* p) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"((uint32_t)kTileBytes) : "memory");
+}
+
 __device__ __forceinline__ void red_add_f32(float* p, float v) {
   asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
@@ -658,17 +678,23 @@ __device__ __forceinline__ uint32_t unit_table_key(const GvParams& P, int64_t u)
 template <int XDT, int NSLOT>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_constant__ GvParams P) {
   extern __shared__ __align__(128) unsigned char gv_smem[];
-  TilesSmem& S = *reinterpret_cast<TilesSmem*>(gv_smem);
+  const uint32_t sbase = smem_u32(gv_smem);
+  const uint32_t tab_addr = (sbase + 0xFFFFu) & ~0xFFFFu;  // table buffer 0; buffer 1 follows at + 64 KiB
+  const uint32_t pad = tab_addr - sbase;
+  float* const tabp = reinterpret_cast<float*>(gv_smem + pad);
+  TilesSmem& S = *reinterpret_cast<TilesSmem*>(pad >= sizeof(TilesSmem) ? gv_smem : gv_smem + pad + 2 * kTabBytes);
+  const uint32_t tk = tab_addr >> 16;
+  const uint32_t tab_toggle = (tk ^ (tk + 1u)) << 16;  // flips byte 2 between buffers 0 and 1
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, a = lane & 3;
   // PRMT operands: byte 0 = byte offset of the bank of the current column,
-  // byte 2 = table buffer (tab[1] starts 64 KiB after tab[0]); the index
+  // byte 2 = shared address of the current table buffer >> 16; the index
   // byte lands in byte 1, i.e. at j * 256.
   uint32_t lc[8];
 #pragma unroll
   for (int q = 0; q < 8; q++)
-    lc[q] = 4u * (8u * a + (uint32_t)((q & 3) ^ (g & 3)) + 4u * (uint32_t)((q >> 2) ^ (g >> 2)));
+    lc[q] = (tk << 16) | (4u * (8u * a + (uint32_t)((q & 3) ^ (g & 3)) + 4u * (uint32_t)((q >> 2) ^ (g >> 2))));
   uint32_t sel[4];
 #pragma unroll
   for (int q = 0; q < 4; q++) sel[q] = 0x7604u | ((uint32_t)((q ^ g) & 3) << 4);
@@ -756,42 +782,39 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
       skey[i] = kNoTable;
     }
   }
+  // L2 prefetch of the kPrefetchUnits index blocks beyond the ring; one more
+  // is requested per unit after this, so the distance stays the same.
+  TileCursor cpf = ci;
+  int64_t upf = u0 + NSLOT;
+  if (tid == 0) {
+    for (int k = 0; k < kPrefetchUnits && upf < u1; k++, upf++) {
+      prefetch_block_l2(cpf.p);
+      tcur_next(P, cpf);
+    }
+  }
 
   // The first table is built at once, while the first index loads are in flight.
-  build_pieces_from<XDT>(S.tab[0], S.cb[0], S.xraw[0], slab_columns(P, key_cur), 0, warp, lane);
+  build_pieces_from<XDT>(tabp, S.cb[0], S.xraw[0], slab_columns(P, key_cur), 0, warp, lane);
   if (tid == 0) barrier_wait(P.hdr, arrival);  // every y is zeroed before the first add
   __syncthreads();
-  int tno = 0;              // number of the current table within this CTA; it lives in tab[tno & 1]
-  int pieces = 0;           // pieces of table tno + 1 this warp has built
-  bool next_ready = false;  // the inputs of table tno + 1 have landed
-  const unsigned char* tb = reinterpret_cast<const unsigned char*>(S.tab[0]);
-
+  int tno = 0;  // number of the current table within this CTA; it lives in table buffer tno & 1
   for (int64_t u = u0; u < u1; u += NSLOT) {
 #pragma unroll
     for (int i = 0; i < NSLOT; i++) {
       if (u + i < u1) {
-        const int nb = (tno + 1) & 1;
-        const uint32_t nparity = (uint32_t)((tno + 1) >> 1) & 1u;
         if (skey[i] != key_cur) {  // switch to table tno + 1 (= key_next)
-          if (!next_ready) ok = mbar_wait_bounded(&S.mbar[nb], nparity) && ok;
-          build_pieces_from<XDT>(S.tab[nb], S.cb[nb], S.xraw[nb], slab_columns(P, key_next), pieces, warp, lane);
+          const int nb = (tno + 1) & 1;
+          ok = mbar_wait_bounded(&S.mbar[nb], (uint32_t)((tno + 1) >> 1) & 1u) && ok;
+          build_pieces_from<XDT>(tabp + nb * kTabWords, S.cb[nb], S.xraw[nb], slab_columns(P, key_next), 0, warp, lane);
           __syncthreads();  // table complete; every warp is done with table tno - 1's buffers
           tno++;
           key_cur = key_next;
           key_next = key_cur == key_last ? kNoTable : next_table_key(P, key_cur);
-          pieces = 0;
-          next_ready = false;
 #pragma unroll
-          for (int q = 0; q < 8; q++) lc[q] ^= 0x10000u;
+          for (int q = 0; q < 8; q++) lc[q] ^= tab_toggle;
           if (tid == 0 && key_next != kNoTable) {
             fence_proxy_async_smem();  // generic reads of the staging buffer precede the async refill
             stage_table<XDT>(P, key_next, S, (tno + 1) & 1);
-          }
-        } else if (key_next != kNoTable && pieces < kBuildChunks) {
-          if (!next_ready) next_ready = __all_sync(0xFFFFFFFFu, mbar_test_wait(&S.mbar[nb], nparity));
-          if (next_ready) {
-            build_piece<XDT>(S.tab[nb], S.cb[nb], S.xraw[nb], slab_columns(P, key_next), pieces, warp, lane);
-            pieces++;
           }
         }
         float* const q = sq[i];
@@ -803,14 +826,22 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
 #pragma unroll
         for (int t = 0; t < 4; t++) {
           const uint32_t w[4] = {r[i][t].x, r[i][t].y, r[i][t].z, r[i][t].w};
-          float sum = 0.0f;
+          float2 s2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-          for (int m = 0; m < 16; m++) {
-            const uint32_t off = __byte_perm(w[m >> 2], lc[(m & 3) | ((m >> 3) << 2)], sel[m & 3]);
-            sum += *reinterpret_cast<const float*>(tb + off + ((m >> 2) & 1) * 128);
+          for (int m = 0; m < 16; m += 2) {
+            const uint32_t o0 = __byte_perm(w[m >> 2], lc[(m & 3) | ((m >> 3) << 2)], sel[m & 3]);
+            const uint32_t o1 = __byte_perm(w[(m + 1) >> 2], lc[((m + 1) & 3) | (((m + 1) >> 3) << 2)], sel[(m + 1) & 3]);
+            const float t0 = ((m >> 2) & 1) ? lds_f32_128(o0) : lds_f32(o0);
+            const float t1 = (((m + 1) >> 2) & 1) ? lds_f32_128(o1) : lds_f32(o1);
+            s2 = __fadd2_rn(s2, make_float2(t0, t1));
           }
-          acc[t] = sum;
+          acc[t] = s2.x + s2.y;
           if (refill) r[i][t] = ldg_stream16(pn + t * 8 * kSlabV, pol);
+        }
+        if (tid == 0 && upf < u1) {  // keep kPrefetchUnits blocks prefetched beyond the ring
+          prefetch_block_l2(cpf.p);
+          tcur_next(P, cpf);
+          upf++;
         }
         if (refill) {
           sq[i] = ci.q;

@@ -209,7 +209,7 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
 // largest range cost; for a given budget, ranges are filled greedily table by
 // table.  Writes P.cta_begin[0..n] and P.n_split = n (ranges past the last
 // unit are empty).
-constexpr int64_t kTableCost = 4;  // a table build, and the stall at a switch, cost about four units
+constexpr int64_t kTableCost = 2;  // a table build at a switch, and its stall, cost about two units
 
 int64_t split_ranges(const GvParams& P, int64_t budget, int n, int64_t* begin) {
   int used = 0;
