@@ -107,10 +107,12 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
  *   vq3r_decode.  Summation order is the library's own: results agree with
  *   an exact (binary64) product to about 1e-4 relative to rms(y), not bit
  *   for bit.  TILES calls below 8 tokens (and all TILES calls with F32 or
- *   F16 x) add each partial sum into y with an atomic add, in the order the
- *   GPU schedules them, so two identical calls may differ in the last bits
- *   of y; PLANES calls and TILES calls of 8 or more bf16 tokens give the
- *   same bits every time.
+ *   F16 x), and TILES calls of 17 or more bf16 tokens whose matrices share
+ *   one codebooks pointer (the tensor-memory kernel, which splits the
+ *   columns of a row block between warp groups), add partial sums into y
+ *   with atomic adds, in the order the GPU schedules them, so two identical
+ *   calls may differ in the last bits of y; PLANES calls and the other TILES
+ *   calls of 8 or more bf16 tokens give the same bits every time.
  *
  * One descriptor per matrix; matrices may differ in shape, codebooks and x.
  * Matrices that share (codebooks, x, cols) share the x-projected tables the
@@ -125,9 +127,12 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
  * Fill a workspace with zeros once before its first call (e.g.
  * cudaMemsetAsync after allocating it); nothing needs clearing between
  * calls, replays of a captured CUDA graph included.  The TILES kernel runs
- * one CTA per SM and needs all of them resident together: if another
- * workload holds SMs for more than about a second, the call finishes with
- * vq3r_device_error() = 2 and y undefined.
+ * one CTA per SM and needs all of them resident together.  The library
+ * checks once per device that one CTA fits on an SM (else VQ3R_ERR_CUDA,
+ * vq3r_last_cuda_error() = cudaErrorCooperativeLaunchTooLarge); it does not
+ * launch cooperatively (that measured about 4 us slower per call), so if
+ * another workload holds SMs for more than about a second, the call
+ * finishes with vq3r_device_error() = 2 and y undefined.
  *   mats      HOST array of n_mats descriptors (copied before return)
  *   B         tokens, 1..32
  *   x_dtype   dtype of every x, {F32, BF16, F16}
@@ -221,7 +226,8 @@ vq3r_status vq3r_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const ui
  *     B = 1 as one call.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before capturing a stream into a graph.
+ *     before capturing a stream into a graph.  If that lookup fails the call
+ *     returns VQ3R_ERR_CUDA and the next call looks it up again.
  *   - All calls share the one array: calls that overlap on the GPU (different
  *     streams, or different host threads on the same device) race and must be
  *     serialised by the caller.  The array is zeroed when the library is

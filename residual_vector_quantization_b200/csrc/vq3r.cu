@@ -9,6 +9,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_mma.cuh"
+#include "gemv_tc.cuh"
 #include "train.cuh"
 #include "outliers.cuh"
 #include "vq3r_common.cuh"
@@ -44,6 +45,11 @@ constexpr int kMaxDevices = 64;
 std::mutex g_dev_mu;
 std::atomic<bool> g_dev_ready[kMaxDevices];  // set once a setup has succeeded; a failed one is retried
 int g_dev_sms[kMaxDevices];
+// The tiled GEMV waits on a grid barrier, so every one of its CTAs (at most
+// one per SM) must be resident at once: a CTA must fit on an SM next to
+// nothing else.  Checked once per device with the occupancy calculator.
+bool g_dev_tiles_fit[kMaxDevices];
+bool g_dev_tc_fit[kMaxDevices];  // the same for the tensor-core GEMV (one persistent CTA per SM, grid barrier)
 
 cudaError_t device_setup(int* sms) {
   int dev = 0;
@@ -91,11 +97,28 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_mma_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, gm);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTgSmemBytes);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTgSmemBytes);
     const int go = (int)outlier_select_smem(kOutMaxCols);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
     if (r != cudaSuccess) return r;
+    int fit = 1;
+    for (int k = 0; k < 3 && r == cudaSuccess; k++) {
+      int n = 0;
+      r = k == 0 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tiles_kernel<VQ3R_F32, kTileSlots>, kGvThreads, gt)
+        : k == 1 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tiles_kernel<VQ3R_BF16, kTileSlots>, kGvThreads, gt)
+                 : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tiles_kernel<VQ3R_F16, kTileSlots>, kGvThreads, gt);
+      if (n < 1) fit = 0;
+    }
+    if (r != cudaSuccess) return r;
+    g_dev_tiles_fit[dev] = fit != 0;
+    int ntc1 = 0, ntc2 = 0;
+    r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ntc1, gemv_tc_kernel<1>, kTgThreads, kTgSmemBytes);
+    if (r == cudaSuccess) r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ntc2, gemv_tc_kernel<2>, kTgThreads, kTgSmemBytes);
+    if (r != cudaSuccess) return r;
+    g_dev_tc_fit[dev] = ntc1 >= 1 && ntc2 >= 1;
   }
   g_dev_ready[dev].store(true, std::memory_order_release);
   *sms = g_dev_sms[dev];
@@ -476,8 +499,35 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   cfg.stream = s;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
+  bool one_codebook = true;
+  for (int g = 1; g < P.n_groups; g++) one_codebook = one_codebook && P.g[g].codebooks == P.g[0].codebooks;
+  if (P.layout == VQ3R_LAYOUT_TILES && x_dtype == VQ3R_BF16 && B >= kTgMinB && one_codebook) {
+    // Several tokens: rebuild the weights into tensor memory and contract on
+    // the tcgen05 tensor cores.  The work is the sequence of K-steps (128-row
+    // tile, 16 columns) of all matrices, split evenly over four warp-groups
+    // per SM; like the lookup-table kernel it zeroes y behind a grid barrier,
+    // so one CTA must fit per SM.
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (!g_dev_tc_fit[dev]) return cuda_fail(cudaErrorCooperativeLaunchTooLarge);
+    int64_t ksteps = 0;
+    for (int i = 0; i < P.n_mats; i++)
+      ksteps += (P.m[i].rows + kTgRows - 1) / kTgRows * ((P.g[P.m[i].group].cols / kDim + 1) / 2);
+    plan.P.total_units = ksteps;
+    cfg.gridDim = dim3((unsigned)sms);
+    cfg.blockDim = dim3(kTgThreads);
+    cfg.dynamicSmemBytes = kTgSmemBytes;
+    e = B <= 16 ? cudaLaunchKernelEx(&cfg, gemv_tc_kernel<1>, plan.P) : cudaLaunchKernelEx(&cfg, gemv_tc_kernel<2>, plan.P);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return check_launch();
+  }
   if (P.layout == VQ3R_LAYOUT_TILES && x_dtype == VQ3R_BF16 && B >= kMmaMinB) {
-    // Several tokens: rebuild the weights and contract on the tensor cores.
+    // 8..16 tokens (or matrices with different codebooks): rebuild the weights
+    // in registers and contract with mma.sync; each CTA owns 256 rows of one
+    // matrix and loads its codebooks.  Measured on the 8-expert decode step:
+    // 213 us at B = 8 against 228 us for the tensor-memory kernel, which wins
+    // from 17 tokens (237 against 279 us at B = 32).
     // One CTA per 128 rows of a matrix; blk_begin numbers those blocks.
     int64_t blocks = 0;
     for (int i = 0; i < P.n_mats; i++) {
@@ -498,6 +548,14 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
     return check_launch();
   }
   if (P.layout == VQ3R_LAYOUT_TILES) {  // one CTA per SM
+    // The kernel's grid barrier needs all CTAs resident at once; the cooperative
+    // launch attribute would guarantee it but measured 3.8 us slower per call
+    // (it gives up most of the programmatic-launch overlap), so the grid is
+    // sized to one CTA per SM and the fit of one CTA per SM is checked instead.
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (!g_dev_tiles_fit[dev]) return cuda_fail(cudaErrorCooperativeLaunchTooLarge);
     const int grid = (int)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms);
     balance_split(plan.P, grid);
     cfg.gridDim = dim3((unsigned)grid);

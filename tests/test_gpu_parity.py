@@ -309,6 +309,44 @@ def test_grouped_gemv_many_tokens(B):
         assert gemv_rel_err(y, ref) <= GEMV_TOL
 
 
+@pytest.mark.parametrize("B", [17, 24, 32])
+def test_grouped_gemv_tensor_memory_kernel(B):
+    """17..32 tokens, bf16 x, tiled layout and one codebook set for the whole call run on the tcgen05 kernel
+    (weights rebuilt in bf16 hi + lo into tensor memory): ragged rows (not multiples of 128), columns that end
+    in the middle of a 16-column step (cols % 16 == 8), partial last slabs, a matrix of one step, mixed x
+    groups, and the K-step split across warp-groups that cuts tiles in the middle."""
+    rng = np.random.default_rng(90 + B)
+    cb = random_codebooks(401)
+    specs = [(300, 1032, 0), (129, 1032, 0), (64, 200, 1), (513, 2048, 2), (33, 1032, 0), (7, 8, 3), (2048, 7168, 4)]
+    xs = {}
+    mats, refs = [], []
+    for rows, cols, xk in specs:
+        if (xk, cols) not in xs:
+            xs[(xk, cols)] = f32_to_bf16_bits(rng.standard_normal((B, cols)).astype(np.float32))
+        x = xs[(xk, cols)]
+        W = f32_to_bf16_bits((rng.standard_normal((rows, cols)) * np.exp(rng.standard_normal((rows, 1)))).astype(np.float32))
+        W_t, idx_t, sc_t, cb_t, idx_o, sc_o = check_encode_decode(W, "bf16", cb)
+        y_t = torch.full((B, rows), float("nan"), dtype=torch.float32, device=DEV)
+        mats.append(dict(idx=idx_t, scales=sc_t, codebooks=cb_t, x=None, y=y_t, key=(xk, cols)))
+        refs.append(oracle.gemv(oracle.decode(idx_o, sc_o, cb), x, "bf16"))
+    xdev = {k: to_dev(v, "bf16") for k, v in xs.items()}
+    cb_t = mats[0]["codebooks"]
+    for m in mats:
+        m["x"] = xdev[m.pop("key")]
+        m["codebooks"] = cb_t  # one codebook tensor for the whole call
+    ws = torch.zeros(4096, dtype=torch.uint8, device=DEV)
+    tiled = as_layout(mats, "tiles")
+    for _ in range(2):  # twice: the second call reuses the workspace's grid-barrier counts
+        for m in mats:
+            m["y"].fill_(float("nan"))
+        vq.vq3r_gemv(tiled, B, workspace=ws)
+        for m, ref in zip(mats, refs):
+            y = m["y"].cpu().numpy()
+            assert np.isfinite(y).all()  # every output written
+            assert gemv_rel_err(y, ref) <= GEMV_TOL
+    assert vq.vq3r_device_error() == 0
+
+
 @pytest.mark.parametrize("B", [1, 3])
 def test_gemv_cuda_graph_replays(B):
     """A tiled GEMV captured once in a CUDA graph and replayed with new inputs: every replay repeats the
