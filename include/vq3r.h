@@ -106,13 +106,13 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
  *   y[b][i] = sum_c w_hat[i][c] * x[b][c], fp32 accumulation, w_hat as in
  *   vq3r_decode.  Summation order is the library's own: results agree with
  *   an exact (binary64) product to about 1e-4 relative to rms(y), not bit
- *   for bit.  TILES calls below 8 tokens (and all TILES calls with F32 or
+ *   for bit.  TILES calls below 11 tokens (and all TILES calls with F32 or
  *   F16 x), and TILES calls of 17 or more bf16 tokens whose matrices share
  *   one codebooks pointer (the tensor-memory kernel, which splits the
  *   columns of a row block between warp groups), add partial sums into y
  *   with atomic adds, in the order the GPU schedules them, so two identical
  *   calls may differ in the last bits of y; PLANES calls and the other TILES
- *   calls of 8 or more bf16 tokens give the same bits every time.
+ *   calls of 11 or more bf16 tokens give the same bits every time.
  *
  * One descriptor per matrix; matrices may differ in shape, codebooks and x.
  * Matrices that share (codebooks, x, cols) share the x-projected tables the

@@ -103,6 +103,8 @@ struct GvParams {
   uint32_t cta_key0[kMaxSplit], cta_key_last[kMaxSplit];
   int32_t cta_m0[kMaxSplit], cta_tile0[kMaxSplit];
   int32_t n_mats, n_groups, B, vec8;  // vec8: rows and planes 8-byte aligned (64-bit index loads)
+  int32_t nb;            // table tokens: B, or ceil(B / 2) when the tiled kernel looks up two tokens per table pair
+  int32_t tokm;          // tokens per table token (1 or 2): table token b covers tokens tokm * b ..
   int64_t total_units;
   int32_t tile_rows;     // rows per work unit: kGvTileRows (planes) or kTileRows (tiles)
   int32_t layout;        // VQ3R_LAYOUT_PLANES or VQ3R_LAYOUT_TILES
@@ -135,9 +137,9 @@ __host__ __device__ __forceinline__ GvCursor unit_cursor(const GvParams& P, int6
   c.g = g;
   const int tab = (int)(lu / G.tiles);
   const int t = (int)(lu - (int64_t)tab * G.tiles);
-  c.b = tab % P.B;
-  c.s = (tab / P.B) % kStages;
-  c.slab = tab / (P.B * kStages);
+  c.b = tab % P.nb;
+  c.s = (tab / P.nb) % kStages;
+  c.slab = tab / (P.nb * kStages);
   int m = G.mat_begin;
   while (m + 1 < G.mat_end && P.m[m + 1].tile_prefix <= t) m++;
   c.m = m;
@@ -150,7 +152,7 @@ __device__ __forceinline__ void unit_advance(const GvParams& P, GvCursor& c) {
   c.tile = 0;
   if (++c.m < P.g[c.g].mat_end) return;
   c.m = P.g[c.g].mat_begin;
-  if (++c.b < P.B) return;
+  if (++c.b < P.nb) return;
   c.b = 0;
   if (++c.s < kStages) return;
   c.s = 0;
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_lut_kernel(const __grid_co
   const unsigned char* tb = reinterpret_cast<const unsigned char*>(tab);
   auto step = [&](int64_t u, GvCursor& c, uint32_t (&wa)[2][4]) {
     const GvGroup& G = P.g[c.g];
-    const int tab_id = (c.slab * kStages + c.s) * P.B + c.b;
+    const int tab_id = (c.slab * kStages + c.s) * P.nb + c.b;
     if (c.g != loaded_g || tab_id != loaded_tab) {
       build_table<XDT>(G, c, tab, xs, cbs, tid);
       loaded_g = c.g;
@@ -345,9 +347,10 @@ __host__ __device__ __forceinline__ uint32_t table_key(int g, int slab, int s, i
 // coordinates needed for the carry to the next matrix or table.
 struct TileCursor {
   const uint8_t* p;
-  float* q;             // y of the unit's token, at the tile's first row
+  float* q;             // y of the unit's (first) token, at the tile's first row
   const uint16_t* sc;   // scales, at the tile's first row
   int32_t rows_left;
+  int32_t mrows;        // rows of the matrix: y's stride from one token to the next
   uint32_t tkey;
   int32_t m, tile, ntiles;
 };
@@ -359,9 +362,10 @@ __device__ __forceinline__ void tcur_fill(const GvParams& P, TileCursor& c) {
   const int64_t n_slabs = P.g[g].n_slabs;
   c.ntiles = M.n_tiles;
   c.p = M.idx + ((int64_t)s * n_slabs + slab) * M.plane_stride + (int64_t)c.tile * kTileBytes;
-  c.q = M.y + (int64_t)b * M.rows + (int64_t)c.tile * kTileRows;
+  c.q = M.y + (int64_t)b * P.tokm * M.rows + (int64_t)c.tile * kTileRows;
   c.sc = M.scales + (int64_t)c.tile * kTileRows;
   c.rows_left = (int32_t)(M.rows - (int64_t)c.tile * kTileRows);
+  c.mrows = (int32_t)M.rows;
 }
 
 __device__ __forceinline__ TileCursor tcur_at(const GvParams& P, int64_t u) {
@@ -388,7 +392,7 @@ __device__ __forceinline__ void tcur_next(const GvParams& P, TileCursor& c) {
   int g = (int)(c.tkey >> 27);
   if (++c.m >= P.g[g].mat_end) {
     int slab = (int)(c.tkey & 0xFFFFFu), s = (int)((c.tkey >> 20) & 3u), b = (int)((c.tkey >> 22) & 31u);
-    if (++b >= P.B) {
+    if (++b >= P.nb) {
       b = 0;
       if (++s >= kStages) {
         s = 0;
@@ -421,7 +425,7 @@ constexpr uint32_t kNoTable = 0xFFFFFFFFu;           // no key has all bits set 
 // Staging area of the tiled kernel's tables (inputs and barriers).
 struct TilesSmem {
   float cb[2][kCodewords * kDim];                // 2 x 8 KiB
-  unsigned char xraw[2][kSlabV * kDim * 4];      // 2 x 2 KiB (f32; 16-bit types use half)
+  unsigned char xraw[2][2][kSlabV * kDim * 4];   // [buffer][token of the pair] 2 KiB each (f32; 16-bit types use half)
   uint64_t mbar[2];
 };
 // The two 64 KiB table buffers start on a 64 KiB boundary of the shared
@@ -440,7 +444,7 @@ __host__ __device__ constexpr int x_elt_bytes() {
 
 __device__ __forceinline__ uint32_t next_table_key(const GvParams& P, uint32_t k) {
   int slab = (int)(k & 0xFFFFFu), s = (int)((k >> 20) & 3u), b = (int)((k >> 22) & 31u), g = (int)(k >> 27);
-  if (++b < P.B) return table_key(g, slab, s, b);
+  if (++b < P.nb) return table_key(g, slab, s, b);
   b = 0;
   if (++s < kStages) return table_key(g, slab, s, b);
   s = 0;
@@ -461,6 +465,7 @@ __device__ __forceinline__ int slab_columns(const GvParams& P, uint32_t k) {
 // griddep_wait.
 struct TableSrc {
   const unsigned char* x;
+  const unsigned char* x2;  // the pair's second token (two-token tables), else null
   const float* cb;
   uint32_t xbytes;
 };
@@ -469,17 +474,22 @@ template <int XDT>
 __device__ __forceinline__ TableSrc table_src(const GvParams& P, uint32_t k) {
   const GvGroup& G = P.g[k >> 27];
   const int slab = (int)(k & 0xFFFFFu), s = (int)((k >> 20) & 3u), b = (int)((k >> 22) & 31u);
+  const int tok = b * P.tokm;
   TableSrc t;
   t.xbytes = (uint32_t)(slab_columns(P, k) * kDim * x_elt_bytes<XDT>());
-  t.x = static_cast<const unsigned char*>(G.x) + ((int64_t)b * G.cols + (int64_t)slab * kSlabV * kDim) * x_elt_bytes<XDT>();
+  const unsigned char* xs = static_cast<const unsigned char*>(G.x) + (int64_t)slab * kSlabV * kDim * x_elt_bytes<XDT>();
+  t.x = xs + (int64_t)tok * G.cols * x_elt_bytes<XDT>();
+  // an odd token count leaves the last pair with one token: its second table repeats the first (never added)
+  t.x2 = P.tokm == 2 ? xs + (int64_t)(tok + 1 < P.B ? tok + 1 : tok) * G.cols * x_elt_bytes<XDT>() : nullptr;
   t.cb = G.codebooks + (size_t)s * kCodewords * kDim;
   return t;
 }
 
-// Bulk copies of a table's inputs into xraw[i] / cb[i], completing on mbar[i].
+// Bulk copies of a table's inputs into xraw[i][..] / cb[i], completing on mbar[i].
 __device__ __forceinline__ void stage_src(const TableSrc& t, TilesSmem& S, int i) {
-  mbar_arrive_expect_tx(&S.mbar[i], t.xbytes + (uint32_t)(kCodewords * kDim * 4));
-  bulk_copy_g2s(S.xraw[i], t.x, t.xbytes, &S.mbar[i]);
+  mbar_arrive_expect_tx(&S.mbar[i], t.xbytes * (t.x2 ? 2u : 1u) + (uint32_t)(kCodewords * kDim * 4));
+  bulk_copy_g2s(S.xraw[i][0], t.x, t.xbytes, &S.mbar[i]);
+  if (t.x2) bulk_copy_g2s(S.xraw[i][1], t.x2, t.xbytes, &S.mbar[i]);
   bulk_copy_g2s(S.cb[i], t.cb, kCodewords * kDim * 4, &S.mbar[i]);
 }
 
@@ -658,6 +668,17 @@ __device__ __forceinline__ float lds_f32_128(uint32_t a) {
   asm volatile("ld.shared.f32 %0, [%1+128];" : "=f"(v) : "r"(a));
   return v;
 }
+// The same entries of table buffer 1 (64 KiB further): the pair's second token.
+__device__ __forceinline__ float lds_f32_t1(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1+65536];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_f32_t1_128(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1+65664];" : "=f"(v) : "r"(a));
+  return v;
+}
 
 // Bulk prefetch of one 32 KiB index block into L2 (a hint: it reads, writes
 // nothing, and may be issued before the inputs are final).
@@ -675,7 +696,26 @@ __device__ __forceinline__ uint32_t unit_table_key(const GvParams& P, int64_t u)
   return table_key(c.g, c.slab, c.s, c.b);
 }
 
-template <int XDT, int NSLOT>
+// A warp's exchange: four lanes (a = 0..3) hold partial sums of rows t = 0..3
+// over their column quarters; two exchange steps leave lane a with the full
+// sum of row t = a.
+__device__ __forceinline__ float rows_exchange(const float (&acc)[4], bool hi2, bool hi1) {
+  float k0 = hi2 ? acc[2] : acc[0], k1 = hi2 ? acc[3] : acc[1];
+  const float s0 = hi2 ? acc[0] : acc[2], s1 = hi2 ? acc[1] : acc[3];
+  k0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 2);
+  k1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
+  float kk = hi1 ? k1 : k0;
+  kk += __shfl_xor_sync(0xFFFFFFFFu, hi1 ? k0 : k1, 1);
+  return kk;
+}
+
+// TOKS = 1: table buffers t & 1 double-buffer the tables of consecutive
+// (slab, stage, token) keys.  TOKS = 2 (2..16 tokens): a key is (slab, stage,
+// token pair); buffer 0 holds the pair's first token's table and buffer 1 the
+// second's, so every index byte is looked up for both tokens at the same
+// offset (+ 64 KiB) and the index stream is read once per pair instead of
+// once per token.
+template <int XDT, int NSLOT, int TOKS>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_constant__ GvParams P) {
   extern __shared__ __align__(128) unsigned char gv_smem[];
   const uint32_t sbase = smem_u32(gv_smem);
@@ -765,6 +805,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   uint32_t ssc[NSLOT];  // binary16 bits of the lane's row scale, converted when the unit's sum is added
   int32_t srows[NSLOT];
   uint32_t skey[NSLOT];
+  int32_t smr[NSLOT];  // the unit's matrix rows (y's stride between the pair's tokens)
 #pragma unroll
   for (int i = 0; i < NSLOT; i++) {
     if (u0 + i < u1) {
@@ -774,12 +815,14 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
       ssc[i] = out_row < ci.rows_left ? (uint32_t)__ldg(ci.sc + out_row) : 0u;
       srows[i] = ci.rows_left;
       skey[i] = ci.tkey;
+      smr[i] = ci.mrows;
       tcur_next(P, ci);
     } else {
       sq[i] = nullptr;
       ssc[i] = 0u;
       srows[i] = 0;
       skey[i] = kNoTable;
+      smr[i] = 0;
     }
   }
   // L2 prefetch of the kPrefetchUnits index blocks beyond the ring; one more
@@ -794,7 +837,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   }
 
   // The first table is built at once, while the first index loads are in flight.
-  build_pieces_from<XDT>(tabp, S.cb[0], S.xraw[0], slab_columns(P, key_cur), 0, warp, lane);
+  build_pieces_from<XDT>(tabp, S.cb[0], S.xraw[0][0], slab_columns(P, key_cur), 0, warp, lane);
+  if constexpr (TOKS == 2) build_pieces_from<XDT>(tabp + kTabWords, S.cb[0], S.xraw[0][1], slab_columns(P, key_cur), 0, warp, lane);
   if (tid == 0) barrier_wait(P.hdr, arrival);  // every y is zeroed before the first add
   __syncthreads();
   int tno = 0;  // number of the current table within this CTA; it lives in table buffer tno & 1
@@ -805,13 +849,22 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
         if (skey[i] != key_cur) {  // switch to table tno + 1 (= key_next)
           const int nb = (tno + 1) & 1;
           ok = mbar_wait_bounded(&S.mbar[nb], (uint32_t)((tno + 1) >> 1) & 1u) && ok;
-          build_pieces_from<XDT>(tabp + nb * kTabWords, S.cb[nb], S.xraw[nb], slab_columns(P, key_next), 0, warp, lane);
+          if constexpr (TOKS == 1) {
+            build_pieces_from<XDT>(tabp + nb * kTabWords, S.cb[nb], S.xraw[nb][0], slab_columns(P, key_next), 0, warp,
+                                   lane);
+          } else {
+            __syncthreads();  // every warp is done with both buffers (the pair's tables of key_cur)
+            build_pieces_from<XDT>(tabp, S.cb[nb], S.xraw[nb][0], slab_columns(P, key_next), 0, warp, lane);
+            build_pieces_from<XDT>(tabp + kTabWords, S.cb[nb], S.xraw[nb][1], slab_columns(P, key_next), 0, warp, lane);
+          }
           __syncthreads();  // table complete; every warp is done with table tno - 1's buffers
           tno++;
           key_cur = key_next;
           key_next = key_cur == key_last ? kNoTable : next_table_key(P, key_cur);
+          if constexpr (TOKS == 1) {
 #pragma unroll
-          for (int q = 0; q < 8; q++) lc[q] ^= tab_toggle;
+            for (int q = 0; q < 8; q++) lc[q] ^= tab_toggle;
+          }
           if (tid == 0 && key_next != kNoTable) {
             fence_proxy_async_smem();  // generic reads of the staging buffer precede the async refill
             stage_table<XDT>(P, key_next, S, (tno + 1) & 1);
@@ -822,20 +875,34 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
         const int32_t rows_valid = srows[i];
         const bool refill = u + i + NSLOT < u1;
         const uint8_t* const pn = ci.p + lane_off;
-        float acc[4];
+        const int32_t mrows = smr[i];
+        const uint32_t ukey = skey[i];
+        float acc[4], acc2[4];
 #pragma unroll
         for (int t = 0; t < 4; t++) {
           const uint32_t w[4] = {r[i][t].x, r[i][t].y, r[i][t].z, r[i][t].w};
           float2 s2 = make_float2(0.0f, 0.0f);
+          if constexpr (TOKS == 1) {
 #pragma unroll
-          for (int m = 0; m < 16; m += 2) {
-            const uint32_t o0 = __byte_perm(w[m >> 2], lc[(m & 3) | ((m >> 3) << 2)], sel[m & 3]);
-            const uint32_t o1 = __byte_perm(w[(m + 1) >> 2], lc[((m + 1) & 3) | (((m + 1) >> 3) << 2)], sel[(m + 1) & 3]);
-            const float t0 = ((m >> 2) & 1) ? lds_f32_128(o0) : lds_f32(o0);
-            const float t1 = (((m + 1) >> 2) & 1) ? lds_f32_128(o1) : lds_f32(o1);
-            s2 = __fadd2_rn(s2, make_float2(t0, t1));
+            for (int m = 0; m < 16; m += 2) {
+              const uint32_t o0 = __byte_perm(w[m >> 2], lc[(m & 3) | ((m >> 3) << 2)], sel[m & 3]);
+              const uint32_t o1 = __byte_perm(w[(m + 1) >> 2], lc[((m + 1) & 3) | (((m + 1) >> 3) << 2)], sel[(m + 1) & 3]);
+              const float t0 = ((m >> 2) & 1) ? lds_f32_128(o0) : lds_f32(o0);
+              const float t1 = (((m + 1) >> 2) & 1) ? lds_f32_128(o1) : lds_f32(o1);
+              s2 = __fadd2_rn(s2, make_float2(t0, t1));
+            }
+            acc[t] = s2.x + s2.y;
+          } else {  // (first token, second token) of the pair, summed in pairs
+#pragma unroll
+            for (int m = 0; m < 16; m++) {
+              const uint32_t o = __byte_perm(w[m >> 2], lc[(m & 3) | ((m >> 3) << 2)], sel[m & 3]);
+              const float t0 = ((m >> 2) & 1) ? lds_f32_128(o) : lds_f32(o);
+              const float t1 = ((m >> 2) & 1) ? lds_f32_t1_128(o) : lds_f32_t1(o);
+              s2 = __fadd2_rn(s2, make_float2(t0, t1));
+            }
+            acc[t] = s2.x;
+            acc2[t] = s2.y;
           }
-          acc[t] = s2.x + s2.y;
           if (refill) r[i][t] = ldg_stream16(pn + t * 8 * kSlabV, pol);
         }
         if (tid == 0 && upf < u1) {  // keep kPrefetchUnits blocks prefetched beyond the ring
@@ -848,18 +915,17 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
           ssc[i] = out_row < ci.rows_left ? (uint32_t)__ldg(ci.sc + out_row) : 0u;
           srows[i] = ci.rows_left;
           skey[i] = ci.tkey;
+          smr[i] = ci.mrows;
           tcur_next(P, ci);
         }
-        // Four lanes (a = 0..3) hold partial sums of rows t = 0..3 over
-        // their column quarters; two exchange steps leave lane a with the
-        // full sum of row t = a.
-        float k0 = hi2 ? acc[2] : acc[0], k1 = hi2 ? acc[3] : acc[1];
-        const float s0 = hi2 ? acc[0] : acc[2], s1 = hi2 ? acc[1] : acc[3];
-        k0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 2);
-        k1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
-        float kk = hi1 ? k1 : k0;
-        kk += __shfl_xor_sync(0xFFFFFFFFu, hi1 ? k0 : k1, 1);
-        if (out_row < rows_valid) red_add_f32(q + out_row, f16_bits_to_f32((uint16_t)scale_bits) * kk);
+        const float sc = f16_bits_to_f32((uint16_t)scale_bits);
+        const float kk = rows_exchange(acc, hi2, hi1);
+        if (out_row < rows_valid) red_add_f32(q + out_row, sc * kk);
+        if constexpr (TOKS == 2) {
+          const float kk2 = rows_exchange(acc2, hi2, hi1);
+          const int tok2 = 2 * (int)((ukey >> 22) & 31u) + 1;  // the pair's second token
+          if (out_row < rows_valid && tok2 < P.B) red_add_f32(q + mrows + out_row, sc * kk2);
+        }
       }
     }
   }

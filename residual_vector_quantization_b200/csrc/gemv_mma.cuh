@@ -40,7 +40,7 @@ constexpr int kMmaRows = kMmaWarps * 16;            // rows per CTA
 constexpr int kMmaMaxTok = VQ3R_GEMV_MAX_B;         // 32 tokens = 4 n-tiles
 constexpr int kXCols = kSlabV * kDim;               // 512 columns of x per slab
 constexpr int kXStride = kXCols + 8;                // bf16 per token row in shared memory (padding: no bank conflicts)
-constexpr int kMmaMinB = 8;                         // smallest batch routed to this kernel
+constexpr int kMmaMinB = 11;                        // smallest bf16 batch routed to the tensor cores (below: two-token tables)
 
 // Codebooks: each codeword stored four times side by side in a 128-byte row,
 // cb[s][j][r][k] = C_s[j][k].  Row group g reads copy g mod 4, so the 16 lanes

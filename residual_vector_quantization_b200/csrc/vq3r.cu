@@ -75,9 +75,12 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F32, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_BF16, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16, kTileSlots>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
     const int gm = (int)kMmaSmemBytes;
     const int gc = (int)(kCbrFloats * sizeof(float));
     if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_bulk_kernel<VQ3R_F32, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_bulk_smem<FMT_VQ3R>());
@@ -105,11 +108,16 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
     if (r != cudaSuccess) return r;
     int fit = 1;
-    for (int k = 0; k < 3 && r == cudaSuccess; k++) {
+    const void* tiles_kernels[6] = {
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 1>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 1>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 1>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 2>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 2>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 2>)};
+    for (int k = 0; k < 6 && r == cudaSuccess; k++) {
       int n = 0;
-      r = k == 0 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tiles_kernel<VQ3R_F32, kTileSlots>, kGvThreads, gt)
-        : k == 1 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tiles_kernel<VQ3R_BF16, kTileSlots>, kGvThreads, gt)
-                 : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tiles_kernel<VQ3R_F16, kTileSlots>, kGvThreads, gt);
+      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, tiles_kernels[k], kGvThreads, gt);
       if (n < 1) fit = 0;
     }
     if (r != cudaSuccess) return r;
@@ -141,10 +149,13 @@ struct GemvPlan {
 // Groups matrices sharing (codebooks, x, cols), lays out the workspace and
 // numbers the work units.  Matrices are stored grouped (each group's
 // matrices contiguous in P.m); empty matrices are dropped.
-vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_base, GemvPlan* plan) {
+// tokm: tokens per table token (2 for the tiled kernel's two-token tables, else 1).
+vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, int tokm, char* ws_base, GemvPlan* plan) {
   GvParams& P = plan->P;
   memset(&P, 0, sizeof(P));
   P.B = B;
+  P.tokm = tokm;
+  P.nb = (B + tokm - 1) / tokm;
   P.vec8 = 1;
   P.layout = mats[0].layout;
   if (P.layout != VQ3R_LAYOUT_PLANES && P.layout != VQ3R_LAYOUT_TILES) return VQ3R_ERR_SHAPE;
@@ -212,7 +223,7 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, char* ws_ba
   for (int g = 0; g < n_groups; g++) {
     GvGroup& G = P.g[g];
     G.unit_begin = units;
-    units += (int64_t)G.n_slabs * kStages * B * G.tiles;
+    units += (int64_t)G.n_slabs * kStages * P.nb * G.tiles;
   }
   // Partial sums of the planes kernel: one float per (token, stage, slab,
   // row).  The tiled kernels add into y directly and need only the header.
@@ -239,7 +250,7 @@ int64_t split_ranges(const GvParams& P, int64_t budget, int n, int64_t* begin) {
   int64_t unit = 0, cost = budget;  // cost of the open range; budget forces a new range first
   for (int g = 0; g < P.n_groups; g++) {
     const GvGroup& G = P.g[g];
-    const int64_t n_tables = (int64_t)G.n_slabs * kStages * P.B;
+    const int64_t n_tables = (int64_t)G.n_slabs * kStages * P.nb;
     for (int64_t t = 0; t < n_tables; t++) {
       int64_t left = G.tiles;
       bool fresh = true;  // this table not yet charged to the open range
@@ -467,7 +478,7 @@ vq3r_status vq3r_decode(const uint8_t* idx, const uint16_t* scales, const float*
 size_t vq3r_gemv_workspace_size(const vq3r_gemv_desc* mats, int n_mats, int B) {
   if (!mats || n_mats < 1 || n_mats > VQ3R_GEMV_MAX_MATS || B < 1 || B > VQ3R_GEMV_MAX_B) return 0;
   GemvPlan plan;
-  if (plan_gemv(mats, n_mats, B, nullptr, &plan) != VQ3R_OK) return 0;
+  if (plan_gemv(mats, n_mats, B, 1, nullptr, &plan) != VQ3R_OK) return 0;  // the table-token count changes no size
   return plan.ws_bytes;
 }
 
@@ -477,7 +488,12 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   if (n_mats < 1 || n_mats > VQ3R_GEMV_MAX_MATS || B < 1 || B > VQ3R_GEMV_MAX_B) return VQ3R_ERR_BATCH;
   if (!valid_dtype(x_dtype)) return VQ3R_ERR_DTYPE;
   GemvPlan plan;
-  vq3r_status st = plan_gemv(mats, n_mats, B, static_cast<char*>(workspace), &plan);
+  // The tiled lookup-table kernel takes 2 or more tokens as pairs (both of a
+  // pair's tables resident, the index stream read once per pair); bf16 x
+  // with more tokens goes to the tensor cores instead.
+  const bool tiles_tables = mats[0].layout == VQ3R_LAYOUT_TILES && (x_dtype != VQ3R_BF16 || B < kMmaMinB);
+  const int tokm = tiles_tables && B >= 2 ? 2 : 1;
+  vq3r_status st = plan_gemv(mats, n_mats, B, tokm, static_cast<char*>(workspace), &plan);
   if (st != VQ3R_OK) return st;
   if (plan.P.total_units == 0) return VQ3R_OK;
   if (!workspace || ws_bytes < plan.ws_bytes) return VQ3R_ERR_WORKSPACE;
@@ -523,10 +539,11 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
     return check_launch();
   }
   if (P.layout == VQ3R_LAYOUT_TILES && x_dtype == VQ3R_BF16 && B >= kMmaMinB) {
-    // 8..16 tokens (or matrices with different codebooks): rebuild the weights
+    // 11..16 tokens (or matrices with different codebooks): rebuild the weights
     // in registers and contract with mma.sync; each CTA owns 256 rows of one
     // matrix and loads its codebooks.  Measured on the 8-expert decode step:
-    // 213 us at B = 8 against 228 us for the tensor-memory kernel, which wins
+    // 231 us at B = 12 (two-token tables: 250 us), 213 us at B = 8 (tables:
+    // 171 us, so B <= 10 stays on the tables); the tensor-memory kernel wins
     // from 17 tokens (237 against 279 us at B = 32).
     // One CTA per 128 rows of a matrix; blk_begin numbers those blocks.
     int64_t blocks = 0;
@@ -561,10 +578,18 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kGvThreads);
     cfg.dynamicSmemBytes = kTilesSmemBytes;
-    switch (x_dtype) {
-      case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, kTileSlots>, P); break;
-      case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, kTileSlots>, P); break;
-      default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, kTileSlots>, P); break;
+    if (P.tokm == 2) {
+      switch (x_dtype) {
+        case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, kTileSlots, 2>, P); break;
+        case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 2>, P); break;
+        default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, kTileSlots, 2>, P); break;
+      }
+    } else {
+      switch (x_dtype) {
+        case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, kTileSlots, 1>, P); break;
+        case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 1>, P); break;
+        default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, kTileSlots, 1>, P); break;
+      }
     }
     if (e != cudaSuccess) return cuda_fail(e);
     return check_launch();  // the tiled kernel reduces its partial sums itself

@@ -281,10 +281,12 @@ def test_grouped_gemv_mixed_matrices(layout):
         assert gemv_rel_err(m["y"].cpu().numpy(), ref) <= GEMV_TOL
 
 
-@pytest.mark.parametrize("B", [8, 9, 24, 32])
+@pytest.mark.parametrize("B", [8, 9, 12, 24, 32])
 def test_grouped_gemv_many_tokens(B):
-    """B >= 8 with bf16 x in the tiled layout runs on the tensor cores (weights rebuilt in bf16 hi + lo):
-    ragged rows (not multiples of 128), partial last slabs, partly filled 8-token tiles, mixed groups."""
+    """Many tokens, bf16 x, tiled layout, matrices with different codebooks: B <= 10 on the two-token lookup
+    tables (an odd B leaves a pair with one token), B >= 11 on the tensor cores with the weights rebuilt in
+    bf16 hi + lo (mma.sync, since the codebooks differ): ragged rows (not multiples of 128), partial last
+    slabs, partly filled 8-token tiles, mixed groups."""
     rng = np.random.default_rng(80 + B)
     specs = [(300, 1032, 0, 0), (129, 1032, 0, 0), (64, 200, 1, 1), (513, 2048, 2, 0), (33, 1032, 0, 2)]
     xs = {}
