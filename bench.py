@@ -669,7 +669,56 @@ def main():
                 "vq3r_decode_f32_ms": dec3_ms, "decode_speedup_vs_vq3r": dec3_ms / dec4_ms,
                 "rel_frobenius_ms": err4_ms, "rel_frobenius_frac_hbm": n_w * 2.375 / err4_ms / 1e6 / hbm_gbs,
                 "error": float(e4.item()), "vq3r_error": float(layer.err[k].item())}
-        del pl, sc4, cb4
+        del pl, sc4
+
+        # the 8-expert decode step with VQ4P weights beside VQ3R's over the same experts and x: experts 0-15 of
+        # every kind, the two 8-expert groups alternating (264 MB of indices, more than L2)
+        t4 = {}
+        for kk in layer.kinds:
+            rows, cols = wl.mat_shape(kk)
+            p4, s4 = vq.vq4p_encode(layer.W[kk][:16 * rows], cb4)
+            t4[kk] = (vq.vq3r_pack_tiles(p4), s4)
+            del p4
+        ws4 = torch.zeros(256, dtype=torch.uint8, device=dev)
+        L4, stream4 = vq.lib(), torch.cuda.current_stream().cuda_stream
+        step4 = {}
+        for B in (1, 4):
+            _, _, xu, xd = layer.moe[B]
+            res = {}
+            for fmt, fn in (("vq3r", L4.vq3r_gemv), ("vq4p", L4.vq4p_gemv)):
+                calls = []
+                for g in range(2):
+                    mats = []
+                    for j in range(8):
+                        for kk in layer.kinds:
+                            rows, cols = wl.mat_shape(kk)
+                            idx_k, sc_k, cb_k = (t4[kk][0], t4[kk][1], cb4) if fmt == "vq4p" else \
+                                (layer.tiles[kk], layer.sc[kk], layer.cb)
+                            mats.append(dict(idx=idx_k, scales=sc_k, codebooks=cb_k, x=xd[j] if kk == wl.W2 else xu,
+                                             row0=(8 * g + j) * rows, rows=rows, layout="tiles", cols=cols,
+                                             y=torch.empty((B, rows), dtype=torch.float32, device=dev)))
+                    calls.append((vq._descs(mats), len(mats), mats))
+
+                def call(i, fn=fn, calls=calls, fmt=fmt):
+                    d, n, _ = calls[i % 2]
+                    st = fn(d, n, B, 1, ws4.data_ptr(), ws4.numel(), stream4)
+                    if st:
+                        raise vq.VQ3RError(st, fmt + "_gemv")
+
+                for i in range(4):
+                    call(i)
+                torch.cuda.synchronize()
+                a, b = ev(), ev()
+                a.record()
+                for i in range(args.gemv_iters):
+                    call(i)
+                b.record()
+                torch.cuda.synchronize()
+                ms = a.elapsed_time(b) / args.gemv_iters
+                res[fmt] = {"us_per_step": 1e3 * ms, "frac_hbm": moe_step_bytes(B) / ms / 1e6 / hbm_gbs}
+            step4[str(B)] = res
+        vq4p["decode_step_8_experts"] = step4
+        del t4, cb4
 
     # outlier-aware variant (page "XFP", 权重分解): a sparse FP16 residual of cols/512 entries per row on top of
     # the layer's VQ3R encoding: selection, decode and error with outliers, the MoE decode step with the sparse add,

@@ -329,6 +329,26 @@ vq3r_status vq4p_decode(const uint8_t* planes, const uint16_t* scales, const flo
 vq3r_status vq4p_rel_frobenius_error(const void* W, vq3r_dtype w_dtype, const uint8_t* planes, const uint16_t* scales,
                                      const float* codebooks, int64_t rows, int64_t cols, double* err_out,
                                      void* workspace, size_t ws_bytes, vq3r_stream stream);
+/*
+ * vq4p_gemv -- vq3r_gemv for VQ4P weights: y[b][i] = sum_c w_hat[i][c] * x[b][c],
+ * w_hat as vq4p_decode writes it, B = 1..32 tokens.  Descriptors, workspace,
+ * errors and the grid-barrier conditions are those of vq3r_gemv with TILES
+ * descriptors, except:
+ *   - every descriptor must be VQ3R_LAYOUT_TILES (VQ3R_ERR_SHAPE otherwise):
+ *     the three byte planes repacked by vq3r_pack_tiles, which moves bytes
+ *     and so serves either format;
+ *   - codebooks are [4][64][8] float;
+ *   - every token count runs on the lookup-table kernel: one 256-row table per
+ *     64-column slab holds the four stages' codewords, and from B = 2 two
+ *     tokens share each pass over the indices.
+ * Partial sums are added into y with atomic adds (last bits of y depend on
+ * scheduling); results agree with a binary64 product of the decoded weights
+ * to about 1e-4 relative to rms(y).
+ *   workspace  at least vq3r_gemv_workspace_size() of the same descriptors
+ *              (256 bytes), zero-filled before its first use
+ */
+vq3r_status vq4p_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype x_dtype, void* workspace,
+                      size_t ws_bytes, vq3r_stream stream);
 /* vq3r_train's Lloyd reading with 64 centroids per stage (initial centroids:
  * the first 64 vectors); n >= 64, nstages 1..4, codebooks [nstages][64][8]. */
 size_t vq4p_train_workspace_size(int64_t n);

@@ -74,6 +74,7 @@ def _lib():
         L.vq3r_gemv.argtypes = [P, I32, I32, I32, P, SZ, P]
         L.vq3r_gemv_workspace_size.argtypes = [P, I32, I32]
         L.vq3r_gemv_noalloc.argtypes = [P, I32, I32, I32, P]
+        L.vq4p_gemv.argtypes = L.vq3r_gemv.argtypes
         L.vq3r_tiles_size.argtypes = [I64, I64]
         L.vq3r_tiles_size.restype = SZ
         L.vq3r_pack_tiles.argtypes = [P, I64, I64, I64, P, P]
@@ -105,7 +106,7 @@ def _lib():
         L.vq3r_selftest_wait_timeout.restype = I32
         for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error",
                   "vq3r_gemv_noalloc", "vq3r_pack_tiles", "vq3r_gemm", "vq3r_train", "vq4p_encode", "vq4p_decode",
-                  "vq4p_rel_frobenius_error", "vq4p_train", "vq3r_outliers", "vq3r_decode_outliers",
+                  "vq4p_rel_frobenius_error", "vq4p_train", "vq4p_gemv", "vq3r_outliers", "vq3r_decode_outliers",
                   "vq3r_rel_frobenius_error_outliers", "vq3r_gemv_outliers"):
             getattr(L, f).restype = I32
         _L = L
@@ -309,6 +310,19 @@ def vq3r_gemv(mats, B, workspace=None, stream=None):
     xdt = _DT[mats[0]["x"].dtype]
     _check(_lib().vq3r_gemv(arr, len(mats), B, xdt, _dev(workspace, "workspace"), workspace.numel(),
                             _stream(stream)), "vq3r_gemv")
+    return [m["y"] for m in mats]
+
+
+def vq4p_gemv(mats, B, workspace=None, stream=None):
+    """y = W_hat . x for VQ4P matrices: descriptor dicts as for vq3r_gemv with layout "tiles" (planes
+    repacked by vq3r_pack_tiles) and codebooks [4][64][8]."""
+    arr = _descs(mats)
+    ws = _lib().vq3r_gemv_workspace_size(arr, len(mats), B)
+    if workspace is None:
+        workspace = torch.zeros(max(ws, 16), dtype=torch.uint8, device=mats[0]["idx"].device)
+    xdt = _DT[mats[0]["x"].dtype]
+    _check(_lib().vq4p_gemv(arr, len(mats), B, xdt, _dev(workspace, "workspace"), workspace.numel(),
+                            _stream(stream)), "vq4p_gemv")
     return [m["y"] for m in mats]
 
 

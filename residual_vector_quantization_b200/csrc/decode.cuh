@@ -17,12 +17,6 @@ namespace vq3r {
 
 constexpr int kDecThreads = 512;
 
-// Index formats.  FMT_VQ3R: three 1-byte indices into 256-entry codebooks
-// [3][256][8], one byte plane per stage.  FMT_VQ4P (page §5, VQ3R's sibling at
-// the same 3.00 bits/weight): four 6-bit indices into 64-entry codebooks
-// [4][64][8], packed into the 24-bit word i1 | i2 << 6 | i3 << 12 | i4 << 18
-// whose byte p is stored in plane p.  Both read three byte planes per vector.
-constexpr int FMT_VQ3R = 0, FMT_VQ4P = 1;
 template <int FMT>
 __host__ __device__ constexpr int fmt_codewords_total() {
   return FMT == FMT_VQ4P ? 4 * 64 : kStages * kCodewords;

@@ -105,6 +105,7 @@ struct GvParams {
   int32_t n_mats, n_groups, B, vec8;  // vec8: rows and planes 8-byte aligned (64-bit index loads)
   int32_t nb;            // table tokens: B, or ceil(B / 2) when the tiled kernel looks up two tokens per table pair
   int32_t tokm;          // tokens per table token (1 or 2): table token b covers tokens tokm * b ..
+  int32_t nst;           // table stages per slab: 3 (VQ3R, one table per stage), 1 (VQ4P, one table for all four)
   int64_t total_units;
   int32_t tile_rows;     // rows per work unit: kGvTileRows (planes) or kTileRows (tiles)
   int32_t layout;        // VQ3R_LAYOUT_PLANES or VQ3R_LAYOUT_TILES
@@ -138,8 +139,8 @@ __host__ __device__ __forceinline__ GvCursor unit_cursor(const GvParams& P, int6
   const int tab = (int)(lu / G.tiles);
   const int t = (int)(lu - (int64_t)tab * G.tiles);
   c.b = tab % P.nb;
-  c.s = (tab / P.nb) % kStages;
-  c.slab = tab / (P.nb * kStages);
+  c.s = (tab / P.nb) % P.nst;
+  c.slab = tab / (P.nb * P.nst);
   int m = G.mat_begin;
   while (m + 1 < G.mat_end && P.m[m + 1].tile_prefix <= t) m++;
   c.m = m;
@@ -154,7 +155,7 @@ __device__ __forceinline__ void unit_advance(const GvParams& P, GvCursor& c) {
   c.m = P.g[c.g].mat_begin;
   if (++c.b < P.nb) return;
   c.b = 0;
-  if (++c.s < kStages) return;
+  if (++c.s < P.nst) return;
   c.s = 0;
   if (++c.slab < P.g[c.g].n_slabs) return;
   c.slab = 0;
@@ -351,6 +352,7 @@ struct TileCursor {
   const uint16_t* sc;   // scales, at the tile's first row
   int32_t rows_left;
   int32_t mrows;        // rows of the matrix: y's stride from one token to the next
+  int64_t pst;          // bytes from one byte plane's blocks to the next (n_slabs * plane_stride)
   uint32_t tkey;
   int32_t m, tile, ntiles;
 };
@@ -366,6 +368,7 @@ __device__ __forceinline__ void tcur_fill(const GvParams& P, TileCursor& c) {
   c.sc = M.scales + (int64_t)c.tile * kTileRows;
   c.rows_left = (int32_t)(M.rows - (int64_t)c.tile * kTileRows);
   c.mrows = (int32_t)M.rows;
+  c.pst = n_slabs * M.plane_stride;
 }
 
 __device__ __forceinline__ TileCursor tcur_at(const GvParams& P, int64_t u) {
@@ -394,7 +397,7 @@ __device__ __forceinline__ void tcur_next(const GvParams& P, TileCursor& c) {
     int slab = (int)(c.tkey & 0xFFFFFu), s = (int)((c.tkey >> 20) & 3u), b = (int)((c.tkey >> 22) & 31u);
     if (++b >= P.nb) {
       b = 0;
-      if (++s >= kStages) {
+      if (++s >= P.nst) {
         s = 0;
         if (++slab >= P.g[g].n_slabs) {
           slab = 0;
@@ -446,7 +449,7 @@ __device__ __forceinline__ uint32_t next_table_key(const GvParams& P, uint32_t k
   int slab = (int)(k & 0xFFFFFu), s = (int)((k >> 20) & 3u), b = (int)((k >> 22) & 31u), g = (int)(k >> 27);
   if (++b < P.nb) return table_key(g, slab, s, b);
   b = 0;
-  if (++s < kStages) return table_key(g, slab, s, b);
+  if (++s < P.nst) return table_key(g, slab, s, b);
   s = 0;
   if (++slab < P.g[g].n_slabs) return table_key(g, slab, s, b);
   return table_key(g + 1, 0, 0, 0);
@@ -680,6 +683,43 @@ __device__ __forceinline__ float lds_f32_t1_128(uint32_t a) {
   return v;
 }
 
+// VQ4P table entries: one 256-row table holds the four stages' 64 codewords
+// (row 64 s + i), so stage s is 16 KiB further; plus 128 bytes for the second
+// column slot and 64 KiB for the pair's second token.  off is a constant
+// once the lookup loop is unrolled.
+template <int OFF>
+__device__ __forceinline__ float lds_at(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(a), "n"(OFF));
+  return v;
+}
+__device__ __forceinline__ float lds_vq4p(uint32_t a, int stage, int slot, int buf) {
+  switch (buf * 8 + stage * 2 + slot) {
+#define VQ4P_LDS_CASE(k) \
+  case k: return lds_at<65536 * ((k) >> 3) + 16384 * (((k) >> 1) & 3) + 128 * ((k) & 1)>(a);
+    VQ4P_LDS_CASE(0) VQ4P_LDS_CASE(1) VQ4P_LDS_CASE(2) VQ4P_LDS_CASE(3)
+    VQ4P_LDS_CASE(4) VQ4P_LDS_CASE(5) VQ4P_LDS_CASE(6) VQ4P_LDS_CASE(7)
+    VQ4P_LDS_CASE(8) VQ4P_LDS_CASE(9) VQ4P_LDS_CASE(10) VQ4P_LDS_CASE(11)
+    VQ4P_LDS_CASE(12) VQ4P_LDS_CASE(13) VQ4P_LDS_CASE(14)
+#undef VQ4P_LDS_CASE
+    default: return lds_at<65536 + 3 * 16384 + 128>(a);
+  }
+}
+
+// Shared addresses of the four table entries of one VQ4P vector.  v holds
+// the vector's plane-0 byte in byte 0 and its plane-1 byte in byte 1, v2 its
+// plane-1 and plane-2 bytes; with the 24-bit word w = e0 | e1 << 8 | e2 << 16
+// the indices are i1 = w[0:6), i2 = w[6:12), i3 = w[12:18), i4 = w[18:24),
+// so i_s << 8 is one shift and mask away: i1 = v[0:6), i2 = v[6:12),
+// i3 = v2[4:10), i4 = v2[10:16).  l supplies the bank offset and the table
+// base (bytes 0 and 2).
+__device__ __forceinline__ void vq4p_addrs(uint32_t v, uint32_t v2, uint32_t l, uint32_t (&ad)[4]) {
+  ad[0] = ((v << 8) & 0x3F00u) | l;
+  ad[1] = ((v << 2) & 0x3F00u) | l;
+  ad[2] = ((v2 << 4) & 0x3F00u) | l;
+  ad[3] = ((v2 >> 2) & 0x3F00u) | l;
+}
+
 // Bulk prefetch of one 32 KiB index block into L2 (a hint: it reads, writes
 // nothing, and may be issued before the inputs are final).
 __device__ __forceinline__ void prefetch_block_l2(const void* p) {
@@ -710,13 +750,17 @@ __device__ __forceinline__ float rows_exchange(const float (&acc)[4], bool hi2, 
 }
 
 // TOKS = 1: table buffers t & 1 double-buffer the tables of consecutive
-// (slab, stage, token) keys.  TOKS = 2 (2..16 tokens): a key is (slab, stage,
-// token pair); buffer 0 holds the pair's first token's table and buffer 1 the
-// second's, so every index byte is looked up for both tokens at the same
-// offset (+ 64 KiB) and the index stream is read once per pair instead of
-// once per token.
-template <int XDT, int NSLOT, int TOKS>
+// (slab, stage, token) keys.  TOKS = 2 (2 or more tokens): a key is (slab,
+// stage, token pair); buffer 0 holds the pair's first token's table and
+// buffer 1 the second's, so every index byte is looked up for both tokens at
+// the same offset (+ 64 KiB) and the index stream is read once per pair
+// instead of once per token.
+// FMT = FMT_VQ4P: a slab has one table (the four stages' 64 codewords seen as
+// 256 rows, built exactly as a VQ3R stage table), a unit reads the three
+// byte planes of its (slab, tile) and makes four lookups per vector.
+template <int XDT, int NSLOT, int TOKS, int FMT = FMT_VQ3R>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_constant__ GvParams P) {
+  constexpr int PL = FMT == FMT_VQ4P ? 3 : 1;  // byte planes read per unit
   extern __shared__ __align__(128) unsigned char gv_smem[];
   const uint32_t sbase = smem_u32(gv_smem);
   const uint32_t tab_addr = (sbase + 0xFFFFu) & ~0xFFFFu;  // table buffer 0; buffer 1 follows at + 64 KiB
@@ -738,6 +782,10 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   uint32_t sel[4];
 #pragma unroll
   for (int q = 0; q < 4; q++) sel[q] = 0x7604u | ((uint32_t)((q ^ g) & 3) << 4);
+  // VQ4P: byte (q ^ g) & 3 of the first register in byte 0, of the second in byte 1
+  uint32_t sel2[4];
+#pragma unroll
+  for (int q = 0; q < 4; q++) sel2[q] = (uint32_t)((q ^ g) & 3) | ((4u + (uint32_t)((q ^ g) & 3)) << 4);
   constexpr int kRowsPerWarpT = kTileRows / kGvWarps;  // 32: rows warp*32 + 8t + g, t = 0..3
   const int lane_off = (warp * kRowsPerWarpT + g) * kSlabV + 16 * a;
   const int out_row = warp * kRowsPerWarpT + 8 * a + g;  // row whose sum this lane holds after the reduction
@@ -800,7 +848,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   if (tid == 0) arrival = barrier_arrive(P.hdr);
   bool ok = mbar_wait_bounded(&S.mbar[0], 0);
 
-  uint4 r[NSLOT][4];
+  uint4 r[NSLOT][PL][4];
   float* sq[NSLOT];
   uint32_t ssc[NSLOT];  // binary16 bits of the lane's row scale, converted when the unit's sum is added
   int32_t srows[NSLOT];
@@ -810,7 +858,9 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   for (int i = 0; i < NSLOT; i++) {
     if (u0 + i < u1) {
 #pragma unroll
-      for (int t = 0; t < 4; t++) r[i][t] = ldg_stream16(ci.p + lane_off + t * 8 * kSlabV, pol);
+      for (int t = 0; t < 4; t++)
+#pragma unroll
+        for (int pl = 0; pl < PL; pl++) r[i][pl][t] = ldg_stream16(ci.p + pl * ci.pst + lane_off + t * 8 * kSlabV, pol);
       sq[i] = ci.q;
       ssc[i] = out_row < ci.rows_left ? (uint32_t)__ldg(ci.sc + out_row) : 0u;
       srows[i] = ci.rows_left;
@@ -831,7 +881,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   int64_t upf = u0 + NSLOT;
   if (tid == 0) {
     for (int k = 0; k < kPrefetchUnits && upf < u1; k++, upf++) {
-      prefetch_block_l2(cpf.p);
+      for (int pl = 0; pl < PL; pl++) prefetch_block_l2(cpf.p + pl * cpf.pst);
       tcur_next(P, cpf);
     }
   }
@@ -875,14 +925,39 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
         const int32_t rows_valid = srows[i];
         const bool refill = u + i + NSLOT < u1;
         const uint8_t* const pn = ci.p + lane_off;
+        const int64_t pstn = ci.pst;
         const int32_t mrows = smr[i];
         const uint32_t ukey = skey[i];
         float acc[4], acc2[4];
 #pragma unroll
         for (int t = 0; t < 4; t++) {
-          const uint32_t w[4] = {r[i][t].x, r[i][t].y, r[i][t].z, r[i][t].w};
+          const uint32_t w[4] = {r[i][0][t].x, r[i][0][t].y, r[i][0][t].z, r[i][0][t].w};
           float2 s2 = make_float2(0.0f, 0.0f);
-          if constexpr (TOKS == 1) {
+          if constexpr (FMT == FMT_VQ4P) {
+            const uint32_t wb[4] = {r[i][PL - 2][t].x, r[i][PL - 2][t].y, r[i][PL - 2][t].z, r[i][PL - 2][t].w};
+            const uint32_t wc[4] = {r[i][PL - 1][t].x, r[i][PL - 1][t].y, r[i][PL - 1][t].z, r[i][PL - 1][t].w};
+#pragma unroll
+            for (int m = 0; m < 16; m++) {
+              const int k = m >> 2, slot = (m >> 2) & 1;
+              uint32_t ad[4];
+              vq4p_addrs(__byte_perm(w[k], wb[k], sel2[m & 3]), __byte_perm(wb[k], wc[k], sel2[m & 3]),
+                         lc[(m & 3) | ((m >> 3) << 2)], ad);
+              if constexpr (TOKS == 1) {  // stages 1 and 3 in one half of the pair sum, 2 and 4 in the other
+                s2 = __fadd2_rn(s2, make_float2(lds_vq4p(ad[0], 0, slot, 0), lds_vq4p(ad[1], 1, slot, 0)));
+                s2 = __fadd2_rn(s2, make_float2(lds_vq4p(ad[2], 2, slot, 0), lds_vq4p(ad[3], 3, slot, 0)));
+              } else {  // (first token, second token)
+#pragma unroll
+                for (int st = 0; st < 4; st++)
+                  s2 = __fadd2_rn(s2, make_float2(lds_vq4p(ad[st], st, slot, 0), lds_vq4p(ad[st], st, slot, 1)));
+              }
+            }
+            if constexpr (TOKS == 1) {
+              acc[t] = s2.x + s2.y;
+            } else {
+              acc[t] = s2.x;
+              acc2[t] = s2.y;
+            }
+          } else if constexpr (TOKS == 1) {
 #pragma unroll
             for (int m = 0; m < 16; m += 2) {
               const uint32_t o0 = __byte_perm(w[m >> 2], lc[(m & 3) | ((m >> 3) << 2)], sel[m & 3]);
@@ -903,10 +978,13 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
             acc[t] = s2.x;
             acc2[t] = s2.y;
           }
-          if (refill) r[i][t] = ldg_stream16(pn + t * 8 * kSlabV, pol);
+          if (refill) {
+#pragma unroll
+            for (int pl = 0; pl < PL; pl++) r[i][pl][t] = ldg_stream16(pn + pl * pstn + t * 8 * kSlabV, pol);
+          }
         }
-        if (tid == 0 && upf < u1) {  // keep kPrefetchUnits blocks prefetched beyond the ring
-          prefetch_block_l2(cpf.p);
+        if (tid == 0 && upf < u1) {  // keep kPrefetchUnits units prefetched beyond the ring
+          for (int pl = 0; pl < PL; pl++) prefetch_block_l2(cpf.p + pl * cpf.pst);
           tcur_next(P, cpf);
           upf++;
         }

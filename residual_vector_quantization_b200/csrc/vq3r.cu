@@ -75,12 +75,21 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
-    if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
+    const void* tiles_kernels[12] = {
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 1>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 1>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 1>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 2>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 2>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 2>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, 1, 1, FMT_VQ4P>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, 1, 1, FMT_VQ4P>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, 1, 1, FMT_VQ4P>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, 1, 2, FMT_VQ4P>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, 1, 2, FMT_VQ4P>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, 1, 2, FMT_VQ4P>)};
+    for (int k = 0; k < 12 && r == cudaSuccess; k++)
+      r = cudaFuncSetAttribute(tiles_kernels[k], cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
     const int gm = (int)kMmaSmemBytes;
     const int gc = (int)(kCbrFloats * sizeof(float));
     if (r == cudaSuccess) r = cudaFuncSetAttribute(decode_bulk_kernel<VQ3R_F32, FMT_VQ3R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_bulk_smem<FMT_VQ3R>());
@@ -108,14 +117,7 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
     if (r != cudaSuccess) return r;
     int fit = 1;
-    const void* tiles_kernels[6] = {
-        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 1>),
-        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 1>),
-        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 1>),
-        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 2>),
-        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 2>),
-        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 2>)};
-    for (int k = 0; k < 6 && r == cudaSuccess; k++) {
+    for (int k = 0; k < 12 && r == cudaSuccess; k++) {
       int n = 0;
       r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, tiles_kernels[k], kGvThreads, gt);
       if (n < 1) fit = 0;
@@ -150,12 +152,16 @@ struct GemvPlan {
 // numbers the work units.  Matrices are stored grouped (each group's
 // matrices contiguous in P.m); empty matrices are dropped.
 // tokm: tokens per table token (2 for the tiled kernel's two-token tables, else 1).
-vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, int tokm, char* ws_base, GemvPlan* plan) {
+// nst: table stages per slab, 3 for VQ3R, 1 for VQ4P (its four 64-codeword
+// stages share one 256-entry table).
+vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, int tokm, char* ws_base, GemvPlan* plan,
+                      int nst = kStages) {
   GvParams& P = plan->P;
   memset(&P, 0, sizeof(P));
   P.B = B;
   P.tokm = tokm;
   P.nb = (B + tokm - 1) / tokm;
+  P.nst = nst;
   P.vec8 = 1;
   P.layout = mats[0].layout;
   if (P.layout != VQ3R_LAYOUT_PLANES && P.layout != VQ3R_LAYOUT_TILES) return VQ3R_ERR_SHAPE;
@@ -223,7 +229,7 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, int tokm, c
   for (int g = 0; g < n_groups; g++) {
     GvGroup& G = P.g[g];
     G.unit_begin = units;
-    units += (int64_t)G.n_slabs * kStages * P.nb * G.tiles;
+    units += (int64_t)G.n_slabs * P.nst * P.nb * G.tiles;
   }
   // Partial sums of the planes kernel: one float per (token, stage, slab,
   // row).  The tiled kernels add into y directly and need only the header.
@@ -250,7 +256,7 @@ int64_t split_ranges(const GvParams& P, int64_t budget, int n, int64_t* begin) {
   int64_t unit = 0, cost = budget;  // cost of the open range; budget forces a new range first
   for (int g = 0; g < P.n_groups; g++) {
     const GvGroup& G = P.g[g];
-    const int64_t n_tables = (int64_t)G.n_slabs * kStages * P.nb;
+    const int64_t n_tables = (int64_t)G.n_slabs * P.nst * P.nb;
     for (int64_t t = 0; t < n_tables; t++) {
       int64_t left = G.tiles;
       bool fresh = true;  // this table not yet charged to the open range
@@ -301,6 +307,40 @@ void balance_split(GvParams& P, int n) {
     P.cta_key_last[c] = table_key(last.g, last.slab, last.s, last.b);
   }
   P.n_split = n;
+}
+
+// Launch of the tiled lookup-table GEMV, one CTA per SM.  The kernel's grid
+// barrier needs all CTAs resident at once; the cooperative launch attribute
+// would guarantee it but measured 3.8 us slower per call (it gives up most of
+// the programmatic-launch overlap), so the grid is sized to one CTA per SM
+// and the fit of one CTA per SM is checked instead.
+template <int FMT, int NSLOT>
+vq3r_status launch_tiles(GemvPlan& plan, vq3r_dtype x_dtype, int sms, cudaLaunchConfig_t& cfg) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!g_dev_tiles_fit[dev]) return cuda_fail(cudaErrorCooperativeLaunchTooLarge);
+  GvParams& P = plan.P;
+  const int grid = (int)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms);
+  balance_split(P, grid);
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = kTilesSmemBytes;
+  if (P.tokm == 2) {
+    switch (x_dtype) {
+      case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, NSLOT, 2, FMT>, P); break;
+      case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, NSLOT, 2, FMT>, P); break;
+      default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, NSLOT, 2, FMT>, P); break;
+    }
+  } else {
+    switch (x_dtype) {
+      case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, NSLOT, 1, FMT>, P); break;
+      case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, NSLOT, 1, FMT>, P); break;
+      default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, NSLOT, 1, FMT>, P); break;
+    }
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  return check_launch();  // the tiled kernel adds its sums into y itself
 }
 
 template <int DT, int FMT>
@@ -564,36 +604,8 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
     if (e != cudaSuccess) return cuda_fail(e);
     return check_launch();
   }
-  if (P.layout == VQ3R_LAYOUT_TILES) {  // one CTA per SM
-    // The kernel's grid barrier needs all CTAs resident at once; the cooperative
-    // launch attribute would guarantee it but measured 3.8 us slower per call
-    // (it gives up most of the programmatic-launch overlap), so the grid is
-    // sized to one CTA per SM and the fit of one CTA per SM is checked instead.
-    int dev = 0;
-    e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e);
-    if (!g_dev_tiles_fit[dev]) return cuda_fail(cudaErrorCooperativeLaunchTooLarge);
-    const int grid = (int)(P.total_units < (int64_t)sms ? P.total_units : (int64_t)sms);
-    balance_split(plan.P, grid);
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kGvThreads);
-    cfg.dynamicSmemBytes = kTilesSmemBytes;
-    if (P.tokm == 2) {
-      switch (x_dtype) {
-        case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, kTileSlots, 2>, P); break;
-        case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 2>, P); break;
-        default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, kTileSlots, 2>, P); break;
-      }
-    } else {
-      switch (x_dtype) {
-        case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, kTileSlots, 1>, P); break;
-        case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 1>, P); break;
-        default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, kTileSlots, 1>, P); break;
-      }
-    }
-    if (e != cudaSuccess) return cuda_fail(e);
-    return check_launch();  // the tiled kernel reduces its partial sums itself
-  } else {  // two CTAs per SM
+  if (P.layout == VQ3R_LAYOUT_TILES) return launch_tiles<FMT_VQ3R, kTileSlots>(plan, x_dtype, sms, cfg);
+  {  // two CTAs per SM
     const int grid = (int)(P.total_units < 2 * (int64_t)sms ? P.total_units : 2 * (int64_t)sms);
     switch (x_dtype) {
       case VQ3R_F32: gemv_lut_kernel<VQ3R_F32><<<grid, kGvThreads, kGvSmemBytes, s>>>(P); break;
@@ -611,6 +623,31 @@ vq3r_status vq3r_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype 
   e = cudaLaunchKernelEx(&cfg, gemv_reduce_kernel, P);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
+}
+
+vq3r_status vq4p_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, vq3r_dtype x_dtype, void* workspace,
+                      size_t ws_bytes, vq3r_stream stream) {
+  if (!mats) return VQ3R_ERR_NULL;
+  if (n_mats < 1 || n_mats > VQ3R_GEMV_MAX_MATS || B < 1 || B > VQ3R_GEMV_MAX_B) return VQ3R_ERR_BATCH;
+  if (!valid_dtype(x_dtype)) return VQ3R_ERR_DTYPE;
+  if (mats[0].layout != VQ3R_LAYOUT_TILES) return VQ3R_ERR_SHAPE;  // plan_gemv checks that all layouts agree
+  GemvPlan plan;
+  vq3r_status st = plan_gemv(mats, n_mats, B, B >= 2 ? 2 : 1, static_cast<char*>(workspace), &plan, 1);
+  if (st != VQ3R_OK) return st;
+  if (plan.P.total_units == 0) return VQ3R_OK;
+  if (!workspace || ws_bytes < plan.ws_bytes) return VQ3R_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return launch_tiles<FMT_VQ4P, 1>(plan, x_dtype, sms, cfg);
 }
 
 vq3r_status vq3r_gemm(const vq3r_gemm_desc* mats, int n_mats, vq3r_dtype x_dtype, vq3r_stream stream) {

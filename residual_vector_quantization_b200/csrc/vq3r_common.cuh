@@ -17,6 +17,13 @@ constexpr int kDim = VQ3R_DIM;
 constexpr int kCodebookFloats = kStages * kCodewords * kDim;  // 6144
 constexpr int kCodebookBytes = kCodebookFloats * 4;           // 24 KiB
 
+// Index formats.  FMT_VQ3R: three 1-byte indices into 256-entry codebooks
+// [3][256][8], one byte plane per stage.  FMT_VQ4P (page §5, VQ3R's sibling at
+// the same 3.00 bits/weight): four 6-bit indices into 64-entry codebooks
+// [4][64][8], packed into the 24-bit word i1 | i2 << 6 | i3 << 12 | i4 << 18
+// whose byte p is stored in plane p.  Both read three byte planes per vector.
+constexpr int FMT_VQ3R = 0, FMT_VQ4P = 1;
+
 // Error codes a kernel may leave in the device error word.
 constexpr int kDevErrMbarTimeout = 1;  // a bulk copy into shared memory did not complete within ~1 s
 constexpr int kDevErrBarrierTimeout = 2;  // not all CTAs of a tiled GEMV reached its grid barrier within ~1 s

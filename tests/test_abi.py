@@ -78,6 +78,20 @@ def test_gemv_batch_and_workspace_checks(lib):
     assert lib.vq3r_gemv_workspace_size(arr, 1, 0) == 0
 
 
+def test_vq4p_gemv_argument_checks(lib):
+    arr = _descs([(2048, 7168, 0x10000, 0x20000)])
+    assert lib.vq4p_gemv(None, 1, 1, 1, 0x500000, 1 << 30, None) == 1
+    assert lib.vq4p_gemv(arr, 1, 1, 1, 0x500000, 1 << 30, None) == 2  # the planes layout is not accepted
+    arr[0].layout = 1
+    assert lib.vq4p_gemv(arr, 1, 0, 1, 0x500000, 1 << 30, None) == 5
+    assert lib.vq4p_gemv(arr, 1, 33, 1, 0x500000, 1 << 30, None) == 5
+    assert lib.vq4p_gemv(arr, 1, 1, 9, 0x500000, 1 << 30, None) == 4
+    assert lib.vq4p_gemv(arr, 1, 1, 1, None, 0, None) == 7
+    assert lib.vq4p_gemv(arr, 1, 1, 1, 0x500000, 255, None) == 7  # the 256-byte header is needed
+    arr[0].plane_stride = 4 * 32768 + 16
+    assert lib.vq4p_gemv(arr, 1, 1, 1, 0x500000, 1 << 30, None) == 2
+
+
 def test_gemv_workspace_holds_the_partial_sums(lib):
     # a 256-byte header, then per matrix: B tokens x 3 stages x ceil(cols / 512) slabs x rows fp32 partial sums
     # (256-byte aligned)

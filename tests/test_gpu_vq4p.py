@@ -11,7 +11,7 @@ import torch
 import oracle
 import synth
 from synth import workloads as wl
-from vq3r_cases import RELFRO_TOL, f32_to_bf16_bits
+from vq3r_cases import GEMV_TOL, RELFRO_TOL, f32_to_bf16_bits, gemv_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -197,3 +197,85 @@ def test_layer_stacked_encode_sampled_rows():
     np.testing.assert_array_equal(pl_t[:, sel, :].cpu().numpy(), pl_o)
     np.testing.assert_array_equal(d_t[sel].cpu().numpy().view(np.uint32),
                                   oracle.vq4p_decode(pl_o, sc_o, cb).view(np.uint32))
+
+
+def _gemv_case(rng, specs, B, x_dtype, seed):
+    """Random VQ4P matrices (every 24-bit index word possible), binary16 scales, per-group codebooks and x;
+    -> (device descriptor dicts in the tiled layout, binary64 oracle outputs)."""
+    xs, mats, refs = {}, [], []
+    for rows, cols, cbk, xk in specs:
+        cb = random_codebooks4(seed + cbk)
+        if (xk, cols) not in xs:
+            xf = rng.standard_normal((B, cols)).astype(np.float32)
+            xs[(xk, cols)] = (xf if x_dtype == "f32" else f32_to_bf16_bits(xf) if x_dtype == "bf16"
+                              else xf.astype(np.float16).view(np.uint16))
+        pl = rng.integers(0, 256, size=(3, rows, cols // 8), dtype=np.uint8)
+        sc = np.float16(np.exp(rng.standard_normal(rows) * 0.5)).view(np.uint16)
+        refs.append(oracle.vq4p_gemv(pl, sc, cb, xs[(xk, cols)], x_dtype))
+        pl_t = torch.from_numpy(pl).to(DEV)
+        mats.append(dict(idx=vq.vq3r_pack_tiles(pl_t), layout="tiles", cols=cols,
+                         scales=torch.from_numpy(sc.view(np.int16)).to(DEV),
+                         codebooks=torch.from_numpy(np.ascontiguousarray(cb)).to(DEV),
+                         x=(xk, cols), y=torch.full((B, rows), float("nan"), device=DEV)))
+    xdev = {k: to_dev(v, x_dtype) for k, v in xs.items()}
+    for m in mats:
+        m["x"] = xdev[m["x"]]
+    return mats, refs
+
+
+@pytest.mark.parametrize("B,x_dtype", [(1, "bf16"), (1, "f32"), (1, "f16"), (2, "bf16"), (3, "f16"), (8, "bf16"),
+                                       (17, "f32"), (32, "bf16")])
+def test_gemv_grouped_matches_oracle(B, x_dtype):
+    """vq4p_gemv over mixed matrices (ragged rows and slabs, two codebook sets, two x per width) against the
+    oracle's binary64 product of the decoded weights; one token (one table per slab), token pairs with an odd
+    count (a pair with one token), every x dtype."""
+    rng = np.random.default_rng(900 + 10 * B + len(x_dtype))
+    specs = [(300, 1032, 0, 0), (129, 1032, 0, 0), (64, 200, 1, 1), (513, 2048, 1, 0), (1, 8, 0, 2)]
+    mats, refs = _gemv_case(rng, specs, B, x_dtype, 70)
+    vq.vq4p_gemv(mats, B)
+    for m, ref in zip(mats, refs):
+        y = m["y"].cpu().numpy()
+        assert np.isfinite(y).all()  # every output written
+        assert gemv_rel_err(y, ref) <= GEMV_TOL
+    assert vq.vq3r_device_error() == 0
+
+
+@pytest.mark.parametrize("B", [1, 4])
+def test_gemv_moe_decode_step_sampled_rows(B):
+    """The 8-expert MoE decode step's shapes (w1, w3: 2048 x 7168; w2: 7168 x 2048; one call, 24 matrices) with
+    random VQ4P indices: 48 sampled rows of every matrix against the oracle."""
+    rng = np.random.default_rng(950 + B)
+    cb = random_codebooks4(5)
+    cb_t = torch.from_numpy(np.ascontiguousarray(cb)).to(DEV)
+    x1 = f32_to_bf16_bits(rng.standard_normal((B, 7168)).astype(np.float32))
+    x2 = f32_to_bf16_bits(rng.standard_normal((B, 2048)).astype(np.float32))
+    x1_t, x2_t = to_dev(x1, "bf16"), to_dev(x2, "bf16")
+    mats, hosts = [], []
+    for e in range(8):
+        for rows, cols, x_t, x in ((2048, 7168, x1_t, x1), (2048, 7168, x1_t, x1), (7168, 2048, x2_t, x2)):
+            pl_t = torch.randint(0, 256, (3, rows, cols // 8), dtype=torch.uint8, device=DEV)
+            sc_t = torch.from_numpy(np.float16(np.exp(rng.standard_normal(rows) * 0.5)).view(np.int16)).to(DEV)
+            mats.append(dict(idx=vq.vq3r_pack_tiles(pl_t), layout="tiles", cols=cols, scales=sc_t, codebooks=cb_t,
+                             x=x_t, y=torch.empty((B, rows), device=DEV)))
+            hosts.append((pl_t, sc_t, x))
+    vq.vq4p_gemv(mats, B)
+    torch.cuda.synchronize()
+    for m, (pl_t, sc_t, x) in zip(mats, hosts):
+        rows = pl_t.shape[1]
+        sample = np.sort(rng.choice(rows, 48, replace=False))
+        sel = torch.from_numpy(sample).to(DEV)
+        pl = pl_t[:, sel, :].cpu().numpy()
+        sc = sc_t[sel].cpu().numpy().view(np.uint16)
+        ref = oracle.vq4p_gemv(pl, sc, cb, x, "bf16")
+        y = m["y"][:, sel].cpu().numpy()
+        # the tolerance's rms term comes from the sampled rows
+        assert gemv_rel_err(y, ref) <= GEMV_TOL
+    assert vq.vq3r_device_error() == 0
+
+
+def test_gemv_rejects_the_planes_layout():
+    pl = torch.zeros((3, 4, 2), dtype=torch.uint8, device=DEV)
+    m = dict(idx=pl, scales=torch.zeros(4, dtype=torch.int16, device=DEV), codebooks=torch.zeros((4, 64, 8), device=DEV),
+             x=torch.zeros((1, 16), dtype=torch.bfloat16, device=DEV), y=torch.empty((1, 4), device=DEV))
+    with pytest.raises(vq.VQ3RError):
+        vq.vq4p_gemv([m], 1)
