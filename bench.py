@@ -754,8 +754,18 @@ def main():
                                                                       layer.cb, oc[k1], ov[k1], out=e1,
                                                                       workspace=layer.err_ws[k1]), 3)
         err_with = float(e1.item())
-        # the MoE decode step (B = 1) with the sparse add: one extra grouped launch over the same 24 matrices
-        plans, _, xu, xd = layer.moe[1]
+        # the MoE decode step (B = 1) with the outliers: one call whose lookup kernel adds them
+        # (vq3r_gemv_with_outliers), and for comparison the two-launch form (vq3r_gemv, then vq3r_gemv_outliers)
+        plans, ws1, xu, xd = layer.moe[1]
+        otl = {k: vq.vq3r_pack_outliers(oc[k], ov[k]) for k in layer.kinds}  # one-time layout for the fused call
+        fdescs = []
+        for g in range(layer.groups):
+            d, n, mats = plans[g][:3]
+            mo = []
+            for i, m in enumerate(mats):
+                kind = (wl.W1, wl.W3)[i % 2] if i < 16 else wl.W2
+                mo.append(dict(m, otiles=otl[kind]))
+            fdescs.append((d, vq._outlier_tiles(mo), n))
         odescs = []
         for g in range(layer.groups):
             mats = plans[g][2]
@@ -772,16 +782,24 @@ def main():
         def step_plain(i):
             layer.gemv(1, i)
 
-        def step_out(i):
+        def step_two_launch(i):
             layer.gemv(1, i)
             d = odescs[i % layer.groups]
             st = L.vq3r_gemv_outliers(d, len(d), 1, 1, torch.cuda.current_stream().cuda_stream)
             if st:
                 raise vq.VQ3RError(st, "vq3r_gemv_outliers")
 
+        def step_out(i):
+            d, od, n = fdescs[i % layer.groups]
+            st = L.vq3r_gemv_with_outliers(d, od, n, 1, 1, ws1.data_ptr(), ws1.numel(),
+                                           torch.cuda.current_stream().cuda_stream)
+            if st:
+                raise vq.VQ3RError(st, "vq3r_gemv_with_outliers")
+
         reps = max(8, args.gemv_iters)
         t_plain = timed_ms(lambda: [step_plain(i) for i in range(reps)], 1) / reps
         t_out = timed_ms(lambda: [step_out(i) for i in range(reps)], 1) / reps
+        t_two = timed_ms(lambda: [step_two_launch(i) for i in range(reps)], 1) / reps
         # error gain on 8 experts' w1 of the sweep distribution
         rows, cols = wl.mat_shape(wl.W1)
         Ws = torch.empty((8 * rows, cols), dtype=torch.bfloat16, device=dev)
@@ -804,8 +822,9 @@ def main():
                 "rel_frobenius_w1_ms": err_o, "rel_frobenius_w1_frac_hbm": n1 * 2.375 / err_o / 1e6 / hbm_gbs,
                 "error_w1": err_with, "error_w1_plain": errs_plain_w1(layer),
                 "moe_step_B1_us": 1e3 * t_out, "moe_step_B1_plain_us": 1e3 * t_plain,
+                "moe_step_B1_two_launch_us": 1e3 * t_two, "moe_step_B1_ratio_to_plain": t_out / t_plain,
                 "sweep_8x_w1_error_plain": es0, "sweep_8x_w1_error_with_outliers": sweep_gain}
-        del oc, ov, odescs
+        del oc, ov, odescs, fdescs, otl
 
     # the single-expert workload's quality table: VQ3R error of w1, w3, w2 (this library, expert codebooks) beside
     # the oracle's rtn4-row error of the same matrices (computed in the CPU leg), outside the timed region

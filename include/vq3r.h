@@ -411,6 +411,43 @@ vq3r_status vq3r_rel_frobenius_error_outliers(const void* W, vq3r_dtype w_dtype,
 vq3r_status vq3r_gemv_outliers(const vq3r_outlier_desc* mats, int n_mats, int B, vq3r_dtype x_dtype,
                                vq3r_stream stream);
 
+/*
+ * Outlier tiles -- the layout vq3r_gemv_with_outliers streams: per 512-row
+ * tile t of a matrix and outlier number q (0 <= q < k), 512 uint32 words
+ *   otiles[(t * k + q) * 512 + r] = ocols[512 t + r][q] | ovals[512 t + r][q] << 16
+ * for rows 512 t + r < rows, and 0xFFFFFFFF past the last row, so the q-th
+ * outliers of a tile's rows are one contiguous 2 KiB block (4 bytes per
+ * outlier, like ocols + ovals).
+ * vq3r_outliers_tiles_size: bytes of that layout, ceil(rows / 512) * k * 2048
+ *   (0 for a negative size or k > 16384).
+ * vq3r_pack_outliers: ocols / ovals [rows][k] (as vq3r_outliers writes them)
+ *   -> otiles (DEVICE, 16-byte aligned).  rows == 0 or k == 0 is a no-op.
+ *
+ * vq3r_gemv_with_outliers -- y = (W_hat + O) . x in one call: vq3r_gemv of
+ * mats and the sparse outlier product of outl[i] for each matrix i.
+ * outl[i].otiles points at the outlier tile block of mats[i]'s first row
+ * (a row range of a larger matrix starts at a multiple of 512 rows, as for
+ * TILES indices); outl[i].k = 0 marks a matrix without outliers (otiles may
+ * then be NULL), otherwise 0 < k <= cols <= 16384.  Workspace, B, x_dtype and
+ * the other conditions are vq3r_gemv's.  Per row i and token b the
+ * outliers' part is sum_q (float)o_iq * x[b][c_iq] in binary32 (fused
+ * multiply-adds, q ascending).  TILES calls that run on the lookup-table
+ * kernel (F32 and F16 x, and bf16 x below 11 tokens) compute it inside that
+ * kernel's single launch, as the value y starts from instead of zero, before
+ * the lookups add into it.  Other calls launch vq3r_gemv and then a sparse
+ * add over the outlier tiles, which adds it to y.
+ */
+typedef struct {
+  const uint32_t* otiles;   /* outlier tiles of the matrix's first row, DEVICE */
+  int64_t k;                /* outliers per row; 0: none */
+} vq3r_outlier_tiles;
+
+size_t vq3r_outliers_tiles_size(int64_t rows, int64_t k);
+vq3r_status vq3r_pack_outliers(const uint16_t* ocols, const uint16_t* ovals, int64_t rows, int64_t k, uint32_t* otiles,
+                               vq3r_stream stream);
+vq3r_status vq3r_gemv_with_outliers(const vq3r_gemv_desc* mats, const vq3r_outlier_tiles* outl, int n_mats, int B,
+                                    vq3r_dtype x_dtype, void* workspace, size_t ws_bytes, vq3r_stream stream);
+
 /* Human-readable name of a status code (static string). */
 const char* vq3r_status_string(vq3r_status s);
 

@@ -102,12 +102,16 @@ def _lib():
         L.vq3r_rel_frobenius_outliers_workspace_size.restype = SZ
         L.vq3r_rel_frobenius_error_outliers.argtypes = [P, I32, P, P, P, P, P, I64, I64, I64, P, P, SZ, P]
         L.vq3r_gemv_outliers.argtypes = [P, I32, I32, I32, P]
+        L.vq3r_gemv_with_outliers.argtypes = [P, P, I32, I32, I32, P, SZ, P]
+        L.vq3r_outliers_tiles_size.argtypes = [I64, I64]
+        L.vq3r_outliers_tiles_size.restype = SZ
+        L.vq3r_pack_outliers.argtypes = [P, P, I64, I64, P, P]
         L.vq3r_selftest_wait_timeout.argtypes = [P]
         L.vq3r_selftest_wait_timeout.restype = I32
         for f in ("vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_rel_frobenius_error", "vq3r_device_error",
                   "vq3r_gemv_noalloc", "vq3r_pack_tiles", "vq3r_gemm", "vq3r_train", "vq4p_encode", "vq4p_decode",
                   "vq4p_rel_frobenius_error", "vq4p_train", "vq4p_gemv", "vq3r_outliers", "vq3r_decode_outliers",
-                  "vq3r_rel_frobenius_error_outliers", "vq3r_gemv_outliers"):
+                  "vq3r_rel_frobenius_error_outliers", "vq3r_gemv_outliers", "vq3r_gemv_with_outliers", "vq3r_pack_outliers"):
             getattr(L, f).restype = I32
         _L = L
     return _L
@@ -431,6 +435,55 @@ def vq3r_gemv_outliers(mats, B, stream=None):
     arr = _outlier_descs(mats)
     xdt = _DT[mats[0]["x"].dtype]
     _check(_lib().vq3r_gemv_outliers(arr, len(mats), B, xdt, _stream(stream)), "vq3r_gemv_outliers")
+    return [m["y"] for m in mats]
+
+
+class OutlierTiles(ctypes.Structure):
+    _fields_ = [("otiles", ctypes.c_void_p), ("k", ctypes.c_int64)]
+
+
+def vq3r_pack_outliers(ocols, ovals, out=None, stream=None):
+    """Outliers [rows][k] (from vq3r_outliers) -> the outlier-tile layout, an int32 tensor [ceil(rows/512)][k][512]
+    of column | value << 16 words."""
+    rows, k = ocols.shape
+    n_tiles = (rows + TILE_ROWS - 1) // TILE_ROWS
+    if out is None:
+        out = torch.empty((n_tiles, k, TILE_ROWS), dtype=torch.int32, device=ocols.device)
+    _check(_lib().vq3r_pack_outliers(_dev(ocols, "ocols"), _dev(ovals, "ovals"), rows, k, _dev(out, "out"),
+                                     _stream(stream)), "vq3r_pack_outliers")
+    return out
+
+
+def _outlier_tiles(mats):
+    """vq3r_outlier_tiles array: a dict's "otiles" (from vq3r_pack_outliers; its row0, a multiple of 512, picks the
+    first tile) or k = 0 where it has none."""
+    arr = (OutlierTiles * len(mats))()
+    for i, m in enumerate(mats):
+        ot = m.get("otiles")
+        if ot is None:
+            arr[i] = OutlierTiles(None, 0)
+            continue
+        if not (ot.is_cuda and ot.is_contiguous() and ot.dim() == 3):
+            raise ValueError("otiles must be a contiguous CUDA tensor from vq3r_pack_outliers")
+        r0 = m.get("row0", 0)
+        if r0 % TILE_ROWS:
+            raise ValueError("row0 of a matrix with outlier tiles must be a multiple of 512")
+        k = ot.shape[1]
+        arr[i] = OutlierTiles(ot.data_ptr() + (r0 // TILE_ROWS) * k * TILE_ROWS * 4, k)
+    return arr
+
+
+def vq3r_gemv_with_outliers(mats, B, workspace=None, stream=None):
+    """y = (W_hat + O) . x: vq3r_gemv's descriptor dicts, each optionally with "otiles" (the matrix's outliers
+    packed by vq3r_pack_outliers; with row0 / rows, rows of that larger matrix as for idx)."""
+    garr = _descs(mats)
+    oarr = _outlier_tiles(mats)
+    ws = _lib().vq3r_gemv_workspace_size(garr, len(mats), B)
+    if workspace is None:
+        workspace = torch.zeros(max(ws, 16), dtype=torch.uint8, device=mats[0]["idx"].device)
+    xdt = _DT[mats[0]["x"].dtype]
+    _check(_lib().vq3r_gemv_with_outliers(garr, oarr, len(mats), B, xdt, _dev(workspace, "workspace"),
+                                          workspace.numel(), _stream(stream)), "vq3r_gemv_with_outliers")
     return [m["y"] for m in mats]
 
 

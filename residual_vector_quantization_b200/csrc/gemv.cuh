@@ -78,6 +78,11 @@ struct GvMat {
   int32_t n_tiles;       // ceil(rows / kGvTileRows) >= 1
   int32_t tile_prefix;   // tiles of the earlier matrices of the same group
   int32_t blk_begin;     // first row block of this matrix in the tensor-core kernel's grid
+  // sparse outlier residual added by the tiled kernel (n_out = 0: none), in the outlier-tile layout
+  // (per 512-row tile and outlier number q, 512 words column | value << 16), n_out <= 3 * n_slabs
+  const uint32_t* otiles;
+  int32_t n_out;
+  int32_t pad_;
 };
 
 struct GvGroup {
@@ -107,6 +112,7 @@ struct GvParams {
   int32_t tokm;          // tokens per table token (1 or 2): table token b covers tokens tokm * b ..
   int32_t nst;           // table stages per slab: 3 (VQ3R, one table per stage), 1 (VQ4P, one table for all four)
   int64_t total_units;
+  int32_t has_out;       // some matrix has outliers (tiled kernel with OUTL)
   int32_t tile_rows;     // rows per work unit: kGvTileRows (planes) or kTileRows (tiles)
   int32_t layout;        // VQ3R_LAYOUT_PLANES or VQ3R_LAYOUT_TILES
   unsigned long long* hdr;  // workspace header: [0] arrival count at the start of the call, [1] arrival count
@@ -592,16 +598,18 @@ __device__ __forceinline__ void build_pieces_from(float* tab, const float* cb, c
 struct ZeroJob {
   float* y;
   int64_t lo, hi;
+  int m;  // the matrix
 };
 
 __device__ __forceinline__ ZeroJob zero_job(const GvParams& P, int j) {
   const int n_mats = P.n_mats, grid = (int)gridDim.x;
   const int parts = grid >= n_mats ? grid / n_mats : 1;
-  ZeroJob z = {nullptr, 0, 0};
+  ZeroJob z = {nullptr, 0, 0, 0};
   if (j < n_mats * parts) {
     const int m = j % n_mats, part = j / n_mats;
     const int64_t n = (int64_t)P.B * P.m[m].rows;
     z.y = P.m[m].y;
+    z.m = m;
     z.lo = n * part / parts;
     z.hi = n * (part + 1) / parts;
   }
@@ -614,6 +622,61 @@ __device__ __forceinline__ void zero_run(const ZeroJob& z, int tid) {
 
 __device__ __forceinline__ void zero_rest(const GvParams& P, int tid) {
   for (int j = blockIdx.x + gridDim.x; j < P.n_mats; j += gridDim.x) zero_run(zero_job(P, j), tid);
+}
+
+// Outliers (OUTL): instead of zero, y[b][i] starts as its row's outlier sum
+// sum_q (float)o_iq * x[b][c_iq] (binary32, q ascending), written by the CTA
+// that would zero it before the grid barrier; the lookup units then add into
+// it, and the lookup loop is that of the kernel without outliers.  Eight
+// words are loaded before their x values are gathered.  The words come from
+// the outlier tiles (a warp's words of one q for consecutive rows are
+// contiguous).  On the 8-expert decode step (14 or 4 outliers per row) this
+// costs 1.16x the step without outliers; measured and slower: the same sums
+// added after the CTA's last unit (1.22x, also with x staged in shared
+// memory, the words prefetched into L2 and the code warmed before
+// griddepcontrol.wait), one outlier per row in each lookup unit (1.25x), per
+// warp chunks between units (2.4x), a second launch (1.29x).
+template <int XDT>
+__device__ __forceinline__ void outlier_init_run(const GvParams& P, const ZeroJob& z, int tid) {
+  const GvMat& M = P.m[z.m];
+  const int k = M.n_out;
+  if (k == 0) {
+    zero_run(z, tid);
+    return;
+  }
+  const GvGroup& G = P.g[M.group];
+  for (int64_t i = z.lo + tid; i < z.hi; i += kGvThreads) {
+    const int64_t b = i / M.rows, row = i - b * M.rows;
+    const uint32_t* p = M.otiles + (row / kTileRows) * k * kTileRows + row % kTileRows;
+    float acc = 0.0f;
+    for (int q0 = 0; q0 < k; q0 += 8) {
+      uint32_t w8[8];
+#pragma unroll
+      for (int u = 0; u < 8; u++) w8[u] = q0 + u < k ? __ldg(p + (int64_t)(q0 + u) * kTileRows) : 0xFFFFFFFFu;
+      float x8[8];
+#pragma unroll
+      for (int u = 0; u < 8; u++) {
+        const int64_t c = w8[u] & 0xFFFFu;
+        x8[u] = c < G.cols ? load1<XDT>(G.x, b * G.cols + c) : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; u++)
+        if ((int64_t)(w8[u] & 0xFFFFu) < G.cols) acc = fmaf(f16_bits_to_f32((uint16_t)(w8[u] >> 16)), x8[u], acc);
+    }
+    z.y[i] = acc;
+  }
+}
+
+// The CTA's share of y: zeros, or with OUTL the outlier sums.
+template <int XDT, bool OUTL>
+__device__ __forceinline__ void init_y(const GvParams& P, const ZeroJob& zj, int tid) {
+  if (OUTL && P.has_out) {
+    if (zj.y) outlier_init_run<XDT>(P, zj, tid);
+    for (int j = blockIdx.x + gridDim.x; j < P.n_mats; j += gridDim.x) outlier_init_run<XDT>(P, zero_job(P, j), tid);
+  } else {
+    zero_run(zj, tid);
+    zero_rest(P, tid);
+  }
 }
 
 struct Arrival {
@@ -758,7 +821,7 @@ __device__ __forceinline__ float rows_exchange(const float (&acc)[4], bool hi2, 
 // FMT = FMT_VQ4P: a slab has one table (the four stages' 64 codewords seen as
 // 256 rows, built exactly as a VQ3R stage table), a unit reads the three
 // byte planes of its (slab, tile) and makes four lookups per vector.
-template <int XDT, int NSLOT, int TOKS, int FMT = FMT_VQ3R>
+template <int XDT, int NSLOT, int TOKS, int FMT = FMT_VQ3R, bool OUTL = false>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_constant__ GvParams P) {
   constexpr int PL = FMT == FMT_VQ4P ? 3 : 1;  // byte planes read per unit
   extern __shared__ __align__(128) unsigned char gv_smem[];
@@ -802,8 +865,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
   const ZeroJob zj = zero_job(P, blockIdx.x);
   if (u0 >= u1) {  // no units: only the share of y to zero
     griddep_wait();
-    zero_run(zj, tid);
-    zero_rest(P, tid);
+    init_y<XDT, OUTL>(P, zj, tid);
     __syncthreads();
     if (tid == 0) barrier_close(P.hdr, barrier_arrive(P.hdr));  // adds nothing, so it need not wait
     return;
@@ -841,8 +903,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_tiles_kernel(const __grid_
     stage_src(src0, S, 0);
     if (key_next != kNoTable) stage_src(src1, S, 1);
   }
-  zero_run(zj, tid);
-  zero_rest(P, tid);
+  init_y<XDT, OUTL>(P, zj, tid);
   __syncthreads();  // the CTA's zeros precede its count
   Arrival arrival = {0ull, 0ull};
   if (tid == 0) arrival = barrier_arrive(P.hdr);

@@ -260,4 +260,64 @@ __global__ void __launch_bounds__(256) outlier_gemv_kernel(const __grid_constant
   }
 }
 
+// Outlier tiles: per 512-row tile t of a matrix and outlier number q, 512
+// words ocols[512 t + r][q] | ovals[512 t + r][q] << 16 (r = 0..511; rows past
+// the end hold kNoOutlierWord), so that the q-th outliers of a tile's rows are
+// one contiguous 2 KiB block.  One thread per output word.
+constexpr int kOutTileRows = 512;
+constexpr uint32_t kNoOutlierWord = 0xFFFFFFFFu;  // column field 0xFFFF: no column (cols <= 16384)
+
+__global__ void __launch_bounds__(256) pack_outliers_kernel(const uint16_t* __restrict__ ocols,
+                                                            const uint16_t* __restrict__ ovals, int64_t rows,
+                                                            int64_t k, int64_t n_tiles, uint32_t* __restrict__ out) {
+  const int64_t n = n_tiles * k * kOutTileRows;
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n; t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = t % kOutTileRows, tq = t / kOutTileRows;
+    const int64_t tile = tq / k, q = tq - tile * k;
+    const int64_t row = tile * kOutTileRows + r;
+    out[t] = row < rows ? (uint32_t)__ldg(ocols + row * k + q) | ((uint32_t)__ldg(ovals + row * k + q) << 16)
+                        : kNoOutlierWord;
+  }
+}
+
+// Grouped sparse add over outlier tiles (the calls the tiled GEMV does not
+// fuse): one thread per row, y[b][i] += sum_q (float)o_iq * x[b][c_iq] in
+// binary32, q ascending; a warp's reads of one q are 128 contiguous bytes.
+struct OutTilesParams {
+  const uint32_t* ot[kOutGemvMaxMats];
+  const void* x[kOutGemvMaxMats];
+  float* y[kOutGemvMaxMats];
+  int64_t rows[kOutGemvMaxMats], k[kOutGemvMaxMats], cols[kOutGemvMaxMats];
+  int64_t row_begin[kOutGemvMaxMats + 1];
+  int n_mats, B;
+};
+
+template <int XDT>
+__global__ void __launch_bounds__(256) outlier_tiles_add_kernel(const __grid_constant__ OutTilesParams P) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= P.row_begin[P.n_mats]) return;
+  int m = 0;
+  while (t >= P.row_begin[m + 1]) m++;
+  const int64_t i = t - P.row_begin[m], k = P.k[m], cols = P.cols[m], rows = P.rows[m];
+  const uint32_t* p = P.ot[m] + (i / kOutTileRows) * k * kOutTileRows + i % kOutTileRows;
+  for (int b = 0; b < P.B; b++) {
+    float acc = 0.0f;
+    for (int64_t q0 = 0; q0 < k; q0 += 8) {
+      uint32_t w8[8];
+#pragma unroll
+      for (int u = 0; u < 8; u++) w8[u] = q0 + u < k ? __ldg(p + (q0 + u) * kOutTileRows) : kNoOutlierWord;
+      float x8[8];
+#pragma unroll
+      for (int u = 0; u < 8; u++) {
+        const int64_t c = w8[u] & 0xFFFFu;
+        x8[u] = c < cols ? load1<XDT>(P.x[m], (int64_t)b * cols + c) : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; u++)
+        if ((w8[u] & 0xFFFFu) < cols) acc = fmaf(f16_bits_to_f32((uint16_t)(w8[u] >> 16)), x8[u], acc);
+    }
+    P.y[m][(int64_t)b * rows + i] += acc;
+  }
+}
+
 }  // namespace vq3r

@@ -51,6 +51,8 @@ int g_dev_sms[kMaxDevices];
 bool g_dev_tiles_fit[kMaxDevices];
 bool g_dev_tc_fit[kMaxDevices];  // the same for the tensor-core GEMV (one persistent CTA per SM, grid barrier)
 
+constexpr int kNumTilesKernels = 18;  // instantiations of gemv_tiles_kernel (occupancy-checked together)
+
 cudaError_t device_setup(int* sms) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -75,7 +77,7 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(gemv_lut_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv);
-    const void* tiles_kernels[12] = {
+    const void* tiles_kernels[kNumTilesKernels] = {
         reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 1>),
         reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 1>),
         reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 1>),
@@ -87,8 +89,14 @@ cudaError_t device_setup(int* sms) {
         reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, 1, 1, FMT_VQ4P>),
         reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, 1, 2, FMT_VQ4P>),
         reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, 1, 2, FMT_VQ4P>),
-        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, 1, 2, FMT_VQ4P>)};
-    for (int k = 0; k < 12 && r == cudaSuccess; k++)
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, 1, 2, FMT_VQ4P>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 1, FMT_VQ3R, true>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 1, FMT_VQ3R, true>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 1, FMT_VQ3R, true>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F32, kTileSlots, 2, FMT_VQ3R, true>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_BF16, kTileSlots, 2, FMT_VQ3R, true>),
+        reinterpret_cast<const void*>(gemv_tiles_kernel<VQ3R_F16, kTileSlots, 2, FMT_VQ3R, true>)};
+    for (int k = 0; k < kNumTilesKernels && r == cudaSuccess; k++)
       r = cudaFuncSetAttribute(tiles_kernels[k], cudaFuncAttributeMaxDynamicSharedMemorySize, gt);
     const int gm = (int)kMmaSmemBytes;
     const int gc = (int)(kCbrFloats * sizeof(float));
@@ -117,7 +125,7 @@ cudaError_t device_setup(int* sms) {
     if (r == cudaSuccess) r = cudaFuncSetAttribute(outlier_select_kernel<VQ3R_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, go);
     if (r != cudaSuccess) return r;
     int fit = 1;
-    for (int k = 0; k < 12 && r == cudaSuccess; k++) {
+    for (int k = 0; k < kNumTilesKernels && r == cudaSuccess; k++) {
       int n = 0;
       r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, tiles_kernels[k], kGvThreads, gt);
       if (n < 1) fit = 0;
@@ -153,9 +161,10 @@ struct GemvPlan {
 // matrices contiguous in P.m); empty matrices are dropped.
 // tokm: tokens per table token (2 for the tiled kernel's two-token tables, else 1).
 // nst: table stages per slab, 3 for VQ3R, 1 for VQ4P (its four 64-codeword
-// stages share one 256-entry table).
+// stages share one 256-entry table).  outl (tiled kernel only, may be null):
+// the matrices' sparse outlier residuals, whose sums start y.
 vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, int tokm, char* ws_base, GemvPlan* plan,
-                      int nst = kStages) {
+                      int nst = kStages, const vq3r_outlier_tiles* outl = nullptr) {
   GvParams& P = plan->P;
   memset(&P, 0, sizeof(P));
   P.B = B;
@@ -213,6 +222,8 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, int tokm, c
                                       : (tiles ? (d.rows + kTileRows - 1) / kTileRows * kTileBytes
                                                : d.rows * (d.cols / kDim));
       M.group = g;
+      M.otiles = outl ? outl[i].otiles : nullptr;
+      M.n_out = outl ? (int32_t)outl[i].k : 0;
       M.n_tiles = (int32_t)((d.rows + P.tile_rows - 1) / P.tile_rows);
       M.tile_prefix = P.g[g].tiles;
       P.g[g].tiles += M.n_tiles;
@@ -239,6 +250,7 @@ vq3r_status plan_gemv(const vq3r_gemv_desc* mats, int n_mats, int B, int tokm, c
     if (!tiles) off = align_up(off + (size_t)B * kStages * P.g[M.group].n_slabs * (size_t)M.rows * sizeof(float));
   }
   P.total_units = units;
+  for (int i = 0; i < nm; i++) P.has_out |= P.m[i].n_out > 0;
   plan->ws_bytes = off;
   return VQ3R_OK;
 }
@@ -314,7 +326,7 @@ void balance_split(GvParams& P, int n) {
 // would guarantee it but measured 3.8 us slower per call (it gives up most of
 // the programmatic-launch overlap), so the grid is sized to one CTA per SM
 // and the fit of one CTA per SM is checked instead.
-template <int FMT, int NSLOT>
+template <int FMT, int NSLOT, bool OUTL = false>
 vq3r_status launch_tiles(GemvPlan& plan, vq3r_dtype x_dtype, int sms, cudaLaunchConfig_t& cfg) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -328,15 +340,15 @@ vq3r_status launch_tiles(GemvPlan& plan, vq3r_dtype x_dtype, int sms, cudaLaunch
   cfg.dynamicSmemBytes = kTilesSmemBytes;
   if (P.tokm == 2) {
     switch (x_dtype) {
-      case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, NSLOT, 2, FMT>, P); break;
-      case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, NSLOT, 2, FMT>, P); break;
-      default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, NSLOT, 2, FMT>, P); break;
+      case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, NSLOT, 2, FMT, OUTL>, P); break;
+      case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, NSLOT, 2, FMT, OUTL>, P); break;
+      default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, NSLOT, 2, FMT, OUTL>, P); break;
     }
   } else {
     switch (x_dtype) {
-      case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, NSLOT, 1, FMT>, P); break;
-      case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, NSLOT, 1, FMT>, P); break;
-      default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, NSLOT, 1, FMT>, P); break;
+      case VQ3R_F32: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F32, NSLOT, 1, FMT, OUTL>, P); break;
+      case VQ3R_BF16: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_BF16, NSLOT, 1, FMT, OUTL>, P); break;
+      default: e = cudaLaunchKernelEx(&cfg, gemv_tiles_kernel<VQ3R_F16, NSLOT, 1, FMT, OUTL>, P); break;
     }
   }
   if (e != cudaSuccess) return cuda_fail(e);
@@ -933,6 +945,99 @@ vq3r_status vq3r_gemv_outliers(const vq3r_outlier_desc* mats, int n_mats, int B,
     default: outlier_gemv_kernel<VQ3R_F16><<<(int)grid, 256, 0, s>>>(P);
   }
   return check_launch();
+}
+
+size_t vq3r_outliers_tiles_size(int64_t rows, int64_t k) {
+  if (rows < 0 || k < 0 || k > kOutMaxCols) return 0;
+  return (size_t)((rows + kOutTileRows - 1) / kOutTileRows) * (size_t)k * kOutTileRows * 4;
+}
+
+vq3r_status vq3r_pack_outliers(const uint16_t* ocols, const uint16_t* ovals, int64_t rows, int64_t k, uint32_t* otiles,
+                               vq3r_stream stream) {
+  if (rows < 0 || k < 0 || k > kOutMaxCols) return VQ3R_ERR_SHAPE;
+  if (rows == 0 || k == 0) return VQ3R_OK;
+  if (!ocols || !ovals || !otiles) return VQ3R_ERR_NULL;
+  if (!aligned16(otiles)) return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int64_t n_tiles = (rows + kOutTileRows - 1) / kOutTileRows;
+  const int64_t n = n_tiles * k * kOutTileRows;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+  pack_outliers_kernel<<<(int)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(ocols, ovals, rows, k, n_tiles,
+                                                                                     otiles);
+  return check_launch();
+}
+
+vq3r_status vq3r_gemv_with_outliers(const vq3r_gemv_desc* mats, const vq3r_outlier_tiles* outl, int n_mats, int B,
+                                    vq3r_dtype x_dtype, void* workspace, size_t ws_bytes, vq3r_stream stream) {
+  if (!mats || !outl) return VQ3R_ERR_NULL;
+  if (n_mats < 1 || n_mats > VQ3R_GEMV_MAX_MATS || B < 1 || B > VQ3R_GEMV_MAX_B) return VQ3R_ERR_BATCH;
+  if (!valid_dtype(x_dtype)) return VQ3R_ERR_DTYPE;
+  bool any = false;
+  for (int i = 0; i < n_mats; i++) {
+    const vq3r_outlier_tiles& o = outl[i];
+    const vq3r_gemv_desc& d = mats[i];
+    if (o.k < 0 || o.k > d.cols || (o.k > 0 && d.cols > kOutMaxCols)) return VQ3R_ERR_SHAPE;
+    if (d.rows <= 0 || o.k == 0) continue;
+    if (!o.otiles) return VQ3R_ERR_NULL;
+    if (!aligned16(o.otiles)) return VQ3R_ERR_ALIGN;
+    any = true;
+  }
+  // The lookup-table kernel starts y at the outliers' sums instead of zero
+  // (before its grid barrier); the other kernels are followed by a separate
+  // sparse add over the outlier tiles.
+  const bool fused = mats[0].layout == VQ3R_LAYOUT_TILES && (x_dtype != VQ3R_BF16 || B < kMmaMinB);
+  if (!fused || !any) {
+    vq3r_status st = vq3r_gemv(mats, n_mats, B, x_dtype, workspace, ws_bytes, stream);
+    if (st != VQ3R_OK || !any) return st;
+    OutTilesParams Q;
+    memset(&Q, 0, sizeof(Q));
+    int m = 0;
+    int64_t total = 0;
+    for (int i = 0; i < n_mats; i++) {
+      if (mats[i].rows <= 0 || outl[i].k == 0) continue;
+      Q.ot[m] = outl[i].otiles;
+      Q.x[m] = mats[i].x;
+      Q.y[m] = mats[i].y;
+      Q.rows[m] = mats[i].rows;
+      Q.k[m] = outl[i].k;
+      Q.cols[m] = mats[i].cols;
+      Q.row_begin[m] = total;
+      total += mats[i].rows;
+      m++;
+    }
+    Q.row_begin[m] = total;
+    Q.n_mats = m;
+    Q.B = B;
+    const int64_t grid = (total + 255) / 256;
+    if (grid > INT32_MAX) return VQ3R_ERR_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (x_dtype) {
+      case VQ3R_F32: outlier_tiles_add_kernel<VQ3R_F32><<<(int)grid, 256, 0, s>>>(Q); break;
+      case VQ3R_BF16: outlier_tiles_add_kernel<VQ3R_BF16><<<(int)grid, 256, 0, s>>>(Q); break;
+      default: outlier_tiles_add_kernel<VQ3R_F16><<<(int)grid, 256, 0, s>>>(Q);
+    }
+    return check_launch();
+  }
+  GemvPlan plan;
+  vq3r_status st = plan_gemv(mats, n_mats, B, B >= 2 ? 2 : 1, static_cast<char*>(workspace), &plan, kStages, outl);
+  if (st != VQ3R_OK) return st;
+  if (plan.P.total_units == 0) return VQ3R_OK;
+  if (!workspace || ws_bytes < plan.ws_bytes) return VQ3R_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return VQ3R_ERR_ALIGN;
+  int sms = 0;
+  cudaError_t e = device_setup(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return launch_tiles<FMT_VQ3R, kTileSlots, true>(plan, x_dtype, sms, cfg);
 }
 
 }  // extern "C"

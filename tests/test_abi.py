@@ -251,3 +251,31 @@ def test_outlier_descriptor_and_budget_checks(lib):
 def test_selftest_symbol_is_exported(lib):
     assert hasattr(lib, "vq3r_selftest_wait_timeout")
     assert "vq3r_selftest_wait_timeout" in vq.EXPORTED
+
+
+def test_gemv_with_outliers_argument_checks(lib):
+    arr = _descs([(2048, 7168, 0x10000, 0x20000)])
+    ot = (vq.OutlierTiles * 1)()
+    ot[0] = vq.OutlierTiles(0x30000, 14)
+    assert lib.vq3r_gemv_with_outliers(arr, None, 1, 1, 1, 0x500000, 1 << 30, None) == 1
+    assert lib.vq3r_gemv_with_outliers(arr, ot, 1, 0, 1, 0x500000, 1 << 30, None) == 5
+    assert lib.vq3r_gemv_with_outliers(arr, ot, 1, 1, 9, 0x500000, 1 << 30, None) == 4
+    ot[0].k = 7169  # more outliers than columns
+    assert lib.vq3r_gemv_with_outliers(arr, ot, 1, 1, 1, 0x500000, 1 << 30, None) == 2
+    ot[0].k = -1
+    assert lib.vq3r_gemv_with_outliers(arr, ot, 1, 1, 1, 0x500000, 1 << 30, None) == 2
+    ot[0].k = 14
+    ot[0].otiles = 0x30004
+    assert lib.vq3r_gemv_with_outliers(arr, ot, 1, 1, 1, 0x500000, 1 << 30, None) == 3
+    ot[0].otiles = None
+    assert lib.vq3r_gemv_with_outliers(arr, ot, 1, 1, 1, 0x500000, 1 << 30, None) == 1
+    ot[0].otiles = 0x30000
+    arr[0].layout = 1
+    assert lib.vq3r_gemv_with_outliers(arr, ot, 1, 1, 1, None, 0, None) == 7
+    assert lib.vq3r_outliers_tiles_size(2048, 14) == 4 * 14 * 2048
+    assert lib.vq3r_outliers_tiles_size(513, 3) == 2 * 3 * 2048
+    assert lib.vq3r_outliers_tiles_size(5, 16385) == 0
+    assert lib.vq3r_pack_outliers(None, 0x100000, 4, 2, 0x200000, None) == 1
+    assert lib.vq3r_pack_outliers(0x100000, 0x100000, 4, 2, 0x200008, None) == 3
+    assert lib.vq3r_pack_outliers(0x100000, 0x100000, 4, -1, 0x200000, None) == 2
+    assert lib.vq3r_pack_outliers(None, None, 0, 2, None, None) == 0

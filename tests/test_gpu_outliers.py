@@ -170,3 +170,115 @@ def test_layer_stacked_outliers_sampled_rows():
     del d
     e = float(vq.vq3r_rel_frobenius_error_outliers(W_t, idx_t, sc_t, cb_t, oc_t, ov_t).cpu()[0])
     assert abs(e - e2) <= 1e-9 * e2
+
+
+def _random_outliers(rng, rows, cols, k):
+    """k distinct ascending columns per row and binary16 values (as vq3r_outliers lays them out)."""
+    oc = np.zeros((rows, k), dtype=np.uint16)
+    for i in range(rows):
+        oc[i] = np.sort(rng.choice(cols, k, replace=False))
+    ov = np.float16(rng.standard_normal((rows, k)) * 0.3).view(np.uint16)
+    return oc, ov
+
+
+@pytest.mark.parametrize("B,x_dtype,layout,per512", [(1, "bf16", "tiles", 3), (2, "bf16", "tiles", 3),
+                                                     (5, "f32", "tiles", 1), (1, "f16", "tiles", 2),
+                                                     (1, "bf16", "tiles", 4), (12, "bf16", "tiles", 3),
+                                                     (3, "bf16", "planes", 3)])
+def test_gemv_with_outliers_one_call(B, x_dtype, layout, per512):
+    """vq3r_gemv_with_outliers over mixed matrices: several 512-row tiles with a ragged last one, a matrix
+    without outliers between two with, a ragged last slab, two inputs x, up to per512 outliers per 512 columns.
+    The lookup-table kernel starts y at the outliers' sums (tiles, B <= 10 or non-bf16 x); bf16 B = 12 and the
+    plane layout take the two-launch path.  Against the oracle's binary64 product of the decoded weights with the
+    outliers applied."""
+    rng = np.random.default_rng(500 + B + per512)
+    cb = random_codebooks(41)
+    cb_t = torch.from_numpy(cb).to(DEV)
+    p = per512
+    specs = [(1030, 1024, 0, 2 * p), (300, 1024, 0, 0), (513, 2048, 1, 4 * p), (64, 1032, 1, 3 * p - 2)]
+    xs = {}
+    mats, refs = [], []
+    for rows, cols, xk, k in specs:
+        if (xk, cols) not in xs:
+            xf = rng.standard_normal((B, cols)).astype(np.float32)
+            xs[(xk, cols)] = (xf if x_dtype == "f32" else f32_to_bf16_bits(xf) if x_dtype == "bf16"
+                              else xf.astype(np.float16).view(np.uint16))
+        idx = rng.integers(0, 256, size=(3, rows, cols // 8), dtype=np.uint8)
+        sc = np.float16(np.exp(rng.standard_normal(rows) * 0.5)).view(np.uint16)
+        What = oracle.decode(idx, sc, cb)
+        m = dict(idx=torch.from_numpy(idx).to(DEV), scales=torch.from_numpy(sc.view(np.int16)).to(DEV),
+                 codebooks=cb_t, x=(xk, cols), y=torch.full((B, rows), float("nan"), device=DEV))
+        if k:
+            oc, ov = _random_outliers(rng, rows, cols, k)
+            What = oracle.outliers_apply(What, oc, ov)
+            m["otiles"] = vq.vq3r_pack_outliers(torch.from_numpy(oc.view(np.int16)).to(DEV),
+                                                torch.from_numpy(ov.view(np.int16)).to(DEV))
+        if layout == "tiles":
+            m.update(idx=vq.vq3r_pack_tiles(m["idx"]), layout="tiles", cols=cols)
+        refs.append(oracle.gemv(What, xs[(xk, cols)], x_dtype))
+        mats.append(m)
+    xdev = {kk: to_dev(v, x_dtype) for kk, v in xs.items()}
+    for m in mats:
+        m["x"] = xdev[m["x"]]
+    vq.vq3r_gemv_with_outliers(mats, B)
+    for m, ref in zip(mats, refs):
+        y = m["y"].cpu().numpy()
+        assert np.isfinite(y).all()
+        assert gemv_rel_err(y, ref) <= GEMV_TOL
+    assert vq.vq3r_device_error() == 0
+
+
+def test_gemv_with_outliers_moe_decode_step_sampled_rows():
+    """The 8-expert MoE decode step (24 matrices, B = 1, cols/512 outliers per row) in one call against the
+    oracle on 32 sampled rows of every matrix.  Outlier columns: one per 512-column stretch of the row."""
+    rng = np.random.default_rng(77)
+    cb = random_codebooks(43)
+    cb_t = torch.from_numpy(cb).to(DEV)
+    B = 1
+    x1 = f32_to_bf16_bits(rng.standard_normal((B, 7168)).astype(np.float32))
+    x1_t = to_dev(x1, "bf16")
+    mats, hosts = [], []
+    for e in range(8):
+        x2 = f32_to_bf16_bits(rng.standard_normal((B, 2048)).astype(np.float32))
+        x2_t = to_dev(x2, "bf16")
+        for rows, cols, x_t, x in ((2048, 7168, x1_t, x1), (2048, 7168, x1_t, x1), (7168, 2048, x2_t, x2)):
+            idx_t = torch.randint(0, 256, (3, rows, cols // 8), dtype=torch.uint8, device=DEV)
+            sc = np.float16(np.exp(rng.standard_normal(rows) * 0.5)).view(np.uint16)
+            k = cols // 512
+            oc = (rng.integers(0, 512, size=(rows, k)) + 512 * np.arange(k)).astype(np.uint16)
+            ov = np.float16(rng.standard_normal((rows, k))).view(np.uint16)
+            m = dict(idx=vq.vq3r_pack_tiles(idx_t), layout="tiles", cols=cols,
+                     scales=torch.from_numpy(sc.view(np.int16)).to(DEV), codebooks=cb_t, x=x_t,
+                     y=torch.empty((B, rows), device=DEV),
+                     otiles=vq.vq3r_pack_outliers(torch.from_numpy(oc.view(np.int16)).to(DEV),
+                                                  torch.from_numpy(ov.view(np.int16)).to(DEV)))
+            mats.append(m)
+            hosts.append((idx_t, sc, oc, ov, x))
+    vq.vq3r_gemv_with_outliers(mats, B)
+    torch.cuda.synchronize()
+    for m, (idx_t, sc, oc, ov, x) in zip(mats, hosts):
+        rows = sc.shape[0]
+        sample = np.sort(rng.choice(rows, 32, replace=False))
+        idx = idx_t[:, torch.from_numpy(sample).to(DEV), :].cpu().numpy()
+        What = oracle.outliers_apply(oracle.decode(idx, sc[sample], cb), oc[sample], ov[sample])
+        ref = oracle.gemv(What, x, "bf16")
+        assert gemv_rel_err(m["y"][:, torch.from_numpy(sample).to(DEV)].cpu().numpy(), ref) <= GEMV_TOL
+    assert vq.vq3r_device_error() == 0
+
+
+@pytest.mark.parametrize("rows,k", [(1, 1), (511, 3), (512, 14), (1300, 5)])
+def test_pack_outliers_layout(rows, k):
+    """The outlier-tile layout written out from its definition: word (t, q, r) = ocols[512 t + r][q] |
+    ovals[512 t + r][q] << 16, all ones past the last row."""
+    rng = np.random.default_rng(rows + k)
+    oc = rng.integers(0, 16384, size=(rows, k)).astype(np.uint16)
+    ov = rng.integers(0, 65536, size=(rows, k)).astype(np.uint16)
+    got = vq.vq3r_pack_outliers(torch.from_numpy(oc.view(np.int16)).to(DEV),
+                                torch.from_numpy(ov.view(np.int16)).to(DEV)).cpu().numpy().view(np.uint32)
+    n_tiles = (rows + 511) // 512
+    want = np.full((n_tiles, k, 512), 0xFFFFFFFF, dtype=np.uint32)
+    for i in range(rows):
+        for q in range(k):
+            want[i // 512, q, i % 512] = int(oc[i, q]) | (int(ov[i, q]) << 16)
+    np.testing.assert_array_equal(got, want)
+    assert vq.lib().vq3r_outliers_tiles_size(rows, k) == got.nbytes
