@@ -238,7 +238,10 @@ class Layer:
 
     def encode(self):
         for k in self.kinds:
-            self.vq.vq3r_encode(self.W[k], self.cb, self.idx[k], self.sc[k])
+            self.encode_kind(k)
+
+    def encode_kind(self, k):
+        self.vq.vq3r_encode(self.W[k], self.cb, self.idx[k], self.sc[k])
 
     def pack(self):
         for k in self.kinds:
@@ -937,8 +940,10 @@ def main():
 
     # end to end through the public API with host buffers: every step uploads the layer from pinned host memory
     # and reads its results back (indices, scales, errors, y).  The device inputs and index outputs are double
-    # buffered, so step i + 1's upload (its own copy stream) and step i's index read-back (a third stream) overlap
-    # step i's compute; every copy still lies between the start and end events.
+    # buffered and the copies are pipelined per matrix kind: a kind's encode starts once its weights have arrived
+    # (upload on its own stream) and its indices are read back as soon as it is encoded (a third stream), so the
+    # copies overlap the compute of the same and the neighbouring steps; every copy lies between the start and
+    # end events.
     e2e = None
     if args.e2e_steps > 0:
         hostW = {k: torch.empty(layer.W[k].shape, dtype=layer.W[k].dtype, pin_memory=True) for k in layer.kinds}
@@ -957,7 +962,9 @@ def main():
         s_comp = torch.cuda.current_stream()
         s_up, s_down = torch.cuda.Stream(), torch.cuda.Stream()
         K = args.e2e_steps
-        ev_up = [ev() for _ in range(K)]
+        nk = len(layer.kinds)
+        ev_up = [[ev() for _ in range(nk)] for _ in range(K)]
+        ev_enc = [[ev() for _ in range(nk)] for _ in range(K)]
         ev_comp = [ev() for _ in range(K)]
         ev_down = [ev() for _ in range(K)]
         barrier()
@@ -969,14 +976,27 @@ def main():
                 s_up.wait_event(a)
                 if i >= 2:
                     s_up.wait_event(ev_comp[i - 2])  # step i - 2 has finished with this input buffer
-                for k in layer.kinds:
+                for j, k in enumerate(layer.kinds):
                     Wbuf[bi][k].copy_(hostW[k], non_blocking=True)
-                ev_up[i].record(s_up)
-            s_comp.wait_event(ev_up[i])
+                    ev_up[i][j].record(s_up)
             if i >= 2:
                 s_comp.wait_event(ev_down[i - 2])  # step i - 2's indices have been read back
             layer.W, layer.idx = Wbuf[bi], Ibuf[bi]
-            step(i)
+            # the step (as in the timed loop), each kind's encode once its weights are on the device and its
+            # index read-back once it is encoded
+            for j, k in enumerate(layer.kinds):
+                s_comp.wait_event(ev_up[i][j])
+                layer.encode_kind(k)
+                ev_enc[i][j].record(s_comp)
+                with torch.cuda.stream(s_down):
+                    s_down.wait_event(ev_enc[i][j])
+                    hostI[k].copy_(Ibuf[bi][k], non_blocking=True)
+            with torch.cuda.stream(s_down):
+                ev_down[i].record(s_down)
+            layer.pack()
+            layer.decode()
+            layer.errors()
+            layer.gemv(1, i)
             for k in layer.kinds:
                 hostS[k].copy_(layer.sc[k], non_blocking=True)
             for j, k in enumerate(layer.kinds):
@@ -988,20 +1008,16 @@ def main():
                 hostY[off:off + n].copy_(m["y"].view(-1), non_blocking=True)
                 off += n
             ev_comp[i].record(s_comp)
-            with torch.cuda.stream(s_down):
-                s_down.wait_event(ev_comp[i])
-                for k in layer.kinds:
-                    hostI[k].copy_(Ibuf[bi][k], non_blocking=True)
-                ev_down[i].record(s_down)
         s_comp.wait_event(ev_down[K - 1])
-        s_comp.wait_event(ev_up[K - 1])
+        s_comp.wait_event(ev_up[K - 1][nk - 1])
         b.record(s_comp)
         torch.cuda.synchronize()
         layer.W, layer.idx = W0, I0
         e2e_ms = max_over_ranks(torch, a.elapsed_time(b) / K, world, dev)
         e2e = {"value": whole_job_rate(world, layer.weights, e2e_ms), "unit": "Gweights/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": K,
-               "overlap": "uploads and index read-backs on their own streams, double-buffered device buffers"}
+               "overlap": "uploads and index read-backs on their own streams, pipelined per matrix kind, "
+                          "double-buffered device buffers"}
         del Wbuf, Ibuf
 
     errs = {str(k): float(layer.err[k].item()) for k in layer.kinds}
