@@ -46,7 +46,7 @@ ALU_LANES_PER_SM = 64
 # DRAM bytes (read + write) per weight of the encode kernel: dram__bytes_read.sum + dram__bytes_write.sum of the
 # ncu capture in profiles/encode_kernel_moe-layer-8-experts.md (117.4 M weights).  Set to None when the encode
 # kernel changes, until it is captured again.
-ENCODE_DRAM_BYTES_PER_WEIGHT = (235268096 + 8084736) / 117440512
+ENCODE_DRAM_BYTES_PER_WEIGHT = (235115264 + 8597760) / 117440512
 SM_COUNT_NOMINAL = 148
 FP32_LANES_PER_SM = 128
 

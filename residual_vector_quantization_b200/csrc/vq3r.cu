@@ -361,7 +361,7 @@ vq3r_status launch_encode(const void* W, int64_t rows, int64_t cols, const float
   const int64_t nvec = rows * (cols / kDim);
   const int g1 = (int)(rows < (int64_t)sms * 16 ? rows : (int64_t)sms * 16);
   row_scale_kernel<DT><<<g1, kScaleThreads, 0, s>>>(W, rows, cols, scales);
-  const int64_t ntiles = (nvec + kEncTile - 1) / kEncTile;
+  const int64_t ntiles = (nvec + enc_tile<FMT>() - 1) / enc_tile<FMT>();
   const int g2 = (int)(ntiles < (int64_t)sms * 2 ? ntiles : (int64_t)sms * 2);
   encode_kernel<DT, FMT><<<g2, kEncThreads, sizeof(EncSmem), s>>>(W, cols, nvec, cb, scales, idx, 0.0f);
   return check_launch();
