@@ -79,7 +79,7 @@ struct GvMat {
   int32_t tile_prefix;   // tiles of the earlier matrices of the same group
   int32_t blk_begin;     // first row block of this matrix in the tensor-core kernel's grid
   // sparse outlier residual added by the tiled kernel (n_out = 0: none), in the outlier-tile layout
-  // (per 512-row tile and outlier number q, 512 words column | value << 16), n_out <= 3 * n_slabs
+  // (per 512-row tile and outlier number q, 512 words column | value << 16)
   const uint32_t* otiles;
   int32_t n_out;
   int32_t pad_;
