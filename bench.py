@@ -58,7 +58,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="vq3r", choices=["vq3r", "reference"])
     ap.add_argument("--experts", type=int, default=64)
-    ap.add_argument("--gemv-iters", type=int, default=40)
+    ap.add_argument("--gemv-iters", type=int, default=200)
     ap.add_argument("--gemm-iters", type=int, default=10,
                     help="timed calls of the prefill product (8 experts' w1, 512 tokens each); 0 skips it")
     ap.add_argument("--e2e-steps", type=int, default=4)
@@ -233,6 +233,7 @@ class Layer:
             wsz = max(p[3] for p in plans)
             ws = torch.zeros(wsz, dtype=torch.uint8, device=dev)
             self.moe[B] = (plans, ws, xu, xd)
+        self._gemv_calls = {}
 
     # --- the parts of a step (each enqueues on the current stream) ---
 
@@ -257,12 +258,24 @@ class Layer:
                                              workspace=self.err_ws[k])
 
     def gemv(self, B, group):
-        plans, ws, _, _ = self.moe[B]
-        d, n = plans[group % len(plans)][:2]
-        L, s = self.vq.lib(), self.torch.cuda.current_stream().cuda_stream
-        st = L.vq3r_gemv(d, n, B, 1, ws.data_ptr(), ws.numel(), s)
-        if st:
-            raise self.vq.VQ3RError(st, "vq3r_gemv")
+        # the C call with its arguments bound once per batch size (on the stream current at that time, the
+        # default stream everywhere in this script): the decode step takes about 30 us, so per-call Python work
+        # (a stream object, tensor attributes) would otherwise starve the GPU
+        call = self._gemv_calls.get(B)
+        if call is None:
+            plans, ws, _, _ = self.moe[B]
+            fn, s = self.vq.lib().vq3r_gemv, self.torch.cuda.current_stream().cuda_stream
+            wp, wn = ws.data_ptr(), ws.numel()
+            args = [p[:2] for p in plans]
+            err = self.vq.VQ3RError
+
+            def call(g):
+                d, n = args[g % len(args)]
+                st = fn(d, n, B, 1, wp, wn, s)
+                if st:
+                    raise err(st, "vq3r_gemv")
+            self._gemv_calls[B] = call
+        call(group)
 
     def layer_gemv_plan(self, B):
         """One grouped call over the stacked w1, w3, w2 of every expert of the layer (shared x per kind):
