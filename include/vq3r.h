@@ -271,7 +271,13 @@ vq3r_status vq3r_train(const float* vecs, int64_t n, int iters, int nstages, flo
  * measurements are per token, page §1); this call is the prefill counterpart
  * of vq3r_gemv and reuses its TILES layout.  Summation order is the
  * library's: results agree with a binary64 product of the same bf16 weights
- * to about 1e-5 relative to rms(Y), not bit for bit.
+ * to about 1e-5 relative to rms(Y), not bit for bit.  The bf16 rounding of
+ * w_hat (relative error up to 2^-9 per weight) makes this product differ
+ * from vq3r_gemv's for the same token by about 1e-3 relative to rms(Y):
+ * vq3r_gemv carries each weight as a bf16 pair hi + lo (about 2^-17) on its
+ * tensor-core paths and in binary32 on its lookup paths.  A caller that needs
+ * the decode step's accuracy for a few prompt tokens can call vq3r_gemv with
+ * up to 32 tokens.
  *
  * One descriptor per matrix (up to VQ3R_GEMV_MAX_MATS), each with its own
  * tokens, e.g. the experts of an MoE layer and the tokens routed to each.
