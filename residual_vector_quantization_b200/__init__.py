@@ -29,7 +29,8 @@ EXPORTED = ["vq3r_encode", "vq3r_decode", "vq3r_gemv", "vq3r_gemv_workspace_size
             "vq3r_train", "vq3r_train_workspace_size", "vq4p_encode", "vq4p_decode", "vq4p_rel_frobenius_error",
             "vq4p_train", "vq4p_train_workspace_size", "vq3r_outliers", "vq3r_decode_outliers",
             "vq3r_rel_frobenius_error_outliers", "vq3r_rel_frobenius_outliers_workspace_size", "vq3r_gemv_outliers",
-            "vq3r_selftest_wait_timeout"]
+            "vq3r_selftest_wait_timeout", "vq4p_gemv", "vq3r_outliers_tiles_size", "vq3r_pack_outliers",
+            "vq3r_gemv_with_outliers"]
 
 
 class VQ3RError(RuntimeError):
