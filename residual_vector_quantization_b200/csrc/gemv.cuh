@@ -635,7 +635,9 @@ __device__ __forceinline__ void zero_rest(const GvParams& P, int tid) {
 // added after the CTA's last unit (1.22x, also with x staged in shared
 // memory, the words prefetched into L2 and the code warmed before
 // griddepcontrol.wait), one outlier per row in each lookup unit (1.25x), per
-// warp chunks between units (2.4x), a second launch (1.29x).
+// warp chunks between units (2.4x), a second launch (1.29x), and passes over
+// up to four outputs at once (all their words requested before any gather:
+// inline they spill the kernel, out of line 1.27x).
 template <int XDT>
 __device__ __forceinline__ void outlier_init_run(const GvParams& P, const ZeroJob& z, int tid) {
   const GvMat& M = P.m[z.m];
